@@ -1,0 +1,410 @@
+/*
+ * jfa_oracle.c -- plain fp64 CPU oracle for jagged attention (test infrastructure).
+ *
+ * THIS FILE IS TEST INFRASTRUCTURE.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg load it.  It shares no code, header or constant
+ * with the CUDA library; it is the written-out definition of what the library
+ * computes, slow on purpose, so that a reader can check it against the sources
+ * by eye:
+ *
+ *  [JT]  "Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a
+ *        Different Stack", FAQ "What is a jagged tensor?": samples are stored
+ *        packed, values plus offsets, with no padding.
+ *  [JFA] same page, "Bottleneck move 1: dense-sequence kernels to jagged
+ *        execution": attention computed directly on variable-length tensors,
+ *        with custom (additive) biases and asymmetric query / key-value lengths.
+ *  [GDPA] same section: attention-like modules whose softmax is replaced by a
+ *        pointwise GELU or SiLU.
+ *  [ASYM] "GEM Training: How Meta Doubled the Efficiency of Its LLM-Scale Ads
+ *        Foundation Model", "Challenge 1: Achieving High Per-GPU Utilization":
+ *        long-query/short-kv and short-query/long-kv shapes.
+ *  [MX]  "GEM Training ...", opening summary, and "Meta Enhances GEM Training
+ *        Efficiency ...", "Leveraging Compute Efficiency through Customized
+ *        Kernels": MXFP8 attention.  The element and scale formats follow the
+ *        OCP Microscaling Formats (MX) v1.0 specification (E4M3 elements, one
+ *        E8M0 power-of-two scale per 32 elements), which the pages only name.
+ *
+ * Everything the pages leave open is fixed by the readings listed in the
+ * design notes of this repository (scale 1/sqrt(d), bias added after scaling,
+ * bottom-right causal alignment, GDPA divided by the sequence's kv length,
+ * empty rows give zero output and LSE = -inf, natural-log LSE).
+ *
+ * Layouts: Q, O, dQ, dO are [total_q][H][d]; K, V, dK, dV are [total_kv][H][d];
+ * LSE is [total_q][H]; sequence b owns query rows [q_off[b], q_off[b+1]) and
+ * key/value rows [kv_off[b], kv_off[b+1]).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_ACT_SOFTMAX = 0, ORC_ACT_SILU = 1, ORC_ACT_GELU_TANH = 2 };
+enum { ORC_BIAS_NONE = 0, ORC_BIAS_RELPOS = 1, ORC_BIAS_DENSE = 2 };
+
+/* SiLU(x) = x * sigmoid(x) (Elfwing et al., 2018). */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+
+static double silu_grad(double x) {
+    double sg = 1.0 / (1.0 + exp(-x));
+    return sg * (1.0 + x * (1.0 - sg));
+}
+
+/* tanh-approximated GELU (Hendrycks & Gimpel, "Gaussian Error Linear Units",
+ * 2016): 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))). */
+static double gelu_tanh(double x) {
+    double c = sqrt(2.0 / M_PI);
+    double t = tanh(c * (x + 0.044715 * x * x * x));
+    return 0.5 * x * (1.0 + t);
+}
+
+static double gelu_tanh_grad(double x) {
+    double c = sqrt(2.0 / M_PI);
+    double t = tanh(c * (x + 0.044715 * x * x * x));
+    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * c * (1.0 + 3.0 * 0.044715 * x * x);
+}
+
+static double act_value(int act, double x) {
+    return act == ORC_ACT_SILU ? silu(x) : gelu_tanh(x);
+}
+
+static double act_derivative(int act, double x) {
+    return act == ORC_ACT_SILU ? silu_grad(x) : gelu_tanh_grad(x);
+}
+
+/* Causal validity with bottom-right alignment: query i may see key j when
+ * j <= i + (n_kv - n_q); for self-attention (n_q == n_kv) this is j <= i. */
+static int is_valid(int causal, int i, int j, int nq, int nkv) {
+    if (!causal) return 1;
+    return (long)j <= (long)i + (long)(nkv - nq);
+}
+
+/* Additive bias beta_h(i, j).
+ *  RELPOS: table[h][clamp(i - j, -C, C) + C], table length T = 2C + 1.
+ *  DENSE : block [H][n_q][n_kv] of sequence b, blocks concatenated in b order
+ *          starting at element dense_off (int64, computed by the caller loop). */
+static double bias_value(int kind, const double* bias, int relpos_len, int H, int h,
+                         int64_t dense_off, int nq, int nkv, int i, int j) {
+    (void)nq;
+    if (kind == ORC_BIAS_RELPOS) {
+        int C = (relpos_len - 1) / 2;
+        long r = (long)i - (long)j;
+        if (r < -C) r = -C;
+        if (r > C) r = C;
+        return bias[(int64_t)h * relpos_len + (r + C)];
+    }
+    if (kind == ORC_BIAS_DENSE) {
+        (void)H;
+        return bias[dense_off + ((int64_t)h * nq + i) * nkv + j];
+    }
+    return 0.0;
+}
+
+static int64_t* dense_offsets(int B, int H, const int32_t* q_off, const int32_t* kv_off) {
+    int64_t* off = (int64_t*)malloc(sizeof(int64_t) * (size_t)(B + 1));
+    off[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t nq = q_off[b + 1] - q_off[b];
+        int64_t nkv = kv_off[b + 1] - kv_off[b];
+        off[b + 1] = off[b] + (int64_t)H * nq * nkv;
+    }
+    return off;
+}
+
+/* OCP MX v1.0 E4M3 element encoding, round-to-nearest-even, saturating to the
+ * largest finite magnitude 448 = 1.75 * 2^8.  E4M3: 1 sign, 4 exponent bits
+ * (bias 7), 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; the
+ * pattern S.1111.111 is NaN and is never produced here. */
+uint8_t jfa_oracle_e4m3_encode(double y) {
+    uint8_t sign = (y < 0.0 || (y == 0.0 && signbit(y))) ? 0x80 : 0x00;
+    double a = fabs(y);
+    if (isnan(y)) return 0x7F;
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int E;
+    frexp(a, &E);              /* a = f * 2^E with f in [0.5, 1) */
+    int e = E - 1;             /* floor(log2 a) */
+    if (e < -6) e = -6;        /* below the smallest normal the quantum is fixed */
+    double quantum = ldexp(1.0, e - 3);
+    double n = nearbyint(a / quantum); /* default rounding mode: ties to even */
+    /* n * quantum is the rounded value; n in [0, 16] */
+    if (e == -6 && n < 8.0) {
+        return sign | (uint8_t)n; /* subnormal (or zero) */
+    }
+    if (n >= 16.0) { n = 8.0; e += 1; }
+    int code = ((e + 7) << 3) | ((int)n - 8);
+    if (code > 0x7E) code = 0x7E;
+    return sign | (uint8_t)code;
+}
+
+double jfa_oracle_e4m3_decode(uint8_t c) {
+    int s = c >> 7, ex = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (ex == 15 && m == 7) return NAN;
+    if (ex == 0) v = ldexp((double)m, -9);
+    else v = ldexp((double)(8 + m), ex - 10);
+    return s ? -v : v;
+}
+
+/* MX block quantisation of n_blocks contiguous blocks of 32 values.
+ * Shared exponent X = floor(log2(amax)) - 8 (8 = largest E4M3 exponent),
+ * clamped to the E8M0 range [-127, 127]; an all-zero block takes X = -127.
+ * Each element becomes E4M3(x * 2^-X); the scale byte is X + 127. */
+void jfa_oracle_quantize_mx(const double* x, int64_t n_blocks, uint8_t* codes, uint8_t* scales) {
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        const double* xb = x + blk * 32;
+        double amax = 0.0;
+        for (int t = 0; t < 32; ++t) amax = fmax(amax, fabs(xb[t]));
+        int X;
+        if (amax == 0.0) {
+            X = -127;
+        } else {
+            int E;
+            frexp(amax, &E);
+            X = (E - 1) - 8;
+            if (X < -127) X = -127;
+            if (X > 127) X = 127;
+        }
+        scales[blk] = (uint8_t)(X + 127);
+        for (int t = 0; t < 32; ++t) codes[blk * 32 + t] = jfa_oracle_e4m3_encode(ldexp(xb[t], -X));
+    }
+}
+
+/* Dequantise: value = E4M3(code) * 2^(scale - 127). */
+void jfa_oracle_dequantize_mx(const uint8_t* codes, const uint8_t* scales, int64_t n_blocks, double* out) {
+    for (int64_t blk = 0; blk < n_blocks; ++blk)
+        for (int t = 0; t < 32; ++t)
+            out[blk * 32 + t] = ldexp(jfa_oracle_e4m3_decode(codes[blk * 32 + t]), (int)scales[blk] - 127);
+}
+
+/* One query row of one (sequence, head): scores s_j for all keys, the softmax
+ * (or activation) weights w_j, and the row's output.  Returns the number of
+ * valid keys.  Work arrays s and w have n_kv entries. */
+typedef struct {
+    int B, H, d;
+    const int32_t *q_off, *kv_off;
+    const double *q, *k, *v;
+    int bias_kind;
+    const double* bias;
+    int relpos_len;
+    const int64_t* dense_off;
+    int act, causal;
+    double scale;
+    int quant_p; /* MXFP8: quantise exp(s - m) per 32 keys before P.V */
+} orc_problem;
+
+static const double* row_ptr(const double* base, int64_t row, int H, int h, int d) {
+    return base + (row * H + h) * (int64_t)d;
+}
+
+/* Computes s_j and the normalised weights p_j (softmax) or a_j (GDPA) of query
+ * row i.  For softmax also returns m (max) and l (sum of exp(s - m)); for a row
+ * without a valid key m = -inf and l = 0.  pv_weight receives the weights that
+ * multiply V in the forward output (equal to w unless P is quantised). */
+static void row_weights(const orc_problem* P, int b, int h, int i, double* s, double* w,
+                        double* pv_weight, double* m_out, double* l_out) {
+    int nq = P->q_off[b + 1] - P->q_off[b];
+    int nkv = P->kv_off[b + 1] - P->kv_off[b];
+    const double* qi = row_ptr(P->q, P->q_off[b] + i, P->H, h, P->d);
+    double m = -INFINITY;
+    for (int j = 0; j < nkv; ++j) {
+        const double* kj = row_ptr(P->k, P->kv_off[b] + j, P->H, h, P->d);
+        double dot = 0.0;
+        for (int c = 0; c < P->d; ++c) dot += qi[c] * kj[c];
+        s[j] = P->scale * dot +
+               bias_value(P->bias_kind, P->bias, P->relpos_len, P->H, h,
+                          P->dense_off ? P->dense_off[b] : 0, nq, nkv, i, j);
+        if (is_valid(P->causal, i, j, nq, nkv) && s[j] > m) m = s[j];
+    }
+    if (P->act == ORC_ACT_SOFTMAX) {
+        double l = 0.0;
+        for (int j = 0; j < nkv; ++j)
+            w[j] = is_valid(P->causal, i, j, nq, nkv) ? exp(s[j] - m) : 0.0;
+        for (int j = 0; j < nkv; ++j) l += w[j];
+        if (pv_weight) {
+            if (P->quant_p) {
+                /* quantise the unnormalised weights exp(s - m_final) in blocks of
+                 * 32 consecutive keys, counted from the sequence's first key */
+                for (int j0 = 0; j0 < nkv; j0 += 32) {
+                    double blk[32];
+                    uint8_t codes[32], sc;
+                    for (int t = 0; t < 32; ++t) blk[t] = (j0 + t < nkv) ? w[j0 + t] : 0.0;
+                    jfa_oracle_quantize_mx(blk, 1, codes, &sc);
+                    double deq[32];
+                    jfa_oracle_dequantize_mx(codes, &sc, 1, deq);
+                    for (int t = 0; t < 32 && j0 + t < nkv; ++t)
+                        pv_weight[j0 + t] = (l > 0.0) ? deq[t] / l : 0.0;
+                }
+            } else {
+                for (int j = 0; j < nkv; ++j) pv_weight[j] = (l > 0.0) ? w[j] / l : 0.0;
+            }
+        }
+        for (int j = 0; j < nkv; ++j) w[j] = (l > 0.0) ? w[j] / l : 0.0;
+        *m_out = m;
+        *l_out = l;
+    } else {
+        for (int j = 0; j < nkv; ++j)
+            w[j] = is_valid(P->causal, i, j, nq, nkv) ? act_value(P->act, s[j]) / (double)nkv : 0.0;
+        if (pv_weight)
+            for (int j = 0; j < nkv; ++j) pv_weight[j] = w[j];
+        *m_out = m;
+        *l_out = 0.0;
+    }
+}
+
+static void forward_item(const orc_problem* P, int b, int h, double* out, double* lse) {
+    int nq = P->q_off[b + 1] - P->q_off[b];
+    int nkv = P->kv_off[b + 1] - P->kv_off[b];
+    int n = nkv > 0 ? nkv : 1;
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* w = (double*)malloc(sizeof(double) * n);
+    double* pw = (double*)malloc(sizeof(double) * n);
+    for (int i = 0; i < nq; ++i) {
+        double m, l;
+        row_weights(P, b, h, i, s, w, pw, &m, &l);
+        double* oi = out + ((int64_t)(P->q_off[b] + i) * P->H + h) * P->d;
+        for (int c = 0; c < P->d; ++c) oi[c] = 0.0;
+        for (int j = 0; j < nkv; ++j) {
+            if (pw[j] == 0.0) continue;
+            const double* vj = row_ptr(P->v, P->kv_off[b] + j, P->H, h, P->d);
+            for (int c = 0; c < P->d; ++c) oi[c] += pw[j] * vj[c];
+        }
+        if (lse && P->act == ORC_ACT_SOFTMAX)
+            lse[(int64_t)(P->q_off[b] + i) * P->H + h] = (l > 0.0) ? m + log(l) : -INFINITY;
+    }
+    free(s);
+    free(w);
+    free(pw);
+}
+
+/* Analytic gradients of the forward above for one (sequence, head).
+ * softmax: D_i = dO_i . o_i, dp_ij = dO_i . v_j, ds_ij = p_ij (dp_ij - D_i)
+ * GDPA   : ds_ij = dp_ij act'(s_ij) / n_kv on valid (i, j), 0 elsewhere
+ * both   : dV_j += w_ij dO_i, dQ_i += scale sum_j ds_ij k_j,
+ *          dK_j += scale ds_ij q_i.
+ * The bias gets no gradient.  With quant_p the quantiser is a straight-through
+ * estimator, so the gradients are those of the unquantised weights. */
+static void backward_item(const orc_problem* P, int b, int h, const double* dout, double* dq,
+                          double* dk, double* dv) {
+    int nq = P->q_off[b + 1] - P->q_off[b];
+    int nkv = P->kv_off[b + 1] - P->kv_off[b];
+    int H = P->H, d = P->d;
+    int n = nkv > 0 ? nkv : 1;
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* w = (double*)malloc(sizeof(double) * n);
+    double* o = (double*)malloc(sizeof(double) * d);
+    for (int j = 0; j < nkv; ++j) {
+        double* dkj = dk + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
+        double* dvj = dv + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
+        for (int c = 0; c < d; ++c) dkj[c] = 0.0, dvj[c] = 0.0;
+    }
+    for (int i = 0; i < nq; ++i) {
+        double m, l;
+        row_weights(P, b, h, i, s, w, NULL, &m, &l);
+        const double* qi = row_ptr(P->q, P->q_off[b] + i, H, h, d);
+        const double* doi = dout + ((int64_t)(P->q_off[b] + i) * H + h) * d;
+        double* dqi = dq + ((int64_t)(P->q_off[b] + i) * H + h) * d;
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+        double Di = 0.0;
+        if (P->act == ORC_ACT_SOFTMAX) {
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int j = 0; j < nkv; ++j) {
+                const double* vj = row_ptr(P->v, P->kv_off[b] + j, H, h, d);
+                for (int c = 0; c < d; ++c) o[c] += w[j] * vj[c];
+            }
+            for (int c = 0; c < d; ++c) Di += doi[c] * o[c];
+        }
+        for (int j = 0; j < nkv; ++j) {
+            if (!is_valid(P->causal, i, j, nq, nkv)) continue;
+            const double* kj = row_ptr(P->k, P->kv_off[b] + j, H, h, d);
+            const double* vj = row_ptr(P->v, P->kv_off[b] + j, H, h, d);
+            double* dkj = dk + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
+            double* dvj = dv + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
+            double dp = 0.0;
+            for (int c = 0; c < d; ++c) dp += doi[c] * vj[c];
+            double ds;
+            if (P->act == ORC_ACT_SOFTMAX) ds = w[j] * (dp - Di);
+            else ds = dp * act_derivative(P->act, s[j]) / (double)nkv;
+            for (int c = 0; c < d; ++c) {
+                dvj[c] += w[j] * doi[c];
+                dqi[c] += P->scale * ds * kj[c];
+                dkj[c] += P->scale * ds * qi[c];
+            }
+        }
+    }
+    free(s);
+    free(w);
+    free(o);
+}
+
+static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_off,
+                         const int32_t* kv_off, const double* q, const double* k, const double* v,
+                         int bias_kind, const double* bias, int relpos_len, int act, int causal,
+                         double scale, int quant_p) {
+    P->B = B; P->H = H; P->d = d;
+    P->q_off = q_off; P->kv_off = kv_off;
+    P->q = q; P->k = k; P->v = v;
+    P->bias_kind = bias_kind; P->bias = bias; P->relpos_len = relpos_len;
+    P->dense_off = (bias_kind == ORC_BIAS_DENSE) ? dense_offsets(B, H, q_off, kv_off) : NULL;
+    P->act = act; P->causal = causal;
+    P->scale = scale > 0.0 ? scale : 1.0 / sqrt((double)d);
+    P->quant_p = quant_p;
+}
+
+/* Forward over all sequences b with seq_mask == NULL or seq_mask[b] != 0.
+ * Rows of sequences that are skipped are left untouched in out / lse. */
+int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
+                       const double* q, const double* k, const double* v, int bias_kind,
+                       const double* bias, int relpos_len, int act, int causal, double scale,
+                       int quant_p, const int32_t* seq_mask, double* out, double* lse,
+                       int nthreads) {
+    orc_problem P;
+    fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
+                 scale, quant_p);
+    long n_items = (long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long it = 0; it < n_items; ++it) {
+        int b = (int)(it / H), h = (int)(it % H);
+        if (seq_mask && !seq_mask[b]) continue;
+        forward_item(&P, b, h, out, lse);
+    }
+    free((void*)P.dense_off);
+    (void)nthreads;
+    return 0;
+}
+
+int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
+                        const double* q, const double* k, const double* v, int bias_kind,
+                        const double* bias, int relpos_len, int act, int causal, double scale,
+                        const int32_t* seq_mask, const double* dout, double* dq, double* dk,
+                        double* dv, int nthreads) {
+    orc_problem P;
+    fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
+                 scale, 0);
+    long n_items = (long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long it = 0; it < n_items; ++it) {
+        int b = (int)(it / H), h = (int)(it % H);
+        if (seq_mask && !seq_mask[b]) continue;
+        backward_item(&P, b, h, dout, dq, dk, dv);
+    }
+    free((void*)P.dense_off);
+    (void)nthreads;
+    return 0;
+}
+
+int jfa_oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
