@@ -1,0 +1,544 @@
+#!/usr/bin/env python
+"""Benchmark of the jagged-attention hot path (libjfa) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {jfa,reference}]
+                    [--workload self_bf16]
+
+One step = the whole path over one synthetic batch held in HBM: schedule +
+forward (scores, bias, mask, online softmax or GDPA activation, P.V, LSE) +
+backward (D = rowsum(dO*O), dQ, dK, dV), all through the C ABI.  The metric is
+TFLOP/s counted on valid (unpadded) query/key pairs only: forward 4*d per pair
+and head, backward 2.5x that (five GEMMs including the score recompute);
+softmax/exp/bias work is not counted.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronisation, timed with CUDA events on the launching stream; the
+max over ranks is reported.  Every input tensor of the default workload is
+larger than L2 (126 MB), so no L2 flush is needed between steps.  Under
+torchrun each rank draws its own batch (seed + rank) of the same workload:
+weak scaling, no collective on the data path.
+
+Also reported on one JSON line: per-kernel launch times from the library's
+event hooks (the dominant kernel's roofline fraction), the end-to-end number
+through the C ABI with host buffers (pinned host -> device copies of the
+inputs and device -> host copies of every result inside the timed region),
+a padded-dense baseline (torch SDPA on the max-padded batch, causal, no
+bias), the CPU oracle on a bounded sample of the same batch, and the SM
+clocks sampled during the timed region.
+
+``--impl reference`` times the fp64 CPU oracle (the only other implementation
+of this method) on the host cores, each step a bounded stratified sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "jagged attn fwd/bwd TFLOP/s (valid tokens); % of B200 dense BF16/FP8 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["jfa", "reference"], default="jfa")
+    ap.add_argument("--workload", default="self_bf16")
+    ap.add_argument("--act", default=None, help="override the workload's activation")
+    ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-padded", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-pairs", type=float, default=8e6,
+                    help="(query, key) pairs x heads in the CPU oracle's sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# work accounting
+# ---------------------------------------------------------------------------
+def visible_pairs(q_lens, kv_lens, causal):
+    """Per-sequence number of (query, key) pairs attention computes."""
+    out = np.zeros(len(q_lens), np.int64)
+    for b, (nq, nk) in enumerate(zip(q_lens, kv_lens)):
+        nq, nk = int(nq), int(nk)
+        if not causal:
+            out[b] = nq * nk
+        else:
+            i = np.arange(nq, dtype=np.int64)
+            out[b] = int(np.clip(i + 1 + nk - nq, 0, nk).sum())
+    return out
+
+
+def flops_of(p, pairs_per_seq=None):
+    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal) if pairs_per_seq is None else pairs_per_seq
+    f_fwd = 4.0 * p.d * p.H * float(pairs.sum())
+    return f_fwd, 2.5 * f_fwd
+
+
+def padded_flops(p):
+    L = int(max(p.max_q_len, p.max_kv_len))
+    per = L * (L + 1) // 2 if p.causal else L * L
+    f_fwd = 4.0 * p.d * p.H * p.B * per
+    return f_fwd, 2.5 * f_fwd
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, profiles
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons (every 200 ms)."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(", ") for r in self.tmp.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        mine = [r for r in rows if len(r) >= 10 and (self.uuid is None or r[1] == self.uuid)]
+        if not mine:
+            mine = [r for r in rows if len(r) >= 10 and r[0] == "0"]
+        if not mine:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        smax = [float(r[3]) for r in mine if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in mine for k in range(4) if r[6 + k].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(mine)}
+
+
+def kernel_source_hash(name):
+    src = {"tc_fwd": "jfa_tc.cu", "tc_bwd": "jfa_tc.cu", "simt_fwd": "jfa_simt.cu",
+           "simt_bwd_dq": "jfa_simt.cu", "simt_bwd_dkdv": "jfa_simt.cu"}.get(name)
+    if src is None:
+        return None
+    path = os.path.join(ROOT, "jagged_attention_recommender_jfa_b200", "csrc", src)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of that kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256") != kernel_source_hash(kernel):
+        return None
+    try:
+        return float(vals["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# reference arm / CPU baseline: the fp64 oracle on a bounded stratified sample
+# ---------------------------------------------------------------------------
+def cpu_sample_mask(p, target_pairs_heads):
+    """Sequences picked evenly over the length-sorted batch (shortest first)
+    until the sample holds ~target (pairs x heads)."""
+    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal) * p.H
+    order = np.argsort(pairs, kind="stable")
+    mask = np.zeros(p.B, np.int32)
+    total = 0
+    for stride in (64, 32, 16, 8, 4, 2, 1):
+        for idx in order[::stride]:
+            if mask[idx]:
+                continue
+            if total + pairs[idx] > target_pairs_heads and total > 0:
+                continue
+            mask[idx] = 1
+            total += int(pairs[idx])
+        if total >= 0.5 * target_pairs_heads:
+            break
+    return mask, pairs
+
+
+def run_oracle_step(p, mask, act):
+    import oracle
+    kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
+              causal=p.causal, seq_mask=mask)
+    o, l = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, **kw)
+    oracle.backward(p.q_off, p.kv_off, p.q, p.k, p.v, p.dout, **kw)
+
+
+def cpu_baseline(p, act, target):
+    import oracle
+    mask, pairs = cpu_sample_mask(p, target)
+    f_fwd = 4.0 * p.d * float((pairs * mask).sum())
+    t0 = time.perf_counter()
+    run_oracle_step(p, mask, act)
+    dt = time.perf_counter() - t0
+    n = int(mask.sum())
+    return {"value": 3.5 * f_fwd / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of {p.B} sequences (all {p.H} heads, stratified by length), "
+                      f"{int((pairs * mask).sum())} pair-heads, fwd+bwd fp64, {dt:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    from jagged_attention_recommender_jfa_b200.inputs import make_problem
+    import oracle
+    p = make_problem(args.workload, args.seed)
+    act = args.act or p.act
+    target = args.cpu_sample_pairs / 4
+    mask, pairs = cpu_sample_mask(p, target)
+    f_sample = 3.5 * 4.0 * p.d * float((pairs * mask).sum())
+    for _ in range(args.warmup):
+        run_oracle_step(p, mask, act)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle_step(p, mask, act)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = f_sample / dt / 1e12
+    n = int(mask.sum())
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "global_batch": p.B, "heads": p.H,
+                   "head_dim": p.d, "act": act, "causal": p.causal,
+                   "sample_sequences": n, "l2": "inputs larger than L2"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: {n} of {p.B} sequences (stratified by length), "
+                                   f"all heads, fwd+bwd fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# padded-dense baseline: torch SDPA on the max-padded batch
+# ---------------------------------------------------------------------------
+def padded_dense_baseline(p, dev, f_valid, iters=3):
+    L = int(max(p.max_q_len, p.max_kv_len))
+    need = 10 * p.B * p.H * L * p.d * 2
+    free, _ = torch.cuda.mem_get_info(dev)
+    if need > 0.6 * free:
+        return {"skipped": f"needs {need / 1e9:.1f} GB"}
+    import torch.nn.functional as F
+    try:
+        q = torch.randn(p.B, p.H, L, p.d, device=dev, dtype=torch.bfloat16, requires_grad=True)
+        k = torch.randn_like(q, requires_grad=True)
+        v = torch.randn_like(q, requires_grad=True)
+        go = torch.randn_like(q)
+
+        def once():
+            o = F.scaled_dot_product_attention(q, k, v, is_causal=p.causal)
+            o.backward(go)
+
+        once()
+        torch.cuda.synchronize(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(iters):
+            once()
+        e.record()
+        torch.cuda.synchronize(dev)
+        ms = s.elapsed_time(e) / iters
+        pf, pb = padded_flops(p)
+        return {"impl": "torch SDPA (padded to max_len, causal, no bias)", "ms_per_step": ms,
+                "valid_token_tflops": f_valid / (ms * 1e-3) / 1e12,
+                "padded_tflops": (pf + pb) / (ms * 1e-3) / 1e12, "max_len": L}
+    finally:
+        for name in ("q", "k", "v", "go"):
+            locals().pop(name, None)
+        torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# main arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl jfa needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from jagged_attention_recommender_jfa_b200 import jfa
+    from jagged_attention_recommender_jfa_b200.inputs import make_problem
+
+    p = make_problem(args.workload, args.seed + rank)
+    act = args.act or p.act
+    prob = jfa.problem_of(p)
+    path = jfa.jfa_path(prob, act, 0), jfa.jfa_path(prob, act, 1)
+    f_fwd, f_bwd = flops_of(p)
+    d = {n: getattr(p, n).to(dev).contiguous() for n in ("q", "k", "v", "dout", "q_off", "kv_off")}
+    bias = p.bias.to(dev).contiguous() if p.bias is not None else None
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+    ws_f = jfa.workspace(prob, False, dev)
+    ws_b = jfa.workspace(prob, True, dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        jfa.jfa_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"], bias, act,
+                        p.causal, out, lse, ws_f, stream=stream)
+        if marks is not None:
+            marks[1].record(stream)
+        jfa.jfa_backward(prob, d["q"], d["k"], d["v"], out, lse, d["dout"], d["q_off"],
+                         d["kv_off"], bias, act, p.causal, dq, dk, dv, ws_b, stream=stream)
+        if marks is not None:
+            marks[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    jfa.jfa_check_error(ws_f, stream)
+    jfa.jfa_check_error(ws_b, stream)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    marks = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    t_start, t_end = ev(), ev()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    jfa.jfa_profile_enable(True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(marks[k])
+    t_end.record(stream)
+    jfa.jfa_profile_enable(False)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    fwd_ms = sum(m[0].elapsed_time(m[1]) for m in marks) / args.steps
+    bwd_ms = sum(m[1].elapsed_time(m[2]) for m in marks) / args.steps
+    launches = jfa.jfa_profile_read()
+    jfa.jfa_check_error(ws_f, stream)
+    jfa.jfa_check_error(ws_b, stream)
+
+    ms_step = ms_total / args.steps
+    flops_rank = f_fwd + f_bwd
+    if world > 1:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step_max = float(t.item())
+        fl = torch.tensor([flops_rank], dtype=torch.float64, device=dev)
+        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
+        flops_all = float(fl.item())
+    else:
+        ms_step_max, flops_all = ms_step, flops_rank
+    value = flops_all / (ms_step_max * 1e-3) / 1e12
+
+    # per-kernel totals over the timed region
+    per = {}
+    for name, ms in launches:
+        c = per.setdefault(name, [0, 0.0])
+        c[0] += 1
+        c[1] += ms
+    dom = max(per.items(), key=lambda kv: kv[1][1])[0] if per else None
+    peaks, peak_src = load_peaks()
+    kernels = {n: {"launches": c, "total_ms": round(t, 4), "share": round(t / ms_total, 4)}
+               for n, (c, t) in sorted(per.items(), key=lambda kv: -kv[1][1])}
+    roofline = None
+    if dom is not None:
+        avg_s = per[dom][1] / per[dom][0] * 1e-3
+        d_ = p.d
+        pairs = f_fwd / (4.0 * d_)
+        algo = {"tc_fwd": f_fwd, "tc_bwd": f_bwd, "simt_fwd": f_fwd,
+                "simt_bwd_dq": 6.0 * d_ * pairs, "simt_bwd_dkdv": 8.0 * d_ * pairs}.get(dom)
+        if dom.startswith("tc_"):
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            bound, unit = "tensor", "TFLOP/s"
+            note = f"bf16 dense, sustained, of {peak_src}"
+        else:
+            mhz = peaks.get("sm_max_mhz", 1965.0)
+            peak = SM_COUNT * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+            bound, unit = "alu", "TFLOP/s"
+            note = f"fp32 FMA: {SM_COUNT} SMs x {FP32_LANES_PER_SM} lanes x 2 x {mhz:.0f} MHz"
+        achieved = algo / avg_s / 1e12 if algo else None
+        traffic = recorded_traffic(dom, args.workload)
+        roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak if achieved else None,
+                    "traffic": traffic, "peak_source": note,
+                    "algorithmic_flops_per_launch": algo, "avg_launch_ms": avg_s * 1e3}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if path[0] == 1 else "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "global_batch": p.B * world, "heads": p.H,
+                   "head_dim": p.d, "act": act, "causal": p.causal, "bias": p.bias_kind,
+                   "total_tokens": p.total_q, "max_len": p.max_q_len,
+                   "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs larger than L2 (each of Q/K/V/dO > 126 MB); no flush",
+                   "kernel_path": {"fwd": "tcgen05" if path[0] == 1 else "cuda-core",
+                                   "bwd": "tcgen05" if path[1] == 1 else "cuda-core"}},
+        "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "pct_of_bf16_burst_peak": {"fwd": 100 * f_fwd / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                   "bwd": 100 * f_bwd / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": len(launches),
+        "clocks": clock_info,
+    }
+
+    # end to end through the C ABI with host buffers
+    if not args.no_e2e:
+        result["e2e"] = e2e_leg(args, p, prob, act, dev, stream, jfa, f_fwd + f_bwd, world)
+    if rank == 0 and world == 1 and not args.no_padded:
+        result["padded_dense_baseline"] = padded_dense_baseline(p, dev, f_fwd + f_bwd)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(p, act, args.cpu_sample_pairs)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
+    """Same metric with pinned host inputs copied in and every result copied
+    out inside the timed region."""
+    host_in = {n: getattr(p, n).contiguous().pin_memory() for n in ("q", "k", "v", "dout")}
+    host_in["q_off"] = p.q_off.contiguous().pin_memory()
+    host_in["kv_off"] = p.kv_off.contiguous().pin_memory()
+    if p.bias is not None:
+        host_in["bias"] = p.bias.contiguous().pin_memory()
+    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    out = torch.empty_like(dev_in["q"])
+    lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
+    dq, dk, dv = torch.empty_like(dev_in["q"]), torch.empty_like(dev_in["k"]), torch.empty_like(dev_in["v"])
+    ws_f = jfa.workspace(prob, False, dev)
+    ws_b = jfa.workspace(prob, True, dev)
+    results = [out, dq, dk, dv] + ([lse] if lse is not None else [])
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in results]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in results)
+
+    def step():
+        for n, t in host_in.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_off"],
+                        dev_in["kv_off"], dev_in.get("bias"), act, p.causal, out, lse, ws_f,
+                        stream=stream)
+        jfa.jfa_backward(prob, dev_in["q"], dev_in["k"], dev_in["v"], out, lse, dev_in["dout"],
+                         dev_in["q_off"], dev_in["kv_off"], dev_in.get("bias"), act, p.causal,
+                         dq, dk, dv, ws_b, stream=stream)
+        for h, t in zip(host_out, results):
+            h.copy_(t, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / args.e2e_steps
+    flops_all = flops_rank
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        fl = torch.tensor([flops_rank], dtype=torch.float64, device=dev)
+        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
+        flops_all = float(fl.item())
+    return {"value": flops_all / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": args.e2e_steps}
+
+
+if __name__ == "__main__":
+    main()

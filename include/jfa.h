@@ -1,0 +1,196 @@
+/*
+ * jfa.h -- C ABI of libjfa: jagged (offsets-indexed, unpadded) attention
+ * forward and backward for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Attention run directly on variable-length user-sequence
+ * tensors stored as values plus offsets, with custom additive biases and
+ * asymmetric query / key-value lengths ("Meta GEM Training Efficiency: Why
+ * LLM-Scale Recommenders Need a Different Stack", section "Bottleneck move 1:
+ * dense-sequence kernels to jagged execution", and its FAQ "What is a jagged
+ * tensor?"); the GDPA variant that replaces softmax with a pointwise SiLU or
+ * GELU (same section); asymmetric shapes as in "GEM Training: How Meta
+ * Doubled the Efficiency of Its LLM-Scale Ads Foundation Model", "Challenge 1:
+ * Achieving High Per-GPU Utilization"; and MXFP8 attention (same page, opening
+ * summary) with the OCP MX v1.0 E4M3 element / E8M0 scale formats.
+ *
+ * For sequence b, query rows are [q_offsets[b], q_offsets[b+1]) and key/value
+ * rows [kv_offsets[b], kv_offsets[b+1]); n_q(b), n_kv(b) are their counts.
+ * With tau = scale (<= 0 selects 1/sqrt(head_dim)) and beta the bias:
+ *   s_ij  = tau * <q_i, k_j> + beta_h(i, j)
+ *   valid = !causal || j <= i + n_kv(b) - n_q(b)      (bottom-right aligned)
+ *   softmax: o_i = sum_valid softmax_j(s_ij) v_j,  lse_i = log sum_valid e^{s_ij}
+ *   GDPA   : o_i = sum_valid act(s_ij) / n_kv(b) * v_j           (no lse)
+ * A query row with no valid key gets o_i = 0 and lse_i = -inf; its gradients
+ * are 0.  The bias receives no gradient.
+ *
+ * Layouts (all row-major, head_dim contiguous):
+ *   q, out, dout, dq : [total_q ][heads][head_dim]
+ *   k, v, dk, dv     : [total_kv][heads][head_dim]
+ *   lse              : [total_q ][heads]  fp32, natural log
+ *   bias RELPOS      : fp32 [heads][relpos_len], beta_h(i,j) =
+ *                      table[h][clamp(i - j, -C, C) + C], C = (relpos_len-1)/2
+ *   bias DENSE_JAGGED: element type of q; for each sequence in order a block
+ *                      [heads][n_q(b)][n_kv(b)] (keys contiguous); blocks are
+ *                      concatenated, so block b starts at
+ *                      sum_{b'<b} heads * n_q(b') * n_kv(b') (int64).
+ * Element type: JFA_F32 -> float; JFA_BF16 and JFA_MXFP8 -> bfloat16 (MXFP8
+ * computes on E4M3 operands quantised inside the call; outputs stay bf16).
+ *
+ * Conventions shared by every entry point:
+ *  - Ownership: the caller owns every buffer.  All tensor, offset and
+ *    workspace pointers are DEVICE pointers (cudaMalloc / torch); the problem
+ *    descriptor is a HOST pointer read during the call only.  The library
+ *    allocates nothing and keeps no state between calls.
+ *  - Inputs are never written.  Outputs are written only on valid rows of
+ *    their own sequences.
+ *  - Streams: all work is enqueued on `stream` (NULL = legacy default stream);
+ *    there is no host synchronisation.  max_q_len / max_kv_len / total_* come
+ *    from the host so that no device->host copy is needed to size grids.
+ *  - Alignment: tensors 16-byte aligned.
+ *  - Errors are returned, never thrown; nothing aborts or traps.  Argument
+ *    errors are detected on the host before anything is enqueued.  Offsets
+ *    are validated ON THE DEVICE (off[0] == 0, non-decreasing, last == total,
+ *    lengths <= max_*_len); a bad batch enqueues no work on invalid rows and
+ *    leaves JFA_ERR_BAD_OFFSETS in the workspace's error word, which
+ *    jfa_check_error() reads.  Asynchronous CUDA faults surface as
+ *    JFA_ERR_CUDA.  jfa_last_error() describes the last non-OK status of the
+ *    calling thread.
+ */
+#ifndef JFA_H_
+#define JFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* jfa_stream_t;
+
+typedef enum {
+    JFA_OK = 0,
+    JFA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size or enum */
+    JFA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. head_dim 96) */
+    JFA_ERR_WORKSPACE = 3,        /* workspace smaller than jfa_workspace_bytes() */
+    JFA_ERR_CUDA = 4,             /* a CUDA launch or runtime call failed */
+    JFA_ERR_TIMEOUT = 5,          /* a bounded on-device wait gave up */
+    JFA_ERR_BAD_OFFSETS = 6       /* offsets failed the on-device validation */
+} jfa_status;
+
+typedef enum { JFA_F32 = 0, JFA_BF16 = 1, JFA_MXFP8 = 2 } jfa_dtype;
+
+typedef enum { JFA_ACT_SOFTMAX = 0, JFA_ACT_SILU = 1, JFA_ACT_GELU_TANH = 2 } jfa_act;
+
+typedef enum { JFA_BIAS_NONE = 0, JFA_BIAS_RELPOS = 1, JFA_BIAS_DENSE_JAGGED = 2 } jfa_bias_kind;
+
+/* Problem descriptor (host memory).  head_dim in {32, 64, 128}; the bf16
+ * tensor-core kernels need head_dim == 128, other sizes run on the CUDA-core
+ * kernels. */
+typedef struct {
+    int32_t batch;       /* number of sequences B >= 0 */
+    int32_t heads;       /* H >= 1 (query and key/value heads are equal) */
+    int32_t head_dim;    /* d */
+    int32_t max_q_len;   /* >= every n_q(b) */
+    int32_t max_kv_len;  /* >= every n_kv(b) */
+    int64_t total_q;     /* q_offsets[B] */
+    int64_t total_kv;    /* kv_offsets[B] */
+    jfa_dtype dtype;
+    float scale;         /* tau; <= 0 selects 1/sqrt(head_dim) */
+    jfa_bias_kind bias_kind;
+    int32_t relpos_len;  /* odd table length for JFA_BIAS_RELPOS, else ignored */
+} jfa_problem;
+
+/* Bytes of device workspace that jfa_forward (backward = 0) or jfa_backward
+ * (backward = 1) needs for this problem; 0 if the descriptor is invalid.
+ * The workspace holds the tile schedule, the error word and, for the
+ * backward, the fp32 dQ accumulator and the row terms D = rowsum(dO * O). */
+size_t jfa_workspace_bytes(const jfa_problem* problem, int backward);
+
+/* Forward pass.  q, k, v: device tensors as above; q_offsets, kv_offsets:
+ * device int32 [batch + 1]; bias: device pointer in the layout of
+ * problem->bias_kind (NULL for JFA_BIAS_NONE); act: softmax or GDPA
+ * activation; causal: 0/1; out: device [total_q][heads][head_dim] in the
+ * element type; lse: device fp32 [total_q][heads] for softmax (may be NULL if
+ * not needed), ignored for GDPA; workspace: device buffer of ws_bytes >=
+ * jfa_workspace_bytes(problem, 0), 16-byte aligned. */
+jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k, const void* v,
+                       const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                       jfa_act act, int causal, void* out, float* lse, void* workspace,
+                       size_t ws_bytes, jfa_stream_t stream);
+
+/* Backward pass: gradients of <dout, out> with respect to q, k and v.
+ * out and lse are the forward's results (softmax needs both; GDPA needs
+ * neither and accepts NULL); dout: device like out.  dq/dk/dv: device
+ * outputs in the element type (every valid row is written).  workspace:
+ * >= jfa_workspace_bytes(problem, 1). */
+jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k,
+                        const void* v, const void* out, const float* lse, const void* dout,
+                        const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                        jfa_act act, int causal, void* dq, void* dk, void* dv, void* workspace,
+                        size_t ws_bytes, jfa_stream_t stream);
+
+/* MX (OCP v1.0) quantisation of a bf16 tensor x [rows][heads][d] to E4M3
+ * codes [rows][heads][d] (same layout, one byte each) and E8M0 scales.
+ * Shared exponent X = floor(log2(amax of the block)) - 8, clamped to
+ * [-127, 127] (-127 for an all-zero block); codes = RNE(x * 2^-X) saturated
+ * to +-448; scale byte = X + 127.
+ *   along_rows == 0: blocks are 32 consecutive elements of d (d % 32 == 0);
+ *                    scales [rows][heads][d/32]; offsets may be NULL.
+ *   along_rows == 1: blocks are 32 consecutive rows of one sequence, counted
+ *                    from its first row (offsets: device int32 [batch+1]);
+ *                    the last block of a sequence is zero-padded; scales
+ *                    [n_blocks][heads][d] with sequence b's blocks starting
+ *                    at sum_{b'<b} ceil(n(b')/32).  The caller sizes scales
+ *                    for rows/32 + batch blocks (an upper bound); max_len
+ *                    bounds every sequence length (it sizes the grid).
+ * Bit-exact with the OCP rounding rules. */
+jfa_status jfa_quantize_mxfp8(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
+                              const int32_t* offsets, int32_t batch, int32_t max_len,
+                              int along_rows, uint8_t* codes, uint8_t* scales,
+                              jfa_stream_t stream);
+
+/* The longest-first tile schedule that jfa_forward (backward = 0: items are
+ * query tiles) or jfa_backward (backward = 1: items are key/value tiles) runs,
+ * written to items (device int32 [capacity][4] = {sequence, head, tile,
+ * cost}) and its length to *count (device int32).  cost = number of (query,
+ * key) pairs the tile computes; order = cost descending, then sequence, tile,
+ * head ascending.  tile is the tile height in rows (16..256, multiple of 16).
+ * Exposed so that the schedule can be checked; the passes build their own.
+ * workspace: >= jfa_workspace_bytes(problem, backward). */
+jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,
+                        const int32_t* kv_offsets, int causal, int backward, int tile,
+                        int32_t* items, int64_t capacity, int32_t* count, void* workspace,
+                        size_t ws_bytes, jfa_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the workspace's device error
+ * word: JFA_OK, JFA_ERR_BAD_OFFSETS or JFA_ERR_TIMEOUT. */
+jfa_status jfa_check_error(void* workspace, jfa_stream_t stream);
+
+/* Thread-local message for the last non-OK status returned to this thread. */
+const char* jfa_last_error(void);
+
+/* Kernel timing for measurement tools.  jfa_profile_enable(1) starts a fresh
+ * record on the calling thread: from then on every kernel that jfa_forward,
+ * jfa_backward, jfa_schedule or jfa_quantize_mxfp8 launches from this thread
+ * is bracketed by two CUDA events recorded on the call's stream (the events
+ * are created by the library and reused; no device memory is allocated).
+ * jfa_profile_enable(0) stops recording and keeps the record.
+ * jfa_profile_read() waits for the recorded events and writes, for up to
+ * `capacity` launches in launch order, the duration in milliseconds and the
+ * kernel id; it returns the number of recorded launches (which may exceed
+ * capacity) or -1 on a CUDA error.  jfa_kernel_name() names a kernel id. */
+jfa_status jfa_profile_enable(int enable);
+int jfa_profile_read(float* ms, int32_t* kernel_ids, int32_t capacity);
+const char* jfa_kernel_name(int32_t kernel_id);
+
+/* Which kernel family jfa_forward / jfa_backward will use for this problem:
+ * 0 = CUDA-core (fp32 arithmetic), 1 = tcgen05 tensor-core. */
+int jfa_path(const jfa_problem* problem, jfa_act act, int backward);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JFA_H_ */

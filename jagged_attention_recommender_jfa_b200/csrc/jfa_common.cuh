@@ -1,0 +1,213 @@
+// Shared device-side definitions of libjfa: workspace layout, kernel argument
+// block, element conversions and the on-device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "jfa.h"
+
+namespace jfa {
+
+// ---------------------------------------------------------------------------
+// Workspace layout.  Everything the passes need between kernels lives in the
+// caller's workspace; offsets are 256-byte aligned.
+//
+//   [header 256 B]  err, item_count, pair_count, queue counters
+//   dense_off       int64 [B + 1]    start of sequence b's dense bias block
+//   pair_bt         int32 [P_max][2] (sequence, tile) of each schedule pair
+//   pair_cost       int64 [P_max]    pairs computed by that tile
+//   items           int4  [P_max*H]  {b, h, tile, cost} in execution order
+//   (backward)      kv_items, D = rowsum(dO*O) fp32 [total_q*H],
+//                   dQ accumulator fp32 [total_q*H*d] (tensor-core path)
+// P_max covers the smallest schedule tile (16 rows), so one workspace serves
+// every tile height.
+// ---------------------------------------------------------------------------
+struct WsHeader {
+    int32_t err;
+    int32_t item_count;
+    int32_t pair_count;
+    int32_t queue;
+    int32_t kv_item_count;
+    int32_t kv_pair_count;
+    int32_t kv_queue;
+    int32_t pad[57];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr int kMinTile = 16;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t dense_off, pair_bt, pair_cost, items;           // forward schedule
+    size_t kv_pair_bt, kv_pair_cost, kv_items;             // backward schedule
+    size_t dterm, dq_acc;                                  // backward rows
+    size_t total;
+    int64_t pairs_max_q, pairs_max_kv;
+};
+
+// Upper bound of sum_b ceil(n(b) / tile) given only host-side sizes.
+inline int64_t pairs_bound(int64_t batch, int64_t max_len, int64_t total, int tile) {
+    int64_t a = batch * ((max_len + tile - 1) / tile);
+    int64_t b = total / tile + batch;
+    return a < b ? a : b;
+}
+
+inline WsLayout ws_layout(const jfa_problem& p, bool backward, bool need_dq_acc) {
+    WsLayout L{};
+    size_t off = sizeof(WsHeader);
+    L.pairs_max_q = pairs_bound(p.batch, p.max_q_len, p.total_q, kMinTile);
+    L.pairs_max_kv = pairs_bound(p.batch, p.max_kv_len, p.total_kv, kMinTile);
+    L.dense_off = off;  off = align256(off + sizeof(int64_t) * (size_t)(p.batch + 1));
+    L.pair_bt = off;    off = align256(off + sizeof(int32_t) * 2 * (size_t)L.pairs_max_q);
+    L.pair_cost = off;  off = align256(off + sizeof(int64_t) * (size_t)L.pairs_max_q);
+    L.items = off;      off = align256(off + sizeof(int4) * (size_t)L.pairs_max_q * p.heads);
+    if (backward) {
+        L.kv_pair_bt = off;   off = align256(off + sizeof(int32_t) * 2 * (size_t)L.pairs_max_kv);
+        L.kv_pair_cost = off; off = align256(off + sizeof(int64_t) * (size_t)L.pairs_max_kv);
+        L.kv_items = off;     off = align256(off + sizeof(int4) * (size_t)L.pairs_max_kv * p.heads);
+        L.dterm = off;        off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads);
+        if (need_dq_acc) {
+            L.dq_acc = off;
+            off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads * p.head_dim);
+        }
+    }
+    L.total = off;
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel arguments (one block for every attention kernel).
+// ---------------------------------------------------------------------------
+struct AttnArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const int32_t* q_off;
+    const int32_t* kv_off;
+    const void* bias;
+    const int64_t* dense_off;  // int64 [B+1] (dense bias only)
+    int bias_kind;
+    int relpos_len;
+    int B, H;
+    int causal;
+    int act;
+    float scale;
+    void* out;
+    float* lse;
+    const int4* items;
+    const int32_t* item_count;
+    WsHeader* hdr;
+    // backward
+    const void* dout;
+    const float* o_for_d;  // unused placeholder (O is read through `out`)
+    float* dterm;          // D = rowsum(dO * O), fp32 [total_q*H]
+    void* dq;
+    void* dk;
+    void* dv;
+    float* dq_acc;
+};
+
+// ---------------------------------------------------------------------------
+// Element conversions.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Load 4 consecutive elements as float4 (16-byte aligned for float, 8-byte
+// for bf16).
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+// ---------------------------------------------------------------------------
+// Launch timing (jfa_profile_*): prof_begin / prof_end bracket every launch.
+// ---------------------------------------------------------------------------
+enum KernelId {
+    K_SCHED_PREPARE = 0,
+    K_SCHED_RANK,
+    K_SIMT_FWD,
+    K_SIMT_BWD_PRE,
+    K_SIMT_BWD_DQ,
+    K_SIMT_BWD_DKDV,
+    K_QUANT_ALONG_D,
+    K_QUANT_ALONG_ROWS,
+    K_TC_FWD,
+    K_TC_BWD_PRE,
+    K_TC_BWD,
+    K_TC_DQ_FINALIZE,
+    K_TC_FWD_MXFP8,
+    K_COUNT
+};
+void prof_begin(cudaStream_t st);
+void prof_end(cudaStream_t st, int kernel_id);
+
+__device__ __forceinline__ void set_error(WsHeader* hdr, int code) {
+    atomicCAS(&hdr->err, 0, code);
+}
+
+// Activations of the GDPA variant.
+//   SiLU(x) = x * sigmoid(x)
+//   GELU_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+__device__ __forceinline__ float act_f(int act, float x) {
+    if (act == JFA_ACT_SILU) return x / (1.0f + expf(-x));
+    const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    float t = tanhf(c * (x + 0.044715f * x * x * x));
+    return 0.5f * x * (1.0f + t);
+}
+
+__device__ __forceinline__ float act_grad_f(int act, float x) {
+    if (act == JFA_ACT_SILU) {
+        float sg = 1.0f / (1.0f + expf(-x));
+        return sg * (1.0f + x * (1.0f - sg));
+    }
+    const float c = 0.7978845608028654f;
+    float t = tanhf(c * (x + 0.044715f * x * x * x));
+    return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * c * (1.0f + 3.0f * 0.044715f * x * x);
+}
+
+// Additive bias beta_h(i, j) of sequence b (i, j relative to the sequence).
+template <typename T>
+__device__ __forceinline__ float bias_at(const AttnArgs& a, int b, int h, int nq, int nkv, int i, int j) {
+    if (a.bias_kind == JFA_BIAS_RELPOS) {
+        const int C = (a.relpos_len - 1) >> 1;
+        int r = i - j;
+        r = r < -C ? -C : (r > C ? C : r);
+        return __ldg(reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len + (r + C));
+    }
+    if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
+        const T* base = reinterpret_cast<const T*>(a.bias);
+        return to_f(base[a.dense_off[b] + ((int64_t)h * nq + i) * nkv + j]);
+    }
+    return 0.0f;
+}
+
+// Bottom-right causal validity.
+__device__ __forceinline__ bool key_visible(int causal, int i, int j, int nq, int nkv) {
+    return !causal || j <= i + (nkv - nq);
+}
+
+}  // namespace jfa

@@ -21,15 +21,18 @@ MXFP8 run):
                     table of 16385 entries; MXFP8 compute, bf16 in/out.
 
 Draw order from ``numpy.random.default_rng(seed)`` (PCG64): query lengths,
-key/value lengths (when separate), Q, K, V, bias, dO.  Values are drawn as
-float32 standard normals and rounded to the stored dtype with round-to-
-nearest-even (torch's conversion); a relative-position table for a bf16 run is
+key/value lengths (when separate), then one 63-bit seed each for Q, K, V, bias
+and dO; each tensor is filled from PCG64 streams spawned from its seed, one
+stream per 2^22 elements (parallel, thread-count independent).  Values are
+drawn as float32 standard normals and rounded to the stored dtype with
+round-to-nearest-even (torch's conversion); a relative-position table for a bf16 run is
 rounded to bf16 and stored as fp32, so that every consumer sees the same
 values.
 """
 from __future__ import annotations
 
 import dataclasses
+import os
 from typing import Optional
 
 import numpy as np
@@ -119,11 +122,34 @@ def _offsets(lens) -> torch.Tensor:
     return torch.from_numpy(off.astype(np.int32))
 
 
-def _normal(rng, shape, std, dtype):
-    x = rng.standard_normal(size=shape, dtype=np.float32)
+_CHUNK = 1 << 22  # elements per independent stream chunk
+
+
+def _fill_chunk(seed_seq, out, lo, hi, std):
+    g = np.random.Generator(np.random.PCG64(seed_seq))
+    g.standard_normal(size=hi - lo, dtype=np.float32, out=out[lo:hi])
     if std != 1.0:
-        x *= np.float32(std)
-    t = torch.from_numpy(x)
+        out[lo:hi] *= np.float32(std)
+
+
+def _normal(rng, shape, std, dtype):
+    """Standard normals (times std) in chunks of 2^22 elements, chunk c drawn
+    from child c of a SeedSequence seeded by one draw of ``rng``, so large
+    tensors fill in parallel and the values do not depend on the thread
+    count."""
+    n = int(np.prod(shape))
+    root = np.random.SeedSequence(int(rng.integers(0, 2**63 - 1)))
+    n_chunks = max(1, (n + _CHUNK - 1) // _CHUNK)
+    children = root.spawn(n_chunks)
+    flat = np.empty(n, np.float32)
+    if n_chunks == 1:
+        _fill_chunk(children[0], flat, 0, n, std)
+    else:
+        import concurrent.futures as cf
+        with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda c: _fill_chunk(children[c], flat, c * _CHUNK,
+                                              min(n, (c + 1) * _CHUNK), std), range(n_chunks)))
+    t = torch.from_numpy(flat.reshape(shape))
     if dtype == "f32":
         return t
     return t.to(torch.bfloat16)

@@ -100,12 +100,24 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _item_mask(seq_mask, B, H):
+    """Per-(sequence, head) mask from a per-sequence [B] or per-item [B*H] mask."""
+    if seq_mask is None:
+        return None
+    m = _i32(seq_mask).reshape(-1)
+    if m.size == B:
+        m = np.repeat(m, H)
+    assert m.size == B * H
+    return np.ascontiguousarray(m.astype(np.int32))
+
+
 def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0,
             act="softmax", causal=False, scale=0.0, quant_p=False, seq_mask=None,
             nthreads=0):
     """fp64 forward.  Returns (out [total_q,H,d], lse [total_q,H] or None).
 
-    Rows of sequences excluded by ``seq_mask`` are NaN in the result."""
+    ``seq_mask`` ([B] per sequence or [B*H] per (sequence, head)) selects what
+    is computed; everything else is NaN in the result."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     q64, k64, v64 = _f64(q), _f64(k), _f64(v)
     B = len(q_off) - 1
@@ -113,7 +125,7 @@ def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0
     b64 = _f64(bias) if bias is not None else None
     out = np.full((total_q, H, d), np.nan)
     lse = np.full((total_q, H), np.nan)
-    mask = _i32(seq_mask) if seq_mask is not None else None
+    mask = _item_mask(seq_mask, B, H)
     _lib().jfa_oracle_forward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                               _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                               ACT[act], int(bool(causal)), float(scale), int(bool(quant_p)),
@@ -133,7 +145,7 @@ def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpo
     dq = np.full((total_q, H, d), np.nan)
     dk = np.full((total_kv, H, d), np.nan)
     dv = np.full((total_kv, H, d), np.nan)
-    mask = _i32(seq_mask) if seq_mask is not None else None
+    mask = _item_mask(seq_mask, B, H)
     _lib().jfa_oracle_backward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                                _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                                ACT[act], int(bool(causal)), float(scale), _ptr(mask),

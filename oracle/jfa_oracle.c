@@ -353,12 +353,12 @@ static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_o
     P->quant_p = quant_p;
 }
 
-/* Forward over all sequences b with seq_mask == NULL or seq_mask[b] != 0.
- * Rows of sequences that are skipped are left untouched in out / lse. */
+/* Forward over all (sequence b, head h) items with item_mask == NULL or
+ * item_mask[b * H + h] != 0.  Skipped items are left untouched in out / lse. */
 int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                        const double* q, const double* k, const double* v, int bias_kind,
                        const double* bias, int relpos_len, int act, int causal, double scale,
-                       int quant_p, const int32_t* seq_mask, double* out, double* lse,
+                       int quant_p, const int32_t* item_mask, double* out, double* lse,
                        int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
@@ -370,7 +370,7 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
 #endif
     for (long it = 0; it < n_items; ++it) {
         int b = (int)(it / H), h = (int)(it % H);
-        if (seq_mask && !seq_mask[b]) continue;
+        if (item_mask && !item_mask[it]) continue;
         forward_item(&P, b, h, out, lse);
     }
     free((void*)P.dense_off);
@@ -381,7 +381,7 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
 int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                         const double* q, const double* k, const double* v, int bias_kind,
                         const double* bias, int relpos_len, int act, int causal, double scale,
-                        const int32_t* seq_mask, const double* dout, double* dq, double* dk,
+                        const int32_t* item_mask, const double* dout, double* dq, double* dk,
                         double* dv, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
@@ -393,7 +393,7 @@ int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t
 #endif
     for (long it = 0; it < n_items; ++it) {
         int b = (int)(it / H), h = (int)(it % H);
-        if (seq_mask && !seq_mask[b]) continue;
+        if (item_mask && !item_mask[it]) continue;
         backward_item(&P, b, h, dout, dq, dk, dv);
     }
     free((void*)P.dense_off);
