@@ -6,6 +6,10 @@ Tolerances (written here, applied element by element on every valid row):
   LSE (fp32 accumulation) : max |err| <= 1e-3
   fp32 CUDA-core path     : max |err| <= 1e-4 (stricter internal target) and the bf16 gate
   schedules / offsets     : bit-exact
+A result stored as bf16 carries, on top of the computation's error, the final
+rounding to bf16 (half an ulp of the value: 2^-9 relative, e.g. 0.031 for a
+gradient entry of 10).  The max bound for a bf16 tensor is therefore
+2e-2 + half_ulp_bf16(|reference|) per element; the mean bound is unchanged.
 """
 import numpy as np
 import pytest
@@ -56,7 +60,14 @@ def _rows(off, seq_mask):
     return np.concatenate(idx) if idx else np.zeros(0, np.int64)
 
 
+def half_ulp_bf16(x):
+    """Half a unit in the last place of bf16 (8 significant bits) at |x|."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(ax)) - 8)
+
+
 def compare(name, gpu, ref, rows, max_tol, mean_tol=None):
+    bf16_out = gpu.dtype == torch.bfloat16
     g = gpu.float().cpu().numpy()[rows].astype(np.float64)
     r = ref[rows]
     if g.size == 0:
@@ -64,9 +75,11 @@ def compare(name, gpu, ref, rows, max_tol, mean_tol=None):
     finite = np.isfinite(r)
     assert np.array_equal(np.isfinite(g), finite), f"{name}: non-finite pattern differs"
     err = np.abs(g[finite] - r[finite])
+    bound = max_tol + (half_ulp_bf16(r[finite]) if bf16_out else 0.0)
     mx = float(err.max()) if err.size else 0.0
     mn = float(err.mean()) if err.size else 0.0
-    assert mx <= max_tol, f"{name}: max abs err {mx:.3e} > {max_tol}"
+    worst = float((err - bound).max()) if err.size else -1.0
+    assert worst <= 0.0, f"{name}: max abs err {mx:.3e} exceeds {max_tol} (+ bf16 half-ulp)"
     if mean_tol is not None:
         assert mn <= mean_tol, f"{name}: mean abs err {mn:.3e} > {mean_tol}"
     # -inf LSE rows must match exactly
