@@ -64,6 +64,10 @@ def parse_args():
     ap.add_argument("--workload", default="self_bf16")
     ap.add_argument("--act", default=None, help="override the workload's activation")
     ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's number of sequences (profiling captures)")
+    ap.add_argument("--max-len", type=int, default=None,
+                    help="override the workload's length clip (profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
@@ -165,7 +169,7 @@ class ClockSampler:
 
 
 def kernel_source_hash(name):
-    src = {"tc_fwd": "jfa_tc.cu", "tc_bwd": "jfa_tc.cu", "simt_fwd": "jfa_simt.cu",
+    src = {"tc_fwd": "jfa_tc_fwd.cu", "tc_bwd": "jfa_tc_bwd.cu", "simt_fwd": "jfa_simt.cu",
            "simt_bwd_dq": "jfa_simt.cu", "simt_bwd_dkdv": "jfa_simt.cu"}.get(name)
     if src is None:
         return None
@@ -244,7 +248,7 @@ def reference_arm(args, rank, world):
         return
     from jagged_attention_recommender_jfa_b200.inputs import make_problem
     import oracle
-    p = make_problem(args.workload, args.seed)
+    p = make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len)
     act = args.act or p.act
     target = args.cpu_sample_pairs / 4
     mask, pairs = cpu_sample_mask(p, target)
@@ -339,7 +343,7 @@ def main():
     from jagged_attention_recommender_jfa_b200 import jfa
     from jagged_attention_recommender_jfa_b200.inputs import make_problem
 
-    p = make_problem(args.workload, args.seed + rank)
+    p = make_problem(args.workload, args.seed + rank, B=args.batch, max_len=args.max_len)
     act = args.act or p.act
     prob = jfa.problem_of(p)
     path = jfa.jfa_path(prob, act, 0), jfa.jfa_path(prob, act, 1)
@@ -451,7 +455,9 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if path[0] == 1 else "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "global_batch": p.B * world, "heads": p.H,
+        "config": {"workload": args.workload if args.batch is None and args.max_len is None
+                   else f"{args.workload} (B={p.B}, max_len={args.max_len})",
+                   "global_batch": p.B * world, "heads": p.H,
                    "head_dim": p.d, "act": act, "causal": p.causal, "bias": p.bias_kind,
                    "total_tokens": p.total_q, "max_len": p.max_q_len,
                    "parallelism": f"dp{world} (independent batches)",

@@ -185,6 +185,31 @@ jfa_status jfa_profile_enable(int enable);
 int jfa_profile_read(float* ms, int32_t* kernel_ids, int32_t capacity);
 const char* jfa_kernel_name(int32_t kernel_id);
 
+/* Forward pass for callers that cannot allocate device memory.
+ *
+ * No counterpart in the source pages: this is a deployment convenience.
+ * Same operation, arguments, layouts and errors as jfa_forward, minus the
+ * workspace.  Some callers have no way to obtain a workspace: a plugin
+ * inside a host framework that owns the whole device memory pool and exposes
+ * no allocator, or a serving loop that forbids allocation after start-up.
+ * This entry point allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library call); its scratch is a fixed 8 MiB __device__ array inside the
+ * library, held by every GPU that loads the library until the process exits.
+ *  - The first call on a device looks up that array's device address with
+ *    that device current (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture.
+ *  - Problems whose jfa_workspace_bytes(problem, 0) exceeds 8 MiB are
+ *    rejected with JFA_ERR_WORKSPACE (e.g. about 16k query tiles x heads).
+ *  - Every call shares the one array and it keeps the last call's contents;
+ *    calls whose work overlaps on the GPU (other streams, other host threads)
+ *    race on it and must be serialised by the caller.
+ *  - The on-device error word lives in that array too; jfa_check_error()
+ *    cannot reach it, so check outputs instead of the error word. */
+jfa_status jfa_forward_fixed_scratch(const jfa_problem* problem, const void* q, const void* k,
+                                     const void* v, const int32_t* q_offsets,
+                                     const int32_t* kv_offsets, const void* bias, jfa_act act,
+                                     int causal, void* out, float* lse, jfa_stream_t stream);
+
 /* Which kernel family jfa_forward / jfa_backward will use for this problem:
  * 0 = CUDA-core (fp32 arithmetic), 1 = tcgen05 tensor-core. */
 int jfa_path(const jfa_problem* problem, jfa_act act, int backward);

@@ -53,6 +53,7 @@ struct Profiler {
     }
 };
 thread_local Profiler g_prof;
+thread_local char g_msg[512] = "";
 
 const char* const kKernelNames[K_COUNT] = {
     "sched_prepare", "sched_rank", "simt_fwd", "simt_bwd_pre", "simt_bwd_dq", "simt_bwd_dkdv",
@@ -62,6 +63,14 @@ const char* const kKernelNames[K_COUNT] = {
 }  // namespace
 
 namespace jfa {
+jfa_status set_last_error(jfa_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
 void prof_begin(cudaStream_t st) {
     if (!g_prof.on) return;
     cudaEvent_t e = g_prof.next();
@@ -76,8 +85,6 @@ void prof_end(cudaStream_t st, int kernel_id) {
 }  // namespace jfa
 
 namespace {
-
-thread_local char g_msg[512] = "";
 
 jfa_status fail(jfa_status s, const char* fmt, ...) {
     va_list ap;

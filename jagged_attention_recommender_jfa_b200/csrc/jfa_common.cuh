@@ -165,6 +165,10 @@ enum KernelId {
 void prof_begin(cudaStream_t st);
 void prof_end(cudaStream_t st, int kernel_id);
 
+// Records the thread-local message jfa_last_error() returns and passes the
+// status through.
+jfa_status set_last_error(jfa_status s, const char* fmt, ...);
+
 __device__ __forceinline__ void set_error(WsHeader* hdr, int code) {
     atomicCAS(&hdr->err, 0, code);
 }

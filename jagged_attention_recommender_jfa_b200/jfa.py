@@ -38,7 +38,8 @@ STATUS_NAMES = {0: "JFA_OK", 1: "JFA_ERR_INVALID_ARGUMENT", 2: "JFA_ERR_UNSUPPOR
 # Every symbol include/jfa.h declares.
 EXPORTS = ("jfa_workspace_bytes", "jfa_forward", "jfa_backward", "jfa_quantize_mxfp8",
            "jfa_schedule", "jfa_check_error", "jfa_last_error", "jfa_path",
-           "jfa_profile_enable", "jfa_profile_read", "jfa_kernel_name")
+           "jfa_profile_enable", "jfa_profile_read", "jfa_kernel_name",
+           "jfa_forward_fixed_scratch")
 
 
 class JfaError(RuntimeError):
@@ -92,6 +93,8 @@ def load():
         lib.jfa_profile_read.restype = i32
         lib.jfa_kernel_name.argtypes = [i32]
         lib.jfa_kernel_name.restype = ctypes.c_char_p
+        lib.jfa_forward_fixed_scratch.argtypes = [PP, P, P, P, P, P, P, i32, i32, P, P, P]
+        lib.jfa_forward_fixed_scratch.restype = i32
         _LIB = lib
         return lib
 
@@ -152,6 +155,16 @@ def jfa_forward(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out,
                               _addr(q_offsets), _addr(kv_offsets), _addr(bias),
                               ACT.get(act, act), int(bool(causal)), _addr(out), _addr(lse),
                               _addr(workspace), int(ws_bytes), _stream(stream)))
+
+
+def jfa_forward_fixed_scratch(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out,
+                              lse, stream=None):
+    """Forward without a workspace: for callers that cannot allocate device
+    memory (scratch is a fixed 8 MiB array inside the library; see jfa.h)."""
+    _check(load().jfa_forward_fixed_scratch(ctypes.byref(problem), _addr(q), _addr(k), _addr(v),
+                                            _addr(q_offsets), _addr(kv_offsets), _addr(bias),
+                                            ACT.get(act, act), int(bool(causal)), _addr(out),
+                                            _addr(lse), _stream(stream)))
 
 
 def jfa_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act, causal,
