@@ -82,6 +82,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
 }
 
+// BIAS: 0 none, 1 relative-position (window in shared memory when it fits,
+// else through L1), 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.
+template <int BIAS, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
@@ -100,12 +103,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     kv_end = max(kv_end, 0);
     const int n_tiles = (kv_end + BN - 1) / BN;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool softmax = a.act == JFA_ACT_SOFTMAX;
+    constexpr bool softmax = SOFTMAX;
 
     // relative-position window: i - j in [lo, lo + tab_len)
     const int tab_lo = row0 - kv_end + 1;
     const int tab_len = kv_end + BM - 1;
-    const bool tab_in_smem = a.bias_kind == JFA_BIAS_RELPOS && tab_len <= P.tab_cap;
+    const bool tab_in_smem = BIAS == 1 && tab_len <= P.tab_cap;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const int C = (a.relpos_len - 1) >> 1;
         const float* tab_g = reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
-        const int64_t dense_row = (a.bias_kind == JFA_BIAS_DENSE_JAGGED && i < nq)
+        const int64_t dense_row = (BIAS == 2 && i < nq)
                                       ? a.dense_off[b] + ((int64_t)h * nq + i) * nkv : 0;
         uint8_t* prow = smem + kOffP + r * 128;
         float m_used = -CUDART_INF_F, l = 0.f;
@@ -247,30 +250,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             // scale, bias, mask (log2 domain for softmax, natural for GDPA)
             const int jmax_vis = a.causal ? min(nkv - 1, i + shift) : nkv - 1;  // last visible key
+            const int nvis = i < nq ? min(BN, jmax_vis - j0 + 1) : 0;  // visible columns: [0, nvis)
+            // bias (log2 units), added in place
+            if (BIAS == 1 && tab_in_smem) {
+                const float* tb = tab + (i - j0 - tab_lo);  // tb[-c] = bias(i, j0 + c)
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = fmaf(x[c], sc, tb[-c]);
+            } else if (BIAS == 1) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    int rr = i - (j0 + c);
+                    rr = rr < -C ? -C : (rr > C ? C : rr);
+                    x[c] = fmaf(x[c], sc, __ldg(tab_g + rr + C) * kLog2e);
+                }
+            } else if (BIAS == 2) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    x[c] = fmaf(x[c], sc, c < nvis ? __bfloat162float(dense[dense_row + j0 + c]) * kLog2e : 0.f);
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] *= sc;
+            }
+            if (__any_sync(0xffffffffu, nvis < BN)) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) x[c] = c < nvis ? x[c] : -CUDART_INF_F;
+            }
             float tmax = -CUDART_INF_F;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const int jj = j0 + c;
-                const bool vis = (jj <= jmax_vis) && (i < nq);
-                float v = -CUDART_INF_F;
-                if (vis) {
-                    float bias = 0.f;
-                    if (a.bias_kind == JFA_BIAS_RELPOS) {
-                        if (tab_in_smem) {
-                            bias = tab[(i - jj) - tab_lo];
-                        } else {
-                            int rr = i - jj;
-                            rr = rr < -C ? -C : (rr > C ? C : rr);
-                            bias = __ldg(tab_g + rr + C) * kLog2e;
-                        }
-                    } else if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
-                        bias = __bfloat162float(dense[dense_row + jj]) * kLog2e;
-                    }
-                    v = fmaf(x[c], sc, bias);
-                }
-                x[c] = v;
-                tmax = fmaxf(tmax, v);
-            }
+            for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
             if (softmax) {
                 // lazy rescale: keep the reference maximum unless it grew by > 2^8
                 const bool need = tmax > m_used + kRescaleThreshold;
@@ -293,19 +300,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     l = 0.f;
                 }
                 m_used = m_new;
-                float psum = 0.f;
+                // ex2(-inf) = 0 masks the invisible columns; a row with no visible
+                // key yet uses reference 0 so that -inf - ref stays -inf
+                const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
+                float psum0 = 0.f, psum1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const float p = (x[c] == -CUDART_INF_F) ? 0.f : ex2(x[c] - m_used);
-                    x[c] = p;
-                    psum += p;
+                for (int c = 0; c < BN; c += 2) {
+                    x[c] = ex2(x[c] - ref);
+                    x[c + 1] = ex2(x[c + 1] - ref);
+                    psum0 += x[c];
+                    psum1 += x[c + 1];
                 }
-                l += psum;
+                l += psum0 + psum1;
             } else {
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
                     const float s_nat = x[c] * (1.0f / kLog2e);
-                    x[c] = (x[c] == -CUDART_INF_F) ? 0.f : act_f(a.act, s_nat) * inv_n;
+                    x[c] = c < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
                 }
             }
             // P row -> shared memory, K-major, 128-byte swizzle (chunk ^ row%8)
@@ -433,13 +444,19 @@ cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStrea
         smem = base;
     }
     P.tab_cap = tab_need;
-    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    if (e != cudaSuccess) return e;
     int64_t grid = pairs_bound(p.batch, p.max_q_len, p.total_q, BM) * p.heads;
     if (grid <= 0) return cudaSuccess;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
+    const bool sm = a.act == JFA_ACT_SOFTMAX;
+    void (*kern)(FwdParams) = nullptr;
+    if (bias == 0) kern = sm ? tc_fwd_kernel<0, true> : tc_fwd_kernel<0, false>;
+    else if (bias == 1) kern = sm ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
+    else kern = sm ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    if (e != cudaSuccess) return e;
     prof_begin(st);
-    tc_fwd_kernel<<<(unsigned)grid, kThreads, smem, st>>>(P);
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(P);
     prof_end(st, K_TC_FWD);
     return cudaGetLastError();
 }
