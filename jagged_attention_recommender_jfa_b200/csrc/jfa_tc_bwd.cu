@@ -14,12 +14,15 @@
 //                      P^T  = exp2(S^T - LSE), dS^T = P^T (dP^T - D)
 //                             (or GDPA: act(S)/n_kv, dP act'(S)/n_kv)
 //                      dV  += P^T dO,  dK += dS^T Q             (TMEM)
-//                      dQ_t = dS K  -> added to the fp32 accumulator with
-//                             vector reductions (red.global.add.v4.f32)
+//                      dQ_t = dS K  -> staged in shared memory (fp32,
+//                             128B-swizzled 32-column chunks) and added to
+//                             the fp32 accumulator by TMA reduce-add
 //   tc_bwd_dq_finalize  dQ = bf16(scale * accumulator).
 //
-// Warp roles as in the forward: warp 0 TMA, warp 1 MMA, warps 2..5 one
-// key row (or, for dQ, one query row) per thread.
+// Warp roles: warp 0 TMA, warp 1 MMA, warps 2..9 score warps in two groups
+// of four; a thread owns one key row (or, for dQ, one query row) and half of
+// its 128 columns (group 0: columns 0-63, group 1: 64-127).  The backward
+// needs no row reduction (LSE and D are given), so the halves never talk.
 // TMEM columns: dV [0,128), dK [128,256), S^T and dQ_t [256,384), dP^T [384,512).
 #include <math_constants.h>
 
@@ -34,7 +37,7 @@ bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, in
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kBox = 128 * 128;
 constexpr uint32_t kTile = 2 * kBox;
 constexpr uint32_t kOffK = 0;
@@ -67,6 +70,7 @@ struct BwdParams {
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     CUtensorMap tm_do;
+    CUtensorMap tm_dq;  // fp32 accumulator, boxes of 32 columns x 128 rows, 128B swizzle
     AttnArgs a;
     int tab_cap;
 };
@@ -86,9 +90,24 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                  : "memory");
 }
 
-__device__ __forceinline__ void named_sync_softmax() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+__device__ __forceinline__ void named_sync_score() {
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
+
+// TMA reduce-add of a shared-memory tile into global memory (no multicast).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x,
+                                                  int y, int z) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+        " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Stores the 32 values of chunk c4 (columns 32*c4 .. +31) of row r into a
 // K-major 128B-swizzled bf16 tile.
@@ -143,9 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->ds_full, 4);
+        mbar_init(&bars->ds_full, 8);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 4);
+        mbar_init(&bars->dq_empty, 1);
         mbar_init(&bars->fin, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -178,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tma_prefetch_desc(&P.tm_k);
             tma_prefetch_desc(&P.tm_v);
             tma_prefetch_desc(&P.tm_do);
+            tma_prefetch_desc(&P.tm_dq);
             mbar_arrive_expect_tx(&bars->kv_full, 2 * kTile);
             tma_load_3d(smem + kOffK, &P.tm_k, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, h, k0 + j0);
@@ -240,23 +260,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------ score warps
-        const int wq = warp & 3;
+        const int wq = warp & 3;                 // TMEM lane quarter
+        const int grp = (warp - 2) >> 2;         // column half: 0 -> [0,64), 1 -> [64,128)
         const int r = wq * 32 + lane;            // key row (S^T, dV, dK) / query row (dQ)
         const int j = j0 + r;                    // key index within the sequence
         const bool jvalid = j < nkv;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-        const uint32_t tdV = tmem + lane_addr, tdK = tmem + lane_addr + 128;
-        const uint32_t tS = tmem + lane_addr + 256, tdP = tmem + lane_addr + 384;
+        const uint32_t cofs = (uint32_t)grp * 64;
+        const uint32_t tdV = tmem + lane_addr + cofs, tdK = tmem + lane_addr + 128 + cofs;
+        const uint32_t tS = tmem + lane_addr + 256 + cofs, tdP = tmem + lane_addr + 384 + cofs;
         const float sc = a.scale * kLog2e;
         const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
         const int C = (a.relpos_len - 1) >> 1;
         const float* tab_g = reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_base = (a.bias_kind == JFA_BIAS_DENSE_JAGGED) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
+        const bool leader = (warp == 2 && lane == 0);
         bool ok = true;
         for (int t = 0; ok && t < nt; ++t) {
             const int qb0 = i_start + t * BM;    // query index of the tile's row 0
-            {
+            if (grp == 0) {
                 const int qi = qb0 + r;
                 float l2 = CUDART_INF_F, dv = 0.f;
                 if (qi < nq && softmax) {
@@ -267,100 +290,141 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 lse2_s[r] = l2;
                 dd_s[r] = dv;
             }
-            named_sync_softmax();
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr));
-            if (!ok) break;
+            named_sync_score();
+            // leave only here, right after a barrier, so that every score warp
+            // runs the same sequence of named barriers; failed waits below only
+            // set the CTA's abort flag
+            if (*abort_flag) { ok = false; break; }
+            mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr);
             tc_fence_after();
             // key rows past the sequence end (neighbour data) must not reach dS K;
             // S^T = K Q^T of the first tile has completed, so K may be edited now
-            if (t == 0 && !jvalid) zero_row(smem + kOffK, r);
+            if (t == 0 && grp == 0 && !jvalid) zero_row(smem + kOffK, r);
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
 #pragma unroll 1
-            for (int c4 = 0; c4 < BM / 32; ++c4) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c4 = grp * 2 + cc;         // 32-column chunk of this thread
                 uint32_t us[32], up[32];
-                tmem_ld32(tS + c4 * 32, us);
-                tmem_ld32(tdP + c4 * 32, up);
+                tmem_ld32(tS + cc * 32, us);
+                tmem_ld32(tdP + cc * 32, up);
                 tmem_wait_ld();
+                const int qc0 = qb0 + c4 * 32;       // query index of the chunk's column 0
+                const bool all_vis = jvalid && (qc0 + 31 < nq) && (qc0 >= imin_vis);
+                const bool none_vis = !jvalid || qc0 >= nq || (qc0 + 31 < imin_vis);
                 float pv[32], dsv[32];
+                if (none_vis) {
 #pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const int il = c4 * 32 + u;
-                    const int qi = qb0 + il;
-                    const bool vis = jvalid && qi < nq && qi >= imin_vis;
-                    float p = 0.f, ds = 0.f;
-                    if (vis) {
-                        float bias = 0.f;
-                        if (a.bias_kind == JFA_BIAS_RELPOS) {
-                            if (tab_in_smem) {
-                                bias = tab[(qi - j) - tab_lo];
-                            } else {
-                                int rr = qi - j;
-                                rr = rr < -C ? -C : (rr > C ? C : rr);
-                                bias = __ldg(tab_g + rr + C) * kLog2e;
-                            }
-                        } else if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
-                            bias = __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e;
+                    for (int u = 0; u < 32; ++u) pv[u] = 0.f, dsv[u] = 0.f;
+                } else {
+                    float s2[32];
+                    if (a.bias_kind == JFA_BIAS_RELPOS && tab_in_smem) {
+                        const float* tb = tab + (qc0 - j - tab_lo);   // tb[u] = bias(qc0 + u, j)
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) s2[u] = fmaf(__uint_as_float(us[u]), sc, tb[u]);
+                    } else if (a.bias_kind == JFA_BIAS_RELPOS) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            int rr = qc0 + u - j;
+                            rr = rr < -C ? -C : (rr > C ? C : rr);
+                            s2[u] = fmaf(__uint_as_float(us[u]), sc, __ldg(tab_g + rr + C) * kLog2e);
                         }
-                        const float s2 = fmaf(__uint_as_float(us[u]), sc, bias);
-                        const float dp = __uint_as_float(up[u]);
-                        if (softmax) {
-                            p = ex2(s2 - lse2_s[il]);
-                            ds = p * (dp - dd_s[il]);
-                        } else {
-                            const float sn = s2 * (1.0f / kLog2e);
-                            p = act_f(a.act, sn) * inv_n;
-                            ds = dp * act_grad_f(a.act, sn) * inv_n;
+                    } else if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const int qi = qc0 + u;
+                            const float bv = (jvalid && qi < nq)
+                                ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
+                            s2[u] = fmaf(__uint_as_float(us[u]), sc, bv);
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) s2[u] = __uint_as_float(us[u]) * sc;
+                    }
+                    const float* l2c = lse2_s + c4 * 32;
+                    const float* ddc = dd_s + c4 * 32;
+                    if (softmax) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float p = ex2(s2[u] - l2c[u]);
+                            pv[u] = p;
+                            dsv[u] = p * (__uint_as_float(up[u]) - ddc[u]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float sn = s2[u] * (1.0f / kLog2e);
+                            pv[u] = act_f(a.act, sn) * inv_n;
+                            dsv[u] = __uint_as_float(up[u]) * act_grad_f(a.act, sn) * inv_n;
                         }
                     }
-                    pv[u] = p;
-                    dsv[u] = ds;
+                    if (!all_vis) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const int qi = qc0 + u;
+                            const bool vis = jvalid && qi < nq && qi >= imin_vis;
+                            pv[u] = vis ? pv[u] : 0.f;
+                            dsv[u] = vis ? dsv[u] : 0.f;
+                        }
+                    }
                 }
                 store_chunk_bf16(smem + kOffPT, r, c4, pv);
                 store_chunk_bf16(smem + kOffDST, r, c4, dsv);
             }
             // query rows past the sequence end must not reach dV / dK
             if (qb0 + r >= nq) {
-                zero_row(smem + kOffQ, r);
-                zero_row(smem + kOffDO, r);
+                if (grp == 0) zero_row(smem + kOffQ, r);
+                else zero_row(smem + kOffDO, r);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->ds_full);
-            // dQ of this query tile: row r of TMEM = query qb0 + r
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr));
-            if (!ok) break;
+            // dQ of this query tile: TMEM row r = query qb0 + r; staged as fp32
+            // 32-column chunks (128B swizzle) over the P^T / dS^T buffers, which
+            // the finished MMAs no longer read
+            mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr);
             tc_fence_after();
-            const int qi = qb0 + r;
-            float* acc = a.dq_acc + ((int64_t)(q0 + qi) * a.H + h) * HD;
+            const bool qvalid = qb0 + r < nq;
 #pragma unroll 1
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c4 = grp * 2 + cc;
                 uint32_t u[32];
-                tmem_ld32(tS + c4 * 32, u);
+                tmem_ld32(tS + cc * 32, u);
                 tmem_wait_ld();
-                if (qi < nq) {
+                uint8_t* row = smem + kOffPT + c4 * (128 * 128) + r * 128;
 #pragma unroll
-                    for (int v = 0; v < 32; v += 4)
-                        red_add_v4(acc + c4 * 32 + v, __uint_as_float(u[v]), __uint_as_float(u[v + 1]),
-                                   __uint_as_float(u[v + 2]), __uint_as_float(u[v + 3]));
+                for (int v = 0; v < 8; ++v) {
+                    uint4 w = qvalid ? make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3])
+                                     : make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(row + ((v ^ (r & 7)) << 4)) = w;
                 }
             }
+            fence_proxy_async_smem();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dq_empty);
+            named_sync_score();
+            if (leader && !*abort_flag) {
+                const int z = q0 + qb0;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    tma_reduce_add_3d(&P.tm_dq, smem + kOffPT + c4 * (128 * 128), c4 * 32, h, z);
+                bulk_commit();
+                bulk_wait_read_all();  // staging may be overwritten once the reads are done
+            }
+            if (leader) mbar_arrive(&bars->dq_empty);
         }
+        if (leader) bulk_wait_all();
         // ------------------------------------------------------ epilogue
         if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort_flag, a.hdr));
-        if (ok) {
+        if (ok && !*abort_flag) {
             tc_fence_after();
-            __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + j) * a.H + h) * HD;
-            __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + ((int64_t)(k0 + j) * a.H + h) * HD;
+            __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
+            __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
 #pragma unroll 1
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t uk[32], uv[32];
                 if (nt > 0) {
-                    tmem_ld32(tdK + c4 * 32, uk);
-                    tmem_ld32(tdV + c4 * 32, uv);
+                    tmem_ld32(tdK + cc * 32, uk);
+                    tmem_ld32(tdV + cc * 32, uv);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
@@ -378,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         wv.y = pack_bf16(__uint_as_float(uv[t + 2]), __uint_as_float(uv[t + 3]));
                         wv.z = pack_bf16(__uint_as_float(uv[t + 4]), __uint_as_float(uv[t + 5]));
                         wv.w = pack_bf16(__uint_as_float(uv[t + 6]), __uint_as_float(uv[t + 7]));
-                        *reinterpret_cast<uint4*>(dkrow + c4 * 32 + t) = wk;
-                        *reinterpret_cast<uint4*>(dvrow + c4 * 32 + t) = wv;
+                        *reinterpret_cast<uint4*>(dkrow + cc * 32 + t) = wk;
+                        *reinterpret_cast<uint4*>(dvrow + cc * 32 + t) = wv;
                     }
                 }
             }
@@ -436,6 +500,31 @@ __global__ void __launch_bounds__(256) tc_bwd_dq_finalize(const float* __restric
 
 constexpr int kSmemLimitBwd = 232448;
 
+// fp32 accumulator [rows][heads][128] as a 3-D tensor (d, head, row); boxes of
+// 32 d x 1 head x 128 rows (128 bytes inner) with the 128-byte swizzle.
+static bool make_tmap_dq_acc(CUtensorMap* map, void* base, int64_t rows, int heads) {
+    typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 4, (cuuint64_t)heads * HD * 4};
+    cuuint32_t box[3] = {32, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                                cudaStream_t st) {
     const int64_t rows = p.total_q * p.heads;
@@ -452,6 +541,7 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
         !make_tmap_rows_heads_d(&P.tm_v, a.v, p.total_kv, p.heads) ||
         !make_tmap_rows_heads_d(&P.tm_do, a.dout, p.total_q, p.heads))
         return cudaErrorInvalidValue;
+    if (!make_tmap_dq_acc(&P.tm_dq, a.dq_acc, p.total_q, p.heads)) return cudaErrorInvalidValue;
     P.a = kv;
     const int base = 1024 + (int)kOffTab;
     int tab_need = (p.bias_kind == JFA_BIAS_RELPOS) ? (p.max_q_len + BN - 1) : 0;

@@ -36,26 +36,26 @@ using namespace sm100;
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NS = 2;                       // key/value stages
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;               // warp 0 TMA, warp 1 MMA, warps 2..9 softmax
 constexpr uint32_t kBox = 128 * 128;        // bytes of one [128 rows][64 bf16] box
 constexpr uint32_t kTile = 2 * kBox;        // one 128 x 128 bf16 tile (two boxes)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;
-constexpr uint32_t kOffV = kOffK + NS * kTile;
-constexpr uint32_t kOffP = kOffV + NS * kTile;
-constexpr uint32_t kOffBar = kOffP + kTile;  // 196608
-constexpr uint32_t kOffTab = kOffBar + 256;
+constexpr uint32_t kOffK = kOffQ + kTile;        // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTile;    // 2 stages
+constexpr uint32_t kOffP = kOffV + 2 * kTile;
+constexpr uint32_t kOffBar = kOffP + kTile;      // 196608
+constexpr uint32_t kOffRed = kOffBar + 256;      // row-max exchange [2][2][128] + l [2][128]
+constexpr uint32_t kOffTab = kOffRed + 3072;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;    // log2 units
+constexpr float kRescaleThreshold = 8.0f;        // log2 units
 
 struct Bars {
     uint64_t q_full;
-    uint64_t kv_full[NS];
-    uint64_t kv_empty[NS];
-    uint64_t s_full;
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full[2];
     uint64_t p_full;
-    uint64_t o_full;
+    uint64_t pv_done;
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -82,16 +82,29 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
 }
 
+__device__ __forceinline__ void named_sync_softmax() {
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
 // BIAS: 0 none, 1 relative-position (window in shared memory when it fits,
 // else through L1), 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.
+//
+// Pipeline (tensor core): QK_0, QK_1, then for each j: [P_j ready] PV_j,
+// QK_{j+2}.  S is double-buffered in TMEM (S_0 at column 0, S_1 at 128), so
+// the score MMA of tile j+1 runs while the softmax warps work on tile j.
+// O lives at column 256.  P goes through shared memory (one buffer): the
+// softmax of tile j writes it only after P.V of tile j-1 has completed.
+// Each softmax thread owns one query row and one 64-column half of it; the
+// two halves exchange their partial row maxima through shared memory.
 template <int BIAS, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
     extern __shared__ uint8_t smem_dyn[];
-    // 1024-byte alignment for the swizzle atoms
     uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+    float* red = reinterpret_cast<float*>(smem + kOffRed);   // [2 parity][2 half][128 rows]
+    float* lred = red + 512;                                   // [2 half][128 rows]
     float* tab = reinterpret_cast<float*>(smem + kOffTab);
 
     const int4 it = a.items[blockIdx.x];
@@ -112,19 +125,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+            mbar_init(&bars->s_full[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 4);
-        mbar_init(&bars->o_full, 1);
+        mbar_init(&bars->p_full, 8);
+        mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&bars->tmem_base, 256);
+        tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
     if (tab_in_smem) {
@@ -154,63 +169,67 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, q0 + row0);
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
-                const int s = j % NS;
-                if (j >= NS && !mbar_wait(&bars->kv_empty[s], ((j / NS) - 1) & 1, abort_flag, a.hdr))
-                    break;
-                uint8_t* kd = smem + kOffK + s * kTile;
-                uint8_t* vd = smem + kOffV + s * kTile;
-                mbar_arrive_expect_tx(&bars->kv_full[s], 2 * kTile);
+                const int s = j & 1;
+                const uint32_t par = ((j >> 1) - 1) & 1;
                 const int z = k0 + j * BN;
-                tma_load_3d(kd, &P.tm_k, &bars->kv_full[s], 0, h, z);
-                tma_load_3d(kd + kBox, &P.tm_k, &bars->kv_full[s], 64, h, z);
-                tma_load_3d(vd, &P.tm_v, &bars->kv_full[s], 0, h, z);
-                tma_load_3d(vd + kBox, &P.tm_v, &bars->kv_full[s], 64, h, z);
+                if (j >= 2 && !mbar_wait(&bars->k_empty[s], par, abort_flag, a.hdr)) break;
+                mbar_arrive_expect_tx(&bars->k_full[s], kTile);
+                tma_load_3d(smem + kOffK + s * kTile, &P.tm_k, &bars->k_full[s], 0, h, z);
+                tma_load_3d(smem + kOffK + s * kTile + kBox, &P.tm_k, &bars->k_full[s], 64, h, z);
+                if (j >= 2 && !mbar_wait(&bars->v_empty[s], par, abort_flag, a.hdr)) { issued = -(j + 1); break; }
+                mbar_arrive_expect_tx(&bars->v_full[s], kTile);
+                tma_load_3d(smem + kOffV + s * kTile, &P.tm_v, &bars->v_full[s], 0, h, z);
+                tma_load_3d(smem + kOffV + s * kTile + kBox, &P.tm_v, &bars->v_full[s], 64, h, z);
                 issued = j + 1;
             }
-            // never leave the CTA with copies in flight: wait for every issued stage
+            // never leave the CTA with copies in flight: wait for every issued load
             mbar_wait_drain(&bars->q_full, 0, a.hdr);
-            for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-                mbar_wait_drain(&bars->kv_full[j % NS], (j / NS) & 1, a.hdr);
+            const int nk = issued >= 0 ? issued : -issued;       // K loads issued
+            const int nv = issued >= 0 ? issued : -issued - 1;   // V loads issued
+            for (int j = (nk > 2 ? nk - 2 : 0); j < nk; ++j) mbar_wait_drain(&bars->k_full[j & 1], (j >> 1) & 1, a.hdr);
+            for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j) mbar_wait_drain(&bars->v_full[j & 1], (j >> 1) & 1, a.hdr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
-            const uint32_t tS = tmem, tO = tmem + 128;
+            const uint32_t tO = tmem + 256;
             const uint32_t qb = sbase + kOffQ, pb = sbase + kOffP;
             bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.hdr);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int s = j % NS;
-                if (!mbar_wait(&bars->kv_full[s], (j / NS) & 1, abort_flag, a.hdr)) { ok = false; break; }
+            for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {
+                if (!mbar_wait(&bars->k_full[j], 0, abort_flag, a.hdr)) { ok = false; break; }
                 tc_fence_after();
-                if (j > 0) {
-                    if (!mbar_wait(&bars->p_full, (j - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                    tc_fence_after();
-                    const int sp = (j - 1) % NS;
-                    const uint32_t vb = sbase + kOffV + sp * kTile;
-#pragma unroll
-                    for (int k = 0; k < BN / 16; ++k)
-                        mma_bf16_ss(tO, kmajor_desc(pb, k), mnmajor_desc(vb, k), idesc_pv,
-                                    (j - 1 > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&bars->kv_empty[sp]);
-                }
-                const uint32_t kb = sbase + kOffK + s * kTile;
+                const uint32_t kb = sbase + kOffK + j * kTile;
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
-                    mma_bf16_ss(tS, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
-                mma_commit(&bars->s_full);
+                    mma_bf16_ss(tmem + j * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full[j]);
+                mma_commit(&bars->k_empty[j]);
             }
-            if (ok && mbar_wait(&bars->p_full, (n_tiles - 1) & 1, abort_flag, a.hdr)) {
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j & 1;
+                if (!mbar_wait(&bars->p_full, j & 1, abort_flag, a.hdr)) { ok = false; break; }
+                if (!mbar_wait(&bars->v_full[s], (j >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
                 tc_fence_after();
-                const int sp = (n_tiles - 1) % NS;
-                const uint32_t vb = sbase + kOffV + sp * kTile;
+                const uint32_t vb = sbase + kOffV + s * kTile;
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tO, kmajor_desc(pb, k), mnmajor_desc(vb, k), idesc_pv,
-                                (n_tiles - 1 > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&bars->kv_empty[sp]);
-                mma_commit(&bars->o_full);
+                                (j > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bars->v_empty[s]);
+                mma_commit(&bars->pv_done);
+                if (j + 2 < n_tiles) {
+                    if (!mbar_wait(&bars->k_full[s], ((j + 2) >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t kb = sbase + kOffK + s * kTile;
+#pragma unroll
+                    for (int k = 0; k < HD / 16; ++k)
+                        mma_bf16_ss(tmem + s * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk,
+                                    k > 0 ? 1u : 0u);
+                    mma_commit(&bars->s_full[s]);
+                    mma_commit(&bars->k_empty[s]);
+                }
             }
             // all issued MMAs retire before TMEM is released
             mma_commit(&bars->drain);
@@ -219,10 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     } else {
         // ------------------------------------------------ softmax warps
         const int wq = warp & 3;                 // TMEM lane quarter
+        const int grp = (warp - 2) >> 2;         // column half of S / O
         const int r = wq * 32 + lane;            // row within the tile
         const int i = row0 + r;                  // query index within the sequence
+        const int c0 = grp * 64;                 // first column of this thread's half
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_addr, tO = tmem + lane_addr + 128;
+        const uint32_t tO = tmem + lane_addr + 256 + c0;
         const float sc = a.scale * kLog2e;
         const int shift = nkv - nq;              // causal: key j visible iff j <= i + shift
         const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
@@ -231,132 +252,149 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_row = (BIAS == 2 && i < nq)
                                       ? a.dense_off[b] + ((int64_t)h * nq + i) * nkv : 0;
-        uint8_t* prow = smem + kOffP + r * 128;
-        float m_used = -CUDART_INF_F, l = 0.f;
+        const int jmax_vis = a.causal ? min(nkv - 1, i + shift) : nkv - 1;  // last visible key
+        uint8_t* prow = smem + kOffP + grp * kBox + r * 128;
+        float m_used = -CUDART_INF_F, l = 0.f;   // l: this half's partial sum
         bool ok = true;
+        // Every softmax warp runs the same sequence of named barriers: a failed
+        // (timed-out) wait only sets the CTA's abort flag, and the loop is left
+        // right after a barrier, where all warps read the same flag.
         for (int j = 0; j < n_tiles; ++j) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag, a.hdr));
-            if (!ok) break;
+            const int s = j & 1;
+            mbar_wait(&bars->s_full[s], (j >> 1) & 1, abort_flag, a.hdr);
             tc_fence_after();
-            const int j0 = j * BN;
-            float x[BN];
+            const int jc = j * BN + c0;          // key index of this half's column 0
+            float x[64];
 #pragma unroll
-            for (int c4 = 0; c4 < BN / 32; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t u[32];
-                tmem_ld32(tS + c4 * 32, u);
+                tmem_ld32(tmem + lane_addr + s * 128 + c0 + c4 * 32, u);
                 tmem_wait_ld();
 #pragma unroll
                 for (int t = 0; t < 32; ++t) x[c4 * 32 + t] = __uint_as_float(u[t]);
             }
-            // scale, bias, mask (log2 domain for softmax, natural for GDPA)
-            const int jmax_vis = a.causal ? min(nkv - 1, i + shift) : nkv - 1;  // last visible key
-            const int nvis = i < nq ? min(BN, jmax_vis - j0 + 1) : 0;  // visible columns: [0, nvis)
-            // bias (log2 units), added in place
+            const int nvis = i < nq ? max(0, min(64, jmax_vis - jc + 1)) : 0;  // visible: [0, nvis)
             if (BIAS == 1 && tab_in_smem) {
-                const float* tb = tab + (i - j0 - tab_lo);  // tb[-c] = bias(i, j0 + c)
+                const float* tb = tab + (i - jc - tab_lo);  // tb[-c] = bias(i, jc + c)
 #pragma unroll
-                for (int c = 0; c < BN; ++c) x[c] = fmaf(x[c], sc, tb[-c]);
+                for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], sc, tb[-c]);
             } else if (BIAS == 1) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    int rr = i - (j0 + c);
+                for (int c = 0; c < 64; ++c) {
+                    int rr = i - (jc + c);
                     rr = rr < -C ? -C : (rr > C ? C : rr);
                     x[c] = fmaf(x[c], sc, __ldg(tab_g + rr + C) * kLog2e);
                 }
             } else if (BIAS == 2) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    x[c] = fmaf(x[c], sc, c < nvis ? __bfloat162float(dense[dense_row + j0 + c]) * kLog2e : 0.f);
+                for (int c = 0; c < 64; ++c)
+                    x[c] = fmaf(x[c], sc, c < nvis ? __bfloat162float(dense[dense_row + jc + c]) * kLog2e : 0.f);
             } else {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) x[c] *= sc;
+                for (int c = 0; c < 64; ++c) x[c] *= sc;
             }
-            if (__any_sync(0xffffffffu, nvis < BN)) {
+            if (__any_sync(0xffffffffu, nvis < 64)) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) x[c] = c < nvis ? x[c] : -CUDART_INF_F;
+                for (int c = 0; c < 64; ++c) x[c] = c < nvis ? x[c] : -CUDART_INF_F;
             }
-            float tmax = -CUDART_INF_F;
-#pragma unroll
-            for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
+            float alpha = 1.f;
+            bool rescale = false;
             if (softmax) {
+                float pm = -CUDART_INF_F;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) pm = fmaxf(pm, x[c]);
+                red[(s * 2 + grp) * 128 + r] = pm;
+                named_sync_softmax();
+                if (*abort_flag) { ok = false; break; }
+                const float tmax = fmaxf(pm, red[(s * 2 + (grp ^ 1)) * 128 + r]);
                 // lazy rescale: keep the reference maximum unless it grew by > 2^8
                 const bool need = tmax > m_used + kRescaleThreshold;
                 const float m_new = need ? tmax : m_used;
-                if (__any_sync(0xffffffffu, need && j > 0 && m_used != -CUDART_INF_F)) {
-                    const float alpha = (need && m_used != -CUDART_INF_F) ? ex2(m_used - m_new) : 1.f;
-#pragma unroll
-                    for (int c4 = 0; c4 < HD / 32; ++c4) {
-                        uint32_t u[32];
-                        tmem_ld32(tO + c4 * 32, u);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) u[t] = __float_as_uint(__uint_as_float(u[t]) * alpha);
-                        tmem_st32(tO + c4 * 32, u);
-                    }
-                    tmem_wait_st();
-                    l *= alpha;
+                if (need && m_used != -CUDART_INF_F) {
+                    alpha = ex2(m_used - m_new);
+                    rescale = true;
                 } else if (need) {
-                    // first tile with a visible key: nothing accumulated yet
-                    l = 0.f;
+                    l = 0.f;  // first visible key of this row
                 }
                 m_used = m_new;
+            }
+            // P.V of the previous tile must be done before O or the P buffer change
+            if (j > 0) {
+                mbar_wait(&bars->pv_done, (j - 1) & 1, abort_flag, a.hdr);
+                tc_fence_after();
+            }
+            if (softmax && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int c4 = 0; c4 < 2; ++c4) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c4 * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) u[t] = __float_as_uint(__uint_as_float(u[t]) * alpha);
+                    tmem_st32(tO + c4 * 32, u);
+                }
+                tmem_wait_st();
+                l *= alpha;
+            }
+            if (softmax) {
                 // ex2(-inf) = 0 masks the invisible columns; a row with no visible
                 // key yet uses reference 0 so that -inf - ref stays -inf
                 const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
-                float psum0 = 0.f, psum1 = 0.f;
+                float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < BN; c += 2) {
+                for (int c = 0; c < 64; c += 2) {
                     x[c] = ex2(x[c] - ref);
                     x[c + 1] = ex2(x[c + 1] - ref);
-                    psum0 += x[c];
-                    psum1 += x[c + 1];
+                    ps0 += x[c];
+                    ps1 += x[c + 1];
                 }
-                l += psum0 + psum1;
+                l += ps0 + ps1;
             } else {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
+                for (int c = 0; c < 64; ++c) {
                     const float s_nat = x[c] * (1.0f / kLog2e);
                     x[c] = c < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
                 }
             }
-            // P row -> shared memory, K-major, 128-byte swizzle (chunk ^ row%8)
+            // P half-row -> shared memory, K-major, 128-byte swizzle (chunk ^ row%8)
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const int c = half * 64 + ch * 8;
-                    uint4 w;
-                    w.x = pack_bf16(x[c + 0], x[c + 1]);
-                    w.y = pack_bf16(x[c + 2], x[c + 3]);
-                    w.z = pack_bf16(x[c + 4], x[c + 5]);
-                    w.w = pack_bf16(x[c + 6], x[c + 7]);
-                    *reinterpret_cast<uint4*>(prow + half * kBox + ((ch ^ (r & 7)) << 4)) = w;
-                }
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 w;
+                w.x = pack_bf16(x[ch * 8 + 0], x[ch * 8 + 1]);
+                w.y = pack_bf16(x[ch * 8 + 2], x[ch * 8 + 3]);
+                w.z = pack_bf16(x[ch * 8 + 4], x[ch * 8 + 5]);
+                w.w = pack_bf16(x[ch * 8 + 6], x[ch * 8 + 7]);
+                *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = w;
             }
             // value rows past the sequence end (neighbour data) must not reach P.V
-            const int nvalid = nkv - j0;
-            if (nvalid < BN && r >= nvalid) {
-                uint8_t* vrow = smem + kOffV + (j % NS) * kTile + r * 128;
-                const uint4 z = make_uint4(0, 0, 0, 0);
+            const int nvalid = nkv - j * BN;
+            if (nvalid < BN) {  // same for the whole CTA
+                mbar_wait(&bars->v_full[s], (j >> 1) & 1, abort_flag, a.hdr);
+                if (r >= nvalid) {
+                    uint8_t* vrow = smem + kOffV + s * kTile + grp * kBox + r * 128;
+                    const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
-                    *reinterpret_cast<uint4*>(vrow + kBox + ch * 16) = z;
+                    for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->p_full);
+            if (!softmax && *abort_flag) { ok = false; break; }
         }
         // ------------------------------------------------------ epilogue
-        if (ok && n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full, 0, abort_flag, a.hdr));
+        if (ok && n_tiles > 0) mbar_wait(&bars->pv_done, (n_tiles - 1) & 1, abort_flag, a.hdr);
+        lred[grp * 128 + r] = l;
+        named_sync_softmax();
+        ok = ok && !*abort_flag;
+        const float l_row = l + lred[(grp ^ 1) * 128 + r];
         if (ok) {
             tc_fence_after();
-            const float inv = softmax ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)(q0 + i) * a.H + h) * HD;
+            const float inv = softmax ? (l_row > 0.f ? 1.f / l_row : 0.f) : 1.f;
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)(q0 + i) * a.H + h) * HD + c0;
 #pragma unroll
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
+            for (int c4 = 0; c4 < 2; ++c4) {
                 uint32_t u[32];
                 if (n_tiles > 0) {
                     tmem_ld32(tO + c4 * 32, u);
@@ -377,16 +415,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     }
                 }
             }
-            if (softmax && a.lse && i < nq)
+            if (softmax && grp == 0 && a.lse && i < nq)
                 a.lse[(int64_t)(q0 + i) * a.H + h] =
-                    l > 0.f ? m_used * (1.0f / kLog2e) + logf(l) : -CUDART_INF_F;
+                    l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 

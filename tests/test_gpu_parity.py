@@ -67,12 +67,16 @@ def half_ulp_bf16(x):
     return np.exp2(np.floor(np.log2(ax)) - 8)
 
 
-def compare(name, gpu, ref, rows, max_tol, mean_tol=None):
+def compare(name, gpu, ref, rows, max_tol, mean_tol=None, rms_scaled=False):
     bf16_out = gpu.dtype == torch.bfloat16
     g = gpu.float().cpu().numpy()[rows].astype(np.float64)
     r = ref[rows]
     if g.size == 0:
         return 0.0
+    if rms_scaled:
+        scale = max(1.0, float(np.sqrt(np.mean(r[np.isfinite(r)] ** 2))))
+        max_tol *= scale
+        mean_tol = None if mean_tol is None else mean_tol * scale
     finite = np.isfinite(r)
     assert np.array_equal(np.isfinite(g), finite), f"{name}: non-finite pattern differs"
     err = np.abs(g[finite] - r[finite])
@@ -93,7 +97,7 @@ def compare(name, gpu, ref, rows, max_tol, mean_tol=None):
     return mx
 
 
-def check_problem(p, dev, act=None, seq_mask=None, strict_f32=False):
+def check_problem(p, dev, act=None, seq_mask=None, strict_f32=False, rms_scaled=False):
     act = act or p.act
     out, lse, (dq, dk, dv) = run_gpu(p, dev, act)
     ro, rl, (rdq, rdk, rdv) = run_oracle(p, act, seq_mask)
@@ -104,9 +108,9 @@ def check_problem(p, dev, act=None, seq_mask=None, strict_f32=False):
     errs["o"] = compare("O", out, ro, qr, mx, mean)
     if act == "softmax":
         errs["lse"] = compare("LSE", lse, rl, qr, LSE_MAX if not strict_f32 else F32_MAX)
-    errs["dq"] = compare("dQ", dq, rdq, qr, mx, mean)
-    errs["dk"] = compare("dK", dk, rdk, kr, mx, mean)
-    errs["dv"] = compare("dV", dv, rdv, kr, mx, mean)
+    errs["dq"] = compare("dQ", dq, rdq, qr, mx, mean, rms_scaled)
+    errs["dk"] = compare("dK", dk, rdk, kr, mx, mean, rms_scaled)
+    errs["dv"] = compare("dV", dv, rdv, kr, mx, mean, rms_scaled)
     return errs
 
 
@@ -182,16 +186,15 @@ EDGE_LENS = [
 @pytest.mark.parametrize("q_lens,kv_lens,causal", EDGE_LENS)
 @pytest.mark.parametrize("act", ["softmax", "silu"])
 def test_edge_lengths(cuda_device, q_lens, kv_lens, causal, act):
-    if act == "silu" and kv_lens == [1, 1, 1, 1]:
-        # GDPA with one key shared by 200 queries makes dK a sum of 200
-        # same-sign terms (|dK| ~ 13); with bf16 MMA operands its error
-        # (~0.5% relative) exceeds an absolute bound stated for O(1) values,
-        # so the single-key GDPA case keeps its query counts moderate.
-        q_lens = [5, 40, 60, 1]
     kv_lens = kv_lens or q_lens
     p = make_problem("cross_bf16", 7, q_lens=q_lens, kv_lens=kv_lens, causal=causal,
                      bias="dense" if act == "silu" else "relpos")
-    check_problem(p, cuda_device, act=act)
+    # GDPA over a single key does not divide the score gradient down
+    # (dS = dP act'(s) / 1, |dS| ~ 11), so dK is a sum of large terms whose
+    # bf16 MMA operands carry ~2^-9 relative error; the absolute bound, meant
+    # for O(1) values, is applied relative to the tensor's RMS there.
+    rms_scaled = act == "silu" and kv_lens == [1, 1, 1, 1]
+    check_problem(p, cuda_device, act=act, rms_scaled=rms_scaled)
 
 
 def test_no_bias(cuda_device):
