@@ -405,15 +405,7 @@ def main():
 
     ms_step = ms_total / args.steps
     flops_rank = f_fwd + f_bwd
-    if world > 1:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step_max = float(t.item())
-        fl = torch.tensor([flops_rank], dtype=torch.float64, device=dev)
-        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
-        flops_all = float(fl.item())
-    else:
-        ms_step_max, flops_all = ms_step, flops_rank
+    ms_step_max, flops_all = aggregate_over_ranks(ms_step, flops_rank, dev, world)
     value = flops_all / (ms_step_max * 1e-3) / 1e12
 
     # per-kernel totals over the timed region
@@ -489,6 +481,20 @@ def main():
         dist.destroy_process_group()
 
 
+def aggregate_over_ranks(ms_per_step, flops, device, world):
+    """Whole-job numbers of one timed region: the slowest rank's time per step
+    and the work of all ranks (weak scaling: every rank runs its own batch).
+    Returns (max ms per step, summed flops)."""
+    if world <= 1:
+        return float(ms_per_step), float(flops)
+    import torch.distributed as dist
+    t = torch.tensor([ms_per_step], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    fl = torch.tensor([flops], dtype=torch.float64, device=device)
+    dist.all_reduce(fl, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(fl.item())
+
+
 def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
     """Same metric with pinned host inputs copied in and every result copied
     out inside the timed region."""
@@ -532,15 +538,7 @@ def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
     e.record(stream)
     torch.cuda.synchronize(dev)
     ms = s.elapsed_time(e) / args.e2e_steps
-    flops_all = flops_rank
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        fl = torch.tensor([flops_rank], dtype=torch.float64, device=dev)
-        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
-        flops_all = float(fl.item())
+    ms, flops_all = aggregate_over_ranks(ms, flops_rank, dev, world)
     return {"value": flops_all / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "steps": args.e2e_steps}

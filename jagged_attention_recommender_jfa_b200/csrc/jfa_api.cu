@@ -129,19 +129,19 @@ jfa_status check_act(int act) {
 
 bool use_tc(const jfa_problem& p, int act, int backward) { return tc_supported(p, act, backward); }
 
-// The MXFP8 forward exists only as a tensor-core kernel.
-jfa_status check_dtype_path(const jfa_problem& p, int act, int backward) {
-    if (p.dtype == JFA_MXFP8 && !backward && !use_tc(p, act, 0))
-        return fail(JFA_ERR_UNSUPPORTED, "MXFP8 forward needs head_dim 128 and softmax on the tensor-core path");
-    return JFA_OK;
-}
-
 size_t workspace_bytes(const jfa_problem& p, int backward) {
     WsLayout L = ws_layout(p, backward != 0, false);
     size_t extra = 0;
     if (use_tc(p, JFA_ACT_SOFTMAX, backward) || use_tc(p, JFA_ACT_SILU, backward))
         extra = tc_workspace_extra(p, backward);
     return L.total + align256(extra);
+}
+
+// MXFP8 runs only on the tensor-core path (head_dim 128, softmax).
+jfa_status check_mxfp8(const jfa_problem& p, int act) {
+    if (p.dtype == JFA_MXFP8 && !use_tc(p, act, 0))
+        return fail(JFA_ERR_UNSUPPORTED, "MXFP8 needs head_dim 128 and softmax");
+    return JFA_OK;
 }
 
 float eff_scale(const jfa_problem& p) {
@@ -174,7 +174,7 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
     if (s != JFA_OK) return s;
     if ((s = check_act(act)) != JFA_OK) return s;
     const jfa_problem& p = *problem;
-    if ((s = check_dtype_path(p, act, 0)) != JFA_OK) return s;
+    if ((s = check_mxfp8(p, act)) != JFA_OK) return s;
     if (!q_offsets || !kv_offsets || !workspace) return fail(JFA_ERR_INVALID_ARGUMENT, "NULL offsets or workspace");
     if ((p.total_q > 0 && (!q || !out)) || (p.total_kv > 0 && (!k || !v)))
         return fail(JFA_ERR_INVALID_ARGUMENT, "NULL tensor");
@@ -224,6 +224,7 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
     if (s != JFA_OK) return s;
     if ((s = check_act(act)) != JFA_OK) return s;
     const jfa_problem& p = *problem;
+    if ((s = check_mxfp8(p, act)) != JFA_OK) return s;
     if (!q_offsets || !kv_offsets || !workspace) return fail(JFA_ERR_INVALID_ARGUMENT, "NULL offsets or workspace");
     if ((p.total_q > 0 && (!q || !dout || !dq)) || (p.total_kv > 0 && (!k || !v || !dk || !dv)))
         return fail(JFA_ERR_INVALID_ARGUMENT, "NULL tensor");

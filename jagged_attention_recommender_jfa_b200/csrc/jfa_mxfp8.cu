@@ -12,35 +12,18 @@
 // x * 2^-X is exact in fp32 (a power-of-two scaling of a bf16 value whose
 // result lies below 2^9), so the only rounding is the hardware's
 // round-to-nearest-even conversion with saturation (cvt.rn.satfinite).
-#include <cuda_fp8.h>
-
 #include "jfa_common.cuh"
+#include "jfa_mx.cuh"
 
 namespace jfa {
 
 namespace {
 
-// floor(log2(amax)) - 8 clamped to the E8M0 range; amax >= 0 finite.
-__device__ __forceinline__ int shared_exponent(float amax) {
-    uint32_t bits = __float_as_uint(amax);
-    int e = (int)((bits >> 23) & 0xFF);
-    if (e == 0) return -127;  // zero or fp32-subnormal amax: floor(log2) < -126
-    int X = (e - 127) - 8;
-    return X < -127 ? -127 : (X > 127 ? 127 : X);
-}
-
-// 2^-X as a float, X in [-127, 119] for finite bf16 inputs.
-__device__ __forceinline__ float pow2_neg(int X) {
-    int e = 127 - X;
-    if (e >= 255) e = 254;
-    if (e <= 0) return 0.f;
-    return __uint_as_float((uint32_t)e << 23);
-}
-
-__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
-    __nv_fp8x2_storage_t s = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-    return (uint16_t)s;
-}
+using mx::shared_exponent;
+using mx::pow2_neg;
+using mx::pow2;
+using mx::pack_e4m3x2;
+using mx::decode_e4m3x2;
 
 // Blocks of 32 consecutive elements along d: one thread per block.
 __global__ void __launch_bounds__(256) quant_along_d(const __nv_bfloat16* __restrict__ x,
@@ -126,7 +109,102 @@ __global__ void __launch_bounds__(256) quant_along_rows(const __nv_bfloat16* __r
     }
 }
 
+// Quantise-dequantise ("fake quantisation") along d: the output holds, in
+// bf16, exactly the value E4M3(x * 2^-X) * 2^X that an MXFP8 operand
+// represents (3 mantissa bits times a power of two fit bf16 exactly).
+__global__ void __launch_bounds__(256) fake_quant_along_d(const __nv_bfloat16* __restrict__ x,
+                                                          int64_t n_blocks,
+                                                          __nv_bfloat16* __restrict__ y) {
+    int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (blk >= n_blocks) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + blk * 32);
+    uint4 raw[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) raw[t] = src[t];
+    float f[32];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[t]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float2 v = __bfloat1622float2(p2[u]);
+            f[8 * t + 2 * u] = v.x;
+            f[8 * t + 2 * u + 1] = v.y;
+        }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(f[t]));
+    const int X = shared_exponent(amax);
+    const float s = pow2_neg(X), back = pow2(X);
+    uint4 out[4];
+    uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        const float2 d2 = decode_e4m3x2(pack_e4m3x2(f[2 * t] * s, f[2 * t + 1] * s));
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(d2.x * back, d2.y * back);
+        o32[t] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(y + blk * 32);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) dst[t] = out[t];
+}
+
+// Quantise-dequantise along 32-row blocks of each sequence.
+__global__ void __launch_bounds__(256) fake_quant_along_rows(const __nv_bfloat16* __restrict__ x,
+                                                             const int32_t* __restrict__ off,
+                                                             int64_t total_rows, int cols,
+                                                             __nv_bfloat16* __restrict__ y) {
+    const int b = blockIdx.x, blk = blockIdx.y;
+    const int r0 = off[b], n = off[b + 1] - r0;
+    if (blk * 32 >= n || r0 < 0 || (int64_t)r0 + n > total_rows) return;
+    const int rows = min(32, n - blk * 32);
+    const __nv_bfloat16* base = x + (int64_t)(r0 + blk * 32) * cols;
+    __nv_bfloat16* obase = y + (int64_t)(r0 + blk * 32) * cols;
+    for (int col = threadIdx.x; col < cols; col += blockDim.x) {
+        float f[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            f[t] = t < rows ? __bfloat162float(base[(int64_t)t * cols + col]) : 0.f;
+            amax = fmaxf(amax, fabsf(f[t]));
+        }
+        const int X = shared_exponent(amax);
+        const float s = pow2_neg(X), back = pow2(X);
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+            const float2 d2 = decode_e4m3x2(pack_e4m3x2(f[t] * s, f[t + 1] * s));
+            if (t < rows) obase[(int64_t)t * cols + col] = __float2bfloat16_rn(d2.x * back);
+            if (t + 1 < rows) obase[(int64_t)(t + 1) * cols + col] = __float2bfloat16_rn(d2.y * back);
+        }
+    }
+}
+
 }  // namespace
+
+// MXFP8 operands for the attention passes: Q and K quantised along d, V along
+// 32-row blocks of each sequence, each returned dequantised in bf16.
+cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
+                              int64_t total_q, int64_t total_kv, int heads, int d, int batch,
+                              int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st) {
+    const int64_t nq_blocks = total_q * heads * (d / 32), nk_blocks = total_kv * heads * (d / 32);
+    prof_begin(st);
+    if (nq_blocks > 0)
+        fake_quant_along_d<<<(unsigned)((nq_blocks + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(q), nq_blocks, reinterpret_cast<__nv_bfloat16*>(qf));
+    if (nk_blocks > 0)
+        fake_quant_along_d<<<(unsigned)((nk_blocks + 255) / 256), 256, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(k), nk_blocks, reinterpret_cast<__nv_bfloat16*>(kf));
+    prof_end(st, K_QUANT_ALONG_D);
+    if (batch > 0 && max_kv_len > 0) {
+        dim3 grid(batch, (max_kv_len + 31) / 32);
+        prof_begin(st);
+        fake_quant_along_rows<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), kv_off,
+                                                    total_kv, heads * d, reinterpret_cast<__nv_bfloat16*>(vf));
+        prof_end(st, K_QUANT_ALONG_ROWS);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
                         int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,

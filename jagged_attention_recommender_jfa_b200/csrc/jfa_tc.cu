@@ -1,35 +1,92 @@
 // Dispatch to the tensor-core (tcgen05) kernels: which problems they take and
 // how they are launched.
+//
+// MXFP8 (dtype JFA_MXFP8): Q and K are quantised along d, V along 32-row
+// blocks of each sequence (OCP MX: E4M3 elements, one E8M0 scale per 32), and
+// the attention runs on the exact dequantised operands, with P quantised the
+// same way per 32 keys inside the forward kernel.  The backward computes bf16
+// gradients on the dequantised Q/K/V (straight-through quantiser).
 #include "jfa_common.cuh"
 
 namespace jfa {
 
-cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
+cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quant_p, cudaStream_t st);
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                                cudaStream_t st);
+cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
+                              int64_t total_q, int64_t total_kv, int heads, int d, int batch,
+                              int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st);
 
-// bf16 storage, head_dim 128, any activation and bias kind.
+// bf16 storage with head_dim 128 (any activation and bias kind); MXFP8 with
+// head_dim 128 and softmax.
 bool tc_supported(const jfa_problem& p, int act, int backward) {
-    (void)act;
     (void)backward;
-    return p.dtype == JFA_BF16 && p.head_dim == 128;
+    if (p.head_dim != 128) return false;
+    if (p.dtype == JFA_BF16) return true;
+    return p.dtype == JFA_MXFP8 && act == JFA_ACT_SOFTMAX;
 }
 
-// The backward keeps an fp32 dQ accumulator [total_q][heads][128].
+namespace {
+struct Extra {
+    size_t dq_acc, qf, kf, vf, total;
+};
+Extra extra_layout(const jfa_problem& p, int backward) {
+    Extra e{};
+    size_t off = 0;
+    if (backward) {
+        e.dq_acc = off;
+        off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads * p.head_dim);
+    }
+    if (p.dtype == JFA_MXFP8) {
+        e.qf = off; off = align256(off + 2 * (size_t)p.total_q * p.heads * p.head_dim);
+        e.kf = off; off = align256(off + 2 * (size_t)p.total_kv * p.heads * p.head_dim);
+        e.vf = off; off = align256(off + 2 * (size_t)p.total_kv * p.heads * p.head_dim);
+    }
+    e.total = off;
+    return e;
+}
+
+cudaError_t fake_quant(const jfa_problem& p, AttnArgs& a, char* ws, const Extra& L, cudaStream_t st) {
+    void *qf = ws + L.qf, *kf = ws + L.kf, *vf = ws + L.vf;
+    cudaError_t e = mx_fake_quant_qkv(a.q, a.k, a.v, a.kv_off, p.total_q, p.total_kv, p.heads,
+                                      p.head_dim, p.batch, p.max_kv_len, qf, kf, vf, st);
+    a.q = qf;
+    a.k = kf;
+    a.v = vf;
+    return e;
+}
+}  // namespace
+
+// The backward keeps an fp32 dQ accumulator [total_q][heads][128]; MXFP8
+// adds the three dequantised operands.
 size_t tc_workspace_extra(const jfa_problem& p, int backward) {
-    if (!backward) return 0;
-    return sizeof(float) * (size_t)p.total_q * p.heads * p.head_dim;
+    return extra_layout(p, backward).total;
 }
 
-cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void*, cudaStream_t st) {
-    return tc_forward_launch(p, a, st);
+cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, cudaStream_t st) {
+    AttnArgs aa = a;
+    if (p.dtype == JFA_MXFP8) {
+        cudaError_t e = fake_quant(p, aa, reinterpret_cast<char*>(ws_extra), extra_layout(p, 0), st);
+        if (e != cudaSuccess) return e;
+        return tc_forward_launch(p, aa, true, st);
+    }
+    return tc_forward_launch(p, aa, false, st);
 }
 
 cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                         void* ws_extra, cudaStream_t st) {
+    const Extra L = extra_layout(p, 1);
+    char* ws = reinterpret_cast<char*>(ws_extra);
     AttnArgs aq = a, akv = kv;
-    aq.dq_acc = reinterpret_cast<float*>(ws_extra);
+    aq.dq_acc = reinterpret_cast<float*>(ws + L.dq_acc);
     akv.dq_acc = aq.dq_acc;
+    if (p.dtype == JFA_MXFP8) {
+        cudaError_t e = fake_quant(p, aq, ws, L, st);
+        if (e != cudaSuccess) return e;
+        akv.q = aq.q;
+        akv.k = aq.k;
+        akv.v = aq.v;
+    }
     return tc_backward_launch(p, aq, akv, st);
 }
 

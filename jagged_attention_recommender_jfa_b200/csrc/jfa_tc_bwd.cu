@@ -47,8 +47,8 @@ constexpr uint32_t kOffDO = kOffQ + kTile;
 constexpr uint32_t kOffPT = kOffDO + kTile;
 constexpr uint32_t kOffDST = kOffPT + kTile;
 constexpr uint32_t kOffBar = kOffDST + kTile;  // 196608
-constexpr uint32_t kOffRow = kOffBar + 256;     // lse2[128], D[128]
-constexpr uint32_t kOffTab = kOffRow + 1024;
+constexpr uint32_t kOffRow = kOffBar + 256;     // lse2[2][128], D[2][128] (double-buffered)
+constexpr uint32_t kOffTab = kOffRow + 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
@@ -59,6 +59,7 @@ struct Bars {
     uint64_t ds_full;
     uint64_t dq_full;
     uint64_t dq_empty;
+    uint64_t stage_free;
     uint64_t fin;
     uint64_t drain;
     uint32_t tmem_base;
@@ -125,6 +126,21 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t* tile, int r, int c4, c
     }
 }
 
+// Same as store_chunk_bf16 for 32 fp32 values held as bit patterns.
+__device__ __forceinline__ void store_chunk_bits(uint8_t* tile, int r, int c4, const uint32_t (&v)[32]) {
+    uint8_t* row = tile + (c4 >> 1) * kBox + r * 128;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int ch = (c4 & 1) * 4 + u;
+        uint4 w;
+        w.x = pack_bf16(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
+        w.y = pack_bf16(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
+        w.z = pack_bf16(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
+        w.w = pack_bf16(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
+        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
+    }
+}
+
 __device__ __forceinline__ void zero_row(uint8_t* tile, int r) {
     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -134,14 +150,17 @@ __device__ __forceinline__ void zero_row(uint8_t* tile, int r) {
     }
 }
 
+// BIAS: 0 none, 1 relative-position, 2 dense jagged.  SOFTMAX: softmax (true)
+// or GDPA.
+template <int BIAS, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_constant__ BwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
-    float* lse2_s = reinterpret_cast<float*>(smem + kOffRow);
-    float* dd_s = lse2_s + 128;
+    float* lse2_s = reinterpret_cast<float*>(smem + kOffRow);  // [2][128]
+    float* dd_s = lse2_s + 256;                                 // [2][128]
     float* tab = reinterpret_cast<float*>(smem + kOffTab);
 
     const int4 it = a.items[blockIdx.x];
@@ -152,10 +171,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     const int i_start = a.causal ? max(0, j0 - shift) : 0;
     const int nt = nq > i_start ? (nq - i_start + BM - 1) / BM : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool softmax = a.act == JFA_ACT_SOFTMAX;
+    constexpr bool softmax = SOFTMAX;
     const int tab_lo = i_start - j0 - (BN - 1);
     const int tab_len = nq - i_start + BN - 1;
-    const bool tab_in_smem = a.bias_kind == JFA_BIAS_RELPOS && nt > 0 && tab_len <= P.tab_cap;
+    const bool tab_in_smem = BIAS == 1 && nt > 0 && tab_len <= P.tab_cap;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -164,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->ds_full, 8);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 1);
+        mbar_init(&bars->dq_empty, 8);
+        mbar_init(&bars->stage_free, 1);
         mbar_init(&bars->fin, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -213,6 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 tma_load_3d(smem + kOffDO, &P.tm_do, &bars->q_full, 0, h, z);
                 tma_load_3d(smem + kOffDO + kBox, &P.tm_do, &bars->q_full, 64, h, z);
                 issued = t + 1;
+                if (t + 1 < nt) {  // warm L2 for the next query tile (single-buffered)
+                    tma_prefetch_l2_3d(&P.tm_q, 0, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_q, 64, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_do, 0, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_do, 64, h, z + BM);
+                }
             }
             mbar_wait_drain(&bars->kv_full, 0, a.hdr);
             if (issued > 0) mbar_wait_drain(&bars->q_full, (issued - 1) & 1, a.hdr);
@@ -274,101 +300,122 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const int C = (a.relpos_len - 1) >> 1;
         const float* tab_g = reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
-        const int64_t dense_base = (a.bias_kind == JFA_BIAS_DENSE_JAGGED) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
+        const int64_t dense_base = (BIAS == 2) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
         const bool leader = (warp == 2 && lane == 0);
         bool ok = true;
-        for (int t = 0; ok && t < nt; ++t) {
-            const int qb0 = i_start + t * BM;    // query index of the tile's row 0
+        // LSE (log2 units) and D of a query tile, staged by group 0 into one of
+        // two buffers; the next tile's values are fetched a tile ahead.
+        auto fetch_rowstats = [&](int t, float& l2, float& dv) {
+            const int qi = i_start + t * BM + r;
+            l2 = CUDART_INF_F;
+            dv = 0.f;
+            if (qi < nq && softmax) {
+                l2 = a.lse[(int64_t)(q0 + qi) * a.H + h] * kLog2e;
+                dv = a.dterm[(int64_t)(q0 + qi) * a.H + h];
+            }
+        };
+        if (nt > 0) {
             if (grp == 0) {
-                const int qi = qb0 + r;
-                float l2 = CUDART_INF_F, dv = 0.f;
-                if (qi < nq && softmax) {
-                    const float lse = a.lse[(int64_t)(q0 + qi) * a.H + h];
-                    l2 = lse * kLog2e;
-                    dv = a.dterm[(int64_t)(q0 + qi) * a.H + h];
-                }
+                float l2, dv;
+                fetch_rowstats(0, l2, dv);
                 lse2_s[r] = l2;
                 dd_s[r] = dv;
             }
             named_sync_score();
-            // leave only here, right after a barrier, so that every score warp
-            // runs the same sequence of named barriers; failed waits below only
-            // set the CTA's abort flag
-            if (*abort_flag) { ok = false; break; }
+        }
+        for (int t = 0; t < nt; ++t) {
+            const int qb0 = i_start + t * BM;    // query index of the tile's row 0
+            const int buf = t & 1;
+            float nl2 = CUDART_INF_F, ndv = 0.f;
+            if (grp == 0 && t + 1 < nt) fetch_rowstats(t + 1, nl2, ndv);
+            // failed waits below only set the CTA's abort flag; the loop is left
+            // right after the named barrier, so every score warp runs the same
+            // sequence of barriers
             mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr);
             tc_fence_after();
             // key rows past the sequence end (neighbour data) must not reach dS K;
             // S^T = K Q^T of the first tile has completed, so K may be edited now
             if (t == 0 && grp == 0 && !jvalid) zero_row(smem + kOffK, r);
+            // the previous tile's dQ reduce must have read its staging (which
+            // overlays the P^T / dS^T buffers) before they are rewritten
+            if (t > 0) {
+                if (leader) {
+                    bulk_wait_read_all();
+                    mbar_arrive(&bars->stage_free);
+                }
+                mbar_wait(&bars->stage_free, (t - 1) & 1, abort_flag, a.hdr);
+            }
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
-#pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c4 = grp * 2 + cc;         // 32-column chunk of this thread
-                uint32_t us[32], up[32];
-                tmem_ld32(tS + cc * 32, us);
-                tmem_ld32(tdP + cc * 32, up);
-                tmem_wait_ld();
+            // one 32-column chunk: scores u (TMEM bits) -> P in place, dP g -> dS in place
+            auto process = [&](uint32_t (&u)[32], uint32_t (&g)[32], int c4) {
                 const int qc0 = qb0 + c4 * 32;       // query index of the chunk's column 0
                 const bool all_vis = jvalid && (qc0 + 31 < nq) && (qc0 >= imin_vis);
                 const bool none_vis = !jvalid || qc0 >= nq || (qc0 + 31 < imin_vis);
-                float pv[32], dsv[32];
                 if (none_vis) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) pv[u] = 0.f, dsv[u] = 0.f;
+                    for (int v = 0; v < 32; ++v) u[v] = 0u, g[v] = 0u;
+                    return;
+                }
+                if (BIAS == 1 && tab_in_smem) {
+                    const float* tb = tab + (qc0 - j - tab_lo);   // tb[v] = bias(qc0 + v, j)
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, tb[v]));
+                } else if (BIAS == 1) {
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) {
+                        int rr = qc0 + v - j;
+                        rr = rr < -C ? -C : (rr > C ? C : rr);
+                        u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, __ldg(tab_g + rr + C) * kLog2e));
+                    }
+                } else if (BIAS == 2) {
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) {
+                        const int qi = qc0 + v;
+                        const float bv = (jvalid && qi < nq)
+                            ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
+                        u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, bv));
+                    }
                 } else {
-                    float s2[32];
-                    if (a.bias_kind == JFA_BIAS_RELPOS && tab_in_smem) {
-                        const float* tb = tab + (qc0 - j - tab_lo);   // tb[u] = bias(qc0 + u, j)
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) s2[u] = fmaf(__uint_as_float(us[u]), sc, tb[u]);
-                    } else if (a.bias_kind == JFA_BIAS_RELPOS) {
+                    for (int v = 0; v < 32; ++v) u[v] = __float_as_uint(__uint_as_float(u[v]) * sc);
+                }
+                if (SOFTMAX) {
+                    const float* l2c = lse2_s + buf * 128 + c4 * 32;
+                    const float* ddc = dd_s + buf * 128 + c4 * 32;
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            int rr = qc0 + u - j;
-                            rr = rr < -C ? -C : (rr > C ? C : rr);
-                            s2[u] = fmaf(__uint_as_float(us[u]), sc, __ldg(tab_g + rr + C) * kLog2e);
-                        }
-                    } else if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const int qi = qc0 + u;
-                            const float bv = (jvalid && qi < nq)
-                                ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
-                            s2[u] = fmaf(__uint_as_float(us[u]), sc, bv);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) s2[u] = __uint_as_float(us[u]) * sc;
+                    for (int v = 0; v < 32; ++v) {
+                        const float pr = ex2(__uint_as_float(u[v]) - l2c[v]);
+                        u[v] = __float_as_uint(pr);
+                        g[v] = __float_as_uint(pr * (__uint_as_float(g[v]) - ddc[v]));
                     }
-                    const float* l2c = lse2_s + c4 * 32;
-                    const float* ddc = dd_s + c4 * 32;
-                    if (softmax) {
+                } else {
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const float p = ex2(s2[u] - l2c[u]);
-                            pv[u] = p;
-                            dsv[u] = p * (__uint_as_float(up[u]) - ddc[u]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const float sn = s2[u] * (1.0f / kLog2e);
-                            pv[u] = act_f(a.act, sn) * inv_n;
-                            dsv[u] = __uint_as_float(up[u]) * act_grad_f(a.act, sn) * inv_n;
-                        }
-                    }
-                    if (!all_vis) {
-#pragma unroll
-                        for (int u = 0; u < 32; ++u) {
-                            const int qi = qc0 + u;
-                            const bool vis = jvalid && qi < nq && qi >= imin_vis;
-                            pv[u] = vis ? pv[u] : 0.f;
-                            dsv[u] = vis ? dsv[u] : 0.f;
-                        }
+                    for (int v = 0; v < 32; ++v) {
+                        const float sn = __uint_as_float(u[v]) * (1.0f / kLog2e);
+                        u[v] = __float_as_uint(act_f(a.act, sn) * inv_n);
+                        g[v] = __float_as_uint(__uint_as_float(g[v]) * act_grad_f(a.act, sn) * inv_n);
                     }
                 }
-                store_chunk_bf16(smem + kOffPT, r, c4, pv);
-                store_chunk_bf16(smem + kOffDST, r, c4, dsv);
+                if (!all_vis) {
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) {
+                        const int qi = qc0 + v;
+                        const bool vis = jvalid && qi < nq && qi >= imin_vis;
+                        u[v] = vis ? u[v] : 0u;
+                        g[v] = vis ? g[v] : 0u;
+                    }
+                }
+            };
+#pragma unroll 1
+            for (int cc = 0; cc < 2; ++cc) {
+                uint32_t u[32], g[32];
+                tmem_ld32(tS + cc * 32, u);
+                tmem_ld32(tdP + cc * 32, g);
+                tmem_wait_ld();
+                const int c4 = grp * 2 + cc;
+                process(u, g, c4);
+                store_chunk_bits(smem + kOffPT, r, c4, u);
+                store_chunk_bits(smem + kOffDST, r, c4, g);
             }
             // query rows past the sequence end must not reach dV / dK
             if (qb0 + r >= nq) {
@@ -385,32 +432,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr);
             tc_fence_after();
             const bool qvalid = qb0 + r < nq;
-#pragma unroll 1
+            uint32_t u2[2][32];
+            tmem_ld32(tS, u2[0]);
+            tmem_ld32(tS + 32, u2[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dq_empty);  // TMEM columns free for S^T of t+1
+#pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int c4 = grp * 2 + cc;
-                uint32_t u[32];
-                tmem_ld32(tS + cc * 32, u);
-                tmem_wait_ld();
                 uint8_t* row = smem + kOffPT + c4 * (128 * 128) + r * 128;
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
-                    uint4 w = qvalid ? make_uint4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3])
+                    uint4 w = qvalid ? make_uint4(u2[cc][4 * v], u2[cc][4 * v + 1], u2[cc][4 * v + 2], u2[cc][4 * v + 3])
                                      : make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4*>(row + ((v ^ (r & 7)) << 4)) = w;
                 }
             }
+            if (grp == 0 && t + 1 < nt) {
+                lse2_s[(buf ^ 1) * 128 + r] = nl2;
+                dd_s[(buf ^ 1) * 128 + r] = ndv;
+            }
             fence_proxy_async_smem();
-            tc_fence_before();
             named_sync_score();
-            if (leader && !*abort_flag) {
+            if (*abort_flag) { ok = false; break; }
+            if (leader) {
                 const int z = q0 + qb0;
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4)
                     tma_reduce_add_3d(&P.tm_dq, smem + kOffPT + c4 * (128 * 128), c4 * 32, h, z);
                 bulk_commit();
-                bulk_wait_read_all();  // staging may be overwritten once the reads are done
             }
-            if (leader) mbar_arrive(&bars->dq_empty);
         }
         if (leader) bulk_wait_all();
         // ------------------------------------------------------ epilogue
@@ -551,13 +604,19 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
         smem = base;
     }
     P.tab_cap = tab_need;
-    cudaError_t e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimitBwd);
+    const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
+    const bool sm = a.act == JFA_ACT_SOFTMAX;
+    void (*kern)(BwdParams) = nullptr;
+    if (bias == 0) kern = sm ? tc_bwd_kernel<0, true> : tc_bwd_kernel<0, false>;
+    else if (bias == 1) kern = sm ? tc_bwd_kernel<1, true> : tc_bwd_kernel<1, false>;
+    else kern = sm ? tc_bwd_kernel<2, true> : tc_bwd_kernel<2, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimitBwd);
     if (e != cudaSuccess) return e;
     int64_t grid = pairs_bound(p.batch, p.max_kv_len, p.total_kv, BN) * p.heads;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
     if (grid > 0) {
         prof_begin(st);
-        tc_bwd_kernel<<<(unsigned)grid, kThreads, smem, st>>>(P);
+        kern<<<(unsigned)grid, kThreads, smem, st>>>(P);
         prof_end(st, K_TC_BWD);
     }
     const int64_t n8 = rows * HD / 8;

@@ -27,6 +27,7 @@
 // TMEM: S at columns [0, 128), O at [128, 256).
 #include <math_constants.h>
 
+#include "jfa_mx.cuh"
 #include "jfa_sm100.cuh"
 
 namespace jfa {
@@ -88,6 +89,9 @@ __device__ __forceinline__ void named_sync_softmax() {
 
 // BIAS: 0 none, 1 relative-position (window in shared memory when it fits,
 // else through L1), 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.
+// QP: MXFP8 attention -- P is quantised to E4M3 with one E8M0 scale per 32
+// keys (counted from the sequence's first key) before P.V; the row sum l
+// uses the unquantised weights.
 //
 // Pipeline (tensor core): QK_0, QK_1, then for each j: [P_j ready] PV_j,
 // QK_{j+2}.  S is double-buffered in TMEM (S_0 at column 0, S_1 at 128), so
@@ -96,7 +100,7 @@ __device__ __forceinline__ void named_sync_softmax() {
 // softmax of tile j writes it only after P.V of tile j-1 has completed.
 // Each softmax thread owns one query row and one 64-column half of it; the
 // two halves exchange their partial row maxima through shared memory.
-template <int BIAS, bool SOFTMAX>
+template <int BIAS, bool SOFTMAX, bool QP>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
@@ -181,6 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 tma_load_3d(smem + kOffV + s * kTile, &P.tm_v, &bars->v_full[s], 0, h, z);
                 tma_load_3d(smem + kOffV + s * kTile + kBox, &P.tm_v, &bars->v_full[s], 64, h, z);
                 issued = j + 1;
+                if (j + 2 < n_tiles) {  // warm L2 for the tiles loaded after the next release
+                    const int zn = z + 2 * BN;
+                    tma_prefetch_l2_3d(&P.tm_k, 0, h, zn);
+                    tma_prefetch_l2_3d(&P.tm_k, 64, h, zn);
+                    tma_prefetch_l2_3d(&P.tm_v, 0, h, zn);
+                    tma_prefetch_l2_3d(&P.tm_v, 64, h, zn);
+                }
             }
             // never leave the CTA with copies in flight: wait for every issued load
             mbar_wait_drain(&bars->q_full, 0, a.hdr);
@@ -265,13 +276,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tc_fence_after();
             const int jc = j * BN + c0;          // key index of this half's column 0
             float x[64];
-#pragma unroll
-            for (int c4 = 0; c4 < 2; ++c4) {
-                uint32_t u[32];
-                tmem_ld32(tmem + lane_addr + s * 128 + c0 + c4 * 32, u);
+            {
+                uint32_t u[2][32];
+                tmem_ld32(tmem + lane_addr + s * 128 + c0, u[0]);
+                tmem_ld32(tmem + lane_addr + s * 128 + c0 + 32, u[1]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int t = 0; t < 32; ++t) x[c4 * 32 + t] = __uint_as_float(u[t]);
+                for (int t = 0; t < 32; ++t) {
+                    x[t] = __uint_as_float(u[0][t]);
+                    x[32 + t] = __uint_as_float(u[1][t]);
+                }
             }
             const int nvis = i < nq ? max(0, min(64, jmax_vis - jc + 1)) : 0;  // visible: [0, nvis)
             if (BIAS == 1 && tab_in_smem) {
@@ -300,16 +314,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             float alpha = 1.f;
             bool rescale = false;
             if (softmax) {
-                float pm = -CUDART_INF_F;
+                float pm8[8];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) pm = fmaxf(pm, x[c]);
+                for (int t = 0; t < 8; ++t) pm8[t] = x[t];
+#pragma unroll
+                for (int c = 8; c < 64; ++c) pm8[c & 7] = fmaxf(pm8[c & 7], x[c]);
+                const float pm = fmaxf(fmaxf(fmaxf(pm8[0], pm8[1]), fmaxf(pm8[2], pm8[3])),
+                                       fmaxf(fmaxf(pm8[4], pm8[5]), fmaxf(pm8[6], pm8[7])));
                 red[(s * 2 + grp) * 128 + r] = pm;
                 named_sync_softmax();
                 if (*abort_flag) { ok = false; break; }
                 const float tmax = fmaxf(pm, red[(s * 2 + (grp ^ 1)) * 128 + r]);
-                // lazy rescale: keep the reference maximum unless it grew by > 2^8
+                // lazy rescale: keep the reference unless the row maximum grew by
+                // more than 8 (a factor 2^8).  With MXFP8 P the reference is an
+                // integer (ceil of the maximum, log2 units), so rescales are exact
+                // powers of two and the block quantisation of P does not depend on
+                // it; otherwise the maximum itself, so the largest weight is 1.
                 const bool need = tmax > m_used + kRescaleThreshold;
-                const float m_new = need ? tmax : m_used;
+                const float m_new = need ? (QP ? ceilf(tmax) : tmax) : m_used;
                 if (need && m_used != -CUDART_INF_F) {
                     alpha = ex2(m_used - m_new);
                     rescale = true;
@@ -340,15 +362,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 // ex2(-inf) = 0 masks the invisible columns; a row with no visible
                 // key yet uses reference 0 so that -inf - ref stays -inf
                 const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
-                float ps0 = 0.f, ps1 = 0.f;
+                float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
+                for (int c = 0; c < 64; ++c) {
                     x[c] = ex2(x[c] - ref);
-                    x[c + 1] = ex2(x[c + 1] - ref);
-                    ps0 += x[c];
-                    ps1 += x[c + 1];
+                    ps8[c & 7] += x[c];
                 }
-                l += ps0 + ps1;
+                l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+                if (QP) {
+                    mx::fake_quant32(x);
+                    mx::fake_quant32(x + 32);
+                }
             } else {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
@@ -467,7 +491,7 @@ bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, in
 
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per CTA
 
-cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st) {
+cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quant_p, cudaStream_t st) {
     FwdParams P{};
     if (!make_tmap_rows_heads_d(&P.tm_q, a.q, p.total_q, p.heads) ||
         !make_tmap_rows_heads_d(&P.tm_k, a.k, p.total_kv, p.heads) ||
@@ -488,14 +512,22 @@ cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStrea
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
     const bool sm = a.act == JFA_ACT_SOFTMAX;
     void (*kern)(FwdParams) = nullptr;
-    if (bias == 0) kern = sm ? tc_fwd_kernel<0, true> : tc_fwd_kernel<0, false>;
-    else if (bias == 1) kern = sm ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
-    else kern = sm ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
+    if (quant_p) {
+        if (!sm) return cudaErrorInvalidValue;
+        kern = bias == 0 ? tc_fwd_kernel<0, true, true>
+                         : (bias == 1 ? tc_fwd_kernel<1, true, true> : tc_fwd_kernel<2, true, true>);
+    } else if (bias == 0) {
+        kern = sm ? tc_fwd_kernel<0, true, false> : tc_fwd_kernel<0, false, false>;
+    } else if (bias == 1) {
+        kern = sm ? tc_fwd_kernel<1, true, false> : tc_fwd_kernel<1, false, false>;
+    } else {
+        kern = sm ? tc_fwd_kernel<2, true, false> : tc_fwd_kernel<2, false, false>;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     prof_begin(st);
     kern<<<(unsigned)grid, kThreads, smem, st>>>(P);
-    prof_end(st, K_TC_FWD);
+    prof_end(st, quant_p ? K_TC_FWD_MXFP8 : K_TC_FWD);
     return cudaGetLastError();
 }
 

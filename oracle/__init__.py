@@ -59,7 +59,7 @@ def _lib():
             lib.jfa_oracle_forward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
                                                i32, f64, i32, P, P, P, i32]
             lib.jfa_oracle_backward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                                i32, f64, P, P, P, P, P, i32]
+                                                i32, f64, P, P, P, P, P, P, i32]
             lib.jfa_oracle_quantize_mx.argtypes = [P, ctypes.c_int64, P, P]
             lib.jfa_oracle_dequantize_mx.argtypes = [P, P, ctypes.c_int64, P]
             lib.jfa_oracle_e4m3_encode.argtypes = [f64]
@@ -134,8 +134,12 @@ def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0
 
 
 def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpos_len=0,
-             act="softmax", causal=False, scale=0.0, seq_mask=None, nthreads=0):
-    """fp64 analytic gradients (dq, dk, dv); the bias receives none."""
+             act="softmax", causal=False, scale=0.0, seq_mask=None, out_for_d=None,
+             nthreads=0):
+    """fp64 analytic gradients (dq, dk, dv); the bias receives none.
+
+    ``out_for_d``: the forward output whose rows give D = rowsum(dO * O)
+    (the MXFP8 forward's output); by default O is recomputed exactly."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     q64, k64, v64, do64 = _f64(q), _f64(k), _f64(v), _f64(dout)
     B = len(q_off) - 1
@@ -146,10 +150,12 @@ def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpo
     dk = np.full((total_kv, H, d), np.nan)
     dv = np.full((total_kv, H, d), np.nan)
     mask = _item_mask(seq_mask, B, H)
+    o64 = _f64(out_for_d) if out_for_d is not None else None
     _lib().jfa_oracle_backward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                                _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                                ACT[act], int(bool(causal)), float(scale), _ptr(mask),
-                               _ptr(do64), _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads))
+                               _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv),
+                               int(nthreads))
     return dq, dk, dv
 
 

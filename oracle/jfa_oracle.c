@@ -225,18 +225,32 @@ static void row_weights(const orc_problem* P, int b, int h, int i, double* s, do
         for (int j = 0; j < nkv; ++j) l += w[j];
         if (pv_weight) {
             if (P->quant_p) {
-                /* quantise the unnormalised weights exp(s - m_final) in blocks of
-                 * 32 consecutive keys, counted from the sequence's first key */
+                /* MXFP8 P: the weights 2^(x_j - R), x_j = s_j log2(e), with the
+                 * integer reference R = ceil(max_j x_j), are quantised in blocks
+                 * of 32 consecutive keys counted from the sequence's first key;
+                 * l sums the unquantised weights.  A power-of-two reference makes
+                 * the codes independent of which integer R a kernel uses. */
+                double xmax = -INFINITY;
+                for (int j = 0; j < nkv; ++j)
+                    if (is_valid(P->causal, i, j, nq, nkv) && s[j] * M_LOG2E > xmax) xmax = s[j] * M_LOG2E;
+                const double R = ceil(xmax);
+                double* w2 = (double*)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
+                double l2 = 0.0;
+                for (int j = 0; j < nkv; ++j) {
+                    w2[j] = is_valid(P->causal, i, j, nq, nkv) ? exp2(s[j] * M_LOG2E - R) : 0.0;
+                    l2 += w2[j];
+                }
                 for (int j0 = 0; j0 < nkv; j0 += 32) {
                     double blk[32];
                     uint8_t codes[32], sc;
-                    for (int t = 0; t < 32; ++t) blk[t] = (j0 + t < nkv) ? w[j0 + t] : 0.0;
+                    for (int t = 0; t < 32; ++t) blk[t] = (j0 + t < nkv) ? w2[j0 + t] : 0.0;
                     jfa_oracle_quantize_mx(blk, 1, codes, &sc);
                     double deq[32];
                     jfa_oracle_dequantize_mx(codes, &sc, 1, deq);
                     for (int t = 0; t < 32 && j0 + t < nkv; ++t)
-                        pv_weight[j0 + t] = (l > 0.0) ? deq[t] / l : 0.0;
+                        pv_weight[j0 + t] = (l2 > 0.0) ? deq[t] / l2 : 0.0;
                 }
+                free(w2);
             } else {
                 for (int j = 0; j < nkv; ++j) pv_weight[j] = (l > 0.0) ? w[j] / l : 0.0;
             }
@@ -284,10 +298,12 @@ static void forward_item(const orc_problem* P, int b, int h, double* out, double
  * GDPA   : ds_ij = dp_ij act'(s_ij) / n_kv on valid (i, j), 0 elsewhere
  * both   : dV_j += w_ij dO_i, dQ_i += scale sum_j ds_ij k_j,
  *          dK_j += scale ds_ij q_i.
- * The bias gets no gradient.  With quant_p the quantiser is a straight-through
- * estimator, so the gradients are those of the unquantised weights. */
-static void backward_item(const orc_problem* P, int b, int h, const double* dout, double* dq,
-                          double* dk, double* dv) {
+ * The bias gets no gradient.  For MXFP8 the quantisers are straight-through
+ * estimators: the gradients are those of the unquantised weights on the
+ * dequantised operands, with D taken from the forward's saved output when
+ * out_for_d is given. */
+static void backward_item(const orc_problem* P, int b, int h, const double* dout,
+                          const double* out_for_d, double* dq, double* dk, double* dv) {
     int nq = P->q_off[b + 1] - P->q_off[b];
     int nkv = P->kv_off[b + 1] - P->kv_off[b];
     int H = P->H, d = P->d;
@@ -309,10 +325,17 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
         for (int c = 0; c < d; ++c) dqi[c] = 0.0;
         double Di = 0.0;
         if (P->act == ORC_ACT_SOFTMAX) {
-            for (int c = 0; c < d; ++c) o[c] = 0.0;
-            for (int j = 0; j < nkv; ++j) {
-                const double* vj = row_ptr(P->v, P->kv_off[b] + j, H, h, d);
-                for (int c = 0; c < d; ++c) o[c] += w[j] * vj[c];
+            if (out_for_d) {
+                /* D from the forward's saved output (MXFP8: the output computed
+                 * with quantised P), as a training step uses it */
+                const double* oi = row_ptr(out_for_d, P->q_off[b] + i, H, h, d);
+                for (int c = 0; c < d; ++c) o[c] = oi[c];
+            } else {
+                for (int c = 0; c < d; ++c) o[c] = 0.0;
+                for (int j = 0; j < nkv; ++j) {
+                    const double* vj = row_ptr(P->v, P->kv_off[b] + j, H, h, d);
+                    for (int c = 0; c < d; ++c) o[c] += w[j] * vj[c];
+                }
             }
             for (int c = 0; c < d; ++c) Di += doi[c] * o[c];
         }
@@ -381,8 +404,8 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
 int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                         const double* q, const double* k, const double* v, int bias_kind,
                         const double* bias, int relpos_len, int act, int causal, double scale,
-                        const int32_t* item_mask, const double* dout, double* dq, double* dk,
-                        double* dv, int nthreads) {
+                        const int32_t* item_mask, const double* dout, const double* out_for_d,
+                        double* dq, double* dk, double* dv, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
                  scale, 0);
@@ -394,7 +417,7 @@ int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t
     for (long it = 0; it < n_items; ++it) {
         int b = (int)(it / H), h = (int)(it % H);
         if (item_mask && !item_mask[it]) continue;
-        backward_item(&P, b, h, dout, dq, dk, dv);
+        backward_item(&P, b, h, dout, out_for_d, dq, dk, dv);
     }
     free((void*)P.dense_off);
     (void)nthreads;

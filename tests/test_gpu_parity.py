@@ -310,3 +310,137 @@ def test_quantize_mxfp8_bit_exact(cuda_device):
     rc, rs = oracle.quantize_mx_along_rows(v, p.kv_off)
     assert np.array_equal(codes.cpu().numpy(), rc)
     assert np.array_equal(scales[:rs.shape[0]].cpu().numpy(), rs)
+
+
+# ---------------------------------------------------------------------------
+# MXFP8: Q/K quantised along d, V along 32-row blocks, P per 32 keys
+# ---------------------------------------------------------------------------
+MX_MAX = 6e-2
+
+
+def mx_dequantised_inputs(p):
+    """The exact operands an MXFP8 kernel sees, from the oracle's quantiser."""
+    qc, qs = oracle.quantize_mx_along_d(p.q)
+    kc, ks = oracle.quantize_mx_along_d(p.k)
+    vc, vs = oracle.quantize_mx_along_rows(p.v, p.kv_off)
+    rows_q, H, d = p.q.shape
+    qd = oracle.dequantize_mx(qc.reshape(-1), np.repeat(qs.reshape(-1), 1)).reshape(rows_q, H, d)
+    kd = oracle.dequantize_mx(kc.reshape(-1), ks.reshape(-1)).reshape(p.k.shape)
+    vd = oracle.dequantize_along_rows(vc, vs, p.kv_off)
+    return qd, kd, vd
+
+
+def check_mxfp8(p, dev, seq_mask=None):
+    out, lse, (dq, dk, dv) = run_gpu(p, dev)
+    qd, kd, vd = mx_dequantised_inputs(p)
+    kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act="softmax",
+              causal=p.causal, seq_mask=seq_mask)
+    ro, rl = oracle.forward(p.q_off, p.kv_off, qd, kd, vd, quant_p=True, **kw)
+    rdq, rdk, rdv = oracle.backward(p.q_off, p.kv_off, qd, kd, vd, p.dout, out_for_d=ro, **kw)
+    qr, kr = _rows(p.q_off, seq_mask), _rows(p.kv_off, seq_mask)
+    compare("O", out, ro, qr, MX_MAX)
+    compare("LSE", lse, rl, qr, LSE_MAX)
+    compare("dQ", dq, rdq, qr, MX_MAX)
+    compare("dK", dk, rdk, kr, MX_MAX)
+    compare("dV", dv, rdv, kr, MX_MAX)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_mxfp8_small(cuda_device, seed):
+    p = make_problem("self_mxfp8", 30 + seed, B=6, max_len=330)
+    assert jfa.jfa_path(jfa.problem_of(p), "softmax", 0) == 1
+    check_mxfp8(p, cuda_device)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, launched as bench.py launches them, checked on sampled
+# (sequence, head) items that the oracle computes in seconds
+# ---------------------------------------------------------------------------
+def _sample_items(p, n_short=3, max_len=1200, heads=(0,)):
+    lens = np.maximum(p.q_lens, p.kv_lens)
+    order = np.argsort(lens, kind="stable")
+    picks = list(order[:n_short])
+    mid = [b for b in order if lens[b] <= max_len][-2:]
+    picks += mid
+    mask = np.zeros(p.B * p.H, np.int32)
+    for b in picks:
+        for h in heads:
+            mask[b * p.H + h] = 1
+    return mask
+
+
+def _item_rows(off, H, mask):
+    """(row index, head) pairs of the selected items."""
+    rows, heads = [], []
+    for b in range(len(off) - 1):
+        for h in range(H):
+            if mask[b * H + h]:
+                r = np.arange(int(off[b]), int(off[b + 1]))
+                rows.append(r)
+                heads.append(np.full(len(r), h))
+    return np.concatenate(rows), np.concatenate(heads)
+
+
+def _check_items(name, gpu, ref, rows, heads, max_tol, mean_tol=None):
+    g = gpu.float().cpu().numpy()[rows, heads].astype(np.float64)
+    r = ref[rows, heads]
+    bound = max_tol + half_ulp_bf16(r)
+    assert np.all(np.abs(g - r) <= bound), f"{name}: max err {np.abs(g - r).max():.3e}"
+    if mean_tol is not None:
+        rb = torch.from_numpy(r).to(torch.bfloat16).double().numpy()
+        assert np.abs(g - rb).mean() <= mean_tol, name
+
+
+@pytest.mark.parametrize("workload,act", [("self_bf16", None), ("cross_bf16", None),
+                                          ("gdpa_bf16", "silu"), ("gdpa_bf16", "gelu_tanh")])
+def test_full_size_sampled(cuda_device, workload, act):
+    p = make_problem(workload, 1)
+    act = act or p.act
+    out, lse, (dq, dk, dv) = run_gpu(p, cuda_device, act)
+    mask = _sample_items(p, heads=(0, p.H - 1))
+    kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
+              causal=p.causal, seq_mask=mask)
+    ro, rl = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, **kw)
+    rdq, rdk, rdv = oracle.backward(p.q_off, p.kv_off, p.q, p.k, p.v, p.dout, **kw)
+    qrows, qh = _item_rows(p.q_off, p.H, mask)
+    krows, kh = _item_rows(p.kv_off, p.H, mask)
+    _check_items("O", out, ro, qrows, qh, BF16_MAX, BF16_MEAN)
+    if act == "softmax":
+        gl = lse.cpu().numpy()[qrows, qh]
+        assert np.all(np.abs(gl - rl[qrows, qh]) <= LSE_MAX)
+    _check_items("dQ", dq, rdq, qrows, qh, BF16_MAX, BF16_MEAN)
+    _check_items("dK", dk, rdk, krows, kh, BF16_MAX, BF16_MEAN)
+    _check_items("dV", dv, rdv, krows, kh, BF16_MAX, BF16_MEAN)
+    # properties over every row: finite outputs, LSE finite where a key is visible
+    assert torch.isfinite(out).all() and torch.isfinite(dq).all()
+    assert torch.isfinite(dk).all() and torch.isfinite(dv).all()
+
+
+def test_full_size_mxfp8_sampled(cuda_device):
+    p = make_problem("self_mxfp8", 1)
+    out, lse, (dq, dk, dv) = run_gpu(p, cuda_device)
+    mask = _sample_items(p, heads=(0,))
+    seqs = sorted({i // p.H for i in np.nonzero(mask)[0]})
+    # dequantised operands of the sampled sequences only (the oracle's V
+    # quantiser walks sequences one by one)
+    sub_q = [np.arange(int(p.q_off[b]), int(p.q_off[b + 1])) for b in seqs]
+    sub = make_problem("self_mxfp8", 1, q_lens=[len(r) for r in sub_q])
+    sub.q = torch.cat([p.q[r] for r in sub_q])
+    sub.k = torch.cat([p.k[r] for r in sub_q])
+    sub.v = torch.cat([p.v[r] for r in sub_q])
+    sub.dout = torch.cat([p.dout[r] for r in sub_q])
+    sub.bias = p.bias
+    sub.relpos_len = p.relpos_len
+    qd, kd, vd = mx_dequantised_inputs(sub)
+    kw = dict(bias=sub.bias, bias_kind="relpos", relpos_len=sub.relpos_len, causal=True,
+              seq_mask=np.array([1 if h == 0 else 0 for _ in seqs for h in range(p.H)], np.int32))
+    ro, rl = oracle.forward(sub.q_off, sub.kv_off, qd, kd, vd, quant_p=True, **kw)
+    rdq, rdk, rdv = oracle.backward(sub.q_off, sub.kv_off, qd, kd, vd, sub.dout, out_for_d=ro,
+                                    **kw)
+    rows = np.concatenate(sub_q)
+    for name, g, r in (("O", out, ro), ("dQ", dq, rdq), ("dK", dk, rdk), ("dV", dv, rdv)):
+        gg = g.float().cpu().numpy()[rows, 0].astype(np.float64)
+        rr = r[:, 0]
+        assert np.all(np.abs(gg - rr) <= MX_MAX + half_ulp_bf16(rr)), name
+    gl = lse.cpu().numpy()[rows, 0]
+    assert np.all(np.abs(gl - rl[:, 0]) <= LSE_MAX)

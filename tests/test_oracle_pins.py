@@ -369,3 +369,21 @@ def test_schedule_covers_every_tile_once_longest_first():
                 assert int(sub.sum()) == c
                 total += c
             assert total == H * oracle.valid_pairs(q_off, kv_off, causal)
+
+
+def test_backward_d_from_saved_output():
+    """D taken from a saved output equals the recomputed one when that output
+    is the oracle's own forward; a perturbed output changes only the softmax
+    score-gradient terms (dQ, dK), never dV."""
+    P = _jagged(10, [6, 9], [6, 9], bias_kind="relpos")
+    kw = dict(bias=P["bias"], bias_kind="relpos", relpos_len=P["relpos_len"], causal=True)
+    out, _ = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
+    ref = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"], **kw)
+    same = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                           out_for_d=out, **kw)
+    for a, b in zip(ref, same):
+        assert np.array_equal(a, b)
+    bumped = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                             out_for_d=out * 1.01, **kw)
+    assert np.array_equal(bumped[2], ref[2])
+    assert not np.allclose(bumped[0], ref[0])
