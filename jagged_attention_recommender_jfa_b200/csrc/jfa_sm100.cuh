@@ -185,6 +185,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -239,6 +250,50 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Round-to-nearest-even to bf16 on the integer pipe (finite inputs): add
+// 0x7FFF plus the lowest kept bit, keep the upper 16 bits; two results are
+// packed with one byte permute.  Used for the P / dS operands, which keeps
+// the conversion off the pipe that also evaluates exp2.
+#ifndef JFA_PACK_ALU
+#define JFA_PACK_ALU 0
+#endif
+__device__ __forceinline__ uint32_t pack_bf16_p(float lo, float hi) {
+#if JFA_PACK_ALU
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a += 0x7FFFu + ((a >> 16) & 1u);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return __byte_perm(a, b, 0x7632);
+#else
+    return pack_bf16(lo, hi);
+#endif
+}
+
+// 2^y on the FMA pipe for y <= 8 (Cody-Waite style split y = n + f with
+// n = round(y), f in [-0.5, 0.5]; 2^f by a cubic fitted here for minimax
+// relative error, max 7.5e-5, well below bf16's 2^-9; 2^n added to the
+// exponent bits).  Inputs below -126 give a value below 2^-125.
+#ifndef JFA_EXP2_POLY_MOD
+#define JFA_EXP2_POLY_MOD 0
+#endif
+__device__ __forceinline__ float exp2_fma(float y) {
+    y = fmaxf(y, -126.0f);
+    const float t = y + 12582912.0f;  // 1.5 * 2^23: the low mantissa bits of t hold round(y)
+    const float n = t - 12582912.0f;
+    const float f = y - n;
+    const float p = fmaf(fmaf(fmaf(0.05517098f, f, 0.24260971f), f, 0.69326097f), f, 0.9999282f);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// exp2 of element c of a row: every JFA_EXP2_POLY_MOD-th element on the FMA
+// pipe, the rest on the MUFU.
+template <int c>
+__device__ __forceinline__ float exp2_mixed(float y) {
+#if JFA_EXP2_POLY_MOD > 0
+    if ((c % JFA_EXP2_POLY_MOD) == JFA_EXP2_POLY_MOD - 1) return exp2_fma(y);
+#endif
+    return ex2(y);
 }
 
 }  // namespace sm100

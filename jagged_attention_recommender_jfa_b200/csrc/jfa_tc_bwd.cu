@@ -19,10 +19,10 @@
 //                             the fp32 accumulator by TMA reduce-add
 //   tc_bwd_dq_finalize  dQ = bf16(scale * accumulator).
 //
-// Warp roles: warp 0 TMA, warp 1 MMA, warps 2..9 score warps in two groups
-// of four; a thread owns one key row (or, for dQ, one query row) and half of
-// its 128 columns (group 0: columns 0-63, group 1: 64-127).  The backward
-// needs no row reduction (LSE and D are given), so the halves never talk.
+// Warp roles: warp 0 TMA, warp 1 MMA, warps 2..17 score warps in four groups
+// of four; a thread owns one key row (or, for dQ, one query row) and one
+// 32-column chunk of it.  The backward needs no row reduction (LSE and D are
+// given), so the chunks never talk.
 // TMEM columns: dV [0,128), dK [128,256), S^T and dQ_t [256,384), dP^T [384,512).
 #include <math_constants.h>
 
@@ -37,7 +37,8 @@ bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, in
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int kThreads = 320;
+constexpr int NG = 4;                 // column groups: a score thread owns one 32-column chunk
+constexpr int kThreads = 64 + NG * 128;
 constexpr uint32_t kBox = 128 * 128;
 constexpr uint32_t kTile = 2 * kBox;
 constexpr uint32_t kOffK = 0;
@@ -55,6 +56,8 @@ struct Bars {
     uint64_t kv_full;
     uint64_t q_full;
     uint64_t q_empty;
+    uint64_t do_full;
+    uint64_t do_empty;
     uint64_t s_full;
     uint64_t ds_full;
     uint64_t dq_full;
@@ -92,7 +95,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 __device__ __forceinline__ void named_sync_score() {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(NG * 128) : "memory");
 }
 
 // TMA reduce-add of a shared-memory tile into global memory (no multicast).
@@ -126,6 +129,35 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t* tile, int r, int c4, c
     }
 }
 
+// P = 2^(s - lse) and dS = P (dP - D) for 32 columns (compile-time column
+// index, so that exp2_mixed can place each element on its pipe).
+template <int v>
+__device__ __forceinline__ void softmax_chunk(uint32_t (&u)[16], uint32_t (&g)[16], const float* l2c,
+                                              const float* ddc) {
+    if constexpr (v < 16) {
+        const float pr = exp2_mixed<v>(__uint_as_float(u[v]) - l2c[v]);
+        u[v] = __float_as_uint(pr);
+        g[v] = __float_as_uint(pr * (__uint_as_float(g[v]) - ddc[v]));
+        softmax_chunk<v + 1>(u, g, l2c, ddc);
+    }
+}
+
+// Stores 16 fp32 values (bit patterns) as bf16: columns 16*c16 .. +15 of row r
+// of a K-major 128B-swizzled tile.
+__device__ __forceinline__ void store_half_chunk_bits(uint8_t* tile, int r, int c16, const uint32_t (&v)[16]) {
+    uint8_t* row = tile + (c16 >> 2) * kBox + r * 128;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int ch = (c16 & 3) * 2 + u;
+        uint4 w;
+        w.x = pack_bf16_p(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
+        w.y = pack_bf16_p(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
+        w.z = pack_bf16_p(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
+        w.w = pack_bf16_p(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
+        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
+    }
+}
+
 // Same as store_chunk_bf16 for 32 fp32 values held as bit patterns.
 __device__ __forceinline__ void store_chunk_bits(uint8_t* tile, int r, int c4, const uint32_t (&v)[32]) {
     uint8_t* row = tile + (c4 >> 1) * kBox + r * 128;
@@ -133,10 +165,10 @@ __device__ __forceinline__ void store_chunk_bits(uint8_t* tile, int r, int c4, c
     for (int u = 0; u < 4; ++u) {
         const int ch = (c4 & 1) * 4 + u;
         uint4 w;
-        w.x = pack_bf16(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
-        w.y = pack_bf16(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
-        w.z = pack_bf16(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
-        w.w = pack_bf16(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
+        w.x = pack_bf16_p(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
+        w.y = pack_bf16_p(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
+        w.z = pack_bf16_p(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
+        w.w = pack_bf16_p(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
         *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
     }
 }
@@ -180,10 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
+        mbar_init(&bars->do_full, 1);
+        mbar_init(&bars->do_empty, 1);
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->ds_full, 8);
+        mbar_init(&bars->ds_full, NG * 4);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 8);
+        mbar_init(&bars->dq_empty, NG * 4);
         mbar_init(&bars->stage_free, 1);
         mbar_init(&bars->fin, 1);
         mbar_init(&bars->drain, 1);
@@ -223,16 +257,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, h, k0 + j0);
             tma_load_3d(smem + kOffV, &P.tm_v, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->kv_full, 64, h, k0 + j0);
-            int issued = 0;
+            // Q of tile t+1 is loaded as soon as dK += dS^T Q of tile t has retired,
+            // dO as soon as dV += P^T dO has (the MMAs of a tile run dK, dV, dQ)
+            int issued_q = 0, issued_do = 0;
             for (int t = 0; t < nt; ++t) {
-                if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
                 const int z = q0 + i_start + t * BM;
-                mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
+                if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
+                mbar_arrive_expect_tx(&bars->q_full, kTile);
                 tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, h, z);
                 tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, z);
-                tma_load_3d(smem + kOffDO, &P.tm_do, &bars->q_full, 0, h, z);
-                tma_load_3d(smem + kOffDO + kBox, &P.tm_do, &bars->q_full, 64, h, z);
-                issued = t + 1;
+                issued_q = t + 1;
+                if (t > 0 && !mbar_wait(&bars->do_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
+                mbar_arrive_expect_tx(&bars->do_full, kTile);
+                tma_load_3d(smem + kOffDO, &P.tm_do, &bars->do_full, 0, h, z);
+                tma_load_3d(smem + kOffDO + kBox, &P.tm_do, &bars->do_full, 64, h, z);
+                issued_do = t + 1;
                 if (t + 1 < nt) {  // warm L2 for the next query tile (single-buffered)
                     tma_prefetch_l2_3d(&P.tm_q, 0, h, z + BM);
                     tma_prefetch_l2_3d(&P.tm_q, 64, h, z + BM);
@@ -241,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
             }
             mbar_wait_drain(&bars->kv_full, 0, a.hdr);
-            if (issued > 0) mbar_wait_drain(&bars->q_full, (issued - 1) & 1, a.hdr);
+            if (issued_q > 0) mbar_wait_drain(&bars->q_full, (issued_q - 1) & 1, a.hdr);
+            if (issued_do > 0) mbar_wait_drain(&bars->do_full, (issued_do - 1) & 1, a.hdr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -260,6 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tS, kmajor_desc(kb, k), kmajor_desc(qb, k), idesc_nt, k > 0 ? 1u : 0u);
+                if (!mbar_wait(&bars->do_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tdP, kmajor_desc(vb, k), kmajor_desc(dob, k), idesc_nt, k > 0 ? 1u : 0u);
@@ -268,16 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)
-                    mma_bf16_ss(tdV, kmajor_desc(ptb, k), mnmajor_desc(dob, k), idesc_nn,
-                                (t > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < BM / 16; ++k)
                     mma_bf16_ss(tdK, kmajor_desc(dsb, k), mnmajor_desc(qb, k), idesc_nn,
                                 (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bars->q_empty);
+#pragma unroll
+                for (int k = 0; k < BM / 16; ++k)
+                    mma_bf16_ss(tdV, kmajor_desc(ptb, k), mnmajor_desc(dob, k), idesc_nn,
+                                (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bars->do_empty);
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tS, mnmajor_desc(dsb, k), mnmajor_desc(kb, k), idesc_tn, k > 0 ? 1u : 0u);
-                mma_commit(&bars->q_empty);
                 mma_commit(&bars->dq_full);
             }
             if (ok) mma_commit(&bars->fin);
@@ -287,12 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     } else {
         // ------------------------------------------------ score warps
         const int wq = warp & 3;                 // TMEM lane quarter
-        const int grp = (warp - 2) >> 2;         // column half: 0 -> [0,64), 1 -> [64,128)
+        const int grp = (warp - 2) >> 2;         // 32-column chunk of the row
         const int r = wq * 32 + lane;            // key row (S^T, dV, dK) / query row (dQ)
         const int j = j0 + r;                    // key index within the sequence
         const bool jvalid = j < nkv;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-        const uint32_t cofs = (uint32_t)grp * 64;
+        const uint32_t cofs = (uint32_t)grp * 32;
         const uint32_t tdV = tmem + lane_addr + cofs, tdK = tmem + lane_addr + 128 + cofs;
         const uint32_t tS = tmem + lane_addr + 256 + cofs, tdP = tmem + lane_addr + 384 + cofs;
         const float sc = a.scale * kLog2e;
@@ -346,30 +389,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 mbar_wait(&bars->stage_free, (t - 1) & 1, abort_flag, a.hdr);
             }
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
-            // one 32-column chunk: scores u (TMEM bits) -> P in place, dP g -> dS in place
-            auto process = [&](uint32_t (&u)[32], uint32_t (&g)[32], int c4) {
-                const int qc0 = qb0 + c4 * 32;       // query index of the chunk's column 0
-                const bool all_vis = jvalid && (qc0 + 31 < nq) && (qc0 >= imin_vis);
-                const bool none_vis = !jvalid || qc0 >= nq || (qc0 + 31 < imin_vis);
+            // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
+            auto process = [&](uint32_t (&u)[16], uint32_t (&g)[16], int c16) {
+                const int qc0 = qb0 + c16 * 16;      // query index of the part's column 0
+                const bool all_vis = jvalid && (qc0 + 15 < nq) && (qc0 >= imin_vis);
+                const bool none_vis = !jvalid || qc0 >= nq || (qc0 + 15 < imin_vis);
                 if (none_vis) {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) u[v] = 0u, g[v] = 0u;
+                    for (int v = 0; v < 16; ++v) u[v] = 0u, g[v] = 0u;
                     return;
                 }
                 if (BIAS == 1 && tab_in_smem) {
                     const float* tb = tab + (qc0 - j - tab_lo);   // tb[v] = bias(qc0 + v, j)
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, tb[v]));
+                    for (int v = 0; v < 16; ++v) u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, tb[v]));
                 } else if (BIAS == 1) {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) {
+                    for (int v = 0; v < 16; ++v) {
                         int rr = qc0 + v - j;
                         rr = rr < -C ? -C : (rr > C ? C : rr);
                         u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, __ldg(tab_g + rr + C) * kLog2e));
                     }
                 } else if (BIAS == 2) {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) {
+                    for (int v = 0; v < 16; ++v) {
                         const int qi = qc0 + v;
                         const float bv = (jvalid && qi < nq)
                             ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
@@ -377,20 +420,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     }
                 } else {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) u[v] = __float_as_uint(__uint_as_float(u[v]) * sc);
+                    for (int v = 0; v < 16; ++v) u[v] = __float_as_uint(__uint_as_float(u[v]) * sc);
                 }
                 if (SOFTMAX) {
-                    const float* l2c = lse2_s + buf * 128 + c4 * 32;
-                    const float* ddc = dd_s + buf * 128 + c4 * 32;
-#pragma unroll
-                    for (int v = 0; v < 32; ++v) {
-                        const float pr = ex2(__uint_as_float(u[v]) - l2c[v]);
-                        u[v] = __float_as_uint(pr);
-                        g[v] = __float_as_uint(pr * (__uint_as_float(g[v]) - ddc[v]));
-                    }
+                    const float* l2c = lse2_s + buf * 128 + c16 * 16;
+                    const float* ddc = dd_s + buf * 128 + c16 * 16;
+                    softmax_chunk<0>(u, g, l2c, ddc);
                 } else {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) {
+                    for (int v = 0; v < 16; ++v) {
                         const float sn = __uint_as_float(u[v]) * (1.0f / kLog2e);
                         u[v] = __float_as_uint(act_f(a.act, sn) * inv_n);
                         g[v] = __float_as_uint(__uint_as_float(g[v]) * act_grad_f(a.act, sn) * inv_n);
@@ -398,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
                 if (!all_vis) {
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) {
+                    for (int v = 0; v < 16; ++v) {
                         const int qi = qc0 + v;
                         const bool vis = jvalid && qi < nq && qi >= imin_vis;
                         u[v] = vis ? u[v] : 0u;
@@ -407,20 +445,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
             };
 #pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
-                uint32_t u[32], g[32];
-                tmem_ld32(tS + cc * 32, u);
-                tmem_ld32(tdP + cc * 32, g);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t u[16], g[16];
+                tmem_ld16(tS + hh * 16, u);
+                tmem_ld16(tdP + hh * 16, g);
                 tmem_wait_ld();
-                const int c4 = grp * 2 + cc;
-                process(u, g, c4);
-                store_chunk_bits(smem + kOffPT, r, c4, u);
-                store_chunk_bits(smem + kOffDST, r, c4, g);
+                const int c16 = grp * 2 + hh;
+                process(u, g, c16);
+                store_half_chunk_bits(smem + kOffPT, r, c16, u);
+                store_half_chunk_bits(smem + kOffDST, r, c16, g);
             }
             // query rows past the sequence end must not reach dV / dK
             if (qb0 + r >= nq) {
                 if (grp == 0) zero_row(smem + kOffQ, r);
-                else zero_row(smem + kOffDO, r);
+                else if (grp == 1) zero_row(smem + kOffDO, r);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -432,20 +470,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr);
             tc_fence_after();
             const bool qvalid = qb0 + r < nq;
-            uint32_t u2[2][32];
-            tmem_ld32(tS, u2[0]);
-            tmem_ld32(tS + 32, u2[1]);
+            uint32_t u2[32];
+            tmem_ld32(tS, u2);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dq_empty);  // TMEM columns free for S^T of t+1
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c4 = grp * 2 + cc;
-                uint8_t* row = smem + kOffPT + c4 * (128 * 128) + r * 128;
+            {
+                uint8_t* row = smem + kOffPT + grp * (128 * 128) + r * 128;
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
-                    uint4 w = qvalid ? make_uint4(u2[cc][4 * v], u2[cc][4 * v + 1], u2[cc][4 * v + 2], u2[cc][4 * v + 3])
+                    uint4 w = qvalid ? make_uint4(u2[4 * v], u2[4 * v + 1], u2[4 * v + 2], u2[4 * v + 3])
                                      : make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4*>(row + ((v ^ (r & 7)) << 4)) = w;
                 }
@@ -472,12 +507,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tc_fence_after();
             __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
             __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
-#pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
+            {
+                const int cc = 0;
                 uint32_t uk[32], uv[32];
                 if (nt > 0) {
-                    tmem_ld32(tdK + cc * 32, uk);
-                    tmem_ld32(tdV + cc * 32, uv);
+                    tmem_ld32(tdK, uk);
+                    tmem_ld32(tdV, uv);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
