@@ -45,8 +45,7 @@ constexpr uint32_t kTile = 2 * kBox;        // one 128 x 128 bf16 tile (two boxe
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;        // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTile;    // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTile;
-constexpr uint32_t kOffBar = kOffP + kTile;      // 196608
+constexpr uint32_t kOffBar = kOffV + 2 * kTile;  // 163840
 constexpr uint32_t kOffRed = kOffBar + 512;      // row-max exchange [2][NG][128] + l [2][NG][128]
 constexpr uint32_t kSmemBytes = kOffRed + 2 * 2 * NG * 128 * 4 + 1024;  // + alignment slack
 constexpr float kLog2e = 1.4426950408889634f;
@@ -224,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
-            const uint32_t qb = sbase + kOffQ, pb = sbase + kOffP;
+            const uint32_t qb = sbase + kOffQ;
             int g = 0, nk = 0, m = 0;
             bool ok = true;
             auto issue_qk = [&](int gg, int n_left_after) -> bool {
@@ -259,9 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     if (!mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t vb = sbase + kOffV + s * kTile;
+                    const uint32_t tP = tmem + s * 128;  // P (bf16 pairs) over columns 0..63 of its S
 #pragma unroll
                     for (int k = 0; k < BN / 16; ++k)
-                        mma_bf16_ss(tO, kmajor_desc(pb, k), mnmajor_desc(vb, k), idesc_pv,
+                        mma_bf16_ts(tO, tP + k * 8, mnmajor_desc(vb, k), idesc_pv,
                                     (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&bars->v_empty[s]);
                     mma_commit(&bars->pv_done);
@@ -281,8 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const float sc = a.scale * kLog2e;
         const int C = (a.relpos_len - 1) >> 1;
-        uint8_t* prow = smem + kOffP + (c0 >> 6) * kBox + r_ * 128;
-        const int ch0 = (c0 & 63) >> 3;          // first 16-byte chunk of the group in its box row
         int g = 0, m = 0;
         bool ok = true;
         // Every softmax warp runs the same sequence of named barriers: a failed
@@ -376,13 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     }
                     m_used = m_new;
                 }
-                // P.V of the previous key tile (any item) must be done before O of
-                // this item or the P buffer change
-                if (g > 0) {
-                    mbar_wait(&bars->pv_done, (g - 1) & 1, abort_flag, a.hdr);
-                    tc_fence_after();
-                }
+                // a rescale of O needs every earlier P.V of this item retired
                 if (softmax && __any_sync(0xffffffffu, rescale)) {
+                    if (g > 0) {
+                        mbar_wait(&bars->pv_done, (g - 1) & 1, abort_flag, a.hdr);
+                        tc_fence_after();
+                    }
                     uint32_t u[32];
                     tmem_ld32(tO, u);
                     tmem_wait_ld();
@@ -410,16 +407,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         const float s_nat = x[c] * (1.0f / kLog2e);
                         x[c] = c < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
                     }
+                    // P overwrites S columns other groups may still be loading
+                    named_sync_softmax();
                 }
-                // P row part -> shared memory, K-major, 128-byte swizzle (chunk ^ row%8)
+                // P row part (bf16 pairs) -> TMEM over the first 64 columns of its own
+                // S buffer: column c0/2 + t holds keys c0 + 2t (low half) and c0 + 2t + 1.
+                // Every group has loaded its S columns (they did so before the barrier
+                // above), and the next write to this buffer is QK_{j+2}, issued after
+                // P.V_j, which reads it.
+                {
+                    uint32_t pw[16];
 #pragma unroll
-                for (int ch = 0; ch < CW / 8; ++ch) {
-                    uint4 wv;
-                    wv.x = pack_bf16(x[ch * 8 + 0], x[ch * 8 + 1]);
-                    wv.y = pack_bf16(x[ch * 8 + 2], x[ch * 8 + 3]);
-                    wv.z = pack_bf16(x[ch * 8 + 4], x[ch * 8 + 5]);
-                    wv.w = pack_bf16(x[ch * 8 + 6], x[ch * 8 + 7]);
-                    *reinterpret_cast<uint4*>(prow + (((ch0 + ch) ^ (r_ & 7)) << 4)) = wv;
+                    for (int t = 0; t < 16; ++t) pw[t] = pack_bf16(x[2 * t], x[2 * t + 1]);
+                    tmem_st16(tmem + lane_addr + s * 128 + (c0 >> 1), pw);
+                    tmem_wait_st();
                 }
                 // value rows past the sequence end (neighbour data) must not reach P.V
                 const int nvalid = w.nkv - j * BN;
