@@ -58,7 +58,7 @@ thread_local char g_msg[512] = "";
 const char* const kKernelNames[K_COUNT] = {
     "sched_prepare", "sched_rank", "simt_fwd", "simt_bwd_pre", "simt_bwd_dq", "simt_bwd_dkdv",
     "quant_along_d", "quant_along_rows", "tc_fwd", "tc_bwd_pre", "tc_bwd", "tc_dq_finalize",
-    "tc_fwd_mxfp8"};
+    "tc_fwd_mxfp8", "tc_bias_prep"};
 
 }  // namespace
 

@@ -108,6 +108,11 @@ struct AttnArgs {
     void* dk;
     void* dv;
     float* dq_acc;
+    // tensor-core path, relative-position bias: four copies of each head's
+    // table scaled by log2(e), copy k shifted left by k entries, so that any
+    // run of table entries can be read with 16-byte-aligned vector loads
+    const float* bias4;
+    int bias4_stride;  // floats per copy (a multiple of 4)
 };
 
 // ---------------------------------------------------------------------------
@@ -160,6 +165,7 @@ enum KernelId {
     K_TC_BWD,
     K_TC_DQ_FINALIZE,
     K_TC_FWD_MXFP8,
+    K_TC_BIAS_PREP,
     K_COUNT
 };
 void prof_begin(cudaStream_t st);

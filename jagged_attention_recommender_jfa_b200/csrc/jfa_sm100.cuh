@@ -10,6 +10,32 @@
 #include "jfa_common.cuh"
 
 namespace jfa {
+// Pipeline timeline hooks.  Compiled out unless JFA_TRACE is defined; then
+// JFA_TRACE_DEFINE(tag) gives a translation unit a clock64 record
+// [cta < 4][role slot < 4][step < 512][event < 8] and an extern "C" reader
+// jfa_trace_read_<tag>(host, n) that copies and clears it.
+#ifdef JFA_TRACE
+#define JFA_TRACE_N (4 * 4 * 512 * 8)
+#define JFA_TRACE_DEFINE(tag)                                                                 \
+    __device__ unsigned long long g_trace_##tag[JFA_TRACE_N];                                 \
+    extern "C" int jfa_trace_read_##tag(unsigned long long* host) {                          \
+        if (cudaMemcpyFromSymbol(host, g_trace_##tag, sizeof(g_trace_##tag)) != cudaSuccess) \
+            return -1;                                                                        \
+        static unsigned long long zero[JFA_TRACE_N];                                          \
+        return cudaMemcpyToSymbol(g_trace_##tag, zero, sizeof(zero)) == cudaSuccess ? JFA_TRACE_N : -1; \
+    }
+#define JFA_TRACE_EV(tag, slot, step, ev)                                                     \
+    do {                                                                                      \
+        if (blockIdx.x < 4 && (unsigned)(step) < 512u)                                       \
+            g_trace_##tag[((blockIdx.x * 4 + (slot)) * 512 + (step)) * 8 + (ev)] = clock64(); \
+    } while (0)
+#else
+#define JFA_TRACE_DEFINE(tag)
+#define JFA_TRACE_EV(tag, slot, step, ev) \
+    do {                                  \
+    } while (0)
+#endif
+
 namespace sm100 {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -274,6 +300,45 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Paired fp32 arithmetic (one instruction for two lanes of work, sm_100):
+// each is exactly two round-to-nearest fp32 operations.
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+    return r;
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t r) {
+    float2 a;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+    return a;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+    return bits_f2(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(d);
+}
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -28,11 +28,16 @@ bool tc_supported(const jfa_problem& p, int act, int backward) {
 
 namespace {
 struct Extra {
-    size_t dq_acc, qf, kf, vf, total;
+    size_t dq_acc, qf, kf, vf, bias4, total;
 };
+int bias4_stride(const jfa_problem& p) { return (p.relpos_len + 3) & ~3; }
 Extra extra_layout(const jfa_problem& p, int backward) {
     Extra e{};
     size_t off = 0;
+    if (p.bias_kind == JFA_BIAS_RELPOS) {
+        e.bias4 = off;
+        off = align256(off + sizeof(float) * 4 * (size_t)p.heads * bias4_stride(p));
+    }
     if (backward) {
         e.dq_acc = off;
         off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads * p.head_dim);
@@ -55,16 +60,48 @@ cudaError_t fake_quant(const jfa_problem& p, AttnArgs& a, char* ws, const Extra&
     a.v = vf;
     return e;
 }
+// out[(h * 4 + k) * stride + t] = log2(e) * table[h][min(t + k, len - 1)]
+__global__ void __launch_bounds__(256) tc_bias_prep(const float* __restrict__ tab, int len, int heads,
+                                                    int stride, float* __restrict__ out) {
+    const int64_t n = (int64_t)heads * 4 * stride;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i % stride);
+        const int hk = (int)(i / stride);
+        const int k = hk & 3, h = hk >> 2;
+        out[i] = tab[(int64_t)h * len + min(t + k, len - 1)] * 1.4426950408889634f;
+    }
+}
+
+cudaError_t prep_bias(const jfa_problem& p, AttnArgs& a, char* ws, const Extra& L, cudaStream_t st) {
+    if (p.bias_kind != JFA_BIAS_RELPOS) return cudaSuccess;
+    const int stride = bias4_stride(p);
+    float* out = reinterpret_cast<float*>(ws + L.bias4);
+    const int64_t n = (int64_t)p.heads * 4 * stride;
+    const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    prof_begin(st);
+    tc_bias_prep<<<blocks, 256, 0, st>>>(reinterpret_cast<const float*>(a.bias), p.relpos_len, p.heads,
+                                          stride, out);
+    prof_end(st, K_TC_BIAS_PREP);
+    a.bias4 = out;
+    a.bias4_stride = stride;
+    return cudaGetLastError();
+}
 }  // namespace
 
 // The backward keeps an fp32 dQ accumulator [total_q][heads][128]; MXFP8
-// adds the three dequantised operands.
+// adds the three dequantised operands; a relative-position bias adds its
+// four shifted, log2(e)-scaled copies.
 size_t tc_workspace_extra(const jfa_problem& p, int backward) {
     return extra_layout(p, backward).total;
 }
 
 cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, cudaStream_t st) {
     AttnArgs aa = a;
+    {
+        cudaError_t e = prep_bias(p, aa, reinterpret_cast<char*>(ws_extra), extra_layout(p, 0), st);
+        if (e != cudaSuccess) return e;
+    }
     if (p.dtype == JFA_MXFP8) {
         cudaError_t e = fake_quant(p, aa, reinterpret_cast<char*>(ws_extra), extra_layout(p, 0), st);
         if (e != cudaSuccess) return e;
@@ -80,6 +117,12 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
     AttnArgs aq = a, akv = kv;
     aq.dq_acc = reinterpret_cast<float*>(ws + L.dq_acc);
     akv.dq_acc = aq.dq_acc;
+    {
+        cudaError_t e = prep_bias(p, akv, ws, L, st);
+        if (e != cudaSuccess) return e;
+        aq.bias4 = akv.bias4;
+        aq.bias4_stride = akv.bias4_stride;
+    }
     if (p.dtype == JFA_MXFP8) {
         cudaError_t e = fake_quant(p, aq, ws, L, st);
         if (e != cudaSuccess) return e;

@@ -34,6 +34,8 @@ using namespace sm100;
 
 bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads);
 
+JFA_TRACE_DEFINE(bwd)
+
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
@@ -49,7 +51,7 @@ constexpr uint32_t kOffPT = kOffDO + kTile;
 constexpr uint32_t kOffDST = kOffPT + kTile;
 constexpr uint32_t kOffBar = kOffDST + kTile;  // 196608
 constexpr uint32_t kOffRow = kOffBar + 256;     // lse2[2][128], D[2][128] (double-buffered)
-constexpr uint32_t kOffTab = kOffRow + 2048;
+constexpr uint32_t kOffEnd = kOffRow + 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
@@ -76,7 +78,7 @@ struct BwdParams {
     CUtensorMap tm_do;
     CUtensorMap tm_dq;  // fp32 accumulator, boxes of 32 columns x 128 rows, 128B swizzle
     AttnArgs a;
-    int tab_cap;
+    int tab_cap;  // bias table entries that fit in shared memory
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
@@ -86,12 +88,6 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
 
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
 }
 
 __device__ __forceinline__ void named_sync_score() {
@@ -113,35 +109,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Stores the 32 values of chunk c4 (columns 32*c4 .. +31) of row r into a
-// K-major 128B-swizzled bf16 tile.
-__device__ __forceinline__ void store_chunk_bf16(uint8_t* tile, int r, int c4, const float (&v)[32]) {
-    uint8_t* row = tile + (c4 >> 1) * kBox + r * 128;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int ch = (c4 & 1) * 4 + u;
-        uint4 w;
-        w.x = pack_bf16(v[8 * u + 0], v[8 * u + 1]);
-        w.y = pack_bf16(v[8 * u + 2], v[8 * u + 3]);
-        w.z = pack_bf16(v[8 * u + 4], v[8 * u + 5]);
-        w.w = pack_bf16(v[8 * u + 6], v[8 * u + 7]);
-        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
-    }
-}
-
-// P = 2^(s - lse) and dS = P (dP - D) for 32 columns (compile-time column
-// index, so that exp2_mixed can place each element on its pipe).
-template <int v>
-__device__ __forceinline__ void softmax_chunk(uint32_t (&u)[16], uint32_t (&g)[16], const float* l2c,
-                                              const float* ddc) {
-    if constexpr (v < 16) {
-        const float pr = exp2_mixed<v>(__uint_as_float(u[v]) - l2c[v]);
-        u[v] = __float_as_uint(pr);
-        g[v] = __float_as_uint(pr * (__uint_as_float(g[v]) - ddc[v]));
-        softmax_chunk<v + 1>(u, g, l2c, ddc);
-    }
-}
-
 // Stores 16 fp32 values (bit patterns) as bf16: columns 16*c16 .. +15 of row r
 // of a K-major 128B-swizzled tile.
 __device__ __forceinline__ void store_half_chunk_bits(uint8_t* tile, int r, int c16, const uint32_t (&v)[16]) {
@@ -149,21 +116,6 @@ __device__ __forceinline__ void store_half_chunk_bits(uint8_t* tile, int r, int 
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         const int ch = (c16 & 3) * 2 + u;
-        uint4 w;
-        w.x = pack_bf16_p(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
-        w.y = pack_bf16_p(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
-        w.z = pack_bf16_p(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
-        w.w = pack_bf16_p(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
-        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
-    }
-}
-
-// Same as store_chunk_bf16 for 32 fp32 values held as bit patterns.
-__device__ __forceinline__ void store_chunk_bits(uint8_t* tile, int r, int c4, const uint32_t (&v)[32]) {
-    uint8_t* row = tile + (c4 >> 1) * kBox + r * 128;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int ch = (c4 & 1) * 4 + u;
         uint4 w;
         w.x = pack_bf16_p(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
         w.y = pack_bf16_p(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
@@ -193,7 +145,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     float* lse2_s = reinterpret_cast<float*>(smem + kOffRow);  // [2][128]
     float* dd_s = lse2_s + 256;                                 // [2][128]
-    float* tab = reinterpret_cast<float*>(smem + kOffTab);
 
     const int4 it = a.items[blockIdx.x];
     const int b = it.x, h = it.y, j0 = it.z * BN;
@@ -204,9 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     const int nt = nq > i_start ? (nq - i_start + BM - 1) / BM : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool softmax = SOFTMAX;
+    // relative-position bias of this CTA's (query, key) range, log2(e)-scaled:
+    // tab[t] = bias(i, j) for i - j = tab_lo + t, kept in shared memory when
+    // it fits
     const int tab_lo = i_start - j0 - (BN - 1);
     const int tab_len = nq - i_start + BN - 1;
     const bool tab_in_smem = BIAS == 1 && nt > 0 && tab_len <= P.tab_cap;
+    float* tab = reinterpret_cast<float*>(smem + kOffEnd);
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -230,12 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     }
     if (tab_in_smem) {
         const int C = (a.relpos_len - 1) >> 1;
-        const float* src = reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len;
-        for (int t = threadIdx.x; t < tab_len; t += kThreads) {
-            int r = tab_lo + t;
-            r = r < -C ? -C : (r > C ? C : r);
-            tab[t] = __ldg(src + r + C) * kLog2e;
-        }
+        const float* src = a.bias4 + (int64_t)h * 4 * a.bias4_stride;   // copy 0
+        for (int t = threadIdx.x; t < tab_len; t += kThreads)
+            tab[t] = __ldg(src + min(max(tab_lo + t, -C), C) + C);
     }
     tc_fence_before();
     __syncthreads();
@@ -263,11 +215,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             for (int t = 0; t < nt; ++t) {
                 const int z = q0 + i_start + t * BM;
                 if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
+                JFA_TRACE_EV(bwd, 0, t, 0);
                 mbar_arrive_expect_tx(&bars->q_full, kTile);
                 tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, h, z);
                 tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, z);
                 issued_q = t + 1;
                 if (t > 0 && !mbar_wait(&bars->do_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
+                JFA_TRACE_EV(bwd, 0, t, 1);
                 mbar_arrive_expect_tx(&bars->do_full, kTile);
                 tma_load_3d(smem + kOffDO, &P.tm_do, &bars->do_full, 0, h, z);
                 tma_load_3d(smem + kOffDO + kBox, &P.tm_do, &bars->do_full, 64, h, z);
@@ -295,18 +249,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.hdr);
             for (int t = 0; ok && t < nt; ++t) {
                 if (!mbar_wait(&bars->q_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwd, 1, t, 0);
                 if (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwd, 1, t, 1);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tS, kmajor_desc(kb, k), kmajor_desc(qb, k), idesc_nt, k > 0 ? 1u : 0u);
                 if (!mbar_wait(&bars->do_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwd, 1, t, 2);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tdP, kmajor_desc(vb, k), kmajor_desc(dob, k), idesc_nt, k > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full);
+                JFA_TRACE_EV(bwd, 1, t, 3);
                 if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwd, 1, t, 4);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)
@@ -322,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tS, mnmajor_desc(dsb, k), mnmajor_desc(kb, k), idesc_tn, k > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
+                JFA_TRACE_EV(bwd, 1, t, 5);
             }
             if (ok) mma_commit(&bars->fin);
             mma_commit(&bars->drain);
@@ -341,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const float sc = a.scale * kLog2e;
         const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
         const int C = (a.relpos_len - 1) >> 1;
-        const float* tab_g = reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len;
+        // log2(e)-scaled table (copy 0 of the four shifted copies)
+        const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)h * 4 * a.bias4_stride : nullptr;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_base = (BIAS == 2) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
         const bool leader = (warp == 2 && lane == 0);
@@ -366,7 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             }
             named_sync_score();
         }
+        const int tslot = (warp == 2 && lane == 0) ? 2 : ((warp == kThreads / 32 - 1 && lane == 0) ? 3 : -1);
+#define SC_EV(ev)                                     \
+    do {                                              \
+        if (tslot >= 0) JFA_TRACE_EV(bwd, tslot, t, ev); \
+    } while (0)
         for (int t = 0; t < nt; ++t) {
+            SC_EV(0);
             const int qb0 = i_start + t * BM;    // query index of the tile's row 0
             const int buf = t & 1;
             float nl2 = CUDART_INF_F, ndv = 0.f;
@@ -375,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // right after the named barrier, so every score warp runs the same
             // sequence of barriers
             mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr);
+            SC_EV(1);
             tc_fence_after();
             // key rows past the sequence end (neighbour data) must not reach dS K;
             // S^T = K Q^T of the first tile has completed, so K may be edited now
@@ -388,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 }
                 mbar_wait(&bars->stage_free, (t - 1) & 1, abort_flag, a.hdr);
             }
+            SC_EV(2);
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
             // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
             auto process = [&](uint32_t (&u)[16], uint32_t (&g)[16], int c16) {
@@ -399,16 +368,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     for (int v = 0; v < 16; ++v) u[v] = 0u, g[v] = 0u;
                     return;
                 }
-                if (BIAS == 1 && tab_in_smem) {
-                    const float* tb = tab + (qc0 - j - tab_lo);   // tb[v] = bias(qc0 + v, j)
+                float x[16];
+                const float2 sc2 = make_float2(sc, sc);
+                if (BIAS == 1) {
+                    float bb[16];
+                    if (tab_in_smem) {
+                        const float* tb = tab + (qc0 - j - tab_lo);   // tb[v] = bias(qc0 + v, j)
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, tb[v]));
-                } else if (BIAS == 1) {
+                        for (int v = 0; v < 16; ++v) bb[v] = tb[v];
+                    } else {
+                        const int s0 = qc0 - j + C;                   // table index of bias(qc0, j)
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        int rr = qc0 + v - j;
-                        rr = rr < -C ? -C : (rr > C ? C : rr);
-                        u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, __ldg(tab_g + rr + C) * kLog2e));
+                        for (int v = 0; v < 16; ++v) bb[v] = __ldg(tab4 + min(max(s0 + v, 0), 2 * C));
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 r2 = fma2(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])),
+                                               sc2, make_float2(bb[2 * e], bb[2 * e + 1]));
+                        x[2 * e] = r2.x, x[2 * e + 1] = r2.y;
                     }
                 } else if (BIAS == 2) {
 #pragma unroll
@@ -416,20 +393,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         const int qi = qc0 + v;
                         const float bv = (jvalid && qi < nq)
                             ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
-                        u[v] = __float_as_uint(fmaf(__uint_as_float(u[v]), sc, bv));
+                        x[v] = fmaf(__uint_as_float(u[v]), sc, bv);
                     }
                 } else {
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) u[v] = __float_as_uint(__uint_as_float(u[v]) * sc);
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 r2 = mul2(make_float2(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1])), sc2);
+                        x[2 * e] = r2.x, x[2 * e + 1] = r2.y;
+                    }
                 }
                 if (SOFTMAX) {
-                    const float* l2c = lse2_s + buf * 128 + c16 * 16;
-                    const float* ddc = dd_s + buf * 128 + c16 * 16;
-                    softmax_chunk<0>(u, g, l2c, ddc);
+                    // P = 2^(x - lse), dS = P (dP - D); lse and D of the 16 query
+                    // columns are broadcast reads of the staged row statistics
+                    const float4* l4 = reinterpret_cast<const float4*>(lse2_s + buf * 128 + c16 * 16);
+                    const float4* d4 = reinterpret_cast<const float4*>(dd_s + buf * 128 + c16 * 16);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 L = l4[q], D = d4[q];
+                        const float2 y0 = sub2(make_float2(x[4 * q], x[4 * q + 1]), make_float2(L.x, L.y));
+                        const float2 y1 = sub2(make_float2(x[4 * q + 2], x[4 * q + 3]), make_float2(L.z, L.w));
+                        const float2 p0 = make_float2(ex2(y0.x), ex2(y0.y));
+                        const float2 p1 = make_float2(ex2(y1.x), ex2(y1.y));
+                        const float2 t0 = sub2(make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])),
+                                               make_float2(D.x, D.y));
+                        const float2 t1 = sub2(make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])),
+                                               make_float2(D.z, D.w));
+                        const float2 d0 = mul2(p0, t0), d1 = mul2(p1, t1);
+                        u[4 * q] = __float_as_uint(p0.x), u[4 * q + 1] = __float_as_uint(p0.y);
+                        u[4 * q + 2] = __float_as_uint(p1.x), u[4 * q + 3] = __float_as_uint(p1.y);
+                        g[4 * q] = __float_as_uint(d0.x), g[4 * q + 1] = __float_as_uint(d0.y);
+                        g[4 * q + 2] = __float_as_uint(d1.x), g[4 * q + 3] = __float_as_uint(d1.y);
+                    }
                 } else {
 #pragma unroll
                     for (int v = 0; v < 16; ++v) {
-                        const float sn = __uint_as_float(u[v]) * (1.0f / kLog2e);
+                        const float sn = x[v] * (1.0f / kLog2e);
                         u[v] = __float_as_uint(act_f(a.act, sn) * inv_n);
                         g[v] = __float_as_uint(__uint_as_float(g[v]) * act_grad_f(a.act, sn) * inv_n);
                     }
@@ -460,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 if (grp == 0) zero_row(smem + kOffQ, r);
                 else if (grp == 1) zero_row(smem + kOffDO, r);
             }
+            SC_EV(3);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -468,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // 32-column chunks (128B swizzle) over the P^T / dS^T buffers, which
             // the finished MMAs no longer read
             mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr);
+            SC_EV(4);
             tc_fence_after();
             const bool qvalid = qb0 + r < nq;
             uint32_t u2[32];
@@ -476,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dq_empty);  // TMEM columns free for S^T of t+1
+            SC_EV(5);
             {
                 uint8_t* row = smem + kOffPT + grp * (128 * 128) + r * 128;
 #pragma unroll
@@ -490,7 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 dd_s[(buf ^ 1) * 128 + r] = ndv;
             }
             fence_proxy_async_smem();
+            SC_EV(6);
             named_sync_score();
+            SC_EV(7);
             if (*abort_flag) { ok = false; break; }
             if (leader) {
                 const int z = q0 + qb0;
@@ -500,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 bulk_commit();
             }
         }
+#undef SC_EV
         if (leader) bulk_wait_all();
         // ------------------------------------------------------ epilogue
         if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort_flag, a.hdr));
@@ -586,7 +590,6 @@ __global__ void __launch_bounds__(256) tc_bwd_dq_finalize(const float* __restric
 
 }  // namespace
 
-constexpr int kSmemLimitBwd = 232448;
 
 // fp32 accumulator [rows][heads][128] as a 3-D tensor (d, head, row); boxes of
 // 32 d x 1 head x 128 rows (128 bytes inner) with the 128-byte swizzle.
@@ -613,6 +616,8 @@ static bool make_tmap_dq_acc(CUtensorMap* map, void* base, int64_t rows, int hea
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr int kSmemLimit = 232448;  // opt-in shared memory per block
+
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                                cudaStream_t st) {
     const int64_t rows = p.total_q * p.heads;
@@ -631,12 +636,12 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
         return cudaErrorInvalidValue;
     if (!make_tmap_dq_acc(&P.tm_dq, a.dq_acc, p.total_q, p.heads)) return cudaErrorInvalidValue;
     P.a = kv;
-    const int base = 1024 + (int)kOffTab;
+    const int base = 1024 + (int)kOffEnd;
     int tab_need = (p.bias_kind == JFA_BIAS_RELPOS) ? (p.max_q_len + BN - 1) : 0;
     int smem = base + 4 * tab_need;
-    if (smem > kSmemLimitBwd) {
-        tab_need = 0;
-        smem = base;
+    if (smem > kSmemLimit) {
+        tab_need = (kSmemLimit - base) / 4;
+        smem = kSmemLimit;
     }
     P.tab_cap = tab_need;
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
@@ -645,7 +650,7 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
     if (bias == 0) kern = sm ? tc_bwd_kernel<0, true> : tc_bwd_kernel<0, false>;
     else if (bias == 1) kern = sm ? tc_bwd_kernel<1, true> : tc_bwd_kernel<1, false>;
     else kern = sm ? tc_bwd_kernel<2, true> : tc_bwd_kernel<2, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimitBwd);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int64_t grid = pairs_bound(p.batch, p.max_kv_len, p.total_kv, BN) * p.heads;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;

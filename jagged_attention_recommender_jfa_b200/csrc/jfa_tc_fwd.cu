@@ -34,6 +34,8 @@ namespace jfa {
 
 using namespace sm100;
 
+JFA_TRACE_DEFINE(fwd)
+
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
@@ -196,11 +198,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     const uint32_t par = ((g >> 1) - 1) & 1;
                     const int z = w.k0 + j * BN;
                     if (g >= 2 && !mbar_wait(&bars->k_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(fwd, 0, g, 0);
                     mbar_arrive_expect_tx(&bars->k_full[s], kTile);
                     tma_load_3d(smem + kOffK + s * kTile, &P.tm_k, &bars->k_full[s], 0, w.h, z);
                     tma_load_3d(smem + kOffK + s * kTile + kBox, &P.tm_k, &bars->k_full[s], 64, w.h, z);
                     ++kq;
                     if (g >= 2 && !mbar_wait(&bars->v_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(fwd, 0, g, 1);
                     mbar_arrive_expect_tx(&bars->v_full[s], kTile);
                     tma_load_3d(smem + kOffV + s * kTile, &P.tm_v, &bars->v_full[s], 0, w.h, z);
                     tma_load_3d(smem + kOffV + s * kTile + kBox, &P.tm_v, &bars->v_full[s], 64, w.h, z);
@@ -229,12 +233,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             auto issue_qk = [&](int gg, int n_left_after) -> bool {
                 const int s = gg & 1;
                 if (!mbar_wait(&bars->k_full[s], (gg >> 1) & 1, abort_flag, a.hdr)) return false;
+                JFA_TRACE_EV(fwd, 1, gg, 0);
                 tc_fence_after();
                 const uint32_t kb = sbase + kOffK + s * kTile;
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tmem + s * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full[s]);
+                JFA_TRACE_EV(fwd, 1, gg, 1);
                 mma_commit(&bars->k_empty[s]);
                 if (n_left_after == 0) mma_commit(&bars->q_free);  // last score MMA of the item
                 return true;
@@ -255,7 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 for (int t = 0; ok && t < n; ++t, ++g) {
                     const int s = g & 1;
                     if (!mbar_wait(&bars->p_full, g & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(fwd, 1, g, 2);
                     if (!mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(fwd, 1, g, 3);
                     tc_fence_after();
                     const uint32_t vb = sbase + kOffV + s * kTile;
                     const uint32_t tP = tmem + s * 128;  // P (bf16 pairs) over columns 0..63 of its S
@@ -265,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                                     (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&bars->v_empty[s]);
                     mma_commit(&bars->pv_done);
+                    JFA_TRACE_EV(fwd, 1, g, 4);
                     if (t + 2 < n) ok = issue_qk(g + 2, n - 1 - (t + 2));
                 }
             }
@@ -283,6 +292,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         const int C = (a.relpos_len - 1) >> 1;
         int g = 0, m = 0;
         bool ok = true;
+        const int tslot = (warp == 2 && lane == 0) ? 2 : ((warp == kThreads / 32 - 1 && lane == 0) ? 3 : -1);
+#define SM_EV(ev)                                     \
+    do {                                              \
+        if (tslot >= 0) JFA_TRACE_EV(fwd, tslot, g, ev); \
+    } while (0)
         // Every softmax warp runs the same sequence of named barriers: a failed
         // (timed-out) wait only sets the CTA's abort flag, and the loops are left
         // right after a barrier, where all warps read the same flag.
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             const int shift = w.nkv - w.nq;        // causal: key j visible iff j <= i + shift
             const float inv_n = w.nkv > 0 ? 1.0f / (float)w.nkv : 0.f;
             const int jmax_vis = a.causal ? min(w.nkv - 1, i + shift) : w.nkv - 1;
-            const float* tab_g = reinterpret_cast<const float*>(a.bias) + (int64_t)w.h * a.relpos_len;
+            const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)w.h * 4 * a.bias4_stride : nullptr;
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
                                           ? a.dense_off[w.b] + ((int64_t)w.h * w.nq + i) * w.nkv : 0;
@@ -302,7 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             float m_used = -CUDART_INF_F, l = 0.f;   // l: this group's partial sum
             for (int j = 0; j < w.n_tiles; ++j, ++g) {
                 const int s = g & 1;
+                SM_EV(0);
                 mbar_wait(&bars->s_full[s], (g >> 1) & 1, abort_flag, a.hdr);
+                SM_EV(1);
                 tc_fence_after();
                 const int jc = j * BN + c0;          // key index of this group's column 0
                 float x[CW];
@@ -315,20 +331,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
                 const int nvis = i < w.nq ? max(0, min(CW, jmax_vis - jc + 1)) : 0;  // visible: [0, nvis)
                 if (BIAS == 1) {
-                    // bias(i, jc + c) = table[clamp(i - jc - c) + C]; within a sequence
-                    // |i - j| <= C, so only tiles reaching past the rows need the clamp
-                    const int hi = i - jc, lo = i - jc - (CW - 1);
-                    if (lo >= -C && hi <= C) {
-                        const float* tb = tab_g + (hi + C);   // tb[-c]
+                    // bias(i, jc + c) = table[i - jc - c + C] (log2(e)-scaled copy);
+                    // within a sequence |i - j| <= C, so only tiles past the rows
+                    // need the clamp
+                    const int hi = i - jc + C;
+                    const float2 sc2 = make_float2(sc, sc);
+                    float bb[CW];
+                    if (hi - (CW - 1) >= 0 && hi <= 2 * C) {
+                        const float* tb = tab4 + hi;   // tb[-c]
 #pragma unroll
-                        for (int c = 0; c < CW; ++c) x[c] = fmaf(x[c], sc, __ldg(tb - c) * kLog2e);
+                        for (int c = 0; c < CW; ++c) bb[c] = __ldg(tb - c);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < CW; ++c) {
-                            int d_ = hi - c;
-                            d_ = d_ < -C ? -C : (d_ > C ? C : d_);
-                            x[c] = fmaf(x[c], sc, __ldg(tab_g + d_ + C) * kLog2e);
-                        }
+                        for (int c = 0; c < CW; ++c) bb[c] = __ldg(tab4 + min(max(hi - c, 0), 2 * C));
+                    }
+#pragma unroll
+                    for (int c = 0; c < CW; c += 2) {
+                        const float2 r2 = fma2(make_float2(x[c], x[c + 1]), sc2, make_float2(bb[c], bb[c + 1]));
+                        x[c] = r2.x, x[c + 1] = r2.y;
                     }
                 } else if (BIAS == 2) {
 #pragma unroll
@@ -336,7 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         x[c] = fmaf(x[c], sc, c < nvis ? __bfloat162float(dense[dense_row + jc + c]) * kLog2e : 0.f);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < CW; ++c) x[c] *= sc;
+                    for (int c = 0; c < CW; c += 2) {
+                        const float2 r2 = mul2(make_float2(x[c], x[c + 1]), make_float2(sc, sc));
+                        x[c] = r2.x, x[c + 1] = r2.y;
+                    }
                 }
                 const bool masked_tile = __any_sync(0xffffffffu, nvis < CW);
                 if (masked_tile) {
@@ -346,15 +369,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 float alpha = 1.f;
                 bool rescale = false;
                 if (softmax) {
-                    float pm8[8];
+                    float pm4[4];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) pm8[t] = x[t];
+                    for (int t = 0; t < 4; ++t) pm4[t] = fmaxf(x[2 * t], x[2 * t + 1]);
 #pragma unroll
-                    for (int c = 8; c < CW; ++c) pm8[c & 7] = fmaxf(pm8[c & 7], x[c]);
-                    const float pm = fmaxf(fmaxf(fmaxf(pm8[0], pm8[1]), fmaxf(pm8[2], pm8[3])),
-                                           fmaxf(fmaxf(pm8[4], pm8[5]), fmaxf(pm8[6], pm8[7])));
+                    for (int c = 8; c < CW; c += 2) pm4[(c >> 1) & 3] = max3(pm4[(c >> 1) & 3], x[c], x[c + 1]);
+                    const float pm = max3(pm4[0], pm4[1], fmaxf(pm4[2], pm4[3]));
                     red[(s * NG + grp) * 128 + r_] = pm;
+                    SM_EV(2);
                     named_sync_softmax();
+                    SM_EV(3);
                     if (*abort_flag) { ok = false; break; }
                     float tmax = pm;
 #pragma unroll
@@ -389,17 +413,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     tmem_wait_st();
                     l *= alpha;
                 }
+                SM_EV(4);
                 if (softmax) {
                     // ex2(-inf) = 0 masks the invisible columns; a row with no visible
                     // key yet uses reference 0 so that -inf - ref stays -inf
                     const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
-                    float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float2 ref2 = make_float2(ref, ref);
+                    float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                    make_float2(0.f, 0.f)};
 #pragma unroll
-                    for (int c = 0; c < CW; ++c) {
-                        x[c] = ex2(x[c] - ref);
-                        ps8[c & 7] += x[c];
+                    for (int c = 0; c < CW; c += 2) {
+                        const float2 y = sub2(make_float2(x[c], x[c + 1]), ref2);
+                        x[c] = ex2(y.x);
+                        x[c + 1] = ex2(y.y);
+                        ps[(c >> 1) & 3] = add2(ps[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
                     }
-                    l += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+                    const float2 s01 = add2(ps[0], ps[1]), s23 = add2(ps[2], ps[3]);
+                    const float2 s4 = add2(s01, s23);
+                    l += s4.x + s4.y;
                     if (QP) mx::fake_quant32(x);  // the group's 32 keys are one MX block
                 } else {
 #pragma unroll
@@ -437,12 +468,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->p_full);
+                SM_EV(5);
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue
             if (w.n_tiles > 0) mbar_wait(&bars->pv_done, (g - 1) & 1, abort_flag, a.hdr);
+            SM_EV(6);
             lred[((m & 1) * NG + grp) * 128 + r_] = l;
             named_sync_softmax();
+            SM_EV(7);
             if (*abort_flag) { ok = false; break; }
             float l_row = 0.f;
 #pragma unroll
@@ -477,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
             }
         }
+#undef SM_EV
     }
     tc_fence_before();
     __syncthreads();
