@@ -14,7 +14,7 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int causal, int backward, int tile, WsHeader* hdr, int64_t* dense_off,
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
-                           cudaStream_t stream);
+                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream);
 cudaError_t simt_forward(const AttnArgs& a, int head_dim, bool bf16, int grid, cudaStream_t st);
 cudaError_t simt_backward(const AttnArgs& a, const AttnArgs& kv_args, int head_dim, bool bf16,
                           int grid_q, int grid_kv, int64_t rows, cudaStream_t st);
@@ -194,7 +194,7 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
                                    reinterpret_cast<int2*>(ws + L.pair_bt),
                                    reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
                                    reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
-                                   &hdr->pair_count, 1, st);
+                                   &hdr->pair_count, 1, nullptr, nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     AttnArgs a{};
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
@@ -248,13 +248,14 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
                                    reinterpret_cast<int2*>(ws + L.pair_bt),
                                    reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
                                    reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
-                                   &hdr->pair_count, 1, st);
+                                   &hdr->pair_count, 1, nullptr, nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     e = build_schedule(p, q_offsets, kv_offsets, causal, 1, ktile, hdr, nullptr,
                        reinterpret_cast<int2*>(ws + L.kv_pair_bt),
                        reinterpret_cast<int64_t*>(ws + L.kv_pair_cost), L.pairs_max_kv,
                        reinterpret_cast<int4*>(ws + L.kv_items), &hdr->kv_item_count,
-                       &hdr->kv_pair_count, 0, st);
+                       &hdr->kv_pair_count, 0, reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp),
+                       reinterpret_cast<int64_t*>(ws + L.kv_seq_start), st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     AttnArgs a{};
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
@@ -323,7 +324,9 @@ jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,
                                    reinterpret_cast<int64_t*>(ws + (backward ? L.kv_pair_cost : L.pair_cost)),
                                    backward ? L.pairs_max_kv : L.pairs_max_q,
                                    reinterpret_cast<int4*>(items), count,
-                                   backward ? &hdr->kv_pair_count : &hdr->pair_count, 1, st);
+                                   backward ? &hdr->kv_pair_count : &hdr->pair_count, 1,
+                                   backward ? reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp) : nullptr,
+                                   backward ? reinterpret_cast<int64_t*>(ws + L.kv_seq_start) : nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     return JFA_OK;
 }

@@ -43,6 +43,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct WsLayout {
     size_t dense_off, pair_bt, pair_cost, items;           // forward schedule
     size_t kv_pair_bt, kv_pair_cost, kv_items;             // backward schedule
+    size_t kv_seq_tmp, kv_seq_start;                       // its sequence order
     size_t dterm, dq_acc;                                  // backward rows
     size_t total;
     int64_t pairs_max_q, pairs_max_kv;
@@ -68,6 +69,8 @@ inline WsLayout ws_layout(const jfa_problem& p, bool backward, bool need_dq_acc)
         L.kv_pair_bt = off;   off = align256(off + sizeof(int32_t) * 2 * (size_t)L.pairs_max_kv);
         L.kv_pair_cost = off; off = align256(off + sizeof(int64_t) * (size_t)L.pairs_max_kv);
         L.kv_items = off;     off = align256(off + sizeof(int4) * (size_t)L.pairs_max_kv * p.heads);
+        L.kv_seq_tmp = off;   off = align256(off + sizeof(int64_t) * (size_t)p.batch);
+        L.kv_seq_start = off; off = align256(off + sizeof(int64_t) * (size_t)p.batch);
         L.dterm = off;        off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads);
         if (need_dq_acc) {
             L.dq_acc = off;

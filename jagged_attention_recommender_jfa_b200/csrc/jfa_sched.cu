@@ -3,11 +3,20 @@
 // Removing padding leaves short and long samples finishing at different times,
 // so tile scheduling becomes the exposed bottleneck ("Meta GEM Training
 // Efficiency: Why LLM-Scale Recommenders Need a Different Stack", section
-// "Bottleneck move 1: dense-sequence kernels to jagged execution").  The
-// schedule lists every (sequence, head, tile) work item longest-first
-// (cost = (query, key) pairs the tile computes; ties by sequence, tile, head
-// ascending), so that a grid or a persistent queue that takes items in order
-// runs the long causal tiles first and fills the tail with short ones.
+// "Bottleneck move 1: dense-sequence kernels to jagged execution").
+//
+// Query-tile schedule (forward): every (sequence, head, tile) work item
+// longest-first (cost = (query, key) pairs the tile computes; ties by
+// sequence, tile, head ascending), so that a grid or a persistent queue that
+// takes items in order runs the long causal tiles first and fills the tail
+// with short ones.
+//
+// Key-tile schedule (backward): the items of one (sequence, head) are kept
+// together, so that the key tiles that read the same query / dO tiles and add
+// into the same dQ rows run at the same time and share them through L2.
+// Sequences longest-first (cost = the sequence's (query, key) pairs; ties by
+// sequence), then heads ascending, then key tiles ascending (for causal
+// attention the first key tile is the longest).
 //
 // Two kernels:
 //   sched_prepare  one CTA: validates the offsets, enumerates the
@@ -52,7 +61,8 @@ __global__ void __launch_bounds__(kPrepThreads)
 sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_off, int B, int H,
               int max_q, int max_kv, int64_t total_q, int64_t total_kv, int causal, int backward,
               int tile, int64_t pairs_cap, int want_dense, WsHeader* hdr, int64_t* dense_off,
-              int2* pair_bt, int64_t* pair_cost, int32_t* pair_count_out, int reset_err) {
+              int2* pair_bt, int64_t* pair_cost, int32_t* pair_count_out, int reset_err,
+              int64_t* seq_tmp, int64_t* seq_start) {
     __shared__ int s_bad;
     __shared__ int64_t s_scan[kPrepThreads];
     __shared__ int64_t s_dscan[kPrepThreads];
@@ -132,6 +142,48 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
         pair_cost[p] = backward ? key_tile_cost(lo, hi, nq, nkv, causal)
                                 : query_tile_cost(lo, hi, nq, nkv, causal);
     }
+    if (seq_start == nullptr) return;
+    // 4. sequence order of the grouped (key-tile) schedule: seq_start[b] =
+    //    tiles of the sequences ranked before b (cost descending, then b)
+    for (int b = tid; b < B; b += kPrepThreads) {
+        const int nq = q_off[b + 1] - q_off[b], nkv = kv_off[b + 1] - kv_off[b];
+        seq_tmp[b] = key_tile_cost(0, nkv, nq, nkv, causal);
+    }
+    __syncthreads();
+    for (int b = tid; b < B; b += kPrepThreads) {
+        const int64_t mine = seq_tmp[b];
+        int64_t rank = 0;
+        for (int o = 0; o < B; ++o) {
+            const int64_t c = seq_tmp[o];
+            rank += (c > mine) | ((c == mine) & (o < b));
+        }
+        seq_start[b] = rank;
+    }
+    __syncthreads();
+    for (int b = tid; b < B; b += kPrepThreads) {
+        const int rows = backward ? kv_off[b + 1] - kv_off[b] : q_off[b + 1] - q_off[b];
+        seq_tmp[seq_start[b]] = (rows + tile - 1) / tile;
+    }
+    __syncthreads();
+    carry = 0;   // exclusive scan of the tile counts in rank order
+    for (int base = 0; base < B; base += kPrepThreads) {
+        const int i = base + tid;
+        const int64_t v = i < B ? seq_tmp[i] : 0;
+        s_scan[tid] = v;
+        __syncthreads();
+        for (int off = 1; off < kPrepThreads; off <<= 1) {
+            int64_t x = tid >= off ? s_scan[tid - off] : 0;
+            __syncthreads();
+            s_scan[tid] += x;
+            __syncthreads();
+        }
+        if (i < B) seq_tmp[i] = carry + s_scan[tid] - v;
+        const int64_t chunk_total = s_scan[kPrepThreads - 1];
+        __syncthreads();
+        carry += chunk_total;
+    }
+    __syncthreads();
+    for (int b = tid; b < B; b += kPrepThreads) seq_start[b] = seq_tmp[seq_start[b]];
 }
 
 constexpr int kRankThreads = 256;
@@ -140,12 +192,24 @@ constexpr int kRankChunk = 2048;
 __global__ void __launch_bounds__(kRankThreads)
 sched_rank(const int2* __restrict__ pair_bt, const int64_t* __restrict__ pair_cost,
            const int32_t* __restrict__ pair_count, int H, int4* __restrict__ items,
-           int32_t* __restrict__ item_count) {
+           int32_t* __restrict__ item_count, const int64_t* __restrict__ seq_start,
+           const int32_t* __restrict__ rows_off, int tile) {
     __shared__ int64_t s_cost[kRankChunk];
     const int n = *pair_count;
     const int p = blockIdx.x * kRankThreads + threadIdx.x;
     if (p == 0) *item_count = n * H;
     if (blockIdx.x * kRankThreads >= n) return;
+    if (seq_start != nullptr) {  // grouped: (sequence, head) blocks of consecutive tiles
+        if (p < n) {
+            const int2 bt = pair_bt[p];
+            const int64_t mine = pair_cost[p];
+            const int cost32 = mine > 0x7fffffff ? 0x7fffffff : (int)mine;
+            const int nt = (rows_off[bt.x + 1] - rows_off[bt.x] + tile - 1) / tile;
+            const int64_t first = seq_start[bt.x] * H;
+            for (int h = 0; h < H; ++h) items[first + (int64_t)h * nt + bt.y] = make_int4(bt.x, h, bt.y, cost32);
+        }
+        return;
+    }
     const int64_t mine = p < n ? pair_cost[p] : 0;
     int rank = 0;
     for (int base = 0; base < n; base += kRankChunk) {
@@ -174,13 +238,13 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int causal, int backward, int tile, WsHeader* hdr, int64_t* dense_off,
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
-                           cudaStream_t stream) {
+                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream) {
     int want_dense = (pb.bias_kind == JFA_BIAS_DENSE_JAGGED && dense_off != nullptr) ? 1 : 0;
     prof_begin(stream);
     sched_prepare<<<1, kPrepThreads, 0, stream>>>(
         q_off, kv_off, pb.batch, pb.heads, pb.max_q_len, pb.max_kv_len, pb.total_q, pb.total_kv,
         causal, backward, tile, pairs_cap, want_dense, hdr, dense_off, pair_bt, pair_cost,
-        pair_count, reset_err);
+        pair_count, reset_err, seq_tmp, seq_start);
     prof_end(stream, K_SCHED_PREPARE);
     int64_t bound = pairs_bound(pb.batch, backward ? pb.max_kv_len : pb.max_q_len,
                                 backward ? pb.total_kv : pb.total_q, tile);
@@ -189,7 +253,8 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
     if (grid < 1) grid = 1;
     prof_begin(stream);
     sched_rank<<<grid, kRankThreads, 0, stream>>>(pair_bt, pair_cost, pair_count, pb.heads, items,
-                                                  item_count);
+                                                  item_count, seq_start, backward ? kv_off : q_off,
+                                                  tile);
     prof_end(stream, K_SCHED_RANK);
     return cudaGetLastError();
 }

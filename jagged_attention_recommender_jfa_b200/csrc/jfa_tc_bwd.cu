@@ -7,23 +7,32 @@
 //   tc_bwd_pre       D[t,h] = sum_d dO*O (softmax) with a warp-shuffle row
 //                    reduction; zeroes the fp32 dQ accumulator rows.
 //   tc_bwd_kernel    one CTA per (sequence, head, 128-key tile) work item of
-//                    the longest-first key-tile schedule.  K and V of the tile
-//                    stay in shared memory; the query tiles that can see the
-//                    keys stream through:
+//                    the key-tile schedule.  K and V of the tile stay in
+//                    shared memory; the query tiles that can see the keys
+//                    stream through (Q single-, dO double-buffered):
 //                      S^T  = K Q^T,  dP^T = V dO^T           (TMEM, fp32)
 //                      P^T  = exp2(S^T - LSE), dS^T = P^T (dP^T - D)
 //                             (or GDPA: act(S)/n_kv, dP act'(S)/n_kv)
-//                      dV  += P^T dO,  dK += dS^T Q             (TMEM)
-//                      dQ_t = dS K  -> staged in shared memory (fp32,
-//                             128B-swizzled 32-column chunks) and added to
-//                             the fp32 accumulator by TMA reduce-add
+//                             P^T (bf16) back to TMEM over S^T, dS^T (bf16)
+//                             to shared memory
+//                      dK  += dS^T Q                         (TMEM)
+//                      dQ^T = K^T dS^T over the dP^T columns, read out by
+//                             the score warps and added to the fp32
+//                             accumulator with coalesced reductions (a warp
+//                             covers 32 consecutive d of one query row)
+//                      dV  += P^T dO    (A operand from TMEM)
+//                    The tensor core runs dK, dQ^T, dV of tile t and then
+//                    S^T, dP^T of tile t+1 back to back: Q(t+1) loads while
+//                    dQ^T and dV run, dO(t+1) was loaded a tile earlier, and
+//                    dP^T(t+1) waits only for the read-out of dQ^T(t).
 //   tc_bwd_dq_finalize  dQ = bf16(scale * accumulator).
 //
 // Warp roles: warp 0 TMA, warp 1 MMA, warps 2..17 score warps in four groups
-// of four; a thread owns one key row (or, for dQ, one query row) and one
-// 32-column chunk of it.  The backward needs no row reduction (LSE and D are
-// given), so the chunks never talk.
-// TMEM columns: dV [0,128), dK [128,256), S^T and dQ_t [256,384), dP^T [384,512).
+// of four; a thread owns one key row (or, for dQ^T, one d row) and one
+// 32-column (query) chunk of it.  The backward needs no row reduction (LSE
+// and D are given), so the chunks never talk.
+// TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384),
+// dP^T / dQ^T [384,512).
 #include <math_constants.h>
 
 #include "jfa_sm100.cuh"
@@ -46,37 +55,35 @@ constexpr uint32_t kTile = 2 * kBox;
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTile;
 constexpr uint32_t kOffQ = kOffV + kTile;
-constexpr uint32_t kOffDO = kOffQ + kTile;
-constexpr uint32_t kOffPT = kOffDO + kTile;
-constexpr uint32_t kOffDST = kOffPT + kTile;
-constexpr uint32_t kOffBar = kOffDST + kTile;  // 196608
-constexpr uint32_t kOffRow = kOffBar + 256;     // lse2[2][128], D[2][128] (double-buffered)
+constexpr uint32_t kOffDO = kOffQ + kTile;        // two buffers
+constexpr uint32_t kOffDST = kOffDO + 2 * kTile;
+constexpr uint32_t kOffBar = kOffDST + kTile;     // 196608
+constexpr uint32_t kOffRow = kOffBar + 256;       // lse2[2][128], D[2][128] (double-buffered)
 constexpr uint32_t kOffEnd = kOffRow + 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
     uint64_t kv_full;
-    uint64_t q_full;
-    uint64_t q_empty;
-    uint64_t do_full;
-    uint64_t do_empty;
+    uint64_t q_full, q_empty;
+    uint64_t do_full[2], do_empty[2];
     uint64_t s_full;
-    uint64_t ds_full;
+    uint64_t ds_full;       // 16 score warps
     uint64_t dq_full;
-    uint64_t dq_empty;
-    uint64_t stage_free;
+    uint64_t dq_empty;      // 16 score warps
+    uint64_t rows_full[2];  // LSE / D of a query tile staged (4 warps of group 0)
+    uint64_t rows_free[2];  // ... and read by every score warp (16)
     uint64_t fin;
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 struct BwdParams {
     CUtensorMap tm_q;
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     CUtensorMap tm_do;
-    CUtensorMap tm_dq;  // fp32 accumulator, boxes of 32 columns x 128 rows, 128B swizzle
     AttnArgs a;
     int tab_cap;  // bias table entries that fit in shared memory
 };
@@ -89,25 +96,6 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
 }
-
-__device__ __forceinline__ void named_sync_score() {
-    asm volatile("bar.sync 1, %0;" ::"n"(NG * 128) : "memory");
-}
-
-// TMA reduce-add of a shared-memory tile into global memory (no multicast).
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x,
-                                                  int y, int z) {
-    asm volatile(
-        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
-        " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
-        : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Stores 16 fp32 values (bit patterns) as bf16: columns 16*c16 .. +15 of row r
 // of a K-major 128B-swizzled tile.
@@ -167,13 +155,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
-        mbar_init(&bars->do_full, 1);
-        mbar_init(&bars->do_empty, 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&bars->do_full[s2], 1);
+            mbar_init(&bars->do_empty[s2], 1);
+            mbar_init(&bars->rows_full[s2], 4);
+            mbar_init(&bars->rows_free[s2], NG * 4);
+        }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->ds_full, NG * 4);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, NG * 4);
-        mbar_init(&bars->stage_free, 1);
         mbar_init(&bars->fin, 1);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -198,44 +189,58 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA
+        // Q(t+1) is loaded once dK += dS^T Q(t) has retired; dO(t+2) into
+        // the buffer of dO(t) once dV += P^T dO(t) has
         if (lane == 0 && nt > 0) {
             tma_prefetch_desc(&P.tm_q);
             tma_prefetch_desc(&P.tm_k);
             tma_prefetch_desc(&P.tm_v);
             tma_prefetch_desc(&P.tm_do);
-            tma_prefetch_desc(&P.tm_dq);
             mbar_arrive_expect_tx(&bars->kv_full, 2 * kTile);
             tma_load_3d(smem + kOffK, &P.tm_k, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, h, k0 + j0);
             tma_load_3d(smem + kOffV, &P.tm_v, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->kv_full, 64, h, k0 + j0);
-            // Q of tile t+1 is loaded as soon as dK += dS^T Q of tile t has retired,
-            // dO as soon as dV += P^T dO has (the MMAs of a tile run dK, dV, dQ)
-            int issued_q = 0, issued_do = 0;
-            for (int t = 0; t < nt; ++t) {
+            auto load_q = [&](int t) {
                 const int z = q0 + i_start + t * BM;
-                if (t > 0 && !mbar_wait(&bars->q_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
-                JFA_TRACE_EV(bwd, 0, t, 0);
                 mbar_arrive_expect_tx(&bars->q_full, kTile);
                 tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, h, z);
                 tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, z);
-                issued_q = t + 1;
-                if (t > 0 && !mbar_wait(&bars->do_empty, (t - 1) & 1, abort_flag, a.hdr)) break;
-                JFA_TRACE_EV(bwd, 0, t, 1);
-                mbar_arrive_expect_tx(&bars->do_full, kTile);
-                tma_load_3d(smem + kOffDO, &P.tm_do, &bars->do_full, 0, h, z);
-                tma_load_3d(smem + kOffDO + kBox, &P.tm_do, &bars->do_full, 64, h, z);
-                issued_do = t + 1;
-                if (t + 1 < nt) {  // warm L2 for the next query tile (single-buffered)
-                    tma_prefetch_l2_3d(&P.tm_q, 0, h, z + BM);
-                    tma_prefetch_l2_3d(&P.tm_q, 64, h, z + BM);
-                    tma_prefetch_l2_3d(&P.tm_do, 0, h, z + BM);
-                    tma_prefetch_l2_3d(&P.tm_do, 64, h, z + BM);
+            };
+            auto load_do = [&](int t) {
+                const int z = q0 + i_start + t * BM;
+                uint8_t* dst = smem + kOffDO + (t & 1) * kTile;
+                mbar_arrive_expect_tx(&bars->do_full[t & 1], kTile);
+                tma_load_3d(dst, &P.tm_do, &bars->do_full[t & 1], 0, h, z);
+                tma_load_3d(dst + kBox, &P.tm_do, &bars->do_full[t & 1], 64, h, z);
+            };
+            load_q(0);
+            load_do(0);
+            if (nt > 1) load_do(1);
+            int issued_q = 1, issued_do = nt > 1 ? 2 : 1;
+            for (int t = 0; t + 1 < nt; ++t) {
+                if (!mbar_wait(&bars->q_empty, t & 1, abort_flag, a.hdr)) break;
+                JFA_TRACE_EV(bwd, 0, t + 1, 0);
+                load_q(t + 1);
+                issued_q = t + 2;
+                if (t + 2 < nt) {
+                    tma_prefetch_l2_3d(&P.tm_q, 0, h, q0 + i_start + (t + 2) * BM);
+                    tma_prefetch_l2_3d(&P.tm_q, 64, h, q0 + i_start + (t + 2) * BM);
+                    if (!mbar_wait(&bars->do_empty[t & 1], (t >> 1) & 1, abort_flag, a.hdr)) break;
+                    JFA_TRACE_EV(bwd, 0, t + 2, 1);
+                    load_do(t + 2);
+                    issued_do = t + 3;
+                    if (t + 3 < nt) {
+                        tma_prefetch_l2_3d(&P.tm_do, 0, h, q0 + i_start + (t + 3) * BM);
+                        tma_prefetch_l2_3d(&P.tm_do, 64, h, q0 + i_start + (t + 3) * BM);
+                    }
                 }
             }
+            // never leave the CTA with copies in flight
             mbar_wait_drain(&bars->kv_full, 0, a.hdr);
-            if (issued_q > 0) mbar_wait_drain(&bars->q_full, (issued_q - 1) & 1, a.hdr);
-            if (issued_do > 0) mbar_wait_drain(&bars->do_full, (issued_do - 1) & 1, a.hdr);
+            mbar_wait_drain(&bars->q_full, (issued_q - 1) & 1, a.hdr);
+            for (int t = issued_do > 2 ? issued_do - 2 : 0; t < issued_do; ++t)
+                mbar_wait_drain(&bars->do_full[t & 1], (t >> 1) & 1, a.hdr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -245,43 +250,64 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             constexpr uint32_t idesc_tn = idesc_bf16(128, 128, 1, 1);  // A and B MN-major
             const uint32_t tdV = tmem, tdK = tmem + 128, tS = tmem + 256, tdP = tmem + 384;
             const uint32_t kb = sbase + kOffK, vb = sbase + kOffV, qb = sbase + kOffQ,
-                           dob = sbase + kOffDO, ptb = sbase + kOffPT, dsb = sbase + kOffDST;
-            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.hdr);
-            for (int t = 0; ok && t < nt; ++t) {
-                if (!mbar_wait(&bars->q_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
-                JFA_TRACE_EV(bwd, 1, t, 0);
-                if (t > 0 && !mbar_wait(&bars->dq_empty, (t - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                JFA_TRACE_EV(bwd, 1, t, 1);
-                tc_fence_after();
+                           dob = sbase + kOffDO, dsb = sbase + kOffDST;
+            auto issue_s = [&]() {  // S^T = K Q^T
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tS, kmajor_desc(kb, k), kmajor_desc(qb, k), idesc_nt, k > 0 ? 1u : 0u);
-                if (!mbar_wait(&bars->do_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
-                JFA_TRACE_EV(bwd, 1, t, 2);
-                tc_fence_after();
+            };
+            auto issue_dp = [&](int t) {  // dP^T = V dO^T
+                const uint32_t d = dob + (uint32_t)(t & 1) * kTile;
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
-                    mma_bf16_ss(tdP, kmajor_desc(vb, k), kmajor_desc(dob, k), idesc_nt, k > 0 ? 1u : 0u);
-                mma_commit(&bars->s_full);
-                JFA_TRACE_EV(bwd, 1, t, 3);
-                if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
-                JFA_TRACE_EV(bwd, 1, t, 4);
+                    mma_bf16_ss(tdP, kmajor_desc(vb, k), kmajor_desc(d, k), idesc_nt, k > 0 ? 1u : 0u);
+            };
+            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.hdr) &&
+                      mbar_wait(&bars->q_full, 0, abort_flag, a.hdr) &&
+                      mbar_wait(&bars->do_full[0], 0, abort_flag, a.hdr);
+            if (ok) {
                 tc_fence_after();
+                issue_s();
+                issue_dp(0);
+                mma_commit(&bars->s_full);
+            }
+            for (int t = 0; ok && t < nt; ++t) {
+                if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwd, 1, t, 0);
+                tc_fence_after();
+                // dK += dS^T Q   (A = dS^T K-major in smem, B = Q MN-major)
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)
                     mma_bf16_ss(tdK, kmajor_desc(dsb, k), mnmajor_desc(qb, k), idesc_nn,
                                 (t > 0 || k > 0) ? 1u : 0u);
                 mma_commit(&bars->q_empty);
-#pragma unroll
-                for (int k = 0; k < BM / 16; ++k)
-                    mma_bf16_ss(tdV, kmajor_desc(ptb, k), mnmajor_desc(dob, k), idesc_nn,
-                                (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&bars->do_empty);
+                // dQ^T = K^T dS^T over the dP^T columns (A = K, B = dS^T, both MN-major)
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
-                    mma_bf16_ss(tS, mnmajor_desc(dsb, k), mnmajor_desc(kb, k), idesc_tn, k > 0 ? 1u : 0u);
+                    mma_bf16_ss(tdP, mnmajor_desc(kb, k), mnmajor_desc(dsb, k), idesc_tn, k > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
-                JFA_TRACE_EV(bwd, 1, t, 5);
+                // dV += P^T dO: A = P^T from TMEM, query step k (16 queries) of group
+                // k/2 in columns 32*(k/2) + 8*(k%2) of the S^T region
+                const uint32_t d = dob + (uint32_t)(t & 1) * kTile;
+#pragma unroll
+                for (int k = 0; k < BM / 16; ++k)
+                    mma_bf16_ts(tdV, tS + 32 * (k >> 1) + 8 * (k & 1), mnmajor_desc(d, k), idesc_nn,
+                                (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&bars->do_empty[t & 1]);
+                JFA_TRACE_EV(bwd, 1, t, 1);
+                if (t + 1 < nt) {
+                    // S^T(t+1) overwrites P^T(t): issued after dV, which reads it
+                    if (!mbar_wait(&bars->q_full, (t + 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(bwd, 1, t, 2);
+                    tc_fence_after();
+                    issue_s();
+                    if (!mbar_wait(&bars->do_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, a.hdr) ||
+                        !mbar_wait(&bars->dq_empty, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    JFA_TRACE_EV(bwd, 1, t, 3);
+                    tc_fence_after();
+                    issue_dp(t + 1);
+                    mma_commit(&bars->s_full);
+                }
             }
             if (ok) mma_commit(&bars->fin);
             mma_commit(&bars->drain);
@@ -291,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         // ------------------------------------------------ score warps
         const int wq = warp & 3;                 // TMEM lane quarter
         const int grp = (warp - 2) >> 2;         // 32-column chunk of the row
-        const int r = wq * 32 + lane;            // key row (S^T, dV, dK) / query row (dQ)
+        const int r = wq * 32 + lane;            // key row (S^T, dV, dK) / d row (dQ^T)
         const int j = j0 + r;                    // key index within the sequence
         const bool jvalid = j < nkv;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
@@ -305,10 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)h * 4 * a.bias4_stride : nullptr;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_base = (BIAS == 2) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
-        const bool leader = (warp == 2 && lane == 0);
+        float* dq_col = a.dq_acc + ((int64_t)q0 * a.H + h) * HD + r;   // + qi * H * HD
         bool ok = true;
-        // LSE (log2 units) and D of a query tile, staged by group 0 into one of
-        // two buffers; the next tile's values are fetched a tile ahead.
+        // LSE (log2 units) and D of a query tile: group 0 stages them into one
+        // of two buffers a tile ahead (rows_full), every warp releases the
+        // buffer after reading it (rows_free)
         auto fetch_rowstats = [&](int t, float& l2, float& dv) {
             const int qi = i_start + t * BM + r;
             l2 = CUDART_INF_F;
@@ -318,44 +345,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 dv = a.dterm[(int64_t)(q0 + qi) * a.H + h];
             }
         };
-        if (nt > 0) {
-            if (grp == 0) {
-                float l2, dv;
-                fetch_rowstats(0, l2, dv);
-                lse2_s[r] = l2;
-                dd_s[r] = dv;
-            }
-            named_sync_score();
+        auto stage_rowstats = [&](int t, float l2, float dv) {
+            lse2_s[(t & 1) * 128 + r] = l2;
+            dd_s[(t & 1) * 128 + r] = dv;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->rows_full[t & 1]);
+        };
+        if (nt > 0 && grp == 0) {
+            float l2, dv;
+            fetch_rowstats(0, l2, dv);
+            stage_rowstats(0, l2, dv);
         }
         const int tslot = (warp == 2 && lane == 0) ? 2 : ((warp == kThreads / 32 - 1 && lane == 0) ? 3 : -1);
 #define SC_EV(ev)                                     \
     do {                                              \
         if (tslot >= 0) JFA_TRACE_EV(bwd, tslot, t, ev); \
     } while (0)
+        // A failed (timed-out) wait sets the CTA's abort flag; every later wait
+        // then returns at once, and the warps leave the loop independently
+        // (the loop has no CTA-wide barrier).
         for (int t = 0; t < nt; ++t) {
             SC_EV(0);
             const int qb0 = i_start + t * BM;    // query index of the tile's row 0
             const int buf = t & 1;
             float nl2 = CUDART_INF_F, ndv = 0.f;
             if (grp == 0 && t + 1 < nt) fetch_rowstats(t + 1, nl2, ndv);
-            // failed waits below only set the CTA's abort flag; the loop is left
-            // right after the named barrier, so every score warp runs the same
-            // sequence of barriers
-            mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr);
+            if (!mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
             SC_EV(1);
             tc_fence_after();
-            // key rows past the sequence end (neighbour data) must not reach dS K;
-            // S^T = K Q^T of the first tile has completed, so K may be edited now
+            // key rows past the sequence end (neighbour data) must not reach
+            // dQ^T = K^T dS^T; S^T = K Q^T of the first tile has completed
             if (t == 0 && grp == 0 && !jvalid) zero_row(smem + kOffK, r);
-            // the previous tile's dQ reduce must have read its staging (which
-            // overlays the P^T / dS^T buffers) before they are rewritten
-            if (t > 0) {
-                if (leader) {
-                    bulk_wait_read_all();
-                    mbar_arrive(&bars->stage_free);
-                }
-                mbar_wait(&bars->stage_free, (t - 1) & 1, abort_flag, a.hdr);
-            }
+            if (!mbar_wait(&bars->rows_full[buf], (t >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
             SC_EV(2);
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
             // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
@@ -442,6 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     }
                 }
             };
+            // Two 16-column halves.  P^T (bf16 pairs) goes back to TMEM over the
+            // first 16 of this group's 32 S^T columns (half hh to columns 8hh..,
+            // which half 0 has already read; no other group reads them); dS^T
+            // goes to shared memory for dK and dQ^T.
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t u[16], g[16];
@@ -450,93 +475,87 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 tmem_wait_ld();
                 const int c16 = grp * 2 + hh;
                 process(u, g, c16);
-                store_half_chunk_bits(smem + kOffPT, r, c16, u);
                 store_half_chunk_bits(smem + kOffDST, r, c16, g);
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
+                tmem_st8(tS + hh * 8, pk);
             }
-            // query rows past the sequence end must not reach dV / dK
+            tmem_wait_st();
+            // query rows past the sequence end (neighbour data) must not reach dV / dK
             if (qb0 + r >= nq) {
                 if (grp == 0) zero_row(smem + kOffQ, r);
-                else if (grp == 1) zero_row(smem + kOffDO, r);
+                else if (grp == 1) zero_row(smem + kOffDO + buf * kTile, r);
             }
             SC_EV(3);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->ds_full);
-            // dQ of this query tile: TMEM row r = query qb0 + r; staged as fp32
-            // 32-column chunks (128B swizzle) over the P^T / dS^T buffers, which
-            // the finished MMAs no longer read
-            mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr);
+            if (lane == 0) {
+                mbar_arrive(&bars->rows_free[buf]);
+                mbar_arrive(&bars->ds_full);
+            }
+            // LSE / D of tile t+1 into the other buffer, whose readers (tile t-1)
+            // have all released it
+            if (grp == 0 && t + 1 < nt) {
+                if (t >= 1 && !mbar_wait(&bars->rows_free[(t + 1) & 1], ((t - 1) >> 1) & 1, abort_flag, a.hdr)) {
+                    ok = false;
+                    break;
+                }
+                stage_rowstats(t + 1, nl2, ndv);
+            }
+            // dQ^T of this query tile: TMEM lane r = d, column c = query qb0 + 32 grp + c
+            if (!mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
             SC_EV(4);
             tc_fence_after();
-            const bool qvalid = qb0 + r < nq;
-            uint32_t u2[32];
-            tmem_ld32(tS, u2);
+            uint32_t dqv[32];
+            tmem_ld32(tdP, dqv);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dq_empty);  // TMEM columns free for S^T of t+1
+            if (lane == 0) mbar_arrive(&bars->dq_empty);  // columns free for dP^T of t+1
             SC_EV(5);
             {
-                uint8_t* row = smem + kOffPT + grp * (128 * 128) + r * 128;
+                const int qc = qb0 + grp * 32;
+                float* dst = dq_col + (int64_t)qc * a.H * HD;
+                const int64_t stride = (int64_t)a.H * HD;
+                const int nvalid = min(32, nq - qc);   // warp-uniform
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    uint4 w = qvalid ? make_uint4(u2[4 * v], u2[4 * v + 1], u2[4 * v + 2], u2[4 * v + 3])
-                                     : make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(row + ((v ^ (r & 7)) << 4)) = w;
-                }
+                for (int c = 0; c < 32; ++c)
+                    if (c < nvalid) atomicAdd(dst + c * stride, __uint_as_float(dqv[c]));
             }
-            if (grp == 0 && t + 1 < nt) {
-                lse2_s[(buf ^ 1) * 128 + r] = nl2;
-                dd_s[(buf ^ 1) * 128 + r] = ndv;
-            }
-            fence_proxy_async_smem();
             SC_EV(6);
-            named_sync_score();
-            SC_EV(7);
-            if (*abort_flag) { ok = false; break; }
-            if (leader) {
-                const int z = q0 + qb0;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    tma_reduce_add_3d(&P.tm_dq, smem + kOffPT + c4 * (128 * 128), c4 * 32, h, z);
-                bulk_commit();
-            }
         }
 #undef SC_EV
-        if (leader) bulk_wait_all();
         // ------------------------------------------------------ epilogue
         if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort_flag, a.hdr));
         if (ok && !*abort_flag) {
             tc_fence_after();
             __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
             __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
-            {
-                const int cc = 0;
-                uint32_t uk[32], uv[32];
-                if (nt > 0) {
-                    tmem_ld32(tdK, uk);
-                    tmem_ld32(tdV, uv);
-                    tmem_wait_ld();
-                } else {
+            uint32_t uk[32], uv[32];
+            if (nt > 0) {
+                tmem_ld32(tdK, uk);
+                tmem_ld32(tdV, uv);
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) uk[t] = 0u, uv[t] = 0u;
-                }
-                if (jvalid) {
+                for (int t = 0; t < 32; ++t) uk[t] = 0u, uv[t] = 0u;
+            }
+            if (jvalid) {
 #pragma unroll
-                    for (int t = 0; t < 32; t += 8) {
-                        uint4 wk, wv;
-                        wk.x = pack_bf16(__uint_as_float(uk[t + 0]) * a.scale, __uint_as_float(uk[t + 1]) * a.scale);
-                        wk.y = pack_bf16(__uint_as_float(uk[t + 2]) * a.scale, __uint_as_float(uk[t + 3]) * a.scale);
-                        wk.z = pack_bf16(__uint_as_float(uk[t + 4]) * a.scale, __uint_as_float(uk[t + 5]) * a.scale);
-                        wk.w = pack_bf16(__uint_as_float(uk[t + 6]) * a.scale, __uint_as_float(uk[t + 7]) * a.scale);
-                        wv.x = pack_bf16(__uint_as_float(uv[t + 0]), __uint_as_float(uv[t + 1]));
-                        wv.y = pack_bf16(__uint_as_float(uv[t + 2]), __uint_as_float(uv[t + 3]));
-                        wv.z = pack_bf16(__uint_as_float(uv[t + 4]), __uint_as_float(uv[t + 5]));
-                        wv.w = pack_bf16(__uint_as_float(uv[t + 6]), __uint_as_float(uv[t + 7]));
-                        *reinterpret_cast<uint4*>(dkrow + cc * 32 + t) = wk;
-                        *reinterpret_cast<uint4*>(dvrow + cc * 32 + t) = wv;
-                    }
+                for (int t = 0; t < 32; t += 8) {
+                    uint4 wk, wv;
+                    wk.x = pack_bf16(__uint_as_float(uk[t + 0]) * a.scale, __uint_as_float(uk[t + 1]) * a.scale);
+                    wk.y = pack_bf16(__uint_as_float(uk[t + 2]) * a.scale, __uint_as_float(uk[t + 3]) * a.scale);
+                    wk.z = pack_bf16(__uint_as_float(uk[t + 4]) * a.scale, __uint_as_float(uk[t + 5]) * a.scale);
+                    wk.w = pack_bf16(__uint_as_float(uk[t + 6]) * a.scale, __uint_as_float(uk[t + 7]) * a.scale);
+                    wv.x = pack_bf16(__uint_as_float(uv[t + 0]), __uint_as_float(uv[t + 1]));
+                    wv.y = pack_bf16(__uint_as_float(uv[t + 2]), __uint_as_float(uv[t + 3]));
+                    wv.z = pack_bf16(__uint_as_float(uv[t + 4]), __uint_as_float(uv[t + 5]));
+                    wv.w = pack_bf16(__uint_as_float(uv[t + 6]), __uint_as_float(uv[t + 7]));
+                    *reinterpret_cast<uint4*>(dkrow + t) = wk;
+                    *reinterpret_cast<uint4*>(dvrow + t) = wv;
                 }
             }
         }
@@ -591,31 +610,6 @@ __global__ void __launch_bounds__(256) tc_bwd_dq_finalize(const float* __restric
 }  // namespace
 
 
-// fp32 accumulator [rows][heads][128] as a 3-D tensor (d, head, row); boxes of
-// 32 d x 1 head x 128 rows (128 bytes inner) with the 128-byte swizzle.
-static bool make_tmap_dq_acc(CUtensorMap* map, void* base, int64_t rows, int heads) {
-    typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return false;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
-    cuuint64_t strides[2] = {(cuuint64_t)HD * 4, (cuuint64_t)heads * HD * 4};
-    cuuint32_t box[3] = {32, 1, 128};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per block
 
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
@@ -634,7 +628,6 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
         !make_tmap_rows_heads_d(&P.tm_v, a.v, p.total_kv, p.heads) ||
         !make_tmap_rows_heads_d(&P.tm_do, a.dout, p.total_q, p.heads))
         return cudaErrorInvalidValue;
-    if (!make_tmap_dq_acc(&P.tm_dq, a.dq_acc, p.total_q, p.heads)) return cudaErrorInvalidValue;
     P.a = kv;
     const int base = 1024 + (int)kOffEnd;
     int tab_need = (p.bias_kind == JFA_BIAS_RELPOS) ? (p.max_q_len + BN - 1) : 0;

@@ -254,8 +254,10 @@ def dequantize_along_rows(codes, scales, offsets):
 # [t*tile, min(n_q, (t+1)*tile)); a backward item is (b, h, key tile t).  Its
 # cost is the number of (query, key) pairs it computes: the number of keys each
 # of its rows may see (bottom-right causal: row i sees keys j <= i + n_kv - n_q),
-# or for a key tile the number of queries that may see each key.  Items are
-# ordered by cost descending, ties by (b, t, h) ascending.
+# or for a key tile the number of queries that may see each key.  Forward
+# items are ordered by cost descending, ties by (b, t, h) ascending; backward
+# items are grouped by (sequence, head) -- sequences by their total cost
+# descending, ties by b -- with the key tiles of a group in ascending order.
 # ---------------------------------------------------------------------------
 
 def _visible_keys(i, nq, nkv, causal):
@@ -286,8 +288,18 @@ def schedule(q_off, kv_off, H, tile, causal, backward=False):
             else:
                 cost = sum(_visible_keys(i, nq, nkv, causal) for i in range(lo, hi))
             pairs.append((cost, b, t))
-    pairs.sort(key=lambda p: (-p[0], p[1], p[2]))
-    out = [(b, h, t, cost) for (cost, b, t) in pairs for h in range(H)]
+    if not backward:
+        pairs.sort(key=lambda p: (-p[0], p[1], p[2]))
+        out = [(b, h, t, cost) for (cost, b, t) in pairs for h in range(H)]
+    else:
+        # key tiles grouped by (sequence, head): sequences by their total pair
+        # count descending (ties by b), then heads, then tiles ascending
+        seq_cost, by_seq = {}, {}
+        for cost, b, t in pairs:
+            seq_cost[b] = seq_cost.get(b, 0) + cost
+            by_seq.setdefault(b, []).append((t, cost))
+        order = sorted(by_seq, key=lambda b: (-seq_cost[b], b))
+        out = [(b, h, t, cost) for b in order for h in range(H) for (t, cost) in sorted(by_seq[b])]
     return np.asarray(out, dtype=np.int32).reshape(-1, 4)
 
 

@@ -357,7 +357,19 @@ def test_schedule_covers_every_tile_once_longest_first():
             got = [tuple(x[:3]) for x in items]
             assert len(got) == len(expect) and set(got) == expect
             costs = items[:, 3]
-            assert np.all(costs[:-1] >= costs[1:])
+            if not backward:
+                assert np.all(costs[:-1] >= costs[1:])
+            else:
+                # (sequence, head) groups are contiguous, their tiles ascending,
+                # and sequences come by total cost descending
+                keys = [(int(b), int(h)) for b, h, _, _ in items]
+                starts = [i for i in range(len(keys)) if i == 0 or keys[i] != keys[i - 1]]
+                assert len(starts) == len(set(keys))
+                for i0, i1 in zip(starts, starts[1:] + [len(keys)]):
+                    assert list(items[i0:i1, 2]) == list(range(i1 - i0))
+                seq_tot = [int(costs[items[:, 0] == b].sum()) for b in range(len(rows))]
+                seq_order = list(dict.fromkeys(int(b) for b in items[:, 0]))
+                assert all(seq_tot[x] >= seq_tot[y] for x, y in zip(seq_order, seq_order[1:]))
             # per-item cost equals the number of pairs of the library's
             # bottom-right causal mask restricted to the tile
             total = 0
