@@ -111,11 +111,12 @@ struct AttnArgs {
     void* dk;
     void* dv;
     float* dq_acc;
-    // tensor-core path, relative-position bias: four copies of each head's
-    // table scaled by log2(e), copy k shifted left by k entries, so that any
-    // run of table entries can be read with 16-byte-aligned vector loads
+    // tensor-core path, relative-position bias: each head's table scaled by
+    // log2(e) as runs of four (float4 entry t = entries t .. t+3), so that any
+    // run of table entries can be read with 16-byte-aligned vector loads;
+    // entry t of head h is bias4[4 * (h * bias4_stride + t) + 0..3]
     const float* bias4;
-    int bias4_stride;  // floats per copy (a multiple of 4)
+    int bias4_stride;  // float4 entries per head (at least 384)
 };
 
 // ---------------------------------------------------------------------------

@@ -136,6 +136,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Contiguous bulk copy global -> shared (no tensor map, no multicast);
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Brings a tile into L2 ahead of its TMA load (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -378,6 +388,21 @@ __device__ __forceinline__ float exp2_fma(float y) {
     const float f = y - n;
     const float p = fmaf(fmaf(fmaf(0.05517098f, f, 0.24260971f), f, 0.69326097f), f, 0.9999282f);
     return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Two lanes of exp2_fma with paired fp32 arithmetic (y >= -126 after the
+// clamp; the scale by 2^n is an integer add to the exponent field).
+__device__ __forceinline__ float2 exp2_fma2(float2 y) {
+    y.x = fmaxf(y.x, -126.0f);
+    y.y = fmaxf(y.y, -126.0f);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
+    const float2 t = add2(y, magic);
+    const float2 f = sub2(y, sub2(t, magic));
+    float2 p = fma2(make_float2(0.05517098f, 0.05517098f), f, make_float2(0.24260971f, 0.24260971f));
+    p = fma2(p, f, make_float2(0.69326097f, 0.69326097f));
+    p = fma2(p, f, make_float2(0.9999282f, 0.9999282f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // exp2 of element c of a row: every JFA_EXP2_POLY_MOD-th element on the FMA

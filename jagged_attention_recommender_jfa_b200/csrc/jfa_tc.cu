@@ -30,13 +30,15 @@ namespace {
 struct Extra {
     size_t dq_acc, qf, kf, vf, bias4, total;
 };
-int bias4_stride(const jfa_problem& p) { return (p.relpos_len + 3) & ~3; }
+// entries per head of the prepared table: the table, and at least the
+// 384-entry window the forward stages per key tile
+int bias4_stride(const jfa_problem& p) { return p.relpos_len < 384 ? 384 : p.relpos_len; }
 Extra extra_layout(const jfa_problem& p, int backward) {
     Extra e{};
     size_t off = 0;
     if (p.bias_kind == JFA_BIAS_RELPOS) {
         e.bias4 = off;
-        off = align256(off + sizeof(float) * 4 * (size_t)p.heads * bias4_stride(p));
+        off = align256(off + sizeof(float4) * (size_t)p.heads * bias4_stride(p));
     }
     if (backward) {
         e.dq_acc = off;
@@ -60,16 +62,19 @@ cudaError_t fake_quant(const jfa_problem& p, AttnArgs& a, char* ws, const Extra&
     a.v = vf;
     return e;
 }
-// out[(h * 4 + k) * stride + t] = log2(e) * table[h][min(t + k, len - 1)]
+// out[h * stride + t] = log2(e) * (table[h][t], table[h][t+1], table[h][t+2],
+// table[h][t+3]), indices clamped to len - 1: entry t is the run of four that
+// starts at t, so any run of the table can be read as 16-byte-aligned float4s
 __global__ void __launch_bounds__(256) tc_bias_prep(const float* __restrict__ tab, int len, int heads,
-                                                    int stride, float* __restrict__ out) {
-    const int64_t n = (int64_t)heads * 4 * stride;
+                                                    int stride, float4* __restrict__ out) {
+    const int64_t n = (int64_t)heads * stride;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int t = (int)(i % stride);
-        const int hk = (int)(i / stride);
-        const int k = hk & 3, h = hk >> 2;
-        out[i] = tab[(int64_t)h * len + min(t + k, len - 1)] * 1.4426950408889634f;
+        const int t = (int)(i % stride), h = (int)(i / stride);
+        const float* row = tab + (int64_t)h * len;
+        const float k = 1.4426950408889634f;
+        out[i] = make_float4(row[min(t, len - 1)] * k, row[min(t + 1, len - 1)] * k,
+                             row[min(t + 2, len - 1)] * k, row[min(t + 3, len - 1)] * k);
     }
 }
 
@@ -77,11 +82,11 @@ cudaError_t prep_bias(const jfa_problem& p, AttnArgs& a, char* ws, const Extra& 
     if (p.bias_kind != JFA_BIAS_RELPOS) return cudaSuccess;
     const int stride = bias4_stride(p);
     float* out = reinterpret_cast<float*>(ws + L.bias4);
-    const int64_t n = (int64_t)p.heads * 4 * stride;
+    const int64_t n = (int64_t)p.heads * stride;
     const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
     prof_begin(st);
     tc_bias_prep<<<blocks, 256, 0, st>>>(reinterpret_cast<const float*>(a.bias), p.relpos_len, p.heads,
-                                          stride, out);
+                                          stride, reinterpret_cast<float4*>(out));
     prof_end(st, K_TC_BIAS_PREP);
     a.bias4 = out;
     a.bias4_stride = stride;
@@ -91,7 +96,7 @@ cudaError_t prep_bias(const jfa_problem& p, AttnArgs& a, char* ws, const Extra& 
 
 // The backward keeps an fp32 dQ accumulator [total_q][heads][128]; MXFP8
 // adds the three dequantised operands; a relative-position bias adds its
-// four shifted, log2(e)-scaled copies.
+// log2(e)-scaled table of runs of four.
 size_t tc_workspace_extra(const jfa_problem& p, int backward) {
     return extra_layout(p, backward).total;
 }
@@ -133,7 +138,7 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
     return tc_backward_launch(p, aq, akv, st);
 }
 
-int tc_fwd_tile() { return 128; }
+int tc_fwd_tile() { return 256; }   // a forward work item is a 256-row query block
 int tc_bwd_tile() { return 128; }
 
 }  // namespace jfa

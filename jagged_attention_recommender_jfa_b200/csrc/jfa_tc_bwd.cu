@@ -59,7 +59,14 @@ constexpr uint32_t kOffDO = kOffQ + kTile;        // two buffers
 constexpr uint32_t kOffDST = kOffDO + 2 * kTile;
 constexpr uint32_t kOffBar = kOffDST + kTile;     // 196608
 constexpr uint32_t kOffRow = kOffBar + 256;       // lse2[2][128], D[2][128] (double-buffered)
-constexpr uint32_t kOffEnd = kOffRow + 2048;
+// Relative-position bias window of a query tile, 2 stages: 272 entries of the
+// prepared table (entry t = table entries t .. t+3, log2(e)-scaled) from the
+// smallest index the tile's (query, key) pairs need; a thread reads its run
+// of 16 entries as four float4s, consecutive key rows consecutive entries.
+constexpr int kWin = 272;
+constexpr uint32_t kWinBytes = kWin * 16;          // 4352
+constexpr uint32_t kOffWin = kOffRow + 2048;
+constexpr uint32_t kOffEnd = kOffWin + 2 * kWinBytes;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
@@ -72,6 +79,7 @@ struct Bars {
     uint64_t dq_empty;      // 16 score warps
     uint64_t rows_full[2];  // LSE / D of a query tile staged (4 warps of group 0)
     uint64_t rows_free[2];  // ... and read by every score warp (16)
+    uint64_t bias_full[2];  // bias window of a query tile loaded
     uint64_t fin;
     uint64_t drain;
     uint32_t tmem_base;
@@ -85,8 +93,14 @@ struct BwdParams {
     CUtensorMap tm_v;
     CUtensorMap tm_do;
     AttnArgs a;
-    int tab_cap;  // bias table entries that fit in shared memory
 };
+
+// First entry of the bias window of the query tile starting at query qb0
+// (keys j0 ..): the smallest table index a pair of the tile can need, clamped
+// so that the window lies inside the prepared table.
+__device__ __forceinline__ int bias_window_start(int qb0, int j0, int C, int stride) {
+    return min(max(qb0 - j0 - (BN - 1) + C, 0), stride - kWin);
+}
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32u, 16u,
@@ -143,13 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     const int nt = nq > i_start ? (nq - i_start + BM - 1) / BM : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool softmax = SOFTMAX;
-    // relative-position bias of this CTA's (query, key) range, log2(e)-scaled:
-    // tab[t] = bias(i, j) for i - j = tab_lo + t, kept in shared memory when
-    // it fits
-    const int tab_lo = i_start - j0 - (BN - 1);
-    const int tab_len = nq - i_start + BN - 1;
-    const bool tab_in_smem = BIAS == 1 && nt > 0 && tab_len <= P.tab_cap;
-    float* tab = reinterpret_cast<float*>(smem + kOffEnd);
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -160,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             mbar_init(&bars->do_empty[s2], 1);
             mbar_init(&bars->rows_full[s2], 4);
             mbar_init(&bars->rows_free[s2], NG * 4);
+            mbar_init(&bars->bias_full[s2], 1);
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->ds_full, NG * 4);
@@ -173,12 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     if (warp == 1) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
-    }
-    if (tab_in_smem) {
-        const int C = (a.relpos_len - 1) >> 1;
-        const float* src = a.bias4 + (int64_t)h * 4 * a.bias4_stride;   // copy 0
-        for (int t = threadIdx.x; t < tab_len; t += kThreads)
-            tab[t] = __ldg(src + min(max(tab_lo + t, -C), C) + C);
     }
     tc_fence_before();
     __syncthreads();
@@ -201,11 +203,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, h, k0 + j0);
             tma_load_3d(smem + kOffV, &P.tm_v, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->kv_full, 64, h, k0 + j0);
+            // Q(t) and, with a relative-position bias, the tile's bias window; the
+            // window's stage (t & 1) was last read for tile t-2, whose score
+            // phase ended before dK(t-2) and so before the q_empty that lets
+            // Q(t) in
             auto load_q = [&](int t) {
                 const int z = q0 + i_start + t * BM;
                 mbar_arrive_expect_tx(&bars->q_full, kTile);
                 tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, h, z);
                 tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, z);
+                if (BIAS == 1) {
+                    const int C = (a.relpos_len - 1) >> 1;
+                    const int w0 = bias_window_start(i_start + t * BM, j0, C, a.bias4_stride);
+                    const float* src = a.bias4 + 4 * ((int64_t)h * a.bias4_stride + w0);
+                    mbar_arrive_expect_tx(&bars->bias_full[t & 1], kWinBytes);
+                    bulk_load(smem + kOffWin + (t & 1) * kWinBytes, src, kWinBytes, &bars->bias_full[t & 1]);
+                }
             };
             auto load_do = [&](int t) {
                 const int z = q0 + i_start + t * BM;
@@ -239,6 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // never leave the CTA with copies in flight
             mbar_wait_drain(&bars->kv_full, 0, a.hdr);
             mbar_wait_drain(&bars->q_full, (issued_q - 1) & 1, a.hdr);
+            if (BIAS == 1)
+                for (int t = issued_q > 2 ? issued_q - 2 : 0; t < issued_q; ++t)
+                    mbar_wait_drain(&bars->bias_full[t & 1], (t >> 1) & 1, a.hdr);
             for (int t = issued_do > 2 ? issued_do - 2 : 0; t < issued_do; ++t)
                 mbar_wait_drain(&bars->do_full[t & 1], (t >> 1) & 1, a.hdr);
         }
@@ -315,6 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------ score warps
+        // waits taken by a whole warp: the result is made warp-uniform, so that a
+        // timed-out wait ends the warp's loop on every lane together
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.hdr));
+        };
         const int wq = warp & 3;                 // TMEM lane quarter
         const int grp = (warp - 2) >> 2;         // 32-column chunk of the row
         const int r = wq * 32 + lane;            // key row (S^T, dV, dK) / d row (dQ^T)
@@ -327,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const float sc = a.scale * kLog2e;
         const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
         const int C = (a.relpos_len - 1) >> 1;
-        // log2(e)-scaled table (copy 0 of the four shifted copies)
+        // log2(e)-scaled table: entry t at tab4[4 t]
         const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)h * 4 * a.bias4_stride : nullptr;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_base = (BIAS == 2) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
@@ -370,14 +391,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             const int buf = t & 1;
             float nl2 = CUDART_INF_F, ndv = 0.f;
             if (grp == 0 && t + 1 < nt) fetch_rowstats(t + 1, nl2, ndv);
-            if (!mbar_wait(&bars->s_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+            if (!wwait(&bars->s_full, t & 1)) { ok = false; break; }
             SC_EV(1);
             tc_fence_after();
             // key rows past the sequence end (neighbour data) must not reach
             // dQ^T = K^T dS^T; S^T = K Q^T of the first tile has completed
             if (t == 0 && grp == 0 && !jvalid) zero_row(smem + kOffK, r);
-            if (!mbar_wait(&bars->rows_full[buf], (t >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+            if (!wwait(&bars->rows_full[buf], (t >> 1) & 1)) { ok = false; break; }
+            if (BIAS == 1 && !wwait(&bars->bias_full[buf], (t >> 1) & 1)) { ok = false; break; }
             SC_EV(2);
+            // bias(qc0 + v, j) = table[qc0 - j + C + v]: window entries
+            // qc0 - j + C - w0 + 4q hold table[... + 4q + 0..3]
+            const int wbase = BIAS == 1 ? (qb0 - j + C) - bias_window_start(qb0, j0, C, a.bias4_stride) : 0;
+            const float4* win = reinterpret_cast<const float4*>(smem + kOffWin + buf * kWinBytes);
             const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
             // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
             auto process = [&](uint32_t (&u)[16], uint32_t (&g)[16], int c16) {
@@ -393,14 +419,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const float2 sc2 = make_float2(sc, sc);
                 if (BIAS == 1) {
                     float bb[16];
-                    if (tab_in_smem) {
-                        const float* tb = tab + (qc0 - j - tab_lo);   // tb[v] = bias(qc0 + v, j)
+                    const int s0 = qc0 - j + C;                       // table index of bias(qc0, j)
+                    const int wr = wbase + c16 * 16;                  // its window entry
+                    if (s0 >= 0 && s0 + 15 <= 2 * C && wr >= 0 && wr + 12 < kWin) {
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) bb[v] = tb[v];
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 t4 = win[wr + 4 * q];
+                            bb[4 * q] = t4.x, bb[4 * q + 1] = t4.y, bb[4 * q + 2] = t4.z, bb[4 * q + 3] = t4.w;
+                        }
                     } else {
-                        const int s0 = qc0 - j + C;                   // table index of bias(qc0, j)
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) bb[v] = __ldg(tab4 + min(max(s0 + v, 0), 2 * C));
+                        for (int v = 0; v < 16; ++v) bb[v] = __ldg(tab4 + 4 * min(max(s0 + v, 0), 2 * C));
                     }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -498,14 +527,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // LSE / D of tile t+1 into the other buffer, whose readers (tile t-1)
             // have all released it
             if (grp == 0 && t + 1 < nt) {
-                if (t >= 1 && !mbar_wait(&bars->rows_free[(t + 1) & 1], ((t - 1) >> 1) & 1, abort_flag, a.hdr)) {
+                if (t >= 1 && !wwait(&bars->rows_free[(t + 1) & 1], ((t - 1) >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 stage_rowstats(t + 1, nl2, ndv);
             }
             // dQ^T of this query tile: TMEM lane r = d, column c = query qb0 + 32 grp + c
-            if (!mbar_wait(&bars->dq_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+            if (!wwait(&bars->dq_full, t & 1)) { ok = false; break; }
             SC_EV(4);
             tc_fence_after();
             uint32_t dqv[32];
@@ -528,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         }
 #undef SC_EV
         // ------------------------------------------------------ epilogue
-        if (ok && nt > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->fin, 0, abort_flag, a.hdr));
+        if (ok && nt > 0) ok = __all_sync(0xffffffffu, wwait(&bars->fin, 0));
         if (ok && !*abort_flag) {
             tc_fence_after();
             __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
@@ -629,14 +658,7 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
         !make_tmap_rows_heads_d(&P.tm_do, a.dout, p.total_q, p.heads))
         return cudaErrorInvalidValue;
     P.a = kv;
-    const int base = 1024 + (int)kOffEnd;
-    int tab_need = (p.bias_kind == JFA_BIAS_RELPOS) ? (p.max_q_len + BN - 1) : 0;
-    int smem = base + 4 * tab_need;
-    if (smem > kSmemLimit) {
-        tab_need = (kSmemLimit - base) / 4;
-        smem = kSmemLimit;
-    }
-    P.tab_cap = tab_need;
+    const int smem = 1024 + (int)kOffEnd;
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
     const bool sm = a.act == JFA_ACT_SOFTMAX;
     void (*kern)(BwdParams) = nullptr;

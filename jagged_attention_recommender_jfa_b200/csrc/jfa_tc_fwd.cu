@@ -1,30 +1,42 @@
 // Tensor-core (tcgen05) jagged attention forward for bf16, head_dim 128.
 //
-// One CTA per work item (sequence, head, 128-row query tile) of the
-// longest-first schedule.  Attention runs directly on the packed jagged
-// buffers ("Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a
-// Different Stack", section "Bottleneck move 1"): TMA fetches the query tile
-// once and streams 128-row key/value tiles of the same sequence through a
-// two-stage ring; rows of a tile that lie past the sequence end belong to the
-// neighbouring sequence and are masked out of the scores (and zeroed in the
-// value tile) before they can contribute.
+// Attention runs directly on the packed jagged buffers ("Meta GEM Training
+// Efficiency: Why LLM-Scale Recommenders Need a Different Stack", section
+// "Bottleneck move 1"): a work item is (sequence, head, 256-row query block),
+// taken from the longest-first schedule.  The block is two 128-row query
+// tiles A and B that share one stream of 128-row key/value tiles (a
+// two-stage ring fetched by TMA); rows of a key tile past the sequence end
+// belong to the neighbouring sequence and are masked out of the scores (and
+// zeroed in the value tile) before they can contribute.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer (one thread)
-//   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2..5  softmax / activation and epilogue; warp w owns TMEM lanes
-//               32*(w%4) .. +31, i.e. one query row per thread
+// Warp roles (576 threads, persistent: one CTA per SM walks its share of the
+// work list):
+//   warps 0..7  softmax / activation and epilogue of tile A, warps 8..15 of
+//               tile B; warp w owns TMEM lanes 32*(w%4) .. +31 and one half
+//               (64 columns) of each of those rows: the two warps that share
+//               rows sit on the same SM sub-partition and exchange their
+//               partial row maxima through shared memory and a two-arrival
+//               mbarrier
+//   warp 16     TMEM allocator and MMA issuer (one thread)
+//   warp 17     TMA producer (one thread)
 //
-// Per key tile j:  S = Q K_j^T  (tcgen05, 128x128x128, fp32 in TMEM)
-//                  softmax warps: scale, bias, mask, online softmax in the
-//                  log2 domain (or GDPA act(s)/n_kv), P (bf16) -> shared
-//                  memory in the 128B-swizzled K-major layout
-//                  O += P V_j   (tcgen05, A = P from smem, B = V MN-major)
-// The rescale of O by exp2(m_old - m_new) is lazy: it happens only when a
-// row's running maximum grows by more than 8 (a factor 256), otherwise the
-// old maximum stays the reference; the final O / l is exact either way.
+// Per key tile j, tile T in {A, B}:
+//   S_T = Q_T K_j^T                  (tcgen05, 128x128x128, fp32 in TMEM)
+//   softmax warps of T: scale + bias + mask and the row maximum (the biased
+//   scores go back to TMEM over S), then the online softmax in the log2
+//   domain (or GDPA act(s)/n_kv); P (bf16) written back to TMEM, each half of
+//   the row over the first half of its own S columns (keys 0..63 to columns
+//   0..31, keys 64..127 to columns 64..95)
+//   O_T += P_T V_j                   (tcgen05, A = P from TMEM, B = V MN-major)
+// The tensor core alternates between the tiles: while the softmax warps of
+// one tile work, it runs P.V and the next Q K^T of the other.  The rescale of
+// O by exp2(m_old - m_new) is lazy: it happens only when a row's running
+// maximum grows by more than 8 (a factor 256), otherwise the old maximum stays
+// the reference; the final O / l is exact either way.
 //
-// TMEM: S at columns [0, 128), O at [128, 256).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).  The
+// warps of a tile never wait on each other except for the pairwise maximum
+// exchange.
 #include <math_constants.h>
 
 #include "jfa_mx.cuh"
@@ -39,17 +51,27 @@ JFA_TRACE_DEFINE(fwd)
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NG = 4;                       // column groups: a softmax thread owns 128/NG columns of a row
-constexpr int CW = 128 / NG;                // columns per softmax thread
-constexpr int kThreads = 64 + NG * 128;     // warp 0 TMA, warp 1 MMA, the rest softmax
+constexpr int kBlockRows = 2 * BM;          // query rows per work item (tiles A and B)
+constexpr int kMmaWarp = 16, kTmaWarp = 17;
+constexpr int kThreads = 32 * 18;
+constexpr int CW = 64;                      // columns of a key tile per softmax thread
 constexpr uint32_t kBox = 128 * 128;        // bytes of one [128 rows][64 bf16] box
 constexpr uint32_t kTile = 2 * kBox;        // one 128 x 128 bf16 tile (two boxes)
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;        // 2 stages
+constexpr uint32_t kOffQ = 0;                    // Q_A, Q_B
+constexpr uint32_t kOffK = kOffQ + 2 * kTile;    // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTile;    // 2 stages
-constexpr uint32_t kOffBar = kOffV + 2 * kTile;  // 163840
-constexpr uint32_t kOffRed = kOffBar + 512;      // row-max exchange [2][NG][128] + l [2][NG][128]
-constexpr uint32_t kSmemBytes = kOffRed + 2 * 2 * NG * 128 * 4 + 1024;  // + alignment slack
+// Relative-position bias window of a key tile, 2 stages: 384 entries of the
+// prepared table (entry t = table entries t .. t+3, log2(e)-scaled) starting
+// at w0, so that a thread's run of 128 entries is read as 16-byte float4s;
+// consecutive rows read consecutive entries, which keeps a quarter-warp's
+// reads on distinct banks.
+constexpr int kWin = 384;                          // float4 entries
+constexpr uint32_t kWinBytes = kWin * 16;          // 6144
+constexpr uint32_t kOffBias = kOffV + 2 * kTile;   // 196608
+constexpr uint32_t kOffRed = kOffBias + 2 * kWinBytes;   // [2 parity][2 tiles][2 halves][128] row maxima
+constexpr uint32_t kOffLred = kOffRed + 2 * 2 * 2 * 128 * 4;     // same shape, row sums at the epilogue
+constexpr uint32_t kOffBar = kOffLred + 2 * 2 * 2 * 128 * 4;
+constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // + alignment slack
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
 
@@ -57,10 +79,12 @@ struct Bars {
     uint64_t q_full, q_free;
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2];
-    uint64_t p_full;
-    uint64_t pv_done;
-    uint64_t o_free[2];
+    uint64_t s_full[2];    // per tile
+    uint64_t p_full[2];    // per tile: its 8 softmax warps
+    uint64_t pv_done[2];   // per tile
+    uint64_t o_free[2];    // per tile: its 8 softmax warps, after the epilogue read O
+    uint64_t bias_full[2]; // per stage: bias window loaded
+    uint64_t pair[8];      // [tile][lane quarter]: the two half-row warps exchanged
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -74,7 +98,7 @@ struct FwdParams {
     AttnArgs a;
 };
 
-// K-major operand (Q, K, P) at K-step k (16 elements): box k/4, +32 B per step.
+// K-major operand (Q, K) at K-step k (16 elements): box k/4, +32 B per step.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32u, 16u,
                            1024u);
@@ -86,10 +110,6 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
     return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
 }
 
-__device__ __forceinline__ void named_sync_softmax() {
-    asm volatile("bar.sync 1, %0;" ::"n"(NG * 128) : "memory");
-}
-
 // The work item a CTA takes at its r-th turn: items are listed longest
 // first and dealt out in snake order (0..G-1, G-1..0, ...), which evens out
 // the per-CTA totals of a decreasing cost list.
@@ -98,7 +118,9 @@ __device__ __forceinline__ int item_of_turn(int r, int c, int G) {
 }
 
 struct Item {
-    int b, h, row0, q0, nq, k0, nkv, n_tiles;
+    int b, h, row0, q0, nq, k0, nkv;
+    int n_t[2];   // key tiles of tile A and tile B (0: the tile has no rows or sees no key)
+    int n;        // key tiles of the block
 };
 
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
@@ -106,32 +128,44 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     Item w;
     w.b = it.x;
     w.h = it.y;
-    w.row0 = it.z * BM;
+    w.row0 = it.z * kBlockRows;
     w.q0 = a.q_off[w.b];
     w.nq = a.q_off[w.b + 1] - w.q0;
     w.k0 = a.kv_off[w.b];
     w.nkv = a.kv_off[w.b + 1] - w.k0;
-    const int rows_hi = min(w.row0 + BM, w.nq);
-    int kv_end = a.causal ? min(w.nkv, rows_hi + (w.nkv - w.nq)) : w.nkv;
-    kv_end = max(kv_end, 0);
-    w.n_tiles = (kv_end + BN - 1) / BN;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int lo = w.row0 + t * BM, hi = min(lo + BM, w.nq);
+        if (hi <= lo) {
+            w.n_t[t] = 0;
+            continue;
+        }
+        int kv_end = a.causal ? min(w.nkv, hi + (w.nkv - w.nq)) : w.nkv;
+        kv_end = max(kv_end, 0);
+        w.n_t[t] = (kv_end + BN - 1) / BN;
+    }
+    w.n = max(w.n_t[0], w.n_t[1]);
     return w;
 }
 
-// Persistent forward: one CTA per SM walks its share of the longest-first
-// work list.  BIAS: 0 none, 1 relative-position (read through L1), 2 dense
-// jagged.  SOFTMAX: softmax (true) or GDPA.  QP: MXFP8 attention -- P is
-// quantised to E4M3 with one E8M0 scale per 32 keys (counted from the
+// First table entry of the bias window of key tile jc for the block at row0:
+// the smallest index any (row, key) pair of the block can need, clamped so
+// that the window lies inside the prepared table.
+__device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int stride) {
+    return min(max(row0 - jc - (BN - 1) + C, 0), stride - kWin);
+}
+
+// BIAS: 0 none, 1 relative-position (log2(e)-scaled table staged per key tile),
+// 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.  QP: MXFP8 attention -- P
+// is quantised to E4M3 with one E8M0 scale per 32 keys (counted from the
 // sequence's first key) before P.V; l uses the unquantised weights.
 //
-// Tensor-core order per item: QK_0, QK_1, then for each tile j: [P_j ready]
-// P.V_j, QK_{j+2}.  S is double-buffered in TMEM (columns 0 / 128), O too
-// (columns 256 / 384, alternating per item) so that an item's epilogue
-// overlaps the next item's score MMAs.  Q is reloaded as soon as the item's
-// last QK has retired.  Barrier phases follow per-CTA counters (g: key tiles
-// so far, nk: items with keys so far, m: items so far).  Each softmax thread
-// owns one query row and one 64-column half of it; the two halves exchange
-// partial row maxima through shared memory.
+// Tensor-core order per item (n key tiles; tile T has n_T <= n of them):
+//   QK_A(0), QK_B(0), then for each j: [P_A(j)] PV_A(j), QK_A(j+1),
+//   [P_B(j)] PV_B(j), QK_B(j+1).
+// Barrier phases follow per-CTA counters: g (key tiles so far, for the K/V
+// ring), gt[T] (steps of tile T so far), mt[T] (items with steps for T so
+// far), nk (items so far, for Q).
 template <int BIAS, bool SOFTMAX, bool QP>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
@@ -140,8 +174,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
-    float* red = reinterpret_cast<float*>(smem + kOffRed);   // [2 parity][NG groups][128 rows]
-    float* lred = red + 2 * NG * 128;                          // [2 item parity][NG groups][128 rows]
     const int G = gridDim.x, cta = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool softmax = SOFTMAX;
@@ -155,15 +187,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             mbar_init(&bars->v_full[s], 1);
             mbar_init(&bars->v_empty[s], 1);
             mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->o_free[s], NG * 4);
+            mbar_init(&bars->p_full[s], 8);
+            mbar_init(&bars->pv_done[s], 1);
+            mbar_init(&bars->o_free[s], 8);
+            mbar_init(&bars->bias_full[s], 1);
         }
-        mbar_init(&bars->p_full, NG * 4);
-        mbar_init(&bars->pv_done, 1);
+        for (int q = 0; q < 8; ++q) mbar_init(&bars->pair[q], 2);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
@@ -174,26 +208,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     volatile int* abort_flag = &bars->abort_flag;
     const uint32_t sbase = smem_u32(smem);
 
-    if (warp == 0) {
+    if (warp == kTmaWarp) {
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             tma_prefetch_desc(&P.tm_q);
             tma_prefetch_desc(&P.tm_k);
             tma_prefetch_desc(&P.tm_v);
             int g = 0, nk = 0;        // key tiles issued, items with keys
-            int kq = 0, kv_i = 0;     // loads issued (for the drain)
             bool ok = true;
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
                 const Item w = load_item(a, idx);
-                if (w.n_tiles == 0) continue;
+                if (w.n == 0) continue;
                 if (nk > 0 && !mbar_wait(&bars->q_free, (nk - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars->q_full, kTile);
-                tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, w.h, w.q0 + w.row0);
-                tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, w.h, w.q0 + w.row0);
+                mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
+                for (int t = 0; t < 2; ++t) {
+                    const int z = w.q0 + w.row0 + t * BM;
+                    tma_load_3d(smem + kOffQ + t * kTile, &P.tm_q, &bars->q_full, 0, w.h, z);
+                    tma_load_3d(smem + kOffQ + t * kTile + kBox, &P.tm_q, &bars->q_full, 64, w.h, z);
+                }
                 ++nk;
-                for (int j = 0; j < w.n_tiles; ++j, ++g) {
+                for (int j = 0; j < w.n; ++j, ++g) {
                     const int s = g & 1;
                     const uint32_t par = ((g >> 1) - 1) & 1;
                     const int z = w.k0 + j * BN;
@@ -202,14 +238,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     mbar_arrive_expect_tx(&bars->k_full[s], kTile);
                     tma_load_3d(smem + kOffK + s * kTile, &P.tm_k, &bars->k_full[s], 0, w.h, z);
                     tma_load_3d(smem + kOffK + s * kTile + kBox, &P.tm_k, &bars->k_full[s], 64, w.h, z);
-                    ++kq;
                     if (g >= 2 && !mbar_wait(&bars->v_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
                     JFA_TRACE_EV(fwd, 0, g, 1);
                     mbar_arrive_expect_tx(&bars->v_full[s], kTile);
                     tma_load_3d(smem + kOffV + s * kTile, &P.tm_v, &bars->v_full[s], 0, w.h, z);
                     tma_load_3d(smem + kOffV + s * kTile + kBox, &P.tm_v, &bars->v_full[s], 64, w.h, z);
-                    ++kv_i;
-                    if (j + 2 < w.n_tiles) {  // warm L2 for the tiles loaded after the next release
+                    if (BIAS == 1) {
+                        // the stage's previous window was read by the softmax warps of
+                        // both tiles before its P.V, hence before v_empty above
+                        const int C = (a.relpos_len - 1) >> 1;
+                        const int w0 = bias_window_start(w.row0, j * BN, C, a.bias4_stride);
+                        const float* src = a.bias4 + 4 * ((int64_t)w.h * a.bias4_stride + w0);
+                        mbar_arrive_expect_tx(&bars->bias_full[s], kWinBytes);
+                        bulk_load(smem + kOffBias + s * kWinBytes, src, kWinBytes, &bars->bias_full[s]);
+                    }
+                    if (j + 2 < w.n) {  // warm L2 for the tiles loaded after the next release
                         tma_prefetch_l2_3d(&P.tm_k, 0, w.h, z + 2 * BN);
                         tma_prefetch_l2_3d(&P.tm_k, 64, w.h, z + 2 * BN);
                         tma_prefetch_l2_3d(&P.tm_v, 0, w.h, z + 2 * BN);
@@ -219,62 +262,78 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             }
             // never leave the CTA with copies in flight: wait for the last loads
             if (nk > 0) mbar_wait_drain(&bars->q_full, (nk - 1) & 1, a.hdr);
-            for (int t = (kq > 2 ? kq - 2 : 0); t < kq; ++t) mbar_wait_drain(&bars->k_full[t & 1], (t >> 1) & 1, a.hdr);
-            for (int t = (kv_i > 2 ? kv_i - 2 : 0); t < kv_i; ++t) mbar_wait_drain(&bars->v_full[t & 1], (t >> 1) & 1, a.hdr);
+            for (int t = (g > 2 ? g - 2 : 0); t < g; ++t) {
+                mbar_wait_drain(&bars->k_full[t & 1], (t >> 1) & 1, a.hdr);
+                mbar_wait_drain(&bars->v_full[t & 1], (t >> 1) & 1, a.hdr);
+                if (BIAS == 1) mbar_wait_drain(&bars->bias_full[t & 1], (t >> 1) & 1, a.hdr);
+            }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
-            const uint32_t qb = sbase + kOffQ;
-            int g = 0, nk = 0, m = 0;
+            int g = 0, nk = 0;
+            int gt[2] = {0, 0}, mt[2] = {0, 0};
             bool ok = true;
-            auto issue_qk = [&](int gg, int n_left_after) -> bool {
-                const int s = gg & 1;
-                if (!mbar_wait(&bars->k_full[s], (gg >> 1) & 1, abort_flag, a.hdr)) return false;
-                JFA_TRACE_EV(fwd, 1, gg, 0);
-                tc_fence_after();
-                const uint32_t kb = sbase + kOffK + s * kTile;
-#pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                    mma_bf16_ss(tmem + s * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
-                mma_commit(&bars->s_full[s]);
-                JFA_TRACE_EV(fwd, 1, gg, 1);
-                mma_commit(&bars->k_empty[s]);
-                if (n_left_after == 0) mma_commit(&bars->q_free);  // last score MMA of the item
-                return true;
-            };
-            for (int r = 0; ok; ++r, ++m) {
+            for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
                 const Item w = load_item(a, idx);
-                if (w.n_tiles == 0) continue;
-                const int ob = m & 1;
-                const uint32_t tO = tmem + 256 + ob * 128;
+                if (w.n == 0) continue;
                 if (!mbar_wait(&bars->q_full, nk & 1, abort_flag, a.hdr)) { ok = false; break; }
                 ++nk;
-                // the epilogue of the item two turns back must be done with this O buffer
-                if (m >= 2 && !mbar_wait(&bars->o_free[ob], ((m >> 1) - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                const int n = w.n_tiles, g0 = g;
-                for (int t = 0; t < 2 && t < n && ok; ++t) ok = issue_qk(g0 + t, n - 1 - t);
-                for (int t = 0; ok && t < n; ++t, ++g) {
-                    const int s = g & 1;
-                    if (!mbar_wait(&bars->p_full, g & 1, abort_flag, a.hdr)) { ok = false; break; }
-                    JFA_TRACE_EV(fwd, 1, g, 2);
-                    if (!mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                    JFA_TRACE_EV(fwd, 1, g, 3);
+                // user of key/value step j: tile A while j < n_A, tile B while j < n_B
+                auto first_user = [&](int j) { return j < w.n_t[0] ? 0 : 1; };
+                auto last_user = [&](int j) { return j < w.n_t[1] ? 1 : 0; };
+                const int g0 = g;
+                // S_T = Q_T K_j^T into S_T; the K stage is released by its last user,
+                // Q by the item's last score MMA
+                auto issue_qk = [&](int t, int j) -> bool {
+                    const int gg = g0 + j, s = gg & 1;
+                    if (t == first_user(j)) {
+                        if (!mbar_wait(&bars->k_full[s], (gg >> 1) & 1, abort_flag, a.hdr)) return false;
+                        JFA_TRACE_EV(fwd, 1, gg, 0);
+                    }
                     tc_fence_after();
-                    const uint32_t vb = sbase + kOffV + s * kTile;
-                    const uint32_t tP = tmem + s * 128;  // P (bf16 pairs) over columns 0..63 of its S
+                    const uint32_t qb = sbase + kOffQ + t * kTile, kb = sbase + kOffK + s * kTile;
 #pragma unroll
-                    for (int k = 0; k < BN / 16; ++k)
-                        mma_bf16_ts(tO, tP + k * 8, mnmajor_desc(vb, k), idesc_pv,
-                                    (t > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&bars->v_empty[s]);
-                    mma_commit(&bars->pv_done);
-                    JFA_TRACE_EV(fwd, 1, g, 4);
-                    if (t + 2 < n) ok = issue_qk(g + 2, n - 1 - (t + 2));
+                    for (int k = 0; k < HD / 16; ++k)
+                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
+                    mma_commit(&bars->s_full[t]);
+                    if (t == last_user(j)) mma_commit(&bars->k_empty[s]);
+                    if (j == w.n - 1 && t == last_user(j)) mma_commit(&bars->q_free);
+                    return true;
+                };
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (w.n_t[t] > 0) ok = issue_qk(t, 0);
+                for (int j = 0; ok && j < w.n; ++j, ++g) {
+                    const int s = g & 1;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= w.n_t[t]) continue;
+                        if (!mbar_wait(&bars->p_full[t], gt[t] & 1, abort_flag, a.hdr)) { ok = false; break; }
+                        JFA_TRACE_EV(fwd, 1, g, 1 + 2 * t);
+                        // the epilogue of this tile's previous item must be done with O_T
+                        if (j == 0 && mt[t] > 0 &&
+                            !mbar_wait(&bars->o_free[t], (mt[t] - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                        if (t == first_user(j) &&
+                            !mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t vb = sbase + kOffV + s * kTile;
+                        const uint32_t tP = tmem + t * 128;   // P (bf16 pairs) over S_T: keys 16k.. at 8k + (k >= 4 ? 32 : 0)
+                        const uint32_t tO = tmem + 256 + t * 128;
+#pragma unroll
+                        for (int k = 0; k < BN / 16; ++k)
+                            mma_bf16_ts(tO, tP + k * 8 + (k >= 4 ? 32 : 0), mnmajor_desc(vb, k), idesc_pv,
+                                        (j > 0 || k > 0) ? 1u : 0u);
+                        mma_commit(&bars->pv_done[t]);
+                        if (t == last_user(j)) mma_commit(&bars->v_empty[s]);
+                        JFA_TRACE_EV(fwd, 1, g, 2 + 2 * t);
+                        ++gt[t];
+                        if (j == 0) ++mt[t];
+                        // S_T(j+1) overwrites P_T(j): issued after the P.V that reads it
+                        if (j + 1 < w.n_t[t]) ok = issue_qk(t, j + 1);
+                    }
                 }
             }
             // all issued MMAs retire before TMEM is released
@@ -283,28 +342,61 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------ softmax warps
+        // waits taken by a whole warp: the result is made warp-uniform, so that a
+        // timed-out wait ends the warp's loop on every lane together
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.hdr));
+        };
+        const int tt = warp >> 3;                // query tile: 0 = A, 1 = B
+        const int hf = (warp >> 2) & 1;          // half of the row: columns 64 hf .. +63
         const int wq = warp & 3;                 // TMEM lane quarter
-        const int grp = (warp - 2) >> 2;         // column group of S / O
         const int r_ = wq * 32 + lane;           // row within the tile
-        const int c0 = grp * CW;                 // first column of this thread's group
+        const int cb = hf * CW;                  // first column of this thread
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + tt * 128;
+        const uint32_t tO = tmem + lane_addr + 256 + tt * 128 + cb;
+        float* red = reinterpret_cast<float*>(smem + kOffRed);
+        float* lred = reinterpret_cast<float*>(smem + kOffLred);
+        // exchange with the warp that holds the other half of these rows: both
+        // write, arrive, and wait (bounded) for the other's arrival
+        uint64_t* pair_bar = &bars->pair[tt * 4 + wq];
+        int n_pair = 0;
+        auto pair_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar);
+            return wwait(pair_bar, (n_pair++) & 1);
+        };
         const float sc = a.scale * kLog2e;
+        const float2 sc2 = make_float2(sc, sc);
         const int C = (a.relpos_len - 1) >> 1;
-        int g = 0, m = 0;
+        int gt = 0, gkv = 0, mt = 0;   // steps of this tile, key tiles of the CTA, items of this tile
         bool ok = true;
-        const int tslot = (warp == 2 && lane == 0) ? 2 : ((warp == kThreads / 32 - 1 && lane == 0) ? 3 : -1);
-#define SM_EV(ev)                                     \
-    do {                                              \
-        if (tslot >= 0) JFA_TRACE_EV(fwd, tslot, g, ev); \
+        const int tslot = (warp == 0 && lane == 0) ? 2 : ((warp == 8 && lane == 0) ? 3 : -1);
+#define SM_EV(ev)                                      \
+    do {                                               \
+        if (tslot >= 0) JFA_TRACE_EV(fwd, tslot, gt, ev); \
     } while (0)
-        // Every softmax warp runs the same sequence of named barriers: a failed
-        // (timed-out) wait only sets the CTA's abort flag, and the loops are left
-        // right after a barrier, where all warps read the same flag.
-        for (int rr = 0; ok; ++rr, ++m) {
+        // Every wait is a bounded mbarrier wait (the pair exchange too), so a
+        // failed (timed-out) wait simply ends this warp's loop.
+        for (int rr = 0; ok; ++rr) {
             const int idx = item_of_turn(rr, cta, G);
             if (idx >= n_items) break;
             const Item w = load_item(a, idx);
-            const int i = w.row0 + r_;             // query index within the sequence
+            const int n = w.n_t[tt];
+            const int gkv_item = gkv;
+            gkv += w.n;
+            const int i = w.row0 + tt * BM + r_;   // query index within the sequence
+            if (n == 0) {
+                // rows that see no key (no keys at all, or causal with n_q > n_kv):
+                // zero output, LSE = -inf; the tensor core never touches this tile
+                if (i < w.nq) {
+                    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)(w.q0 + i) * a.H + w.h) * HD + cb;
+#pragma unroll
+                    for (int t = 0; t < CW; t += 8) *reinterpret_cast<uint4*>(orow + t) = make_uint4(0, 0, 0, 0);
+                    if (softmax && a.lse && hf == 0) a.lse[(int64_t)(w.q0 + i) * a.H + w.h] = -CUDART_INF_F;
+                }
+                continue;
+            }
             const int shift = w.nkv - w.nq;        // causal: key j visible iff j <= i + shift
             const float inv_n = w.nkv > 0 ? 1.0f / (float)w.nkv : 0.f;
             const int jmax_vis = a.causal ? min(w.nkv - 1, i + shift) : w.nkv - 1;
@@ -312,84 +404,95 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
                                           ? a.dense_off[w.b] + ((int64_t)w.h * w.nq + i) * w.nkv : 0;
-            const uint32_t tO = tmem + lane_addr + 256 + (m & 1) * 128 + c0;
-            float m_used = -CUDART_INF_F, l = 0.f;   // l: this group's partial sum
-            for (int j = 0; j < w.n_tiles; ++j, ++g) {
-                const int s = g & 1;
+            float m_used = -CUDART_INF_F, l = 0.f;
+            for (int j = 0; j < n; ++j, ++gt) {
                 SM_EV(0);
-                mbar_wait(&bars->s_full[s], (g >> 1) & 1, abort_flag, a.hdr);
+                if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
                 SM_EV(1);
                 tc_fence_after();
-                const int jc = j * BN + c0;          // key index of this group's column 0
-                float x[CW];
-                {
-                    uint32_t u[32];
-                    tmem_ld32(tmem + lane_addr + s * 128 + c0, u);
+                const int jc = j * BN;               // key index of column 0
+                const int gk = gkv_item + j, sk = gk & 1;   // key / value / bias stage
+                if (BIAS == 1 && !wwait(&bars->bias_full[sk], (gk >> 1) & 1)) { ok = false; break; }
+                const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;   // visible: [0, nvis)
+                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW);
+                // bias(i, jc + c) = table[lo + 127 - c], lo = i - jc - 127 + C: the run
+                // table[lo .. lo+127] as the window entries lo - w0 + 4q, or clamped
+                // reads of the table when the run leaves the table or the window
+                const int lo = i - jc - (BN - 1) + C;
+                const int wrel = BIAS == 1 ? lo - bias_window_start(w.row0, jc, C, a.bias4_stride) : 0;
+                const bool win_ok = BIAS == 1 && lo >= 0 && lo + (BN - 1) <= 2 * C && wrel >= 0 && wrel + BN - 4 < kWin;
+                const float4* win = reinterpret_cast<const float4*>(smem + kOffBias + sk * kWinBytes) + wrel;
+                // ---- pass 1: x = scale * s + bias (log2 units), masked to -inf, back
+                //      to TMEM over s; the maximum of this half of the row
+                float pm = -CUDART_INF_F;
+#pragma unroll 1
+                for (int c = 0; c < CW / 16; ++c) {
+                    const int cc = cb + c * 16;      // first column of the chunk
+                    float x[16];
+                    uint32_t* u = reinterpret_cast<uint32_t*>(x);
+                    tmem_ld16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
                     tmem_wait_ld();
+                    if (BIAS == 1) {
+                        float bb[16];   // bb[v] = bias(i, jc + cc + v) = table[lo + 127 - cc - v]
+                        if (win_ok) {
+                            // window entries lo - w0 + 124 - cc - 4q hold table[lo + 124 - cc - 4q + 0..3]
 #pragma unroll
-                    for (int t = 0; t < CW; ++t) x[t] = __uint_as_float(u[t]);
-                }
-                const int nvis = i < w.nq ? max(0, min(CW, jmax_vis - jc + 1)) : 0;  // visible: [0, nvis)
-                if (BIAS == 1) {
-                    // bias(i, jc + c) = table[i - jc - c + C] (log2(e)-scaled copy);
-                    // within a sequence |i - j| <= C, so only tiles past the rows
-                    // need the clamp
-                    const int hi = i - jc + C;
-                    const float2 sc2 = make_float2(sc, sc);
-                    float bb[CW];
-                    if (hi - (CW - 1) >= 0 && hi <= 2 * C) {
-                        const float* tb = tab4 + hi;   // tb[-c]
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 t4 = win[(BN - 4) - cc - 4 * q];
+                                bb[4 * q] = t4.w, bb[4 * q + 1] = t4.z, bb[4 * q + 2] = t4.y, bb[4 * q + 3] = t4.x;
+                            }
+                        } else {
+                            const int hi = lo + (BN - 1) - cc;
 #pragma unroll
-                        for (int c = 0; c < CW; ++c) bb[c] = __ldg(tb - c);
+                            for (int v = 0; v < 16; ++v) bb[v] = __ldg(tab4 + 4 * min(max(hi - v, 0), 2 * C));
+                        }
+#pragma unroll
+                        for (int v = 0; v < 16; v += 2) {
+                            const float2 r2 = fma2(make_float2(x[v], x[v + 1]), sc2, make_float2(bb[v], bb[v + 1]));
+                            x[v] = r2.x, x[v + 1] = r2.y;
+                        }
+                    } else if (BIAS == 2) {
+#pragma unroll
+                        for (int v = 0; v < 16; ++v)
+                            x[v] = fmaf(x[v], sc,
+                                        cc + v < nvis ? __bfloat162float(dense[dense_row + jc + cc + v]) * kLog2e : 0.f);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < CW; ++c) bb[c] = __ldg(tab4 + min(max(hi - c, 0), 2 * C));
+                        for (int v = 0; v < 16; v += 2) {
+                            const float2 r2 = mul2(make_float2(x[v], x[v + 1]), sc2);
+                            x[v] = r2.x, x[v + 1] = r2.y;
+                        }
                     }
+                    if (masked_half) {
 #pragma unroll
-                    for (int c = 0; c < CW; c += 2) {
-                        const float2 r2 = fma2(make_float2(x[c], x[c + 1]), sc2, make_float2(bb[c], bb[c + 1]));
-                        x[c] = r2.x, x[c + 1] = r2.y;
+                        for (int v = 0; v < 16; ++v) x[v] = cc + v < nvis ? x[v] : -CUDART_INF_F;
                     }
-                } else if (BIAS == 2) {
-#pragma unroll
-                    for (int c = 0; c < CW; ++c)
-                        x[c] = fmaf(x[c], sc, c < nvis ? __bfloat162float(dense[dense_row + jc + c]) * kLog2e : 0.f);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < CW; c += 2) {
-                        const float2 r2 = mul2(make_float2(x[c], x[c + 1]), make_float2(sc, sc));
-                        x[c] = r2.x, x[c + 1] = r2.y;
+                    if (softmax) {
+                        const float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
+                        const float m2 = max3(x[6], x[7], x[8]), m3 = max3(x[9], x[10], x[11]);
+                        const float m4 = max3(x[12], x[13], x[14]);
+                        pm = max3(pm, max3(m0, m1, m2), max3(m3, m4, x[15]));
                     }
+                    tmem_st16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
                 }
-                const bool masked_tile = __any_sync(0xffffffffu, nvis < CW);
-                if (masked_tile) {
-#pragma unroll
-                    for (int c = 0; c < CW; ++c) x[c] = c < nvis ? x[c] : -CUDART_INF_F;
-                }
-                float alpha = 1.f;
-                bool rescale = false;
+                SM_EV(2);
+                float ref = 0.f;
                 if (softmax) {
-                    float pm4[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) pm4[t] = fmaxf(x[2 * t], x[2 * t + 1]);
-#pragma unroll
-                    for (int c = 8; c < CW; c += 2) pm4[(c >> 1) & 3] = max3(pm4[(c >> 1) & 3], x[c], x[c + 1]);
-                    const float pm = max3(pm4[0], pm4[1], fmaxf(pm4[2], pm4[3]));
-                    red[(s * NG + grp) * 128 + r_] = pm;
-                    SM_EV(2);
-                    named_sync_softmax();
-                    SM_EV(3);
-                    if (*abort_flag) { ok = false; break; }
-                    float tmax = pm;
-#pragma unroll
-                    for (int q = 0; q < NG; ++q) tmax = fmaxf(tmax, red[(s * NG + q) * 128 + r_]);
+                    // row maximum of both halves (exchange buffer by step parity)
+                    float* rp = red + ((gt & 1) * 4 + tt * 2) * 128;
+                    rp[hf * 128 + r_] = pm;
+                    if (!pair_sync()) { ok = false; break; }
+                    pm = fmaxf(pm, rp[(hf ^ 1) * 128 + r_]);
                     // lazy rescale: keep the reference unless the row maximum grew by
                     // more than 8 (a factor 2^8).  With MXFP8 P the reference is an
                     // integer (ceil of the maximum, log2 units), so rescales are exact
                     // powers of two and the block quantisation of P does not depend on
                     // it; otherwise the maximum itself, so the largest weight is 1.
-                    const bool need = tmax > m_used + kRescaleThreshold;
-                    const float m_new = need ? (QP ? ceilf(tmax) : tmax) : m_used;
+                    // Both halves of a row take the same decision.
+                    float alpha = 1.f;
+                    bool rescale = false;
+                    const bool need = pm > m_used + kRescaleThreshold;
+                    const float m_new = need ? (QP ? ceilf(pm) : pm) : m_used;
                     if (need && m_used != -CUDART_INF_F) {
                         alpha = ex2(m_used - m_new);
                         rescale = true;
@@ -397,125 +500,156 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         l = 0.f;  // first visible key of this row
                     }
                     m_used = m_new;
-                }
-                // a rescale of O needs every earlier P.V of this item retired
-                if (softmax && __any_sync(0xffffffffu, rescale)) {
-                    if (g > 0) {
-                        mbar_wait(&bars->pv_done, (g - 1) & 1, abort_flag, a.hdr);
-                        tc_fence_after();
-                    }
-                    uint32_t u[32];
-                    tmem_ld32(tO, u);
-                    tmem_wait_ld();
+                    // a rescale of O needs every earlier P.V of this tile retired
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        if (j > 0) {
+                            if (!wwait(&bars->pv_done[tt], (gt - 1) & 1)) { ok = false; break; }
+                            tc_fence_after();
+#pragma unroll 1
+                            for (int c = 0; c < CW / 32; ++c) {
+                                uint32_t u[32];
+                                tmem_ld32(tO + c * 32, u);
+                                tmem_wait_ld();
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) u[t] = __float_as_uint(__uint_as_float(u[t]) * alpha);
-                    tmem_st32(tO, u);
-                    tmem_wait_st();
-                    l *= alpha;
-                }
-                SM_EV(4);
-                if (softmax) {
+                                for (int t = 0; t < 32; t += 2) {
+                                    const float2 r2 = mul2(make_float2(__uint_as_float(u[t]), __uint_as_float(u[t + 1])),
+                                                           make_float2(alpha, alpha));
+                                    u[t] = __float_as_uint(r2.x), u[t + 1] = __float_as_uint(r2.y);
+                                }
+                                tmem_st32(tO + c * 32, u);
+                            }
+                        }
+                        l *= alpha;
+                    }
                     // ex2(-inf) = 0 masks the invisible columns; a row with no visible
                     // key yet uses reference 0 so that -inf - ref stays -inf
-                    const float ref = m_used == -CUDART_INF_F ? 0.f : m_used;
-                    const float2 ref2 = make_float2(ref, ref);
-                    float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                    make_float2(0.f, 0.f)};
-#pragma unroll
-                    for (int c = 0; c < CW; c += 2) {
-                        const float2 y = sub2(make_float2(x[c], x[c + 1]), ref2);
-                        x[c] = ex2(y.x);
-                        x[c + 1] = ex2(y.y);
-                        ps[(c >> 1) & 3] = add2(ps[(c >> 1) & 3], make_float2(x[c], x[c + 1]));
-                    }
-                    const float2 s01 = add2(ps[0], ps[1]), s23 = add2(ps[2], ps[3]);
-                    const float2 s4 = add2(s01, s23);
-                    l += s4.x + s4.y;
-                    if (QP) mx::fake_quant32(x);  // the group's 32 keys are one MX block
-                } else {
-#pragma unroll
-                    for (int c = 0; c < CW; ++c) {
-                        const float s_nat = x[c] * (1.0f / kLog2e);
-                        x[c] = c < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
-                    }
-                    // P overwrites S columns other groups may still be loading
-                    named_sync_softmax();
+                    ref = m_used == -CUDART_INF_F ? 0.f : m_used;
                 }
-                // P row part (bf16 pairs) -> TMEM over the first 64 columns of its own
-                // S buffer: column c0/2 + t holds keys c0 + 2t (low half) and c0 + 2t + 1.
-                // Every group has loaded its S columns (they did so before the barrier
-                // above), and the next write to this buffer is QK_{j+2}, issued after
-                // P.V_j, which reads it.
+                tmem_wait_st();
+                SM_EV(3);
+                // ---- pass 2: P (bf16 pairs) -> TMEM over the first half of this
+                //      thread's own S columns: keys cb + 16c .. +15 to columns
+                //      cb + 8c .. +7, which hold x of chunks already read
                 {
-                    uint32_t pw[16];
+                    const float2 ref2 = make_float2(ref, ref);
+                    float2 ps = make_float2(0.f, 0.f), ps2 = make_float2(0.f, 0.f);
+                    float qbuf[QP ? 32 : 1];   // MXFP8: one 32-key block
+                    (void)qbuf;
+#pragma unroll 1
+                    for (int c = 0; c < CW / 16; ++c) {
+                        const int cc = cb + c * 16;
+                        float x[16];
+                        uint32_t* u = reinterpret_cast<uint32_t*>(x);
+                        tmem_ld16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
+                        tmem_wait_ld();
+                        if (softmax) {
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) pw[t] = pack_bf16(x[2 * t], x[2 * t + 1]);
-                    tmem_st16(tmem + lane_addr + s * 128 + (c0 >> 1), pw);
+                            for (int v = 0; v < 16; v += 2) {
+                                const float2 y = sub2(make_float2(x[v], x[v + 1]), ref2);
+                                x[v] = ex2(y.x);
+                                x[v + 1] = ex2(y.y);
+                                if (v & 2) ps2 = add2(ps2, make_float2(x[v], x[v + 1]));
+                                else ps = add2(ps, make_float2(x[v], x[v + 1]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 16; ++v) {
+                                const float s_nat = x[v] * (1.0f / kLog2e);
+                                x[v] = cc + v < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
+                            }
+                        }
+                        if (QP) {
+                            // the 32 keys of an MX block span two chunks: quantise once
+                            // both halves are in (pairs of chunks, even then odd)
+                            if ((c & 1) == 0) {
+#pragma unroll
+                                for (int v = 0; v < 16; ++v) qbuf[v] = x[v];
+                                continue;
+                            }
+#pragma unroll
+                            for (int v = 0; v < 16; ++v) qbuf[16 + v] = x[v];
+                            mx::fake_quant32(qbuf);
+                            uint32_t pw[16];
+#pragma unroll
+                            for (int t = 0; t < 16; ++t) pw[t] = pack_bf16(qbuf[2 * t], qbuf[2 * t + 1]);
+                            tmem_st16(tS + cb + (c - 1) * 8, pw);
+                        } else {
+                            uint32_t pw[8];
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) pw[t] = pack_bf16(x[2 * t], x[2 * t + 1]);
+                            tmem_st8(tS + cb + c * 8, pw);
+                        }
+                    }
                     tmem_wait_st();
+                    const float2 s4 = add2(ps, ps2);
+                    l += s4.x + s4.y;
                 }
-                // value rows past the sequence end (neighbour data) must not reach P.V
-                const int nvalid = w.nkv - j * BN;
-                if (nvalid < BN) {  // same for the whole CTA
-                    mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr);
-                    if (r_ >= nvalid && (grp & 1) == 0) {  // groups 0 and 2 clear the two boxes
-                        uint8_t* vrow = smem + kOffV + s * kTile + (grp >> 1) * kBox + r_ * 128;
+                // value rows past the sequence end (neighbour data) must not reach P.V;
+                // the first tile that uses this key tile clears them before its P is
+                // released (both tiles read the same V stage)
+                const int nvalid = w.nkv - jc;
+                const int clearer = (j < w.n_t[0]) ? 0 : 1;
+                if (nvalid < BN && tt == clearer) {  // same for the whole tile
+                    if (!wwait(&bars->v_full[sk], (gk >> 1) & 1)) { ok = false; break; }
+                    if (r_ >= nvalid) {
+                        uint8_t* vrow = smem + kOffV + sk * kTile + hf * kBox + r_ * 128;
                         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
                         for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
                     }
                 }
+                SM_EV(4);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full);
-                SM_EV(5);
+                if (lane == 0) mbar_arrive(&bars->p_full[tt]);
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue
-            if (w.n_tiles > 0) mbar_wait(&bars->pv_done, (g - 1) & 1, abort_flag, a.hdr);
-            SM_EV(6);
-            lred[((m & 1) * NG + grp) * 128 + r_] = l;
-            named_sync_softmax();
-            SM_EV(7);
-            if (*abort_flag) { ok = false; break; }
-            float l_row = 0.f;
-#pragma unroll
-            for (int q = 0; q < NG; ++q) l_row += lred[((m & 1) * NG + q) * 128 + r_];
+            if (!wwait(&bars->pv_done[tt], (gt - 1) & 1)) { ok = false; break; }
+            SM_EV(5);
             tc_fence_after();
-            const float inv = softmax ? (l_row > 0.f ? 1.f / l_row : 0.f) : 1.f;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)(w.q0 + i) * a.H + w.h) * HD + c0;
-            uint32_t u[32];
-            if (w.n_tiles > 0) {
-                tmem_ld32(tO, u);
-                tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int t = 0; t < 32; ++t) u[t] = 0u;
+            float l_row = l;
+            if (softmax) {
+                float* lp = lred + ((mt & 1) * 4 + tt * 2) * 128;
+                lp[hf * 128 + r_] = l;
+                if (!pair_sync()) { ok = false; break; }
+                l_row += lp[(hf ^ 1) * 128 + r_];
             }
-            // O buffer free for the item two turns ahead
+            ++mt;
+            const float inv = softmax ? (l_row > 0.f ? 1.f / l_row : 0.f) : 1.f;
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)(w.q0 + i) * a.H + w.h) * HD + cb;
+#pragma unroll 1
+            for (int c = 0; c < CW / 32; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tO + c * 32, u);
+                tmem_wait_ld();
+                if (i < w.nq) {
+#pragma unroll
+                    for (int t = 0; t < 32; t += 8) {
+                        uint4 wv;
+                        wv.x = pack_bf16(__uint_as_float(u[t + 0]) * inv, __uint_as_float(u[t + 1]) * inv);
+                        wv.y = pack_bf16(__uint_as_float(u[t + 2]) * inv, __uint_as_float(u[t + 3]) * inv);
+                        wv.z = pack_bf16(__uint_as_float(u[t + 4]) * inv, __uint_as_float(u[t + 5]) * inv);
+                        wv.w = pack_bf16(__uint_as_float(u[t + 6]) * inv, __uint_as_float(u[t + 7]) * inv);
+                        *reinterpret_cast<uint4*>(orow + c * 32 + t) = wv;
+                    }
+                }
+            }
+            // O_T free for this tile's next item
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->o_free[m & 1]);
-            if (i < w.nq) {
-#pragma unroll
-                for (int t = 0; t < 32; t += 8) {
-                    uint4 wv;
-                    wv.x = pack_bf16(__uint_as_float(u[t + 0]) * inv, __uint_as_float(u[t + 1]) * inv);
-                    wv.y = pack_bf16(__uint_as_float(u[t + 2]) * inv, __uint_as_float(u[t + 3]) * inv);
-                    wv.z = pack_bf16(__uint_as_float(u[t + 4]) * inv, __uint_as_float(u[t + 5]) * inv);
-                    wv.w = pack_bf16(__uint_as_float(u[t + 6]) * inv, __uint_as_float(u[t + 7]) * inv);
-                    *reinterpret_cast<uint4*>(orow + t) = wv;
-                }
-                if (softmax && grp == 0 && a.lse)
-                    a.lse[(int64_t)(w.q0 + i) * a.H + w.h] =
-                        l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
-            }
+            if (lane == 0) mbar_arrive(&bars->o_free[tt]);
+            if (softmax && hf == 0 && i < w.nq && a.lse)
+                a.lse[(int64_t)(w.q0 + i) * a.H + w.h] =
+                    l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
+            SM_EV(6);
         }
 #undef SM_EV
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -568,7 +702,7 @@ cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quan
         return cudaErrorInvalidValue;
     P.a = a;
     const int smem = (int)kSmemBytes;
-    const int64_t items_bound = pairs_bound(p.batch, p.max_q_len, p.total_q, BM) * p.heads;
+    const int64_t items_bound = pairs_bound(p.batch, p.max_q_len, p.total_q, kBlockRows) * p.heads;
     if (items_bound <= 0) return cudaSuccess;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
