@@ -358,29 +358,19 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // Round-to-nearest-even to bf16 on the integer pipe (finite inputs): add
 // 0x7FFF plus the lowest kept bit, keep the upper 16 bits; two results are
-// packed with one byte permute.  Used for the P / dS operands, which keeps
-// the conversion off the pipe that also evaluates exp2.
-#ifndef JFA_PACK_ALU
-#define JFA_PACK_ALU 0
-#endif
-__device__ __forceinline__ uint32_t pack_bf16_p(float lo, float hi) {
-#if JFA_PACK_ALU
+// packed with one byte permute.  Keeps the conversion of P off the pipe that
+// also evaluates exp2.
+__device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
     uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
     a += 0x7FFFu + ((a >> 16) & 1u);
     b += 0x7FFFu + ((b >> 16) & 1u);
     return __byte_perm(a, b, 0x7632);
-#else
-    return pack_bf16(lo, hi);
-#endif
 }
 
 // 2^y on the FMA pipe for y <= 8 (Cody-Waite style split y = n + f with
 // n = round(y), f in [-0.5, 0.5]; 2^f by a cubic fitted here for minimax
 // relative error, max 7.5e-5, well below bf16's 2^-9; 2^n added to the
 // exponent bits).  Inputs below -126 give a value below 2^-125.
-#ifndef JFA_EXP2_POLY_MOD
-#define JFA_EXP2_POLY_MOD 0
-#endif
 __device__ __forceinline__ float exp2_fma(float y) {
     y = fmaxf(y, -126.0f);
     const float t = y + 12582912.0f;  // 1.5 * 2^23: the low mantissa bits of t hold round(y)
@@ -403,16 +393,6 @@ __device__ __forceinline__ float2 exp2_fma2(float2 y) {
     p = fma2(p, f, make_float2(0.9999282f, 0.9999282f));
     return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
                        __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// exp2 of element c of a row: every JFA_EXP2_POLY_MOD-th element on the FMA
-// pipe, the rest on the MUFU.
-template <int c>
-__device__ __forceinline__ float exp2_mixed(float y) {
-#if JFA_EXP2_POLY_MOD > 0
-    if ((c % JFA_EXP2_POLY_MOD) == JFA_EXP2_POLY_MOD - 1) return exp2_fma(y);
-#endif
-    return ex2(y);
 }
 
 }  // namespace sm100

@@ -119,10 +119,10 @@ __device__ __forceinline__ void store_half_chunk_bits(uint8_t* tile, int r, int 
     for (int u = 0; u < 2; ++u) {
         const int ch = (c16 & 3) * 2 + u;
         uint4 w;
-        w.x = pack_bf16_p(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
-        w.y = pack_bf16_p(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
-        w.z = pack_bf16_p(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
-        w.w = pack_bf16_p(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
+        w.x = pack_bf16(__uint_as_float(v[8 * u + 0]), __uint_as_float(v[8 * u + 1]));
+        w.y = pack_bf16(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3]));
+        w.z = pack_bf16(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5]));
+        w.w = pack_bf16(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]));
         *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) = w;
     }
 }

@@ -425,13 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 // ---- pass 1: x = scale * s + bias (log2 units), masked to -inf, back
                 //      to TMEM over s; the maximum of this half of the row
                 float pm = -CUDART_INF_F;
-#pragma unroll 1
+                // chunk c + 1 is loaded while chunk c is worked on (a wait covers
+                // every earlier load, so the next chunk's load goes out after it)
+                uint32_t ub[2][16];
+                tmem_ld16(tS + cb, ub[0]);
+#pragma unroll
                 for (int c = 0; c < CW / 16; ++c) {
                     const int cc = cb + c * 16;      // first column of the chunk
-                    float x[16];
-                    uint32_t* u = reinterpret_cast<uint32_t*>(x);
-                    tmem_ld16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
                     tmem_wait_ld();
+                    if (c + 1 < CW / 16) tmem_ld16(tS + cc + 16, ub[(c + 1) & 1]);
+                    float* x = reinterpret_cast<float*>(ub[c & 1]);
+                    uint32_t* u = ub[c & 1];
                     if (BIAS == 1) {
                         float bb[16];   // bb[v] = bias(i, jc + cc + v) = table[lo + 127 - cc - v]
                         if (win_ok) {
@@ -535,13 +539,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     float2 ps = make_float2(0.f, 0.f), ps2 = make_float2(0.f, 0.f);
                     float qbuf[QP ? 32 : 1];   // MXFP8: one 32-key block
                     (void)qbuf;
-#pragma unroll 1
+                    uint32_t ub[2][16];
+                    tmem_ld16(tS + cb, ub[0]);
+#pragma unroll
                     for (int c = 0; c < CW / 16; ++c) {
                         const int cc = cb + c * 16;
-                        float x[16];
-                        uint32_t* u = reinterpret_cast<uint32_t*>(x);
-                        tmem_ld16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
                         tmem_wait_ld();
+                        if (c + 1 < CW / 16) tmem_ld16(tS + cc + 16, ub[(c + 1) & 1]);
+                        float* x = reinterpret_cast<float*>(ub[c & 1]);
                         if (softmax) {
 #pragma unroll
                             for (int v = 0; v < 16; v += 2) {
