@@ -243,18 +243,25 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
     const bool tc = use_tc(p, act, 1);
     const int qtile = tc ? tc_fwd_tile() : kSimtFwdTile;
     const int ktile = tc ? tc_bwd_tile() : kSimtBwdTile;
-    cudaError_t e = build_schedule(p, q_offsets, kv_offsets, causal, 0, qtile, hdr,
-                                   reinterpret_cast<int64_t*>(ws + L.dense_off),
-                                   reinterpret_cast<int2*>(ws + L.pair_bt),
-                                   reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
-                                   reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
-                                   &hdr->pair_count, 1, nullptr, nullptr, st);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule");
-    e = build_schedule(p, q_offsets, kv_offsets, causal, 1, ktile, hdr, nullptr,
+    // the CUDA-core backward walks both schedules; the tensor-core backward only
+    // the key-tile one (its first build resets the error word and, for a dense
+    // bias, writes the sequences' bias offsets)
+    cudaError_t e = cudaSuccess;
+    if (!tc) {
+        e = build_schedule(p, q_offsets, kv_offsets, causal, 0, qtile, hdr,
+                           reinterpret_cast<int64_t*>(ws + L.dense_off),
+                           reinterpret_cast<int2*>(ws + L.pair_bt),
+                           reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
+                           reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
+                           &hdr->pair_count, 1, nullptr, nullptr, st);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule");
+    }
+    e = build_schedule(p, q_offsets, kv_offsets, causal, 1, ktile, hdr,
+                       tc ? reinterpret_cast<int64_t*>(ws + L.dense_off) : nullptr,
                        reinterpret_cast<int2*>(ws + L.kv_pair_bt),
                        reinterpret_cast<int64_t*>(ws + L.kv_pair_cost), L.pairs_max_kv,
                        reinterpret_cast<int4*>(ws + L.kv_items), &hdr->kv_item_count,
-                       &hdr->kv_pair_count, 0, reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp),
+                       &hdr->kv_pair_count, tc ? 1 : 0, reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp),
                        reinterpret_cast<int64_t*>(ws + L.kv_seq_start), st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     AttnArgs a{};
