@@ -367,33 +367,5 @@ __device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
     return __byte_perm(a, b, 0x7632);
 }
 
-// 2^y on the FMA pipe for y <= 8 (Cody-Waite style split y = n + f with
-// n = round(y), f in [-0.5, 0.5]; 2^f by a cubic fitted here for minimax
-// relative error, max 7.5e-5, well below bf16's 2^-9; 2^n added to the
-// exponent bits).  Inputs below -126 give a value below 2^-125.
-__device__ __forceinline__ float exp2_fma(float y) {
-    y = fmaxf(y, -126.0f);
-    const float t = y + 12582912.0f;  // 1.5 * 2^23: the low mantissa bits of t hold round(y)
-    const float n = t - 12582912.0f;
-    const float f = y - n;
-    const float p = fmaf(fmaf(fmaf(0.05517098f, f, 0.24260971f), f, 0.69326097f), f, 0.9999282f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
-// Two lanes of exp2_fma with paired fp32 arithmetic (y >= -126 after the
-// clamp; the scale by 2^n is an integer add to the exponent field).
-__device__ __forceinline__ float2 exp2_fma2(float2 y) {
-    y.x = fmaxf(y.x, -126.0f);
-    y.y = fmaxf(y.y, -126.0f);
-    const float2 magic = make_float2(12582912.0f, 12582912.0f);
-    const float2 t = add2(y, magic);
-    const float2 f = sub2(y, sub2(t, magic));
-    float2 p = fma2(make_float2(0.05517098f, 0.05517098f), f, make_float2(0.24260971f, 0.24260971f));
-    p = fma2(p, f, make_float2(0.69326097f, 0.69326097f));
-    p = fma2(p, f, make_float2(0.9999282f, 0.9999282f));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 }  // namespace sm100
 }  // namespace jfa
