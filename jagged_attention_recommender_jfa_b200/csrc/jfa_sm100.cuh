@@ -294,6 +294,23 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo
     return d;
 }
 
+// The same descriptor split in two 32-bit words, so that an MMA issue loop
+// builds it with one add: the upper word (stride, version, swizzle) is a
+// constant, and the lower word is (start >> 4) | (LBO >> 4) << 16, where a K
+// step only adds to the start field (shared-memory addresses stay below
+// 256 KB, so the 14-bit field never carries).
+__host__ __device__ constexpr uint32_t sw128_desc_hi(uint32_t sbo) {
+    return ((sbo >> 4) & 0x3FFF) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t start, uint32_t lbo) {
+    return ((start & 0x3FFFF) >> 4) | (((lbo >> 4) & 0x3FFF) << 16);
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t lo, uint32_t hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
 //   a_mn / b_mn: 1 if the operand is MN-major (else K-major)
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {

@@ -9,7 +9,7 @@
 //   tc_bwd_kernel    one CTA per (sequence, head, 128-key tile) work item of
 //                    the key-tile schedule.  K and V of the tile stay in
 //                    shared memory; the query tiles that can see the keys
-//                    stream through (Q single-, dO double-buffered):
+//                    stream through (Q and dO in a three-buffer ring):
 //                      S^T  = K Q^T,  dP^T = V dO^T           (TMEM, fp32)
 //                      P^T  = exp2(S^T - LSE), dS^T = P^T (dP^T - D)
 //                             (or GDPA: act(S)/n_kv, dP act'(S)/n_kv)
@@ -22,9 +22,10 @@
 //                             covers 32 consecutive d of one query row)
 //                      dV  += P^T dO    (A operand from TMEM)
 //                    The tensor core runs dK, dQ^T, dV of tile t and then
-//                    S^T, dP^T of tile t+1 back to back: Q(t+1) loads while
-//                    dQ^T and dV run, dO(t+1) was loaded a tile earlier, and
-//                    dP^T(t+1) waits only for the read-out of dQ^T(t).
+//                    S^T, dP^T of tile t+1 back to back: dQ^T(t) is read out
+//                    while dV runs, and Q / dO come from a three-buffer ring
+//                    that fetches Q(t+1) two tiles ahead and dO(t+1) once
+//                    dK(t) has retired (both warmed in L2 a tile earlier).
 //   tc_bwd_dq_finalize  dQ = bf16(scale * accumulator).
 //
 // Warp roles: warp 0 TMA, warp 1 MMA, warps 2..17 score warps in four groups
@@ -54,9 +55,12 @@ constexpr uint32_t kBox = 128 * 128;
 constexpr uint32_t kTile = 2 * kBox;
 constexpr uint32_t kOffK = 0;
 constexpr uint32_t kOffV = kOffK + kTile;
-constexpr uint32_t kOffQ = kOffV + kTile;
-constexpr uint32_t kOffDO = kOffQ + kTile;        // two buffers
-constexpr uint32_t kOffDST = kOffDO + 2 * kTile;
+// Q and dO of the query tiles share a ring of three tile buffers, filled in
+// the order Q(0), dO(0), Q(1), dO(1), ...: load n (Q(n/2) for even n, dO(n/2)
+// for odd n) goes to buffer n % 3, once load n - 3 has been consumed -- so
+// Q(t) is fetched as soon as dV(t-2) has retired and dO(t) once dK(t-1) has.
+constexpr uint32_t kOffQD = kOffV + kTile;        // three buffers
+constexpr uint32_t kOffDST = kOffQD + 3 * kTile;
 constexpr uint32_t kOffBar = kOffDST + kTile;     // 196608
 constexpr uint32_t kOffRow = kOffBar + 256;       // lse2[2][128], D[2][128] (double-buffered)
 // Relative-position bias window of a query tile, 2 stages: 272 entries of the
@@ -71,8 +75,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
     uint64_t kv_full;
-    uint64_t q_full, q_empty;
-    uint64_t do_full[2], do_empty[2];
+    uint64_t buf_full[3], buf_empty[3];   // the Q / dO ring
     uint64_t s_full;
     uint64_t ds_full;       // 16 score warps
     uint64_t dq_full;
@@ -102,13 +105,19 @@ __device__ __forceinline__ int bias_window_start(int qb0, int j0, int C, int str
     return min(max(qb0 - j0 - (BN - 1) + C, 0), stride - kWin);
 }
 
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
-    return smem_desc_sw128(tile_base + (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32u, 16u,
-                           1024u);
+// Shared-memory operand descriptors of a 128 x 128 bf16 tile (two 64-column
+// 128B-swizzled boxes) at K step k (16 elements), from the tile's precomputed
+// lower word: K-major (rows = M or N, 64 K per box row) steps 32 B within a
+// row and kBox to the next box; MN-major (rows = K) steps 16 rows = 2048 B,
+// its two 64-element halves kBox apart (LBO).
+constexpr uint32_t kDescHi = sw128_desc_hi(1024u);
+__device__ __forceinline__ uint32_t kmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, 16u); }
+__device__ __forceinline__ uint32_t mnmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, kBox); }
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t lo, int k) {
+    return sw128_desc(lo + (uint32_t)(k >> 2) * (kBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
 }
-
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
-    return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t lo, int k) {
+    return sw128_desc(lo + (uint32_t)k * 128u, kDescHi);
 }
 
 // Stores 16 fp32 values (bit patterns) as bf16: columns 16*c16 .. +15 of row r
@@ -160,11 +169,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_empty, 1);
+        for (int s3 = 0; s3 < 3; ++s3) {
+            mbar_init(&bars->buf_full[s3], 1);
+            mbar_init(&bars->buf_empty[s3], 1);
+        }
         for (int s2 = 0; s2 < 2; ++s2) {
-            mbar_init(&bars->do_full[s2], 1);
-            mbar_init(&bars->do_empty[s2], 1);
             mbar_init(&bars->rows_full[s2], 4);
             mbar_init(&bars->rows_free[s2], NG * 4);
             mbar_init(&bars->bias_full[s2], 1);
@@ -203,60 +212,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, h, k0 + j0);
             tma_load_3d(smem + kOffV, &P.tm_v, &bars->kv_full, 0, h, k0 + j0);
             tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->kv_full, 64, h, k0 + j0);
-            // Q(t) and, with a relative-position bias, the tile's bias window; the
-            // window's stage (t & 1) was last read for tile t-2, whose score
-            // phase ended before dK(t-2) and so before the q_empty that lets
-            // Q(t) in
-            auto load_q = [&](int t) {
+            // load n of the ring: Q(n/2) (with a relative-position bias also the
+            // tile's bias window) or dO(n/2); the window's stage (t & 1) was last
+            // read for tile t-2, whose score phase ended before dV(t-2), which
+            // frees the buffer that Q(t) goes to
+            const int n_loads = 2 * nt;
+            int issued = 0;
+            for (int n = 0; n < n_loads; ++n) {
+                const int bf = n % 3, use = n / 3, t = n >> 1;
+                if (use > 0 && !mbar_wait(&bars->buf_empty[bf], (use - 1) & 1, abort_flag, a.hdr)) break;
+                JFA_TRACE_EV(bwd, 0, t, n & 1);
                 const int z = q0 + i_start + t * BM;
-                mbar_arrive_expect_tx(&bars->q_full, kTile);
-                tma_load_3d(smem + kOffQ, &P.tm_q, &bars->q_full, 0, h, z);
-                tma_load_3d(smem + kOffQ + kBox, &P.tm_q, &bars->q_full, 64, h, z);
-                if (BIAS == 1) {
+                uint8_t* dst = smem + kOffQD + bf * kTile;
+                const CUtensorMap* map = (n & 1) ? &P.tm_do : &P.tm_q;
+                mbar_arrive_expect_tx(&bars->buf_full[bf], kTile);
+                tma_load_3d(dst, map, &bars->buf_full[bf], 0, h, z);
+                tma_load_3d(dst + kBox, map, &bars->buf_full[bf], 64, h, z);
+                if ((n & 1) == 0 && t + 1 < nt) {  // warm L2 for the next tile's Q and dO
+                    tma_prefetch_l2_3d(&P.tm_q, 0, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_q, 64, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_do, 0, h, z + BM);
+                    tma_prefetch_l2_3d(&P.tm_do, 64, h, z + BM);
+                }
+                if (BIAS == 1 && (n & 1) == 0) {
                     const int C = (a.relpos_len - 1) >> 1;
                     const int w0 = bias_window_start(i_start + t * BM, j0, C, a.bias4_stride);
                     const float* src = a.bias4 + 4 * ((int64_t)h * a.bias4_stride + w0);
                     mbar_arrive_expect_tx(&bars->bias_full[t & 1], kWinBytes);
                     bulk_load(smem + kOffWin + (t & 1) * kWinBytes, src, kWinBytes, &bars->bias_full[t & 1]);
                 }
-            };
-            auto load_do = [&](int t) {
-                const int z = q0 + i_start + t * BM;
-                uint8_t* dst = smem + kOffDO + (t & 1) * kTile;
-                mbar_arrive_expect_tx(&bars->do_full[t & 1], kTile);
-                tma_load_3d(dst, &P.tm_do, &bars->do_full[t & 1], 0, h, z);
-                tma_load_3d(dst + kBox, &P.tm_do, &bars->do_full[t & 1], 64, h, z);
-            };
-            load_q(0);
-            load_do(0);
-            if (nt > 1) load_do(1);
-            int issued_q = 1, issued_do = nt > 1 ? 2 : 1;
-            for (int t = 0; t + 1 < nt; ++t) {
-                if (!mbar_wait(&bars->q_empty, t & 1, abort_flag, a.hdr)) break;
-                JFA_TRACE_EV(bwd, 0, t + 1, 0);
-                load_q(t + 1);
-                issued_q = t + 2;
-                if (t + 2 < nt) {
-                    tma_prefetch_l2_3d(&P.tm_q, 0, h, q0 + i_start + (t + 2) * BM);
-                    tma_prefetch_l2_3d(&P.tm_q, 64, h, q0 + i_start + (t + 2) * BM);
-                    if (!mbar_wait(&bars->do_empty[t & 1], (t >> 1) & 1, abort_flag, a.hdr)) break;
-                    JFA_TRACE_EV(bwd, 0, t + 2, 1);
-                    load_do(t + 2);
-                    issued_do = t + 3;
-                    if (t + 3 < nt) {
-                        tma_prefetch_l2_3d(&P.tm_do, 0, h, q0 + i_start + (t + 3) * BM);
-                        tma_prefetch_l2_3d(&P.tm_do, 64, h, q0 + i_start + (t + 3) * BM);
-                    }
-                }
+                issued = n + 1;
             }
             // never leave the CTA with copies in flight
             mbar_wait_drain(&bars->kv_full, 0, a.hdr);
-            mbar_wait_drain(&bars->q_full, (issued_q - 1) & 1, a.hdr);
+            for (int n = issued > 3 ? issued - 3 : 0; n < issued; ++n)
+                mbar_wait_drain(&bars->buf_full[n % 3], (n / 3) & 1, a.hdr);
             if (BIAS == 1)
-                for (int t = issued_q > 2 ? issued_q - 2 : 0; t < issued_q; ++t)
-                    mbar_wait_drain(&bars->bias_full[t & 1], (t >> 1) & 1, a.hdr);
-            for (int t = issued_do > 2 ? issued_do - 2 : 0; t < issued_do; ++t)
-                mbar_wait_drain(&bars->do_full[t & 1], (t >> 1) & 1, a.hdr);
+                for (int t = 0; t < (issued + 1) / 2; ++t)
+                    if (t + 2 >= (issued + 1) / 2) mbar_wait_drain(&bars->bias_full[t & 1], (t >> 1) & 1, a.hdr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -265,25 +258,30 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             constexpr uint32_t idesc_nn = idesc_bf16(128, 128, 0, 1);  // B MN-major
             constexpr uint32_t idesc_tn = idesc_bf16(128, 128, 1, 1);  // A and B MN-major
             const uint32_t tdV = tmem, tdK = tmem + 128, tS = tmem + 256, tdP = tmem + 384;
-            const uint32_t kb = sbase + kOffK, vb = sbase + kOffV, qb = sbase + kOffQ,
-                           dob = sbase + kOffDO, dsb = sbase + kOffDST;
-            auto issue_s = [&]() {  // S^T = K Q^T
+            // descriptor lower words of every operand tile, computed once
+            const uint32_t kK = kmajor_lo(sbase + kOffK), kM = mnmajor_lo(sbase + kOffK);
+            const uint32_t vK = kmajor_lo(sbase + kOffV);
+            // the ring's buffers, K-major (S^T, dP^T) and MN-major (dK, dV) views
+            auto ringK = [&](int bf) { return kmajor_lo(sbase + kOffQD + (uint32_t)bf * kTile); };
+            auto ringM = [&](int bf) { return mnmajor_lo(sbase + kOffQD + (uint32_t)bf * kTile); };
+            const uint32_t dsK = kmajor_lo(sbase + kOffDST), dsM = mnmajor_lo(sbase + kOffDST);
+            auto issue_s = [&](int t) {  // S^T = K Q^T, Q(t) = load 2t
+                const uint32_t q = ringK((2 * t) % 3);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
-                    mma_bf16_ss(tS, kmajor_desc(kb, k), kmajor_desc(qb, k), idesc_nt, k > 0 ? 1u : 0u);
+                    mma_bf16_ss(tS, kmajor_desc(kK, k), kmajor_desc(q, k), idesc_nt, k > 0 ? 1u : 0u);
             };
-            auto issue_dp = [&](int t) {  // dP^T = V dO^T
-                const uint32_t d = dob + (uint32_t)(t & 1) * kTile;
+            auto issue_dp = [&](int t) {  // dP^T = V dO^T, dO(t) = load 2t + 1
+                const uint32_t d = ringK((2 * t + 1) % 3);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
-                    mma_bf16_ss(tdP, kmajor_desc(vb, k), kmajor_desc(d, k), idesc_nt, k > 0 ? 1u : 0u);
+                    mma_bf16_ss(tdP, kmajor_desc(vK, k), kmajor_desc(d, k), idesc_nt, k > 0 ? 1u : 0u);
             };
-            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.hdr) &&
-                      mbar_wait(&bars->q_full, 0, abort_flag, a.hdr) &&
-                      mbar_wait(&bars->do_full[0], 0, abort_flag, a.hdr);
+            auto wait_load = [&](int n) { return mbar_wait(&bars->buf_full[n % 3], (n / 3) & 1, abort_flag, a.hdr); };
+            bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.hdr) && wait_load(0) && wait_load(1);
             if (ok) {
                 tc_fence_after();
-                issue_s();
+                issue_s(0);
                 issue_dp(0);
                 mma_commit(&bars->s_full);
             }
@@ -292,33 +290,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 JFA_TRACE_EV(bwd, 1, t, 0);
                 tc_fence_after();
                 // dK += dS^T Q   (A = dS^T K-major in smem, B = Q MN-major)
+                {
+                    const uint32_t qM = ringM((2 * t) % 3);
 #pragma unroll
-                for (int k = 0; k < BM / 16; ++k)
-                    mma_bf16_ss(tdK, kmajor_desc(dsb, k), mnmajor_desc(qb, k), idesc_nn,
-                                (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&bars->q_empty);
+                    for (int k = 0; k < BM / 16; ++k)
+                        mma_bf16_ss(tdK, kmajor_desc(dsK, k), mnmajor_desc(qM, k), idesc_nn,
+                                    (t > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&bars->buf_empty[(2 * t) % 3]);
                 // dQ^T = K^T dS^T over the dP^T columns (A = K, B = dS^T, both MN-major)
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
-                    mma_bf16_ss(tdP, mnmajor_desc(kb, k), mnmajor_desc(dsb, k), idesc_tn, k > 0 ? 1u : 0u);
+                    mma_bf16_ss(tdP, mnmajor_desc(kM, k), mnmajor_desc(dsM, k), idesc_tn, k > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
                 // dV += P^T dO: A = P^T from TMEM, query step k (16 queries) of group
                 // k/2 in columns 32*(k/2) + 8*(k%2) of the S^T region
-                const uint32_t d = dob + (uint32_t)(t & 1) * kTile;
+                const uint32_t d = ringM((2 * t + 1) % 3);
 #pragma unroll
                 for (int k = 0; k < BM / 16; ++k)
                     mma_bf16_ts(tdV, tS + 32 * (k >> 1) + 8 * (k & 1), mnmajor_desc(d, k), idesc_nn,
                                 (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&bars->do_empty[t & 1]);
+                mma_commit(&bars->buf_empty[(2 * t + 1) % 3]);
                 JFA_TRACE_EV(bwd, 1, t, 1);
                 if (t + 1 < nt) {
                     // S^T(t+1) overwrites P^T(t): issued after dV, which reads it
-                    if (!mbar_wait(&bars->q_full, (t + 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    if (!wait_load(2 * t + 2)) { ok = false; break; }
                     JFA_TRACE_EV(bwd, 1, t, 2);
                     tc_fence_after();
-                    issue_s();
-                    if (!mbar_wait(&bars->do_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag, a.hdr) ||
-                        !mbar_wait(&bars->dq_empty, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                    issue_s(t + 1);
+                    if (!wait_load(2 * t + 3) || !mbar_wait(&bars->dq_empty, t & 1, abort_flag, a.hdr)) {
+                        ok = false;
+                        break;
+                    }
                     JFA_TRACE_EV(bwd, 1, t, 3);
                     tc_fence_after();
                     issue_dp(t + 1);
@@ -513,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             tmem_wait_st();
             // query rows past the sequence end (neighbour data) must not reach dV / dK
             if (qb0 + r >= nq) {
-                if (grp == 0) zero_row(smem + kOffQ, r);
-                else if (grp == 1) zero_row(smem + kOffDO + buf * kTile, r);
+                if (grp == 0) zero_row(smem + kOffQD + ((2 * t) % 3) * kTile, r);
+                else if (grp == 1) zero_row(smem + kOffQD + ((2 * t + 1) % 3) * kTile, r);
             }
             SC_EV(3);
             fence_proxy_async_smem();

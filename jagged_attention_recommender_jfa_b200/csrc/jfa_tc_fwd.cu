@@ -98,16 +98,18 @@ struct FwdParams {
     AttnArgs a;
 };
 
-// K-major operand (Q, K) at K-step k (16 elements): box k/4, +32 B per step.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_base, int k) {
-    return smem_desc_sw128(tile_base + (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32u, 16u,
-                           1024u);
+// Shared-memory operand descriptors at K step k (16 elements), from the
+// tile's precomputed lower word.  K-major (Q, K): box k/4, +32 B per step.
+// MN-major (V: keys x d, d contiguous): 16 keys = 2048 B per step, 8-key
+// groups 1024 B apart (SBO), the two 64-column halves kBox apart (LBO).
+constexpr uint32_t kDescHi = sw128_desc_hi(1024u);
+__device__ __forceinline__ uint32_t kmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, 16u); }
+__device__ __forceinline__ uint32_t mnmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, kBox); }
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t lo, int k) {
+    return sw128_desc(lo + (uint32_t)(k >> 2) * (kBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
 }
-
-// MN-major operand (V: keys x d, d contiguous) at K-step k (16 keys):
-// 8-key groups 1024 B apart (SBO), the two 64-column halves kBox apart (LBO).
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile_base, int k) {
-    return smem_desc_sw128(tile_base + (uint32_t)k * 2048u, kBox, 1024u);
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t lo, int k) {
+    return sw128_desc(lo + (uint32_t)k * 128u, kDescHi);
 }
 
 // The work item a CTA takes at its r-th turn: items are listed longest
@@ -276,6 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             int g = 0, nk = 0;
             int gt[2] = {0, 0}, mt[2] = {0, 0};
             bool ok = true;
+            // descriptor lower words of every operand tile, computed once
+            const uint32_t qK0 = kmajor_lo(sbase + kOffQ), qK1 = kmajor_lo(sbase + kOffQ + kTile);
+            const uint32_t kK0 = kmajor_lo(sbase + kOffK), kK1 = kmajor_lo(sbase + kOffK + kTile);
+            const uint32_t vM0 = mnmajor_lo(sbase + kOffV), vM1 = mnmajor_lo(sbase + kOffV + kTile);
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
@@ -296,10 +302,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         JFA_TRACE_EV(fwd, 1, gg, 0);
                     }
                     tc_fence_after();
-                    const uint32_t qb = sbase + kOffQ + t * kTile, kb = sbase + kOffK + s * kTile;
+                    const uint32_t qd = t ? qK1 : qK0, kd = s ? kK1 : kK0;
 #pragma unroll
                     for (int k = 0; k < HD / 16; ++k)
-                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qb, k), kmajor_desc(kb, k), idesc_qk, k > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qd, k), kmajor_desc(kd, k), idesc_qk, k > 0 ? 1u : 0u);
                     mma_commit(&bars->s_full[t]);
                     if (t == last_user(j)) mma_commit(&bars->k_empty[s]);
                     if (j == w.n - 1 && t == last_user(j)) mma_commit(&bars->q_free);
@@ -319,12 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         if (t == first_user(j) &&
                             !mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t vb = sbase + kOffV + s * kTile;
+                        const uint32_t vd = s ? vM1 : vM0;
                         const uint32_t tP = tmem + t * 128;   // P (bf16 pairs) over S_T: keys 16k.. at 8k + (k >= 4 ? 32 : 0)
                         const uint32_t tO = tmem + 256 + t * 128;
 #pragma unroll
                         for (int k = 0; k < BN / 16; ++k)
-                            mma_bf16_ts(tO, tP + k * 8 + (k >= 4 ? 32 : 0), mnmajor_desc(vb, k), idesc_pv,
+                            mma_bf16_ts(tO, tP + k * 8 + (k >= 4 ? 32 : 0), mnmajor_desc(vd, k), idesc_pv,
                                         (j > 0 || k > 0) ? 1u : 0u);
                         mma_commit(&bars->pv_done[t]);
                         if (t == last_user(j)) mma_commit(&bars->v_empty[s]);
