@@ -82,38 +82,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// ~1 s of wall-clock time (or as soon as another warp of the CTA has given
-// up), recording JFA_ERR_TIMEOUT; returns false in that case.
+// ~1 s of wall-clock time (or as soon as another warp of the CTA, or another
+// CTA, has given up), recording JFA_ERR_TIMEOUT; returns false in that case.
+// The spin polls only the barrier and the CTA's shared abort flag; the
+// grid's error word (an L2 round trip) and the clock are read every
+// kPollEvery spins, so that a completed phase is seen within one
+// shared-memory round trip rather than one global-memory round trip.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr uint32_t kPollEvery = 1024;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           WsHeader* hdr) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     volatile int* grid_err = &hdr->err;
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag || *grid_err == JFA_ERR_TIMEOUT) {
-            *abort_flag = 1;
-            return false;
-        }
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            set_error(hdr, JFA_ERR_TIMEOUT);
-            return false;
+        if (*abort_flag) return false;
+        if (it % kPollEvery == 0) {
+            if (*grid_err == JFA_ERR_TIMEOUT) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                set_error(hdr, JFA_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
 }
 
 // Bounded wait used before the CTA exits to let its own asynchronous copies
 // and MMAs retire; ignores the abort flag (those operations are in flight
-// whatever the other warps decided).
+// whatever happened), still gives up after the wall-clock limit.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, WsHeader* hdr) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (it % kPollEvery == 0 && globaltimer() - t0 > kWaitLimitNs) {
             set_error(hdr, JFA_ERR_TIMEOUT);
             return false;
         }

@@ -16,22 +16,25 @@
 //                             P^T (bf16) back to TMEM over S^T, dS^T (bf16)
 //                             to shared memory
 //                      dK  += dS^T Q                         (TMEM)
+//                      dV  += P^T dO    (A operand from TMEM)
 //                      dQ^T = K^T dS^T over the dP^T columns, read out by
 //                             the score warps and added to the fp32
 //                             accumulator with coalesced reductions (a warp
 //                             covers 32 consecutive d of one query row)
-//                      dV  += P^T dO    (A operand from TMEM)
-//                    The tensor core runs dK, dQ^T, dV of tile t and then
-//                    S^T, dP^T of tile t+1 back to back: dQ^T(t) is read out
-//                    while dV runs, and Q / dO come from a three-buffer ring
-//                    that fetches Q(t+1) two tiles ahead and dO(t+1) once
-//                    dK(t) has retired (both warmed in L2 a tile earlier).
+//                    dK and dV run over the tile's two query halves, the
+//                    first while the score warps form the second; then dQ^T
+//                    of tile t and S^T, dP^T of tile t+1 follow back to back:
+//                    dQ^T(t) is read out while S^T(t+1) runs, and Q / dO
+//                    come from a three-buffer ring that fetches Q(t+1) two
+//                    tiles ahead and dO(t+1) once dK(t) has retired (both
+//                    warmed in L2 a tile earlier).
 //   tc_bwd_dq_finalize  dQ = bf16(scale * accumulator).
 //
 // Warp roles: warp 0 TMA, warp 1 MMA, warps 2..17 score warps in four groups
-// of four; a thread owns one key row (or, for dQ^T, one d row) and one
-// 32-column (query) chunk of it.  The backward needs no row reduction (LSE
-// and D are given), so the chunks never talk.
+// of four; a thread of group g owns one key row and its 16-query chunks g
+// and g + 4 (for the dQ^T read-out: one d row and queries 32g .. 32g + 31).
+// The backward needs no row reduction (LSE and D are given), so the chunks
+// never talk.
 // TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384),
 // dP^T / dQ^T [384,512).
 #include <math_constants.h>
@@ -77,6 +80,7 @@ struct Bars {
     uint64_t kv_full;
     uint64_t buf_full[3], buf_empty[3];   // the Q / dO ring
     uint64_t s_full;
+    uint64_t ds_half;       // 16 score warps: queries 0..63 of the tile done
     uint64_t ds_full;       // 16 score warps
     uint64_t dq_full;
     uint64_t dq_empty;      // 16 score warps
@@ -179,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             mbar_init(&bars->bias_full[s2], 1);
         }
         mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->ds_half, NG * 4);
         mbar_init(&bars->ds_full, NG * 4);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, NG * 4);
@@ -285,32 +290,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 issue_dp(0);
                 mma_commit(&bars->s_full);
             }
+            // dK += dS^T Q and dV += P^T dO run over the tile's query halves:
+            // the first four K steps (queries 0..63) as soon as the score
+            // warps have formed that half, the rest after the whole tile
+            auto issue_dk = [&](int t, int k_lo) {  // A = dS^T K-major in smem, B = Q MN-major
+                const uint32_t qM = ringM((2 * t) % 3);
+#pragma unroll
+                for (int k = k_lo; k < k_lo + 4; ++k)
+                    mma_bf16_ss(tdK, kmajor_desc(dsK, k), mnmajor_desc(qM, k), idesc_nn,
+                                (t > 0 || k > 0) ? 1u : 0u);
+            };
+            auto issue_dv = [&](int t, int k_lo) {  // A = P^T from TMEM: queries 16k.. at column 16k
+                const uint32_t d = ringM((2 * t + 1) % 3);
+#pragma unroll
+                for (int k = k_lo; k < k_lo + 4; ++k)
+                    mma_bf16_ts(tdV, tS + 16 * k, mnmajor_desc(d, k), idesc_nn, (t > 0 || k > 0) ? 1u : 0u);
+            };
             for (int t = 0; ok && t < nt; ++t) {
+                if (!mbar_wait(&bars->ds_half, t & 1, abort_flag, a.hdr)) { ok = false; break; }
+                tc_fence_after();
+                issue_dk(t, 0);
+                issue_dv(t, 0);
                 if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
                 JFA_TRACE_EV(bwd, 1, t, 0);
                 tc_fence_after();
-                // dK += dS^T Q   (A = dS^T K-major in smem, B = Q MN-major)
-                {
-                    const uint32_t qM = ringM((2 * t) % 3);
-#pragma unroll
-                    for (int k = 0; k < BM / 16; ++k)
-                        mma_bf16_ss(tdK, kmajor_desc(dsK, k), mnmajor_desc(qM, k), idesc_nn,
-                                    (t > 0 || k > 0) ? 1u : 0u);
-                }
+                issue_dk(t, 4);
                 mma_commit(&bars->buf_empty[(2 * t) % 3]);
+                issue_dv(t, 4);
+                mma_commit(&bars->buf_empty[(2 * t + 1) % 3]);
                 // dQ^T = K^T dS^T over the dP^T columns (A = K, B = dS^T, both MN-major)
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tdP, mnmajor_desc(kM, k), mnmajor_desc(dsM, k), idesc_tn, k > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
-                // dV += P^T dO: A = P^T from TMEM, query step k (16 queries) of group
-                // k/2 in columns 32*(k/2) + 8*(k%2) of the S^T region
-                const uint32_t d = ringM((2 * t + 1) % 3);
-#pragma unroll
-                for (int k = 0; k < BM / 16; ++k)
-                    mma_bf16_ts(tdV, tS + 32 * (k >> 1) + 8 * (k & 1), mnmajor_desc(d, k), idesc_nn,
-                                (t > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&bars->buf_empty[(2 * t + 1) % 3]);
                 JFA_TRACE_EV(bwd, 1, t, 1);
                 if (t + 1 < nt) {
                     // S^T(t+1) overwrites P^T(t): issued after dV, which reads it
@@ -347,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const uint32_t cofs = (uint32_t)grp * 32;
         const uint32_t tdV = tmem + lane_addr + cofs, tdK = tmem + lane_addr + 128 + cofs;
-        const uint32_t tS = tmem + lane_addr + 256 + cofs, tdP = tmem + lane_addr + 384 + cofs;
+        const uint32_t tS = tmem + lane_addr + 256, tdP = tmem + lane_addr + 384 + cofs;
         const float sc = a.scale * kLog2e;
         const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
         const int C = (a.relpos_len - 1) >> 1;
@@ -495,30 +507,40 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     }
                 }
             };
-            // Two 16-column halves.  P^T (bf16 pairs) goes back to TMEM over the
-            // first 16 of this group's 32 S^T columns (half hh to columns 8hh..,
-            // which half 0 has already read; no other group reads them); dS^T
-            // goes to shared memory for dK and dQ^T.
+            // Two 16-column halves: half hh of group grp is query chunk
+            // c16 = 4 hh + grp (columns 16 c16 ..), so that every group's first
+            // half together covers queries 0..63 and dK / dV can start on them.
+            // P^T (bf16 pairs) goes back to TMEM over the first 8 of the
+            // chunk's own S^T columns (no other warp reads them), dS^T to
+            // shared memory for dK and dQ^T.  Query rows past the sequence end
+            // (neighbour data) must not reach dV / dK: S^T and dP^T of the
+            // tile have completed, so Q and dO may be edited.
+            if (qb0 + r >= nq) {
+                if (grp == 0) zero_row(smem + kOffQD + ((2 * t) % 3) * kTile, r);
+                else if (grp == 1) zero_row(smem + kOffQD + ((2 * t + 1) % 3) * kTile, r);
+            }
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t u[16], g[16];
-                tmem_ld16(tS + hh * 16, u);
-                tmem_ld16(tdP + hh * 16, g);
+                const int c16 = hh * 4 + grp;
+                tmem_ld16(tS + c16 * 16, u);
+                tmem_ld16(tdP - cofs + c16 * 16, g);
                 tmem_wait_ld();
-                const int c16 = grp * 2 + hh;
                 process(u, g, c16);
                 store_half_chunk_bits(smem + kOffDST, r, c16, g);
                 uint32_t pk[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-                tmem_st8(tS + hh * 8, pk);
+                tmem_st8(tS + c16 * 16, pk);
+                if (hh == 0) {
+                    tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->ds_half);
+                }
             }
             tmem_wait_st();
-            // query rows past the sequence end (neighbour data) must not reach dV / dK
-            if (qb0 + r >= nq) {
-                if (grp == 0) zero_row(smem + kOffQD + ((2 * t) % 3) * kTile, r);
-                else if (grp == 1) zero_row(smem + kOffQD + ((2 * t + 1) % 3) * kTile, r);
-            }
             SC_EV(3);
             fence_proxy_async_smem();
             tc_fence_before();
