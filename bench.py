@@ -68,7 +68,7 @@ def parse_args():
                     help="override the workload's number of sequences (profiling captures)")
     ap.add_argument("--max-len", type=int, default=None,
                     help="override the workload's length clip (profiling captures)")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -497,51 +497,82 @@ def aggregate_over_ranks(ms_per_step, flops, device, world):
 
 def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
     """Same metric with pinned host inputs copied in and every result copied
-    out inside the timed region."""
+    out inside the timed region, pipelined the way a training input loop is:
+    two sets of device buffers, the inputs of step i+1 copied in (one copy
+    stream) and the results of step i-1 copied out (another) while step i
+    computes; every step still moves all of its inputs and results."""
     host_in = {n: getattr(p, n).contiguous().pin_memory() for n in ("q", "k", "v", "dout")}
     host_in["q_off"] = p.q_off.contiguous().pin_memory()
     host_in["kv_off"] = p.kv_off.contiguous().pin_memory()
     if p.bias is not None:
         host_in["bias"] = p.bias.contiguous().pin_memory()
-    dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
-    out = torch.empty_like(dev_in["q"])
-    lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
-    dq, dk, dv = torch.empty_like(dev_in["q"]), torch.empty_like(dev_in["k"]), torch.empty_like(dev_in["v"])
+    sets = []
+    for _ in range(2):
+        dev_in = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+        out = torch.empty_like(dev_in["q"])
+        lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
+        dq, dk, dv = torch.empty_like(dev_in["q"]), torch.empty_like(dev_in["k"]), torch.empty_like(dev_in["v"])
+        sets.append((dev_in, out, lse, dq, dk, dv))
     ws_f = jfa.workspace(prob, False, dev)
     ws_b = jfa.workspace(prob, True, dev)
-    results = [out, dq, dk, dv] + ([lse] if lse is not None else [])
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in results]
+
+    def results_of(st):
+        _, out, lse, dq, dk, dv = st
+        return [out, dq, dk, dv] + ([lse] if lse is not None else [])
+
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in results_of(sets[0])]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in results)
+    d2h = sum(t.numel() * t.element_size() for t in results_of(sets[0]))
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_ready, comp_done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def step():
-        for n, t in host_in.items():
-            dev_in[n].copy_(t, non_blocking=True)
-        jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_off"],
-                        dev_in["kv_off"], dev_in.get("bias"), act, p.causal, out, lse, ws_f,
-                        stream=stream)
-        jfa.jfa_backward(prob, dev_in["q"], dev_in["k"], dev_in["v"], out, lse, dev_in["dout"],
-                         dev_in["q_off"], dev_in["kv_off"], dev_in.get("bias"), act, p.causal,
-                         dq, dk, dv, ws_b, stream=stream)
-        for h, t in zip(host_out, results):
-            h.copy_(t, non_blocking=True)
+    def run(nsteps):
+        for i in range(nsteps):
+            b = i % 2
+            dev_in, out, lse, dq, dk, dv = sets[b]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[b])       # step i-2 has finished reading set b
+                for n, t in host_in.items():
+                    dev_in[n].copy_(t, non_blocking=True)
+                in_ready[b].record(up)
+            stream.wait_event(in_ready[b])
+            if i >= 2:
+                stream.wait_event(out_free[b])        # results of step i-2 are out
+            jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_off"],
+                            dev_in["kv_off"], dev_in.get("bias"), act, p.causal, out, lse, ws_f,
+                            stream=stream)
+            jfa.jfa_backward(prob, dev_in["q"], dev_in["k"], dev_in["v"], out, lse, dev_in["dout"],
+                             dev_in["q_off"], dev_in["kv_off"], dev_in.get("bias"), act, p.causal,
+                             dq, dk, dv, ws_b, stream=stream)
+            comp_done[b].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[b])
+                for h, t in zip(host_out, results_of(sets[b])):
+                    h.copy_(t, non_blocking=True)
+                out_free[b].record(down)
 
-    step()
+    run(2)
     torch.cuda.synchronize(dev)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     s.record(stream)
-    for _ in range(args.e2e_steps):
-        step()
+    up.wait_event(s)
+    run(args.e2e_steps)
+    stream.wait_stream(down)
+    stream.wait_stream(up)
     e.record(stream)
     torch.cuda.synchronize(dev)
     ms = s.elapsed_time(e) / args.e2e_steps
     ms, flops_all = aggregate_over_ranks(ms, flops_rank, dev, world)
     return {"value": flops_all / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": args.e2e_steps}
+            "steps": args.e2e_steps,
+            "pipeline": "two buffer sets; inputs of step i+1 in and results of step i-1 out "
+                        "on two copy streams while step i computes"}
 
 
 if __name__ == "__main__":
