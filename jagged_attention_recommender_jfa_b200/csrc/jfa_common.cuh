@@ -186,21 +186,34 @@ __device__ __forceinline__ void set_error(WsHeader* hdr, int code) {
 // Activations of the GDPA variant.
 //   SiLU(x) = x * sigmoid(x)
 //   GELU_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
-__device__ __forceinline__ float act_f(int act, float x) {
-    if (act == JFA_ACT_SILU) return x / (1.0f + expf(-x));
-    const float c = 0.7978845608028654f;  // sqrt(2/pi)
-    float t = tanhf(c * (x + 0.044715f * x * x * x));
-    return 0.5f * x * (1.0f + t);
+// Both are x * sigmoid(k(x)): k = x for SiLU and, since 0.5 (1 + tanh z) =
+// sigmoid(2 z), k = 2 sqrt(2/pi) (x + 0.044715 x^3) for tanh-GELU.  The
+// sigmoid is 1 / (1 + 2^(-k log2 e)) from the hardware base-2 exponential and
+// a fast reciprocal (a few ulp; a large negative k gives 0, a large positive 1).
+__device__ __forceinline__ float sigmoid_fast(float k) {
+    float e;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-k * 1.4426950408889634f));
+    return __fdividef(1.0f, 1.0f + e);
+}
+
+__device__ __forceinline__ float act_arg(int act, float x) {
+    return act == JFA_ACT_SILU ? x : 1.5957691216057308f * fmaf(0.044715f * x, x * x, x);
+}
+
+__device__ __forceinline__ float act_f(int act, float x) { return x * sigmoid_fast(act_arg(act, x)); }
+
+// Derivatives, from s = sigmoid(k(x)):
+//   SiLU'(x)      = s (1 + x (1 - s))
+//   GELU_tanh'(x) = 0.5 (1 + t) + 0.5 x (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 x^2)
+//                 = s + 2 x s (1 - s) sqrt(2/pi) (1 + 3 * 0.044715 x^2)
+//   (t = tanh z = 2 s - 1, so 1 + t = 2 s and 1 - t^2 = 4 s (1 - s))
+__device__ __forceinline__ float act_grad_from(int act, float x, float s) {
+    if (act == JFA_ACT_SILU) return s * fmaf(x, 1.0f - s, 1.0f);
+    return fmaf(2.0f * x * s * (1.0f - s), 0.7978845608028654f * fmaf(3.0f * 0.044715f, x * x, 1.0f), s);
 }
 
 __device__ __forceinline__ float act_grad_f(int act, float x) {
-    if (act == JFA_ACT_SILU) {
-        float sg = 1.0f / (1.0f + expf(-x));
-        return sg * (1.0f + x * (1.0f - sg));
-    }
-    const float c = 0.7978845608028654f;
-    float t = tanhf(c * (x + 0.044715f * x * x * x));
-    return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * c * (1.0f + 3.0f * 0.044715f * x * x);
+    return act_grad_from(act, x, sigmoid_fast(act_arg(act, x)));
 }
 
 // Additive bias beta_h(i, j) of sequence b (i, j relative to the sequence).

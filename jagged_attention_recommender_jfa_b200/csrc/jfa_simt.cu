@@ -181,8 +181,9 @@ __device__ __forceinline__ void weight_and_dscore(int act, float s, float lse_i,
         w = (lse_i == -CUDART_INF_F) ? 0.f : expf(s - lse_i);
         ds = w * (dp - d_i);
     } else {
-        w = act_f(act, s) * inv_n;
-        ds = dp * act_grad_f(act, s) * inv_n;
+        const float sg = sigmoid_fast(act_arg(act, s));
+        w = s * sg * inv_n;
+        ds = dp * act_grad_from(act, s, sg) * inv_n;
     }
 }
 

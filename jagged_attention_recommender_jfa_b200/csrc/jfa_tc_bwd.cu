@@ -406,6 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             const int buf = t & 1;
             float nl2 = CUDART_INF_F, ndv = 0.f;
             if (grp == 0 && t + 1 < nt) fetch_rowstats(t + 1, nl2, ndv);
+            // the next query tile's dense bias block (read once from HBM) into
+            // L2: query row r, keys j0 .. j0 + 127 span at most three lines
+            if (BIAS == 2 && grp < 3 && t + 1 < nt && qb0 + BM + r < nq)
+                prefetch_l2(dense + dense_base + (int64_t)(qb0 + BM + r) * nkv + min(j0 + 63 * grp + grp / 2, nkv - 1));
             if (!wwait(&bars->s_full, t & 1)) { ok = false; break; }
             SC_EV(1);
             tc_fence_after();
@@ -493,8 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 #pragma unroll
                     for (int v = 0; v < 16; ++v) {
                         const float sn = x[v] * (1.0f / kLog2e);
-                        u[v] = __float_as_uint(act_f(a.act, sn) * inv_n);
-                        g[v] = __float_as_uint(__uint_as_float(g[v]) * act_grad_f(a.act, sn) * inv_n);
+                        const float sg = sigmoid_fast(act_arg(a.act, sn));
+                        u[v] = __float_as_uint(sn * sg * inv_n);
+                        g[v] = __float_as_uint(__uint_as_float(g[v]) * act_grad_from(a.act, sn, sg) * inv_n);
                     }
                 }
                 if (!all_vis) {

@@ -411,6 +411,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
                                           ? a.dense_off[w.b] + ((int64_t)w.h * w.nq + i) * w.nkv : 0;
             float m_used = -CUDART_INF_F, l = 0.f;
+            // a dense bias row segment (this thread's 64 keys of a key tile, read
+            // once from HBM) is brought into L2 a key tile ahead
+            auto prefetch_bias_seg = [&](int jt) {
+                if (BIAS == 2 && i < w.nq && jt < n) {
+                    const int k_lo = min(jt * BN + cb, w.nkv - 1), k_hi = min(jt * BN + cb + CW - 1, w.nkv - 1);
+                    prefetch_l2(dense + dense_row + k_lo);
+                    prefetch_l2(dense + dense_row + k_hi);
+                }
+            };
+            prefetch_bias_seg(0);
             for (int j = 0; j < n; ++j, ++gt) {
                 SM_EV(0);
                 if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
@@ -486,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     tmem_st16(tS + cc, *reinterpret_cast<uint32_t(*)[16]>(u));
                 }
                 SM_EV(2);
+                prefetch_bias_seg(j + 1);
                 float ref = 0.f;
                 if (softmax) {
                     // row maximum of both halves (exchange buffer by step parity)
