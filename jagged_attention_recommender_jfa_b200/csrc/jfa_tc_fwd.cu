@@ -119,6 +119,32 @@ __device__ __forceinline__ int item_of_turn(int r, int c, int G) {
     return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
+// 16 consecutive bf16 starting at p (2-byte aligned) as floats, read as the
+// three 16-byte blocks that cover them (the last only when needed).  Reading
+// whole aligned blocks never leaves the allocation that holds the 32 bytes.
+// Word s + k of the blocks, shifted right by 16 p bits across its neighbour,
+// is the pair (2k, 2k+1), with s, p the word and half offset of p.
+__device__ __forceinline__ void dense_bias16(const __nv_bfloat16* p, float (&bb)[16]) {
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(p);
+    const uint4* blk = reinterpret_cast<const uint4*>(addr & ~static_cast<uintptr_t>(15));
+    const int e0 = (int)(addr & 15) >> 1;      // element offset in the first block, 0..7
+    const uint4 b0 = __ldg(blk), b1 = __ldg(blk + 1);
+    const uint4 b2 = e0 ? __ldg(blk + 2) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t W[12] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w, b2.x, b2.y, b2.z, b2.w};
+    const int s = e0 >> 1, sh = (e0 & 1) * 16;
+    uint32_t V1[10], V2[9];
+#pragma unroll
+    for (int k = 0; k < 10; ++k) V1[k] = (s & 2) ? W[k + 2] : W[k];
+#pragma unroll
+    for (int k = 0; k < 9; ++k) V2[k] = (s & 1) ? V1[k + 1] : V1[k];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t pr = __funnelshift_r(V2[k], V2[k + 1], sh);
+        bb[2 * k] = __uint_as_float(pr << 16);
+        bb[2 * k + 1] = __uint_as_float(pr & 0xffff0000u);
+    }
+}
+
 struct Item {
     int b, h, row0, q0, nq, k0, nkv;
     int n_t[2];   // key tiles of tile A and tile B (0: the tile has no rows or sees no key)
@@ -472,10 +498,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             x[v] = r2.x, x[v + 1] = r2.y;
                         }
                     } else if (BIAS == 2) {
+                        if (cc + 16 <= nvis) {
+                            // the row's 16 bf16 (32 bytes, any 2-byte alignment) from
+                            // the three 16-byte blocks that hold them: three loads
+                            // instead of sixteen (a warp's lanes are on 32 rows)
+                            float bb[16];
+                            dense_bias16(dense + dense_row + jc + cc, bb);
 #pragma unroll
-                        for (int v = 0; v < 16; ++v)
-                            x[v] = fmaf(x[v], sc,
-                                        cc + v < nvis ? __bfloat162float(dense[dense_row + jc + cc + v]) * kLog2e : 0.f);
+                            for (int v = 0; v < 16; v += 2) {
+                                const float2 r2 = fma2(make_float2(x[v], x[v + 1]), sc2,
+                                                       mul2(make_float2(bb[v], bb[v + 1]), make_float2(kLog2e, kLog2e)));
+                                x[v] = r2.x, x[v + 1] = r2.y;
+                            }
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 16; ++v)
+                                x[v] = fmaf(x[v], sc,
+                                            cc + v < nvis ? __bfloat162float(dense[dense_row + jc + cc + v]) * kLog2e : 0.f);
+                        }
                     } else {
 #pragma unroll
                         for (int v = 0; v < 16; v += 2) {
