@@ -387,6 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->rows_full[t & 1]);
         };
+        // the first query tile's dense bias block (read once from HBM) into L1
+        // and L2 while the K / V / Q / dO loads are in flight: query row r,
+        // keys j0 .. j0 + 127 span at most three lines
+        if (BIAS == 2 && grp < 3 && nt > 0 && i_start + r < nq)
+            prefetch_l1(dense + dense_base + (int64_t)(i_start + r) * nkv + min(j0 + 63 * grp + grp / 2, nkv - 1));
         if (nt > 0 && grp == 0) {
             float l2, dv;
             fetch_rowstats(0, l2, dv);
