@@ -212,10 +212,6 @@ __device__ __forceinline__ float act_grad_from(int act, float x, float s) {
     return fmaf(2.0f * x * s * (1.0f - s), 0.7978845608028654f * fmaf(3.0f * 0.044715f, x * x, 1.0f), s);
 }
 
-__device__ __forceinline__ float act_grad_f(int act, float x) {
-    return act_grad_from(act, x, sigmoid_fast(act_arg(act, x)));
-}
-
 // Additive bias beta_h(i, j) of sequence b (i, j relative to the sequence).
 template <typename T>
 __device__ __forceinline__ float bias_at(const AttnArgs& a, int b, int h, int nq, int nkv, int i, int j) {

@@ -299,24 +299,15 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // ---------------------------------------------------------------------------
 // Descriptors
 // ---------------------------------------------------------------------------
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
-//   start : byte address of the (1024-byte aligned) swizzle atom + offset
-//   lbo   : leading byte offset, sbo: stride byte offset (bytes)
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((start & 0x3FFFF) >> 4);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-    d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-    return d;
-}
-
-// The same descriptor split in two 32-bit words, so that an MMA issue loop
-// builds it with one add: the upper word (stride, version, swizzle) is a
-// constant, and the lower word is (start >> 4) | (LBO >> 4) << 16, where a K
-// step only adds to the start field (shared-memory addresses stay below
-// 256 KB, so the 14-bit field never carries).
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits:
+// bits [0,14) start address >> 4 (the 1024-byte aligned swizzle atom plus an
+// offset), [16,30) leading byte offset >> 4, [32,46) stride byte offset >> 4,
+// bit 46 the sm_100 descriptor version, bits [61,64) the layout (2 = 128-byte
+// swizzle).  It is built as two 32-bit words, so that an MMA issue loop makes
+// it with one add: the upper word (stride, version, swizzle) is a constant,
+// and the lower word is (start >> 4) | (LBO >> 4) << 16, where a K step only
+// adds to the start field (shared-memory addresses stay below 256 KB, so the
+// 14-bit field never carries).
 __host__ __device__ constexpr uint32_t sw128_desc_hi(uint32_t sbo) {
     return ((sbo >> 4) & 0x3FFF) | (1u << 14) | (2u << 29);
 }
@@ -389,17 +380,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Round-to-nearest-even to bf16 on the integer pipe (finite inputs): add
-// 0x7FFF plus the lowest kept bit, keep the upper 16 bits; two results are
-// packed with one byte permute.  Keeps the conversion of P off the pipe that
-// also evaluates exp2.
-__device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
-    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-    a += 0x7FFFu + ((a >> 16) & 1u);
-    b += 0x7FFFu + ((b >> 16) & 1u);
-    return __byte_perm(a, b, 0x7632);
 }
 
 }  // namespace sm100
