@@ -462,13 +462,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         x[2 * e] = r2.x, x[2 * e + 1] = r2.y;
                     }
                 } else if (BIAS == 2) {
+                    // bias(qc0 + v, j): sixteen unconditional loads (rows and key
+                    // clamped into the sequence, invalid entries masked below), so
+                    // that they are all in flight together
+                    const __nv_bfloat16* col = dense + dense_base + min(j, nkv - 1);
+                    __nv_bfloat16 bh[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) {
-                        const int qi = qc0 + v;
-                        const float bv = (jvalid && qi < nq)
-                            ? __bfloat162float(dense[dense_base + (int64_t)qi * nkv + j]) * kLog2e : 0.f;
-                        x[v] = fmaf(__uint_as_float(u[v]), sc, bv);
-                    }
+                    for (int v = 0; v < 16; ++v) bh[v] = col[(int64_t)min(qc0 + v, nq - 1) * nkv];
+#pragma unroll
+                    for (int v = 0; v < 16; ++v)
+                        x[v] = fmaf(__uint_as_float(u[v]), sc, __bfloat162float(bh[v]) * kLog2e);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
