@@ -147,3 +147,161 @@ def test_mxfp8_attention_oracle():
     o, _ = oracle.forward(off, off, q, k, v, causal=True)
     assert np.abs(o_q - o).max() <= 2.0 ** -4 * np.abs(v.numpy()).max()
     assert np.abs(o_q - o).max() > 0.0
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 P quantisation, pinned on hand-built rows.
+#
+# With q = 0 the scores are the dense bias; a bias of (k_j + 1/2) ln 2 puts the
+# log2-domain score of key j at x_j = k_j + 1/2 (k_j an integer).  The
+# reference is R = ceil(max x) = k_max + 1, so the weights are
+# w_j = 2^(e_j - 1/2), e_j = k_j - k_max.  In an MX block whose largest
+# weight has exponent e_max the shared exponent is floor(log2 w_max) - 8 =
+# e_max - 9, and the scaled element is sqrt(2) 2^p with p = 8 + e_j - e_max.
+# E4M3 rounds sqrt(2) 2^p to 1.375 2^p in the normal range (p >= -6: 1.4142
+# lies nearer 1.375 than 1.5) and to n 2^-9 below it, n = 6, 3, 1, 1, 0 for
+# p = -7 .. -11.  The output is sum_j deq_j v_j / sum_j w_j (the unquantised
+# sum).  Blocks hold 32 consecutive keys counted from the sequence's first
+# key; the sequence below starts at packed row 5, so counting blocks from the
+# packed row index instead would put key 31 (the row maximum) into the block
+# of keys 32.. and flush those to zero.
+# ---------------------------------------------------------------------------
+_SUBNORMAL_N = {-7: 6, -8: 3, -9: 1, -10: 1}
+
+
+def _e4m3_sqrt2_pow(p):
+    """E4M3 value of sqrt(2) * 2^p (hand table above)."""
+    if p >= -6:
+        return 1.375 * 2.0 ** p
+    return _SUBNORMAL_N.get(p, 0) * 2.0 ** -9
+
+
+def test_e4m3_sqrt2_table_matches_torch_float8():
+    for p in range(-14, 9):
+        t = torch.tensor([math.sqrt(2.0) * 2.0 ** p], dtype=torch.float64)
+        assert float(t.float().to(torch.float8_e4m3fn).double()) == _e4m3_sqrt2_pow(p), p
+        assert oracle.e4m3_decode(oracle.e4m3_encode(math.sqrt(2.0) * 2.0 ** p)) == _e4m3_sqrt2_pow(p)
+
+
+def _expected_row(e, vis, v, block_start):
+    """Closed form of one output row: e[j] integer exponents (0 at the row
+    maximum), vis[j] visibility, blocks of 32 keys starting at key
+    -block_start (0 = the sequence's first key)."""
+    n = len(e)
+    w = np.array([2.0 ** (e[j] - 0.5) if vis[j] else 0.0 for j in range(n)])
+    deq = np.zeros(n)
+    for lo in range(-block_start, n, 32):
+        js = [j for j in range(max(lo, 0), min(lo + 32, n)) if vis[j]]
+        if not js:
+            continue
+        emax = max(e[j] for j in js)
+        for j in js:
+            deq[j] = _e4m3_sqrt2_pow(8 + e[j] - emax) * 2.0 ** (emax - 9)
+    return (deq[:, None] * v).sum(0) / w.sum()
+
+
+def _quant_p_case():
+    rng = np.random.default_rng(11)
+    n0, nq, nkv = 5, 3, 70            # sequence 0: 5 filler rows; sequence 1 under test
+    H, d = 1, 8
+    q_off = np.array([0, n0, n0 + nq], np.int32)
+    kv_off = np.array([0, n0, n0 + nkv], np.int32)
+    e = np.zeros((nq, nkv), np.int64)
+    for i in range(nq):
+        for j in range(nkv):
+            if j < 31:
+                e[i, j] = -((j + i) % 5)               # block 0: near the maximum
+            elif j == 31:
+                e[i, j] = 0                            # the row maximum, last key of block 0
+            elif j < 64:
+                e[i, j] = -20 - ((j + i) % 4)          # block 1: far below it
+            else:
+                e[i, j] = -3 - (j % 2)                 # block 2 (6 keys)
+    e[2, 40] = -20 - 10                                # a subnormal inside block 1 (p = -2 - 10 + 2)
+    x = e + 0.5                                        # k_max = 0 for every row
+    dense = np.concatenate([rng.standard_normal(H * n0 * n0), (x * math.log(2.0)).reshape(-1)])
+    k = rng.standard_normal((n0 + nkv, H, d))
+    v = rng.standard_normal((n0 + nkv, H, d))
+    q = np.zeros((n0 + nq, H, d))
+    q[:n0] = rng.standard_normal((n0, H, d))
+    return q_off, kv_off, q, k, v, dense, e
+
+
+def test_mxfp8_p_quantisation_closed_form():
+    q_off, kv_off, q, k, v, dense, e = _quant_p_case()
+    nq, nkv = e.shape
+    o, lse = oracle.forward(q_off, kv_off, q, k, v, bias=dense, bias_kind="dense",
+                            quant_p=True)
+    vs = v[5:5 + nkv, 0]
+    for i in range(nq):
+        want = _expected_row(e[i], np.ones(nkv, bool), vs, 0)
+        np.testing.assert_allclose(o[5 + i, 0], want, rtol=0, atol=1e-12)
+        # the pin separates the plausible mistakes by far more than its tolerance
+        wrong_blocks = _expected_row(e[i], np.ones(nkv, bool), vs, 5)   # packed-row blocks
+        assert np.abs(wrong_blocks - want).max() > 1e-9
+        w = 2.0 ** (e[i] - 0.5)
+        wrong_ref = (2.0 ** e[i])[:, None] * vs                      # R = max x, not ceil
+        assert np.abs(wrong_ref.sum(0) / (2.0 ** e[i]).sum() - want).max() > 1e-3
+        deq_sum = _expected_row(e[i], np.ones(nkv, bool), np.ones((nkv, 1)), 0)[0] * w.sum()
+        assert abs(deq_sum / w.sum() - 1.0) > 1e-2                   # dividing by sum(deq)
+        # LSE is that of the unquantised scores: ln sum_j e^{s_j}
+        s = (e[i] + 0.5) * math.log(2.0)
+        assert abs(lse[5 + i, 0] - np.log(np.exp(s).sum())) <= 1e-12
+
+
+def test_mxfp8_p_quantisation_causal_blocks():
+    # causal self-attention of one sequence of 40 starting at packed row 9:
+    # row i sees keys 0..i; the block of keys 32..39 is quantised on its own
+    rng = np.random.default_rng(12)
+    n0, n = 9, 40
+    off = np.array([0, n0, n0 + n], np.int32)
+    H, d = 1, 4
+    e = np.array([[-((i - j) % 3) if j != i else 0 for j in range(n)] for i in range(n)])
+    e[:, 32:] -= 12
+    for i in range(32, n):
+        e[i, i] = 0
+    x = (e + 0.5) * math.log(2.0)
+    dense = np.concatenate([rng.standard_normal(n0 * n0), x.reshape(-1)])
+    k = rng.standard_normal((n0 + n, H, d))
+    v = rng.standard_normal((n0 + n, H, d))
+    q = np.zeros((n0 + n, H, d))
+    o, _ = oracle.forward(off, off, q, k, v, bias=dense, bias_kind="dense", causal=True,
+                          quant_p=True)
+    vs = v[n0:, 0]
+    for i in range(n):
+        vis = np.arange(n) <= i
+        want = _expected_row(e[i], vis, vs, 0)
+        np.testing.assert_allclose(o[n0 + i, 0], want, rtol=0, atol=1e-12)
+
+
+def test_dequantize_along_rows_round_trip():
+    # values exactly representable after MX quantisation along rows: per
+    # (head, column) block of 32 rows, E4M3 mantissas in [1, 1.75] times
+    # powers of two within 2^6 of the block maximum (a block maximum with
+    # mantissa 1.875 would saturate to 1.75: 1.875 * 2^8 > 448)
+    rng = np.random.default_rng(13)
+    lens = [5, 70, 0, 33]
+    off = np.array([0] + list(np.cumsum(lens)), np.int32)
+    rows, H, d = int(off[-1]), 2, 32
+    mant = 1.0 + rng.integers(0, 7, (rows, H, d)) / 8.0
+    expo = rng.integers(-6, 1, (rows, H, d)).astype(np.float64)
+    sign = rng.choice([-1.0, 1.0], (rows, H, d))
+    x = sign * mant * 2.0 ** (expo + rng.integers(-3, 4, (1, H, d)))
+    codes, scales = oracle.quantize_mx_along_rows(x, off)
+    back = oracle.dequantize_along_rows(codes, scales, off)
+    assert np.array_equal(back, x)
+    # and row by row it is dequantize_mx of the same blocks: block c of
+    # sequence b covers rows off[b] + 32 c .. + 31 (zero-padded at the end)
+    blk0 = 0
+    for b in range(len(lens)):
+        nb = (lens[b] + 31) // 32
+        for c in range(nb):
+            lo, hi = int(off[b]) + 32 * c, min(int(off[b + 1]), int(off[b]) + 32 * c + 32)
+            for h in range(H):
+                for col in (0, 7, d - 1):
+                    cb = np.zeros(32, np.uint8)
+                    cb[:hi - lo] = codes[lo:hi, h, col]
+                    ref = oracle.dequantize_mx(cb, np.array([scales[blk0 + c, h, col]], np.uint8))
+                    assert np.array_equal(back[lo:hi, h, col], ref[:hi - lo])
+        blk0 += nb
+    assert blk0 == scales.shape[0]
