@@ -15,8 +15,12 @@ Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronisation, timed with CUDA events on the launching stream; the
 max over ranks is reported.  Every input tensor of the default workload is
 larger than L2 (126 MB), so no L2 flush is needed between steps.  Under
-torchrun each rank draws its own batch (seed + rank) of the same workload:
-weak scaling, no collective on the data path.
+torchrun (N ranks) the job is one global batch of N x B sequences of the
+workload: every rank draws the same global lengths, splits them with
+jfa_partition (base batch shuffling by default, or LPT), and draws and runs
+only its own sequences -- weak scaling, no collective on the data path.  The
+line reports the split's rank imbalance (heaviest rank's visible pairs over
+the mean) beside that of a plain contiguous split.
 
 Also reported on one JSON line: per-kernel launch times from the library's
 event hooks (the dominant kernel's roofline fraction), the end-to-end number
@@ -68,6 +72,10 @@ def parse_args():
                     help="override the workload's number of sequences (profiling captures)")
     ap.add_argument("--max-len", type=int, default=None,
                     help="override the workload's length clip (profiling captures)")
+    ap.add_argument("--partition", choices=["bbs", "lpt"], default="bbs",
+                    help="split of the global batch across ranks (N > 1)")
+    ap.add_argument("--sub-batch", type=int, default=8,
+                    help="sequences per sub-batch for --partition bbs")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
@@ -341,9 +349,9 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     from jagged_attention_recommender_jfa_b200 import jfa
-    from jagged_attention_recommender_jfa_b200.inputs import make_problem
+    from jagged_attention_recommender_jfa_b200.inputs import WORKLOADS, draw_lengths
 
-    p = make_problem(args.workload, args.seed + rank, B=args.batch, max_len=args.max_len)
+    p, split = rank_problem(args, rank, world, jfa)
     act = args.act or p.act
     prob = jfa.problem_of(p)
     path = jfa.jfa_path(prob, act, 0), jfa.jfa_path(prob, act, 1)
@@ -449,10 +457,12 @@ def main():
         "data": "synthetic",
         "config": {"workload": args.workload if args.batch is None and args.max_len is None
                    else f"{args.workload} (B={p.B}, max_len={args.max_len})",
-                   "global_batch": p.B * world, "heads": p.H,
+                   "global_batch": (args.batch or WORKLOADS[args.workload]["B"]) * world,
+                   "heads": p.H,
                    "head_dim": p.d, "act": act, "causal": p.causal, "bias": p.bias_kind,
                    "total_tokens": p.total_q, "max_len": p.max_q_len,
-                   "parallelism": f"dp{world} (independent batches)",
+                   "parallelism": (f"dp{world} ({args.partition} split of one global batch)"
+                                   if world > 1 else "dp1"),
                    "l2": "inputs larger than L2 (each of Q/K/V/dO > 126 MB); no flush",
                    "kernel_path": {"fwd": "tcgen05" if path[0] == 1 else "cuda-core",
                                    "bwd": "tcgen05" if path[1] == 1 else "cuda-core"}},
@@ -467,6 +477,15 @@ def main():
         "clocks": clock_info,
     }
 
+    # rank balance of the split: this run's (N > 1), and what an 8-rank split
+    # of 8 x B sequences of this workload would give (host-side only)
+    if split is not None:
+        result["partition"] = split
+    else:
+        gq, gk = draw_lengths(args.workload, args.seed, B=8 * p.B, max_len=args.max_len)
+        result["partition_8_ranks"] = {
+            m: split_report(gq, gk, p.causal, 8, m, args.sub_batch, jfa)[1] for m in ("bbs", "lpt")}
+
     # end to end through the C ABI with host buffers
     if not args.no_e2e:
         result["e2e"] = e2e_leg(args, p, prob, act, dev, stream, jfa, f_fwd + f_bwd, world)
@@ -479,6 +498,40 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def split_report(q_lens, kv_lens, causal, ranks, method, sub_batch, jfa):
+    """Rank imbalance (heaviest rank's visible pairs / mean) of the chosen
+    split and of a contiguous split (rank r takes the r-th run of B/N)."""
+    rank_of, cost = jfa.jfa_partition(q_lens, kv_lens, causal, ranks, method, sub_batch)
+    per = len(q_lens) // ranks
+    contiguous = np.minimum(np.arange(len(q_lens)) // max(per, 1), ranks - 1).astype(np.int32)
+    pairs = visible_pairs(q_lens, kv_lens, causal)
+    c_cost = np.bincount(contiguous, weights=pairs, minlength=ranks)
+    imb = lambda c: float(np.max(c) / np.mean(c)) if np.mean(c) > 0 else 1.0
+    return rank_of, {"method": method, "sub_batch": sub_batch if method == "bbs" else None,
+                     "ranks": ranks, "sequences": int(len(q_lens)),
+                     "imbalance_max_over_mean": imb(cost),
+                     "contiguous_imbalance_max_over_mean": imb(c_cost)}
+
+
+def rank_problem(args, rank, world, jfa):
+    """This rank's batch.  One rank: the workload's batch (seed args.seed).
+    N ranks: the global batch of N x B sequences (lengths from args.seed, the
+    same on every rank), split by jfa_partition; this rank draws the tensors
+    of its own sequences only (seed args.seed + 1 + rank)."""
+    from jagged_attention_recommender_jfa_b200.inputs import WORKLOADS, draw_lengths, make_problem
+    if world == 1:
+        return make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len), None
+    B = args.batch or WORKLOADS[args.workload]["B"]
+    q_lens, kv_lens = draw_lengths(args.workload, args.seed, B=B * world, max_len=args.max_len)
+    causal = WORKLOADS[args.workload]["causal"]
+    rank_of, report = split_report(q_lens, kv_lens, causal, world, args.partition,
+                                   args.sub_batch, jfa)
+    mine = np.nonzero(rank_of == rank)[0]
+    p = make_problem(args.workload, args.seed + 1 + rank, q_lens=q_lens[mine],
+                     kv_lens=kv_lens[mine], max_len=args.max_len)
+    return p, report
 
 
 def aggregate_over_ranks(ms_per_step, flops, device, world):

@@ -164,6 +164,32 @@ jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,
                         int32_t* items, int64_t capacity, int32_t* count, void* workspace,
                         size_t ws_bytes, jfa_stream_t stream);
 
+/* Data-parallel split of one global batch across ranks (HOST function: every
+ * pointer is host memory, nothing touches a GPU).  Sequences are independent,
+ * so each rank runs jfa_forward / jfa_backward on its own sequences with no
+ * collective; the split only has to balance the work, which jagged batches
+ * make uneven ("Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need
+ * a Different Stack", section "Bottleneck move 4: memory relief to load
+ * balance": heaviest rank ~15% above the average; base batch shuffling
+ * pairs heavy and light sub-batches without cross-rank communication).
+ * Every rank computes the same split from the lengths alone.
+ *   q_lens, kv_lens : int32 [batch] sequence lengths (>= 0)
+ *   causal          : cost = visible (query, key) pairs, bottom-right causal
+ *   method          : JFA_PARTITION_LPT -- sequences by cost descending (ties
+ *                     by index), each to the least-loaded rank (ties: lowest);
+ *                     JFA_PARTITION_BBS -- sub-batches of `sub_batch`
+ *                     consecutive sequences sorted by total length (sum of
+ *                     n_q + n_kv, descending, ties by index) and dealt in
+ *                     snake order 0..R-1, R-1..0, ...
+ *   rank_of         : int32 [batch] out, the rank of each sequence
+ *   rank_cost       : int64 [ranks] out (may be NULL), visible pairs per rank
+ *                     (per head)
+ * Returns JFA_ERR_INVALID_ARGUMENT for a bad size, pointer or method. */
+typedef enum { JFA_PARTITION_LPT = 0, JFA_PARTITION_BBS = 1 } jfa_partition_method;
+jfa_status jfa_partition(int32_t batch, const int32_t* q_lens, const int32_t* kv_lens, int causal,
+                         int32_t ranks, int method, int32_t sub_batch, int32_t* rank_of,
+                         int64_t* rank_cost);
+
 /* Synchronises `stream`, then reads and clears the workspace's device error
  * word: JFA_OK, JFA_ERR_BAD_OFFSETS or JFA_ERR_TIMEOUT. */
 jfa_status jfa_check_error(void* workspace, jfa_stream_t stream);
@@ -199,12 +225,20 @@ const char* jfa_kernel_name(int32_t kernel_id);
  *    that device current (cudaGetSymbolAddress) and caches it; make that
  *    first call before any stream capture.
  *  - Problems whose jfa_workspace_bytes(problem, 0) exceeds 8 MiB are
- *    rejected with JFA_ERR_WORKSPACE (e.g. about 16k query tiles x heads).
+ *    rejected with JFA_ERR_WORKSPACE before anything is launched.  That
+ *    count is the tile schedule (about 16 * heads bytes per 16 query rows,
+ *    plus 16 bytes per 16 rows and 8 per sequence), the relative-position
+ *    table prepared for the kernels (16 * heads * max(relpos_len, 384)
+ *    bytes) and, for JFA_MXFP8, the quantised operands: so bf16 batches of a
+ *    few hundred thousand query rows fit, MXFP8 only small ones.
  *  - Every call shares the one array and it keeps the last call's contents;
  *    calls whose work overlaps on the GPU (other streams, other host threads)
  *    race on it and must be serialised by the caller.
- *  - The on-device error word lives in that array too; jfa_check_error()
- *    cannot reach it, so check outputs instead of the error word. */
+ *  - The on-device error word lives in that array too, out of reach of
+ *    jfa_check_error().  Bad offsets (or a timed-out device wait) still
+ *    return JFA_OK here and leave the outputs of the affected rows
+ *    unwritten, so a caller that needs to detect them pre-fills out and lse
+ *    with NaN and treats any row still NaN afterwards as a failed call. */
 jfa_status jfa_forward_fixed_scratch(const jfa_problem* problem, const void* q, const void* k,
                                      const void* v, const int32_t* q_offsets,
                                      const int32_t* kv_offsets, const void* bias, jfa_act act,

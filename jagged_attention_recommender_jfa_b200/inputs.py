@@ -155,6 +155,23 @@ def _normal(rng, shape, std, dtype):
     return t.to(torch.bfloat16)
 
 
+def draw_lengths(workload: str, seed: int = 0, *, B: Optional[int] = None,
+                 max_len: Optional[int] = None):
+    """The (q_lens, kv_lens) that make_problem(workload, seed, B=B,
+    max_len=max_len) draws (the lengths are its first draws), without the
+    tensors: every rank of a data-parallel run can draw the global batch's
+    lengths and split it without drawing the tensors of other ranks."""
+    spec = dict(WORKLOADS[workload])
+    B = spec["B"] if B is None else B
+    rng = np.random.default_rng(seed)
+    q_lens = _lengths(rng, spec["q_len"], B, max_len if spec["kv_len"] is None else None)
+    if spec["kv_len"] is None:
+        kv_lens = q_lens.copy()
+    else:
+        kv_lens = _lengths(rng, spec["kv_len"], B, max_len)
+    return q_lens, kv_lens
+
+
 def make_problem(workload: str, seed: int = 0, *, B: Optional[int] = None,
                  max_len: Optional[int] = None, q_lens=None, kv_lens=None,
                  act: Optional[str] = None, causal: Optional[bool] = None,

@@ -39,7 +39,8 @@ STATUS_NAMES = {0: "JFA_OK", 1: "JFA_ERR_INVALID_ARGUMENT", 2: "JFA_ERR_UNSUPPOR
 EXPORTS = ("jfa_workspace_bytes", "jfa_forward", "jfa_backward", "jfa_quantize_mxfp8",
            "jfa_schedule", "jfa_check_error", "jfa_last_error", "jfa_path",
            "jfa_profile_enable", "jfa_profile_read", "jfa_kernel_name",
-           "jfa_forward_fixed_scratch")
+           "jfa_forward_fixed_scratch", "jfa_partition")
+PARTITION = {"lpt": 0, "bbs": 1}
 
 
 class JfaError(RuntimeError):
@@ -95,6 +96,8 @@ def load():
         lib.jfa_kernel_name.restype = ctypes.c_char_p
         lib.jfa_forward_fixed_scratch.argtypes = [PP, P, P, P, P, P, P, i32, i32, P, P, P]
         lib.jfa_forward_fixed_scratch.restype = i32
+        lib.jfa_partition.argtypes = [i32, P, P, i32, i32, i32, i32, P, P]
+        lib.jfa_partition.restype = i32
         _LIB = lib
         return lib
 
@@ -195,6 +198,22 @@ def jfa_schedule(problem, q_offsets, kv_offsets, causal, backward, tile, items, 
                                _stream(stream)))
 
 
+def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
+    """Host-side split of a global batch across ``ranks``: returns (rank_of
+    int32 [batch], rank_cost int64 [ranks]) as numpy arrays."""
+    import numpy as np
+    ql = np.ascontiguousarray(np.asarray(q_lens, np.int32))
+    kl = np.ascontiguousarray(np.asarray(kv_lens, np.int32))
+    assert ql.shape == kl.shape and ql.ndim == 1
+    rank_of = np.zeros(len(ql), np.int32)
+    rank_cost = np.zeros(int(ranks), np.int64)
+    c = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(load().jfa_partition(len(ql), c(ql), c(kl), int(bool(causal)), int(ranks),
+                                PARTITION.get(method, method), int(sub_batch), c(rank_of),
+                                c(rank_cost)))
+    return rank_of, rank_cost
+
+
 def jfa_profile_enable(enable: bool):
     _check(load().jfa_profile_enable(int(bool(enable))))
 
@@ -233,7 +252,12 @@ def workspace(problem: jfa_problem, backward: bool, device) -> torch.Tensor:
 
 
 def attention_forward(problem, q, k, v, q_offsets, kv_offsets, bias=None, act="softmax",
-                      causal=False, ws=None, stream=None):
+                      causal=False, ws=None, stream=None, check=True):
+    """Allocates out / lse (and the workspace unless ``ws`` is given) and runs
+    jfa_forward.  With ``check`` (the default) the stream is synchronised and
+    the workspace's device error word is read, so that bad offsets or a timed
+    out device wait raise :class:`JfaError` here; ``check=False`` leaves that
+    to the caller (``jfa_check_error(ws)``) and keeps the call asynchronous."""
     out = torch.empty_like(q)
     lse = None
     if act == "softmax":
@@ -242,14 +266,20 @@ def attention_forward(problem, q, k, v, q_offsets, kv_offsets, bias=None, act="s
         ws = workspace(problem, False, q.device)
     jfa_forward(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out, lse, ws,
                 stream=stream)
+    if check:
+        jfa_check_error(ws, stream)
     return out, lse
 
 
 def attention_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias=None,
-                       act="softmax", causal=False, ws=None, stream=None):
+                       act="softmax", causal=False, ws=None, stream=None, check=True):
+    """Allocates dq / dk / dv (and the workspace unless ``ws`` is given) and
+    runs jfa_backward; ``check`` as in :func:`attention_forward`."""
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if ws is None:
         ws = workspace(problem, True, q.device)
     jfa_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act, causal,
                  dq, dk, dv, ws, stream=stream)
+    if check:
+        jfa_check_error(ws, stream)
     return dq, dk, dv

@@ -356,12 +356,20 @@ def test_mxfp8_small(cuda_device, seed):
 # full-size workloads, launched as bench.py launches them, checked on sampled
 # (sequence, head) items that the oracle computes in seconds
 # ---------------------------------------------------------------------------
-def _sample_items(p, n_short=3, max_len=1200, heads=(0,)):
+def _sample_items(p, n_short=3, max_len=1200, heads=None, seed=0):
+    """(sequence, head) items the oracle checks on a full-size batch: the
+    ``n_short`` shortest sequences, the two longest of length <= ``max_len``
+    and the longest of all (the longest key range: many key tiles per row,
+    repeated lazy rescales, relative-position windows clamped at the table's
+    ends, many-way dQ accumulation), each on heads 0, H-1 and one drawn head."""
     lens = np.maximum(p.q_lens, p.kv_lens)
     order = np.argsort(lens, kind="stable")
     picks = list(order[:n_short])
-    mid = [b for b in order if lens[b] <= max_len][-2:]
-    picks += mid
+    picks += [b for b in order if lens[b] <= max_len][-2:]
+    picks.append(order[-1])
+    if heads is None:
+        rng = np.random.default_rng(seed)
+        heads = sorted({0, p.H - 1, int(rng.integers(0, p.H))})
     mask = np.zeros(p.B * p.H, np.int32)
     for b in picks:
         for h in heads:
@@ -397,7 +405,8 @@ def test_full_size_sampled(cuda_device, workload, act):
     p = make_problem(workload, 1)
     act = act or p.act
     out, lse, (dq, dk, dv) = run_gpu(p, cuda_device, act)
-    mask = _sample_items(p, heads=(0, p.H - 1))
+    mask = _sample_items(p)
+    assert mask.reshape(p.B, p.H).any(1)[int(np.argmax(np.maximum(p.q_lens, p.kv_lens)))]
     kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
               causal=p.causal, seq_mask=mask)
     ro, rl = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, **kw)

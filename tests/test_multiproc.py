@@ -1,5 +1,5 @@
-"""The N > 1 path of bench.py on CPU: two gloo ranks, each with its own batch
-(seed + rank), combine their timings the way the benchmark does -- the
+"""The N > 1 path of bench.py on CPU: two gloo ranks, each with its own share
+of the global batch, combine their timings the way the benchmark does -- the
 slowest rank's time and the sum of the ranks' work."""
 import os
 import socket
