@@ -59,7 +59,7 @@ def _lib():
             lib.jfa_oracle_forward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
                                                i32, f64, i32, P, P, P, i32]
             lib.jfa_oracle_backward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                                i32, f64, P, P, P, P, P, P, i32]
+                                                i32, f64, P, P, P, P, P, P, P, i32]
             lib.jfa_oracle_quantize_mx.argtypes = [P, ctypes.c_int64, P, P]
             lib.jfa_oracle_dequantize_mx.argtypes = [P, P, ctypes.c_int64, P]
             lib.jfa_oracle_e4m3_encode.argtypes = [f64]
@@ -135,8 +135,12 @@ def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0
 
 def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpos_len=0,
              act="softmax", causal=False, scale=0.0, seq_mask=None, out_for_d=None,
-             nthreads=0):
-    """fp64 analytic gradients (dq, dk, dv); the bias receives none.
+             dbias=False, nthreads=0):
+    """fp64 analytic gradients (dq, dk, dv), and with ``dbias`` also the bias
+    gradient as a fourth result: for a dense bias an array like ``bias``
+    (ds of each valid pair, 0 at masked pairs, NaN in items not computed),
+    for a relative-position bias the table gradient [H, relpos_len] summed
+    over the computed items.
 
     ``out_for_d``: the forward output whose rows give D = rowsum(dO * O)
     (the MXFP8 forward's output); by default O is recomputed exactly."""
@@ -151,11 +155,18 @@ def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpo
     dv = np.full((total_kv, H, d), np.nan)
     mask = _item_mask(seq_mask, B, H)
     o64 = _f64(out_for_d) if out_for_d is not None else None
+    db = None
+    if dbias and bias_kind == "dense":
+        db = np.full(b64.shape, np.nan)
+    elif dbias and bias_kind == "relpos":
+        db = np.zeros((H, int(relpos_len)))
     _lib().jfa_oracle_backward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                                _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                                ACT[act], int(bool(causal)), float(scale), _ptr(mask),
-                               _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(db),
                                int(nthreads))
+    if dbias:
+        return dq, dk, dv, db
     return dq, dk, dv
 
 

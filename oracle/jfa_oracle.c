@@ -298,12 +298,20 @@ static void forward_item(const orc_problem* P, int b, int h, double* out, double
  * GDPA   : ds_ij = dp_ij act'(s_ij) / n_kv on valid (i, j), 0 elsewhere
  * both   : dV_j += w_ij dO_i, dQ_i += scale sum_j ds_ij k_j,
  *          dK_j += scale ds_ij q_i.
- * The bias gets no gradient.  For MXFP8 the quantisers are straight-through
- * estimators: the gradients are those of the unquantised weights on the
- * dequantised operands, with D taken from the forward's saved output when
- * out_for_d is given. */
+ * Bias ("custom biases", [JFA]): s_ij = scale q_i.k_j + beta_h(i, j), so the
+ * gradient of an additive bias entry is the sum of ds_ij over the pairs that
+ * read it:
+ *   DENSE : dbias at the pair's own position = ds_ij (0 for a masked pair);
+ *   RELPOS: dtable[h][clamp(i - j, -C, C) + C] += ds_ij over valid pairs.
+ * The RELPOS partial sums of this item go to dtab_item (relpos_len entries,
+ * summed over items by the caller in item order); the DENSE gradient goes
+ * straight into dbias_dense (blocks of different items are disjoint).
+ * For MXFP8 the quantisers are straight-through estimators: the gradients
+ * are those of the unquantised weights on the dequantised operands, with D
+ * taken from the forward's saved output when out_for_d is given. */
 static void backward_item(const orc_problem* P, int b, int h, const double* dout,
-                          const double* out_for_d, double* dq, double* dk, double* dv) {
+                          const double* out_for_d, double* dq, double* dk, double* dv,
+                          double* dtab_item, double* dbias_dense) {
     int nq = P->q_off[b + 1] - P->q_off[b];
     int nkv = P->kv_off[b + 1] - P->kv_off[b];
     int H = P->H, d = P->d;
@@ -315,6 +323,11 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
         double* dkj = dk + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
         double* dvj = dv + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
         for (int c = 0; c < d; ++c) dkj[c] = 0.0, dvj[c] = 0.0;
+    }
+    double* dbias_blk = NULL;
+    if (dbias_dense) {
+        dbias_blk = dbias_dense + P->dense_off[b] + (int64_t)h * nq * nkv;
+        for (int64_t e = 0; e < (int64_t)nq * nkv; ++e) dbias_blk[e] = 0.0;
     }
     for (int i = 0; i < nq; ++i) {
         double m, l;
@@ -350,6 +363,14 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
             double ds;
             if (P->act == ORC_ACT_SOFTMAX) ds = w[j] * (dp - Di);
             else ds = dp * act_derivative(P->act, s[j]) / (double)nkv;
+            if (dbias_blk) dbias_blk[(int64_t)i * nkv + j] = ds;
+            if (dtab_item) {
+                int C = (P->relpos_len - 1) / 2;
+                long r = (long)i - (long)j;
+                if (r < -C) r = -C;
+                if (r > C) r = C;
+                dtab_item[r + C] += ds;
+            }
             for (int c = 0; c < d; ++c) {
                 dvj[c] += w[j] * doi[c];
                 dqi[c] += P->scale * ds * kj[c];
@@ -401,15 +422,19 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
     return 0;
 }
 
+/* dbias (may be NULL): DENSE -> same layout as bias; RELPOS -> [H][relpos_len],
+ * overwritten with the sum over the computed items (item order). */
 int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                         const double* q, const double* k, const double* v, int bias_kind,
                         const double* bias, int relpos_len, int act, int causal, double scale,
                         const int32_t* item_mask, const double* dout, const double* out_for_d,
-                        double* dq, double* dk, double* dv, int nthreads) {
+                        double* dq, double* dk, double* dv, double* dbias, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
                  scale, 0);
     long n_items = (long)B * H;
+    const int want_tab = dbias && bias_kind == ORC_BIAS_RELPOS;
+    double** parts = want_tab ? (double**)calloc((size_t)(n_items > 0 ? n_items : 1), sizeof(double*)) : NULL;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -417,7 +442,19 @@ int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t
     for (long it = 0; it < n_items; ++it) {
         int b = (int)(it / H), h = (int)(it % H);
         if (item_mask && !item_mask[it]) continue;
-        backward_item(&P, b, h, dout, out_for_d, dq, dk, dv);
+        if (want_tab) parts[it] = (double*)calloc((size_t)relpos_len, sizeof(double));
+        backward_item(&P, b, h, dout, out_for_d, dq, dk, dv, want_tab ? parts[it] : NULL,
+                      (dbias && bias_kind == ORC_BIAS_DENSE) ? dbias : NULL);
+    }
+    if (want_tab) {
+        for (long e = 0; e < (long)H * relpos_len; ++e) dbias[e] = 0.0;
+        for (long it = 0; it < n_items; ++it) {
+            if (!parts[it]) continue;
+            int h = (int)(it % H);
+            for (int c = 0; c < relpos_len; ++c) dbias[(long)h * relpos_len + c] += parts[it][c];
+            free(parts[it]);
+        }
+        free(parts);
     }
     free((void*)P.dense_off);
     (void)nthreads;

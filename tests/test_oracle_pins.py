@@ -399,3 +399,96 @@ def test_backward_d_from_saved_output():
                              out_for_d=out * 1.01, **kw)
     assert np.array_equal(bumped[2], ref[2])
     assert not np.allclose(bumped[0], ref[0])
+
+
+# ---------------------------------------------------------------------------
+# Bias gradient ("custom biases": s = scale q.k + beta, so d loss / d beta is
+# the score gradient summed over the pairs that read each bias entry)
+# ---------------------------------------------------------------------------
+BIAS_CASES = [c for c in CASES if c[3] != "none"]
+
+
+@pytest.mark.parametrize("act", ["softmax", "silu", "gelu_tanh"])
+@pytest.mark.parametrize("q_lens,kv_lens,causal,bias_kind", BIAS_CASES)
+def test_bias_gradient_equals_autograd(act, q_lens, kv_lens, causal, bias_kind):
+    P = _jagged(12, q_lens, kv_lens, bias_kind=bias_kind)
+    got = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                          bias=P["bias"], bias_kind=bias_kind, relpos_len=P["relpos_len"],
+                          act=act, causal=causal, dbias=True)
+    P = dict(P)
+    P["bias"] = P["bias"].clone().requires_grad_()
+    if act == "softmax":
+        qp, kp, vp, mask, valid = _padded_sdpa(P, causal)
+        row_ok = valid.any(-1, keepdim=True)
+        # rows that see no key take a zero mask (their output is discarded
+        # below), so that no NaN of an all -inf row enters the backward
+        mask = torch.where(row_ok, mask, torch.zeros_like(mask))
+        ref = F.scaled_dot_product_attention(qp, kp, vp, attn_mask=mask)
+        ref = torch.where(row_ok, ref, torch.zeros_like(ref))
+    else:
+        ref = _padded_gdpa(P, causal, act, P["q"], P["k"], P["v"])
+    o = _unpad(ref, P["q_off"])
+    (o * P["do"]).sum().backward()
+    np.testing.assert_allclose(got[3], P["bias"].grad.numpy(), atol=1e-12, rtol=0)
+    # and the other gradients are unchanged by asking for it
+    base = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                           bias=P["bias"].detach(), bias_kind=bias_kind,
+                           relpos_len=P["relpos_len"], act=act, causal=causal)
+    for a, b in zip(base, got[:3]):
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("act", ["softmax", "gelu_tanh"])
+@pytest.mark.parametrize("bias_kind", ["relpos", "dense"])
+def test_bias_gradient_matches_central_differences(act, bias_kind):
+    # relpos_len 5 < 2 * max_len + 1: the clamped end entries collect every
+    # pair beyond the table
+    P = _jagged(13, [4, 5], [5, 3], H=1, d=4, bias_kind=bias_kind, relpos_len=5)
+    kw = dict(bias_kind=bias_kind, relpos_len=P["relpos_len"], act=act, causal=True)
+    do = P["do"].numpy()
+    base = P["bias"].numpy().copy()
+
+    def loss(bias):
+        o, _ = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], bias=bias, **kw)
+        return float(np.sum(o * do))
+
+    _, _, _, db = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                                  bias=P["bias"], dbias=True, **kw)
+    h = 1e-6
+    fd = np.zeros_like(base)
+    for idx in np.ndindex(*base.shape):
+        plus, minus = base.copy(), base.copy()
+        plus[idx] += h
+        minus[idx] -= h
+        fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
+    assert np.abs(fd - db).max() / max(1.0, np.abs(fd).max()) < 1e-6
+    if bias_kind == "relpos":
+        # bottom-right causal: i - j >= -1 in sequence 0 (n_kv = n_q + 1) and
+        # >= 2 in sequence 1, so the clamped upper end collects pairs and the
+        # lower end (i - j <= -2) is read by none
+        assert db[0, -1] != 0.0 and db[0, 0] == 0.0
+
+
+def test_bias_gradient_closed_form_uniform_scores():
+    # Q = 0, zero bias, softmax: p_ij = 1 / n_vis(i) and, with V = 0,
+    # dp = 0 and D = 0, so ds = 0; with dO = 1 and V = e_j-th basis-like
+    # values ds_ij = p_ij (v_j . 1 - mean_vis(v . 1)).  Summed over a row the
+    # bias gradient vanishes (softmax is shift-invariant): sum_j ds_ij = 0.
+    P = _jagged(14, [6, 3], [6, 3], H=2, d=4, bias_kind="dense")
+    q0 = torch.zeros_like(P["q"])
+    b0 = torch.zeros_like(P["bias"])
+    _, _, _, db = oracle.backward(P["q_off"], P["kv_off"], q0, P["k"], P["v"], P["do"],
+                                  bias=b0, bias_kind="dense", causal=True, dbias=True)
+    pos = 0
+    for b, n in enumerate([6, 3]):
+        blk = db[pos:pos + 2 * n * n].reshape(2, n, n)
+        vb = P["v"][int(P["kv_off"][b]):int(P["kv_off"][b]) + n].numpy()
+        dob = P["do"][int(P["q_off"][b]):int(P["q_off"][b]) + n].numpy()
+        for h in range(2):
+            np.testing.assert_allclose(blk[h].sum(1), 0.0, atol=1e-14)
+            for i in range(n):
+                dpv = vb[:i + 1, h] @ dob[i, h]            # dp_ij, j <= i
+                want = (dpv - dpv.mean()) / (i + 1)
+                np.testing.assert_allclose(blk[h, i, :i + 1], want, atol=1e-14)
+                assert np.all(blk[h, i, i + 1:] == 0.0)    # masked pairs
+        pos += 2 * n * n
