@@ -57,9 +57,9 @@ def _lib():
             P = ctypes.c_void_p
             i32, f64 = ctypes.c_int, ctypes.c_double
             lib.jfa_oracle_forward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                               i32, f64, i32, P, P, P, i32]
+                                               i32, f64, i32, i32, P, P, P, i32]
             lib.jfa_oracle_backward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                                i32, f64, P, P, P, P, P, P, P, i32]
+                                                i32, f64, i32, P, P, P, P, P, P, P, i32]
             lib.jfa_oracle_quantize_mx.argtypes = [P, ctypes.c_int64, P, P]
             lib.jfa_oracle_dequantize_mx.argtypes = [P, P, ctypes.c_int64, P]
             lib.jfa_oracle_e4m3_encode.argtypes = [f64]
@@ -113,11 +113,14 @@ def _item_mask(seq_mask, B, H):
 
 def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0,
             act="softmax", causal=False, scale=0.0, quant_p=False, seq_mask=None,
-            nthreads=0):
+            block=0, nthreads=0):
     """fp64 forward.  Returns (out [total_q,H,d], lse [total_q,H] or None).
 
     ``seq_mask`` ([B] per sequence or [B*H] per (sequence, head)) selects what
-    is computed; everything else is NaN in the result."""
+    is computed; everything else is NaN in the result.  ``block`` > 0:
+    BlockAttention, each query sees only the keys of its own block of
+    ``block`` consecutive positions (GDPA then divides by the block's key
+    count)."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     q64, k64, v64 = _f64(q), _f64(k), _f64(v)
     B = len(q_off) - 1
@@ -129,13 +132,13 @@ def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0
     _lib().jfa_oracle_forward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                               _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                               ACT[act], int(bool(causal)), float(scale), int(bool(quant_p)),
-                              _ptr(mask), _ptr(out), _ptr(lse), int(nthreads))
+                              int(block), _ptr(mask), _ptr(out), _ptr(lse), int(nthreads))
     return out, (lse if act == "softmax" else None)
 
 
 def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpos_len=0,
              act="softmax", causal=False, scale=0.0, seq_mask=None, out_for_d=None,
-             dbias=False, nthreads=0):
+             dbias=False, block=0, nthreads=0):
     """fp64 analytic gradients (dq, dk, dv), and with ``dbias`` also the bias
     gradient as a fourth result: for a dense bias an array like ``bias``
     (ds of each valid pair, 0 at masked pairs, NaN in items not computed),
@@ -162,9 +165,9 @@ def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpo
         db = np.zeros((H, int(relpos_len)))
     _lib().jfa_oracle_backward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                                _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
-                               ACT[act], int(bool(causal)), float(scale), _ptr(mask),
-                               _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(db),
-                               int(nthreads))
+                               ACT[act], int(bool(causal)), float(scale), int(block),
+                               _ptr(mask), _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(db), int(nthreads))
     if dbias:
         return dq, dk, dv, db
     return dq, dk, dv

@@ -76,10 +76,25 @@ static double act_derivative(int act, double x) {
 
 /* Causal validity with bottom-right alignment: query i may see key j when
  * j <= i + (n_kv - n_q); for self-attention (n_q == n_kv) this is j <= i. */
-static int is_valid(int causal, int i, int j, int nq, int nkv) {
+static int causal_ok(int causal, int i, int j, int nq, int nkv) {
     if (!causal) return 1;
     return (long)j <= (long)i + (long)(nkv - nq);
 }
+
+/* BlockAttention ("Meta Enhances GEM Training Efficiency ...", "Exploring the
+ * Customized Kernel Library" -> "BlockAttention": windows instead of full
+ * attention over the user history; "Meta GEM Training Efficiency ...",
+ * "Bottleneck move 1": long-sequence attention as independent fixed-size
+ * blocks).  With block length W > 0 the keys of a sequence form blocks
+ * [c W, (c + 1) W) and query i, at the bottom-right aligned position
+ * p = i + n_kv - n_q (p = i for self-attention), sees only the keys of block
+ * floor(p / W) (none when p < 0); the causal rule applies on top. */
+static int block_of(int W, int i, int nq, int nkv) {
+    long p = (long)i + (long)(nkv - nq);
+    return p < 0 ? -1 : (int)(p / W);
+}
+
+
 
 /* Additive bias beta_h(i, j).
  *  RELPOS: table[h][clamp(i - j, -C, C) + C], table length T = 2C + 1.
@@ -193,7 +208,24 @@ typedef struct {
     int act, causal;
     double scale;
     int quant_p; /* MXFP8: quantise exp(s - m) per 32 keys before P.V */
+    int block;   /* BlockAttention block length; 0 = full attention */
 } orc_problem;
+
+static int is_valid(const orc_problem* P, int i, int j, int nq, int nkv) {
+    if (!causal_ok(P->causal, i, j, nq, nkv)) return 0;
+    if (P->block > 0 && block_of(P->block, i, nq, nkv) != j / P->block) return 0;
+    return 1;
+}
+
+/* The GDPA normaliser: the sequence's n_kv, or with BlockAttention the
+ * number of keys in the query's block. */
+static double gdpa_norm(const orc_problem* P, int i, int nq, int nkv) {
+    if (P->block <= 0) return (double)nkv;
+    int c = block_of(P->block, i, nq, nkv);
+    if (c < 0) return 1.0;  /* the row sees no key; nothing is divided */
+    int n = nkv - c * P->block;
+    return (double)(n < P->block ? n : P->block);
+}
 
 static const double* row_ptr(const double* base, int64_t row, int H, int h, int d) {
     return base + (row * H + h) * (int64_t)d;
@@ -216,12 +248,12 @@ static void row_weights(const orc_problem* P, int b, int h, int i, double* s, do
         s[j] = P->scale * dot +
                bias_value(P->bias_kind, P->bias, P->relpos_len, P->H, h,
                           P->dense_off ? P->dense_off[b] : 0, nq, nkv, i, j);
-        if (is_valid(P->causal, i, j, nq, nkv) && s[j] > m) m = s[j];
+        if (is_valid(P, i, j, nq, nkv) && s[j] > m) m = s[j];
     }
     if (P->act == ORC_ACT_SOFTMAX) {
         double l = 0.0;
         for (int j = 0; j < nkv; ++j)
-            w[j] = is_valid(P->causal, i, j, nq, nkv) ? exp(s[j] - m) : 0.0;
+            w[j] = is_valid(P, i, j, nq, nkv) ? exp(s[j] - m) : 0.0;
         for (int j = 0; j < nkv; ++j) l += w[j];
         if (pv_weight) {
             if (P->quant_p) {
@@ -232,12 +264,12 @@ static void row_weights(const orc_problem* P, int b, int h, int i, double* s, do
                  * the codes independent of which integer R a kernel uses. */
                 double xmax = -INFINITY;
                 for (int j = 0; j < nkv; ++j)
-                    if (is_valid(P->causal, i, j, nq, nkv) && s[j] * M_LOG2E > xmax) xmax = s[j] * M_LOG2E;
+                    if (is_valid(P, i, j, nq, nkv) && s[j] * M_LOG2E > xmax) xmax = s[j] * M_LOG2E;
                 const double R = ceil(xmax);
                 double* w2 = (double*)malloc(sizeof(double) * (size_t)(nkv > 0 ? nkv : 1));
                 double l2 = 0.0;
                 for (int j = 0; j < nkv; ++j) {
-                    w2[j] = is_valid(P->causal, i, j, nq, nkv) ? exp2(s[j] * M_LOG2E - R) : 0.0;
+                    w2[j] = is_valid(P, i, j, nq, nkv) ? exp2(s[j] * M_LOG2E - R) : 0.0;
                     l2 += w2[j];
                 }
                 for (int j0 = 0; j0 < nkv; j0 += 32) {
@@ -260,7 +292,7 @@ static void row_weights(const orc_problem* P, int b, int h, int i, double* s, do
         *l_out = l;
     } else {
         for (int j = 0; j < nkv; ++j)
-            w[j] = is_valid(P->causal, i, j, nq, nkv) ? act_value(P->act, s[j]) / (double)nkv : 0.0;
+            w[j] = is_valid(P, i, j, nq, nkv) ? act_value(P->act, s[j]) / gdpa_norm(P, i, nq, nkv) : 0.0;
         if (pv_weight)
             for (int j = 0; j < nkv; ++j) pv_weight[j] = w[j];
         *m_out = m;
@@ -353,7 +385,7 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
             for (int c = 0; c < d; ++c) Di += doi[c] * o[c];
         }
         for (int j = 0; j < nkv; ++j) {
-            if (!is_valid(P->causal, i, j, nq, nkv)) continue;
+            if (!is_valid(P, i, j, nq, nkv)) continue;
             const double* kj = row_ptr(P->k, P->kv_off[b] + j, H, h, d);
             const double* vj = row_ptr(P->v, P->kv_off[b] + j, H, h, d);
             double* dkj = dk + ((int64_t)(P->kv_off[b] + j) * H + h) * d;
@@ -362,7 +394,7 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
             for (int c = 0; c < d; ++c) dp += doi[c] * vj[c];
             double ds;
             if (P->act == ORC_ACT_SOFTMAX) ds = w[j] * (dp - Di);
-            else ds = dp * act_derivative(P->act, s[j]) / (double)nkv;
+            else ds = dp * act_derivative(P->act, s[j]) / gdpa_norm(P, i, nq, nkv);
             if (dbias_blk) dbias_blk[(int64_t)i * nkv + j] = ds;
             if (dtab_item) {
                 int C = (P->relpos_len - 1) / 2;
@@ -386,7 +418,7 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
 static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_off,
                          const int32_t* kv_off, const double* q, const double* k, const double* v,
                          int bias_kind, const double* bias, int relpos_len, int act, int causal,
-                         double scale, int quant_p) {
+                         double scale, int quant_p, int block) {
     P->B = B; P->H = H; P->d = d;
     P->q_off = q_off; P->kv_off = kv_off;
     P->q = q; P->k = k; P->v = v;
@@ -395,6 +427,7 @@ static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_o
     P->act = act; P->causal = causal;
     P->scale = scale > 0.0 ? scale : 1.0 / sqrt((double)d);
     P->quant_p = quant_p;
+    P->block = block;
 }
 
 /* Forward over all (sequence b, head h) items with item_mask == NULL or
@@ -402,11 +435,11 @@ static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_o
 int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                        const double* q, const double* k, const double* v, int bias_kind,
                        const double* bias, int relpos_len, int act, int causal, double scale,
-                       int quant_p, const int32_t* item_mask, double* out, double* lse,
-                       int nthreads) {
+                       int quant_p, int block, const int32_t* item_mask, double* out,
+                       double* lse, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
-                 scale, quant_p);
+                 scale, quant_p, block);
     long n_items = (long)B * H;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -427,11 +460,12 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
 int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                         const double* q, const double* k, const double* v, int bias_kind,
                         const double* bias, int relpos_len, int act, int causal, double scale,
-                        const int32_t* item_mask, const double* dout, const double* out_for_d,
-                        double* dq, double* dk, double* dv, double* dbias, int nthreads) {
+                        int block, const int32_t* item_mask, const double* dout,
+                        const double* out_for_d, double* dq, double* dk, double* dv,
+                        double* dbias, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
-                 scale, 0);
+                 scale, 0, block);
     long n_items = (long)B * H;
     const int want_tab = dbias && bias_kind == ORC_BIAS_RELPOS;
     double** parts = want_tab ? (double**)calloc((size_t)(n_items > 0 ? n_items : 1), sizeof(double*)) : NULL;

@@ -492,3 +492,77 @@ def test_bias_gradient_closed_form_uniform_scores():
                 np.testing.assert_allclose(blk[h, i, :i + 1], want, atol=1e-14)
                 assert np.all(blk[h, i, i + 1:] == 0.0)    # masked pairs
         pos += 2 * n * n
+
+
+# ---------------------------------------------------------------------------
+# BlockAttention: each query sees only the keys of its own block of W
+# consecutive positions (causal on top)
+# ---------------------------------------------------------------------------
+def _block_mask(P, Lq, Lk, causal, W):
+    valid = _valid_mask(P, Lq, Lk, causal)
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    return valid & ((i // W) == (j // W))[None, None]
+
+
+@pytest.mark.parametrize("W", [1, 3, 4, 16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_attention_equals_block_masked_sdpa(W, causal):
+    lens = [5, 1, 9, 12]
+    P = _jagged(15, lens, lens, bias_kind="relpos")
+    kw = dict(bias=P["bias"], bias_kind="relpos", relpos_len=P["relpos_len"], causal=causal,
+              block=W)
+    out, lse = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
+    dq, dk, dv, db = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                                     dbias=True, **kw)
+    L = max(lens)
+    q = P["q"].clone().requires_grad_()
+    k = P["k"].clone().requires_grad_()
+    v = P["v"].clone().requires_grad_()
+    Pb = dict(P)
+    Pb["bias"] = P["bias"].clone().requires_grad_()
+    qp = _pad(q, P["q_off"], L).transpose(1, 2)
+    kp = _pad(k, P["kv_off"], L).transpose(1, 2)
+    vp = _pad(v, P["kv_off"], L).transpose(1, 2)
+    valid = _block_mask(P, L, L, causal, W)
+    row_ok = valid.any(-1, keepdim=True)
+    mask = _padded_bias(Pb, L, L).masked_fill(~valid, float("-inf"))
+    mask = torch.where(row_ok, mask, torch.zeros_like(mask))
+    ref = F.scaled_dot_product_attention(qp, kp, vp, attn_mask=mask)
+    ref = torch.where(row_ok, ref, torch.zeros_like(ref))
+    scores = (qp @ kp.transpose(-1, -2) / math.sqrt(P["d"]) + mask).masked_fill(~valid, float("-inf"))
+    ref_lse = _unpad(torch.logsumexp(scores, -1)[..., None], P["q_off"])[..., 0]
+    o = _unpad(ref, P["q_off"])
+    np.testing.assert_allclose(out, o.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, ref_lse.detach().numpy(), atol=1e-12, rtol=0)
+    (o * P["do"]).sum().backward()
+    np.testing.assert_allclose(dq, q.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(db, Pb["bias"].grad.numpy(), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("act", ["softmax", "silu", "gelu_tanh"])
+def test_block_attention_is_attention_on_the_blocks(act):
+    # independent fixed-size blocks: the same as plain jagged attention over
+    # the sequences cut into blocks of W (the last one shorter), bit for bit;
+    # GDPA divides by the block's key count
+    lens, W = [7, 1, 16, 10], 4
+    P = _jagged(16, lens, lens, bias_kind="relpos")
+    kw = dict(bias=P["bias"], bias_kind="relpos", relpos_len=P["relpos_len"], act=act,
+              causal=True)
+    out, lse = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], block=W, **kw)
+    grads = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"], block=W,
+                            **kw)
+    cut = [min(W, n - c) for n in lens for c in range(0, n, W)]
+    off = torch.tensor([0] + list(np.cumsum(cut)), dtype=torch.int32)
+    out2, lse2 = oracle.forward(off, off, P["q"], P["k"], P["v"], **kw)
+    grads2 = oracle.backward(off, off, P["q"], P["k"], P["v"], P["do"], **kw)
+    assert np.array_equal(out, out2)
+    if act == "softmax":
+        assert np.array_equal(lse, lse2)
+    for a, b in zip(grads, grads2):
+        assert np.array_equal(a, b)
+    # and it differs from full attention whenever a sequence spans blocks
+    full, _ = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
+    assert not np.allclose(full, out)
