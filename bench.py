@@ -72,6 +72,8 @@ def parse_args():
                     help="override the workload's number of sequences (profiling captures)")
     ap.add_argument("--max-len", type=int, default=None,
                     help="override the workload's length clip (profiling captures)")
+    ap.add_argument("--block", type=int, default=0,
+                    help="BlockAttention block length (self-attention workloads); 0 = full")
     ap.add_argument("--partition", choices=["bbs", "lpt"], default="bbs",
                     help="split of the global batch across ranks (N > 1)")
     ap.add_argument("--sub-batch", type=int, default=8,
@@ -88,12 +90,16 @@ def parse_args():
 # ---------------------------------------------------------------------------
 # work accounting
 # ---------------------------------------------------------------------------
-def visible_pairs(q_lens, kv_lens, causal):
-    """Per-sequence number of (query, key) pairs attention computes."""
+def visible_pairs(q_lens, kv_lens, causal, block=0):
+    """Per-sequence number of (query, key) pairs attention computes; with
+    BlockAttention (block > 0, self-attention) only pairs inside a block."""
     out = np.zeros(len(q_lens), np.int64)
     for b, (nq, nk) in enumerate(zip(q_lens, kv_lens)):
         nq, nk = int(nq), int(nk)
-        if not causal:
+        if block > 0:
+            m = np.minimum(block, nq - np.arange(0, nq, block)).astype(np.int64)
+            out[b] = int((m * (m + 1) // 2).sum() if causal else (m * m).sum())
+        elif not causal:
             out[b] = nq * nk
         else:
             i = np.arange(nq, dtype=np.int64)
@@ -101,8 +107,8 @@ def visible_pairs(q_lens, kv_lens, causal):
     return out
 
 
-def flops_of(p, pairs_per_seq=None):
-    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal) if pairs_per_seq is None else pairs_per_seq
+def flops_of(p, pairs_per_seq=None, block=0):
+    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block) if pairs_per_seq is None else pairs_per_seq
     f_fwd = 4.0 * p.d * p.H * float(pairs.sum())
     return f_fwd, 2.5 * f_fwd
 
@@ -209,10 +215,10 @@ def recorded_traffic(kernel, workload):
 # ---------------------------------------------------------------------------
 # reference arm / CPU baseline: the fp64 oracle on a bounded stratified sample
 # ---------------------------------------------------------------------------
-def cpu_sample_mask(p, target_pairs_heads):
+def cpu_sample_mask(p, target_pairs_heads, block=0):
     """Sequences picked evenly over the length-sorted batch (shortest first)
     until the sample holds ~target (pairs x heads)."""
-    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal) * p.H
+    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block) * p.H
     order = np.argsort(pairs, kind="stable")
     mask = np.zeros(p.B, np.int32)
     total = 0
@@ -229,20 +235,20 @@ def cpu_sample_mask(p, target_pairs_heads):
     return mask, pairs
 
 
-def run_oracle_step(p, mask, act):
+def run_oracle_step(p, mask, act, block=0):
     import oracle
     kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
-              causal=p.causal, seq_mask=mask)
+              causal=p.causal, seq_mask=mask, block=block)
     o, l = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, **kw)
     oracle.backward(p.q_off, p.kv_off, p.q, p.k, p.v, p.dout, **kw)
 
 
-def cpu_baseline(p, act, target):
+def cpu_baseline(p, act, target, block=0):
     import oracle
-    mask, pairs = cpu_sample_mask(p, target)
+    mask, pairs = cpu_sample_mask(p, target, block)
     f_fwd = 4.0 * p.d * float((pairs * mask).sum())
     t0 = time.perf_counter()
-    run_oracle_step(p, mask, act)
+    run_oracle_step(p, mask, act, block)
     dt = time.perf_counter() - t0
     n = int(mask.sum())
     return {"value": 3.5 * f_fwd / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
@@ -259,13 +265,13 @@ def reference_arm(args, rank, world):
     p = make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len)
     act = args.act or p.act
     target = args.cpu_sample_pairs / 4
-    mask, pairs = cpu_sample_mask(p, target)
+    mask, pairs = cpu_sample_mask(p, target, args.block)
     f_sample = 3.5 * 4.0 * p.d * float((pairs * mask).sum())
     for _ in range(args.warmup):
-        run_oracle_step(p, mask, act)
+        run_oracle_step(p, mask, act, args.block)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        run_oracle_step(p, mask, act)
+        run_oracle_step(p, mask, act, args.block)
     dt = (time.perf_counter() - t0) / max(1, args.steps)
     value = f_sample / dt / 1e12
     n = int(mask.sum())
@@ -275,7 +281,7 @@ def reference_arm(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "global_batch": p.B, "heads": p.H,
-                   "head_dim": p.d, "act": act, "causal": p.causal,
+                   "head_dim": p.d, "act": act, "causal": p.causal, "block": args.block or None,
                    "sample_sequences": n, "l2": "inputs larger than L2"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
@@ -355,8 +361,16 @@ def main():
     act = args.act or p.act
     prob = jfa.problem_of(p)
     path = jfa.jfa_path(prob, act, 0), jfa.jfa_path(prob, act, 1)
-    f_fwd, f_bwd = flops_of(p)
+    f_fwd, f_bwd = flops_of(p, block=args.block)
     d = {n: getattr(p, n).to(dev).contiguous() for n in ("q", "k", "v", "dout", "q_off", "kv_off")}
+    seq_off = d["q_off"]
+    if args.block:
+        # BlockAttention: the same kernels over the blocks; the offsets are
+        # rewritten inside every timed step
+        if not torch.equal(p.q_off, p.kv_off):
+            raise SystemExit("--block needs a self-attention workload")
+        prob, boff = jfa.block_attention(prob, seq_off, args.block)
+        d["q_off"] = d["kv_off"] = boff
     bias = p.bias.to(dev).contiguous() if p.bias is not None else None
     out = torch.empty_like(d["q"])
     lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
@@ -369,6 +383,8 @@ def main():
     def step(marks=None):
         if marks is not None:
             marks[0].record(stream)
+        if args.block:
+            jfa.jfa_block_offsets(seq_off, p.B, p.total_q, args.block, d["q_off"], stream=stream)
         jfa.jfa_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"], bias, act,
                         p.causal, out, lse, ws_f, stream=stream)
         if marks is not None:
@@ -431,12 +447,20 @@ def main():
         avg_s = per[dom][1] / per[dom][0] * 1e-3
         d_ = p.d
         pairs = f_fwd / (4.0 * d_)
-        algo = {"tc_fwd": f_fwd, "tc_bwd": f_bwd, "simt_fwd": f_fwd,
+        algo = {"tc_fwd": f_fwd, "tc_fwd_mxfp8": f_fwd, "tc_bwd": f_bwd, "simt_fwd": f_fwd,
                 "simt_bwd_dq": 6.0 * d_ * pairs, "simt_bwd_dkdv": 8.0 * d_ * pairs}.get(dom)
-        if dom.startswith("tc_"):
-            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        if dom == "tc_fwd_mxfp8":
+            # E4M3 block-scaled MMAs: the measured bf16 peak x the nominal
+            # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+            peak = 2.0 * peaks["bf16_tflops"]
             bound, unit = "tensor", "TFLOP/s"
-            note = f"bf16 dense, sustained, of {peak_src}"
+            note = f"fp8 dense = 2 x bf16 burst of {peak_src}"
+        elif dom.startswith("tc_"):
+            # the kernel runs for milliseconds inside a sub-second timed
+            # region: the burst figure applies
+            peak = peaks["bf16_tflops"]
+            bound, unit = "tensor", "TFLOP/s"
+            note = f"bf16 dense, burst, of {peak_src}"
         else:
             mhz = peaks.get("sm_max_mhz", 1965.0)
             peak = SM_COUNT * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
@@ -461,6 +485,7 @@ def main():
                    "heads": p.H,
                    "head_dim": p.d, "act": act, "causal": p.causal, "bias": p.bias_kind,
                    "total_tokens": p.total_q, "max_len": p.max_q_len,
+                   "block": args.block or None,
                    "parallelism": (f"dp{world} ({args.partition} split of one global batch)"
                                    if world > 1 else "dp1"),
                    "l2": "inputs larger than L2 (each of Q/K/V/dO > 126 MB); no flush",
@@ -471,6 +496,9 @@ def main():
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
         "pct_of_bf16_burst_peak": {"fwd": 100 * f_fwd / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                                    "bwd": 100 * f_bwd / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+        # the MXFP8 forward against the fp8 peak (2 x the measured bf16 burst)
+        "pct_of_fp8_burst_peak": ({"fwd": 50 * f_fwd / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+                                  if p.dtype == "mxfp8" else None),
         "roofline": roofline,
         "kernels": kernels,
         "gpu_launches": len(launches),
@@ -489,10 +517,10 @@ def main():
     # end to end through the C ABI with host buffers
     if not args.no_e2e:
         result["e2e"] = e2e_leg(args, p, prob, act, dev, stream, jfa, f_fwd + f_bwd, world)
-    if rank == 0 and world == 1 and not args.no_padded:
+    if rank == 0 and world == 1 and not args.no_padded and not args.block:
         result["padded_dense_baseline"] = padded_dense_baseline(p, dev, f_fwd + f_bwd)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(p, act, args.cpu_sample_pairs)
+        result["cpu_baseline"] = cpu_baseline(p, act, args.cpu_sample_pairs, args.block)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -568,6 +596,8 @@ def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
         sets.append((dev_in, out, lse, dq, dk, dv))
     ws_f = jfa.workspace(prob, False, dev)
     ws_b = jfa.workspace(prob, True, dev)
+    # BlockAttention: block offsets rebuilt from each step's sequence offsets
+    boffs = [torch.empty(prob.batch + 1, dtype=torch.int32, device=dev) for _ in range(2)]
 
     def results_of(st):
         _, out, lse, dq, dk, dv = st
@@ -593,12 +623,15 @@ def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
             stream.wait_event(in_ready[b])
             if i >= 2:
                 stream.wait_event(out_free[b])        # results of step i-2 are out
-            jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["q_off"],
-                            dev_in["kv_off"], dev_in.get("bias"), act, p.causal, out, lse, ws_f,
-                            stream=stream)
+            qo, ko = dev_in["q_off"], dev_in["kv_off"]
+            if args.block:
+                jfa.jfa_block_offsets(qo, p.B, p.total_q, args.block, boffs[b], stream=stream)
+                qo = ko = boffs[b]
+            jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], qo, ko,
+                            dev_in.get("bias"), act, p.causal, out, lse, ws_f, stream=stream)
             jfa.jfa_backward(prob, dev_in["q"], dev_in["k"], dev_in["v"], out, lse, dev_in["dout"],
-                             dev_in["q_off"], dev_in["kv_off"], dev_in.get("bias"), act, p.causal,
-                             dq, dk, dv, ws_b, stream=stream)
+                             qo, ko, dev_in.get("bias"), act, p.causal, dq, dk, dv, ws_b,
+                             stream=stream)
             comp_done[b].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(comp_done[b])

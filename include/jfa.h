@@ -21,7 +21,8 @@
  *   softmax: o_i = sum_valid softmax_j(s_ij) v_j,  lse_i = log sum_valid e^{s_ij}
  *   GDPA   : o_i = sum_valid act(s_ij) / n_kv(b) * v_j           (no lse)
  * A query row with no valid key gets o_i = 0 and lse_i = -inf; its gradients
- * are 0.  The bias receives no gradient.
+ * are 0.  jfa_backward leaves the bias alone; jfa_backward_dbias also returns
+ * its gradient.
  *
  * Layouts (all row-major, head_dim contiguous):
  *   q, out, dout, dq : [total_q ][heads][head_dim]
@@ -34,7 +35,8 @@
  *                      concatenated, so block b starts at
  *                      sum_{b'<b} heads * n_q(b') * n_kv(b') (int64).
  * Element type: JFA_F32 -> float; JFA_BF16 and JFA_MXFP8 -> bfloat16 (MXFP8
- * computes on E4M3 operands quantised inside the call; outputs stay bf16).
+ * quantises Q, K and V to E4M3 with E8M0 scales per 32 inside the call and
+ * runs block-scaled E4M3 MMAs; outputs stay bf16).
  *
  * Conventions shared by every entry point:
  *  - Ownership: the caller owns every buffer.  All tensor, offset and
@@ -120,6 +122,27 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
                        jfa_act act, int causal, void* out, float* lse, void* workspace,
                        size_t ws_bytes, jfa_stream_t stream);
 
+/* MXFP8 forward on operands that their producer has already quantised (a
+ * normalisation or projection kernel that writes MX directly, such as
+ * jfa_norm_quantize_mxfp8), so that no separate cast pass runs ("Meta GEM
+ * Training Efficiency: Why LLM-Scale Recommenders Need a Different Stack",
+ * "Bottleneck move 2": scale generation and casting must not eat the
+ * low-precision gain).  Softmax attention with block-scaled E4M3 MMAs, P
+ * quantised per 32 keys in the kernel; problem->dtype must be JFA_MXFP8 and
+ * head_dim 128 (else JFA_ERR_UNSUPPORTED).  Device inputs, in the layouts of
+ * jfa_quantize_mxfp8:
+ *   q8, k8, v8         E4M3 codes [rows][heads][128]
+ *   q_scales, k_scales E8M0 [rows][heads][4], blocks of 32 along d
+ *   v_scales           E8M0 [blocks][heads][128], blocks of 32 keys of each
+ *                      sequence counted from its first key (along_rows = 1)
+ * Everything else (offsets, bias, causal, out bf16, lse, workspace of
+ * jfa_workspace_bytes(problem, 0), stream, errors) is as for jfa_forward. */
+jfa_status jfa_forward_mxfp8(const jfa_problem* problem, const uint8_t* q8, const uint8_t* q_scales,
+                             const uint8_t* k8, const uint8_t* k_scales, const uint8_t* v8,
+                             const uint8_t* v_scales, const int32_t* q_offsets,
+                             const int32_t* kv_offsets, const void* bias, int causal, void* out,
+                             float* lse, void* workspace, size_t ws_bytes, jfa_stream_t stream);
+
 /* Backward pass: gradients of <dout, out> with respect to q, k and v.
  * out and lse are the forward's results (softmax needs both; GDPA needs
  * neither and accepts NULL); dout: device like out.  dq/dk/dv: device
@@ -130,6 +153,28 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
                         const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
                         jfa_act act, int causal, void* dq, void* dk, void* dv, void* workspace,
                         size_t ws_bytes, jfa_stream_t stream);
+
+/* Backward pass that also returns the gradient of the additive bias
+ * ("custom biases", "Meta GEM Training Efficiency: Why LLM-Scale Recommenders
+ * Need a Different Stack", section "Bottleneck move 1": a trainable bias needs
+ * one).  With s_ij = tau <q_i, k_j> + beta_h(i, j) the gradient of a bias
+ * entry is the sum of the score gradients ds_ij of the valid pairs that read
+ * it:
+ *   JFA_BIAS_RELPOS      : dbias fp32 [heads][relpos_len] (the table's
+ *                          layout), dbias[h][clamp(i - j, -C, C) + C] =
+ *                          sum of ds_ij over every sequence; overwritten.
+ *   JFA_BIAS_DENSE_JAGGED: dbias in the bias's layout and element type: ds_ij
+ *                          at each valid pair, 0 at each masked pair of the
+ *                          sequence's [heads][n_q][n_kv] block.
+ * dbias is a device pointer, 16-byte aligned; NULL gives jfa_backward.  The
+ * other arguments, outputs and errors are those of jfa_backward; a problem
+ * with JFA_BIAS_NONE and a non-NULL dbias is JFA_ERR_INVALID_ARGUMENT. */
+jfa_status jfa_backward_dbias(const jfa_problem* problem, const void* q, const void* k,
+                              const void* v, const void* out, const float* lse, const void* dout,
+                              const int32_t* q_offsets, const int32_t* kv_offsets,
+                              const void* bias, jfa_act act, int causal, void* dq, void* dk,
+                              void* dv, void* dbias, void* workspace, size_t ws_bytes,
+                              jfa_stream_t stream);
 
 /* MX (OCP v1.0) quantisation of a bf16 tensor x [rows][heads][d] to E4M3
  * codes [rows][heads][d] (same layout, one byte each) and E8M0 scales.
@@ -151,6 +196,25 @@ jfa_status jfa_quantize_mxfp8(const void* x_bf16, int64_t rows, int32_t heads, i
                               int along_rows, uint8_t* codes, uint8_t* scales,
                               jfa_stream_t stream);
 
+/* Normalisation fused with MX quantisation, for the producer of MXFP8
+ * operands ("Meta Enhances GEM Training Efficiency with Advanced LLM-Scale
+ * Innovations", "Implementing Ultra-Low-Precision Methods"; "Meta GEM
+ * Training Efficiency: Why LLM-Scale Recommenders Need a Different Stack",
+ * "Bottleneck move 2": scale generation and casting fused into the kernel
+ * that produces the tensor, not a separate pass).  For each of `rows` rows of
+ * D elements (bf16 x, device, [rows][D], 16-byte aligned):
+ *   layernorm == 0 (RMSNorm): y = x * gamma / sqrt(mean(x^2) + eps)
+ *   layernorm != 0          : y = (x - mean) * gamma / sqrt(var + eps) + beta
+ * computed in fp32, then MX-quantised along the row in blocks of 32 exactly
+ * as jfa_quantize_mxfp8 (along_rows = 0): codes E4M3 [rows][D], scales E8M0
+ * [rows][D / 32].  gamma, beta: device fp32 [D], NULL for 1 and 0.  With
+ * rows = tokens x heads and D = head_dim this is a per-head Q or K norm
+ * whose outputs are jfa_forward_mxfp8's q8 / q_scales (or k8 / k_scales).
+ * D a multiple of 32 in [32, 16384], eps > 0, else JFA_ERR_INVALID_ARGUMENT. */
+jfa_status jfa_norm_quantize_mxfp8(const void* x, int64_t rows, int32_t D, const float* gamma,
+                                   const float* beta, float eps, int layernorm, uint8_t* codes,
+                                   uint8_t* scales, jfa_stream_t stream);
+
 /* The longest-first tile schedule that jfa_forward (backward = 0: items are
  * query tiles) or jfa_backward (backward = 1: items are key/value tiles) runs,
  * written to items (device int32 [capacity][4] = {sequence, head, tile,
@@ -163,6 +227,33 @@ jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,
                         const int32_t* kv_offsets, int causal, int backward, int tile,
                         int32_t* items, int64_t capacity, int32_t* count, void* workspace,
                         size_t ws_bytes, jfa_stream_t stream);
+
+/* BlockAttention ("Meta Enhances GEM Training Efficiency with Advanced
+ * LLM-Scale Innovations", "Exploring the Customized Kernel Library" ->
+ * "BlockAttention": windows instead of full attention over long user
+ * histories; "Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a
+ * Different Stack", "Bottleneck move 1": long-sequence attention as
+ * independent fixed-size blocks).  With block length W, query i of a
+ * self-attention sequence sees only the keys j with floor(j / W) ==
+ * floor(i / W) (and j <= i when causal); GDPA divides by the block's key
+ * count.  That is jagged attention over the sequences cut into blocks, so this
+ * call only rewrites the offsets (on the device, enqueued on `stream`):
+ *   offsets        : device int32 [batch + 1], the sequences' offsets
+ *   total          : offsets[batch] (host value)
+ *   block_offsets  : device int32 [batch + total / block + 1] out: the blocks
+ *                    [c W, min((c + 1) W, n)) of every sequence in order,
+ *                    then empty blocks up to that fixed count
+ * Then jfa_forward / jfa_backward / jfa_backward_dbias with q_offsets =
+ * kv_offsets = block_offsets and a problem of batch' = batch + total / block,
+ * max_q_len' = max_kv_len' = min(block, max_len), the same totals, compute
+ * BlockAttention; only tiles inside the blocks are scheduled.  A dense bias
+ * is then laid out per block ([heads][n][n] for each block in order).  Bad
+ * offsets (offsets[0] != 0, decreasing, offsets[batch] != total) make
+ * block_offsets[0] = -1, which the attention call reports as
+ * JFA_ERR_BAD_OFFSETS.  JFA_ERR_INVALID_ARGUMENT for block < 1 or a NULL
+ * pointer. */
+jfa_status jfa_block_offsets(const int32_t* offsets, int32_t batch, int64_t total,
+                             int32_t block, int32_t* block_offsets, jfa_stream_t stream);
 
 /* Data-parallel split of one global batch across ranks (HOST function: every
  * pointer is host memory, nothing touches a GPU).  Sequences are independent,
@@ -243,6 +334,18 @@ jfa_status jfa_forward_fixed_scratch(const jfa_problem* problem, const void* q, 
                                      const void* v, const int32_t* q_offsets,
                                      const int32_t* kv_offsets, const void* bias, jfa_act act,
                                      int causal, void* out, float* lse, jfa_stream_t stream);
+
+/* Failure injection for tests of the bounded device waits (no GPU fault is
+ * made: a load is left out and the waits on it give up).  what =
+ * JFA_TEST_FWD_SKIP_LOAD arms the calling thread's NEXT jfa_forward that runs
+ * the tensor-core kernel: CTA 0 skips its first key-tile load and the waits
+ * give up after 5 ms instead of 1 s, so the call ends with JFA_ERR_TIMEOUT in
+ * the workspace's error word (jfa_check_error) while every copy the kernel
+ * did issue completes.  what = 0 disarms.  The hook is used up by that call
+ * (or by any jfa_forward on the CUDA-core path).  JFA_ERR_INVALID_ARGUMENT
+ * for another value. */
+enum { JFA_TEST_FWD_SKIP_LOAD = 1 };
+jfa_status jfa_test_inject(int what);
 
 /* Which kernel family jfa_forward / jfa_backward will use for this problem:
  * 0 = CUDA-core (fp32 arithmetic), 1 = tcgen05 tensor-core. */

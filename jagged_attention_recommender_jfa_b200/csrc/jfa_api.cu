@@ -14,7 +14,8 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int causal, int backward, int tile, WsHeader* hdr, int64_t* dense_off,
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
-                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream);
+                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream,
+                           int wait_limit_us = 0);
 cudaError_t simt_forward(const AttnArgs& a, int head_dim, bool bf16, int grid, cudaStream_t st);
 cudaError_t simt_backward(const AttnArgs& a, const AttnArgs& kv_args, int head_dim, bool bf16,
                           int grid_q, int grid_kv, int64_t rows, cudaStream_t st);
@@ -28,6 +29,11 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
                         void* ws_extra, cudaStream_t st);
 int tc_fwd_tile();
 int tc_bwd_tile();
+cudaError_t dbias_zero_masked(const AttnArgs& a, int elem_bytes, cudaStream_t st);
+cudaError_t tc_forward_mx_prequant(const jfa_problem& p, const AttnArgs& a, const void* q8,
+                                   const uint8_t* qs, const void* k8, const uint8_t* ks,
+                                   const void* v8, const uint8_t* vs, void* ws_extra,
+                                   cudaStream_t st);
 }  // namespace jfa
 
 using namespace jfa;
@@ -54,11 +60,13 @@ struct Profiler {
 };
 thread_local Profiler g_prof;
 thread_local char g_msg[512] = "";
+thread_local int g_test_hook = 0;       // jfa_test_inject: armed for the next forward
+constexpr int kTestWaitLimitUs = 5000;  // the injected failure's wait limit
 
 const char* const kKernelNames[K_COUNT] = {
     "sched_prepare", "sched_rank", "simt_fwd", "simt_bwd_pre", "simt_bwd_dq", "simt_bwd_dkdv",
     "quant_along_d", "quant_along_rows", "tc_fwd", "tc_bwd_pre", "tc_bwd", "tc_dq_finalize",
-    "tc_fwd_mxfp8", "tc_bias_prep"};
+    "tc_fwd_mxfp8", "tc_bias_prep", "dbias_zero_masked", "norm_quantize_mxfp8"};
 
 }  // namespace
 
@@ -166,10 +174,19 @@ int jfa_path(const jfa_problem* problem, jfa_act act, int backward) {
     return use_tc(*problem, act, backward) ? 1 : 0;
 }
 
-jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k, const void* v,
-                       const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
-                       jfa_act act, int causal, void* out, float* lse, void* workspace,
-                       size_t ws_bytes, jfa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// MXFP8 operands quantised by their producer (jfa_forward_mxfp8)
+struct PreQuant {
+    const uint8_t *q8, *qs, *k8, *ks, *v8, *vs;
+};
+
+jfa_status forward_impl(const jfa_problem* problem, const void* q, const void* k, const void* v,
+                        const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                        jfa_act act, int causal, void* out, float* lse, void* workspace,
+                        size_t ws_bytes, jfa_stream_t stream, const PreQuant* pq) {
     jfa_status s = check_problem(problem);
     if (s != JFA_OK) return s;
     if ((s = check_act(act)) != JFA_OK) return s;
@@ -189,12 +206,15 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     const bool tc = use_tc(p, act, 0);
     const int tile = tc ? tc_fwd_tile() : kSimtFwdTile;
+    const bool inject = tc && g_test_hook == JFA_TEST_FWD_SKIP_LOAD;
+    g_test_hook = 0;
     cudaError_t e = build_schedule(p, q_offsets, kv_offsets, causal, 0, tile, hdr,
                                    reinterpret_cast<int64_t*>(ws + L.dense_off),
                                    reinterpret_cast<int2*>(ws + L.pair_bt),
                                    reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
                                    reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
-                                   &hdr->pair_count, 1, nullptr, nullptr, st);
+                                   &hdr->pair_count, 1, nullptr, nullptr, st,
+                                   inject ? kTestWaitLimitUs : 0);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     AttnArgs a{};
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
@@ -204,7 +224,11 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
     a.out = out; a.lse = (act == JFA_ACT_SOFTMAX) ? lse : nullptr;
     a.items = reinterpret_cast<const int4*>(ws + L.items); a.item_count = &hdr->item_count;
     a.hdr = hdr;
-    if (tc) {
+    a.test_skip_load = inject ? 1 : 0;
+    if (pq) {
+        e = tc_forward_mx_prequant(p, a, pq->q8, pq->qs, pq->k8, pq->ks, pq->v8, pq->vs,
+                                   ws + L.total, st);
+    } else if (tc) {
         e = tc_forward(p, a, ws + L.total, st);
     } else {
         int64_t grid = pairs_bound(p.batch, p.max_q_len, p.total_q, tile) * p.heads;
@@ -215,11 +239,43 @@ jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k,
     return JFA_OK;
 }
 
-jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k, const void* v,
-                        const void* out, const float* lse, const void* dout,
-                        const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
-                        jfa_act act, int causal, void* dq, void* dk, void* dv, void* workspace,
-                        size_t ws_bytes, jfa_stream_t stream) {
+}  // namespace
+
+extern "C" {
+
+jfa_status jfa_forward(const jfa_problem* problem, const void* q, const void* k, const void* v,
+                       const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                       jfa_act act, int causal, void* out, float* lse, void* workspace,
+                       size_t ws_bytes, jfa_stream_t stream) {
+    return forward_impl(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out, lse,
+                        workspace, ws_bytes, stream, nullptr);
+}
+
+jfa_status jfa_forward_mxfp8(const jfa_problem* problem, const uint8_t* q8, const uint8_t* q_scales,
+                             const uint8_t* k8, const uint8_t* k_scales, const uint8_t* v8,
+                             const uint8_t* v_scales, const int32_t* q_offsets,
+                             const int32_t* kv_offsets, const void* bias, int causal, void* out,
+                             float* lse, void* workspace, size_t ws_bytes, jfa_stream_t stream) {
+    jfa_status s = check_problem(problem);
+    if (s != JFA_OK) return s;
+    if (problem->dtype != JFA_MXFP8 || problem->head_dim != 128)
+        return fail(JFA_ERR_UNSUPPORTED, "jfa_forward_mxfp8 needs dtype JFA_MXFP8 and head_dim 128");
+    if ((problem->total_q > 0 && (!q8 || !q_scales)) || (problem->total_kv > 0 && (!k8 || !k_scales || !v8 || !v_scales)))
+        return fail(JFA_ERR_INVALID_ARGUMENT, "NULL quantised operand or scales");
+    const PreQuant pq{q8, q_scales, k8, k_scales, v8, v_scales};
+    return forward_impl(problem, q8, k8, v8, q_offsets, kv_offsets, bias, JFA_ACT_SOFTMAX, causal,
+                        out, lse, workspace, ws_bytes, stream, &pq);
+}
+
+}  // extern "C"
+
+namespace {
+
+jfa_status backward_impl(const jfa_problem* problem, const void* q, const void* k, const void* v,
+                         const void* out, const float* lse, const void* dout,
+                         const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                         jfa_act act, int causal, void* dq, void* dk, void* dv, void* dbias,
+                         void* workspace, size_t ws_bytes, jfa_stream_t stream) {
     jfa_status s = check_problem(problem);
     if (s != JFA_OK) return s;
     if ((s = check_act(act)) != JFA_OK) return s;
@@ -235,8 +291,16 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
         !ALIGNED16(dk) || !ALIGNED16(dv) || !ALIGNED16(workspace) || !ALIGNED16(out))
         return fail(JFA_ERR_INVALID_ARGUMENT, "tensors and workspace must be 16-byte aligned");
     if (ws_bytes < workspace_bytes(p, 1)) return fail(JFA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, workspace_bytes(p, 1));
+    if (dbias && p.bias_kind == JFA_BIAS_NONE)
+        return fail(JFA_ERR_INVALID_ARGUMENT, "dbias given for a problem without a bias");
+    if (dbias && !ALIGNED16(dbias)) return fail(JFA_ERR_INVALID_ARGUMENT, "dbias must be 16-byte aligned");
     if (p.batch == 0) return JFA_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dbias && p.bias_kind == JFA_BIAS_RELPOS) {
+        // the kernels add every pair's score gradient into the table
+        cudaError_t e0 = cudaMemsetAsync(dbias, 0, sizeof(float) * (size_t)p.heads * p.relpos_len, st);
+        if (e0 != cudaSuccess) return cuda_fail(e0, "dbias zero");
+    }
     char* ws = reinterpret_cast<char*>(workspace);
     WsLayout L = ws_layout(p, true, false);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
@@ -274,6 +338,12 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
     a.hdr = hdr;
     a.dout = dout; a.dterm = reinterpret_cast<float*>(ws + L.dterm);
     a.dq = dq; a.dk = dk; a.dv = dv;
+    a.dbias = dbias;
+    if (dbias && p.bias_kind == JFA_BIAS_DENSE_JAGGED && causal) {
+        // masked pairs of a causal block get 0; the kernels write the rest
+        e = dbias_zero_masked(a, p.dtype == JFA_F32 ? 4 : 2, st);
+        if (e != cudaSuccess) return cuda_fail(e, "dbias zero");
+    }
     AttnArgs kv = a;
     kv.items = reinterpret_cast<const int4*>(ws + L.kv_items);
     kv.item_count = &hdr->kv_item_count;
@@ -288,6 +358,29 @@ jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward");
     return JFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+jfa_status jfa_backward(const jfa_problem* problem, const void* q, const void* k, const void* v,
+                        const void* out, const float* lse, const void* dout,
+                        const int32_t* q_offsets, const int32_t* kv_offsets, const void* bias,
+                        jfa_act act, int causal, void* dq, void* dk, void* dv, void* workspace,
+                        size_t ws_bytes, jfa_stream_t stream) {
+    return backward_impl(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act,
+                         causal, dq, dk, dv, nullptr, workspace, ws_bytes, stream);
+}
+
+jfa_status jfa_backward_dbias(const jfa_problem* problem, const void* q, const void* k,
+                              const void* v, const void* out, const float* lse, const void* dout,
+                              const int32_t* q_offsets, const int32_t* kv_offsets,
+                              const void* bias, jfa_act act, int causal, void* dq, void* dk,
+                              void* dv, void* dbias, void* workspace, size_t ws_bytes,
+                              jfa_stream_t stream) {
+    return backward_impl(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act,
+                         causal, dq, dk, dv, dbias, workspace, ws_bytes, stream);
 }
 
 jfa_status jfa_quantize_mxfp8(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
@@ -335,6 +428,13 @@ jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,
                                    backward ? reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp) : nullptr,
                                    backward ? reinterpret_cast<int64_t*>(ws + L.kv_seq_start) : nullptr, st);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
+    return JFA_OK;
+}
+
+jfa_status jfa_test_inject(int what) {
+    if (what != 0 && what != JFA_TEST_FWD_SKIP_LOAD)
+        return fail(JFA_ERR_INVALID_ARGUMENT, "unknown test injection %d", what);
+    g_test_hook = what;
     return JFA_OK;
 }
 

@@ -32,7 +32,8 @@ struct WsHeader {
     int32_t kv_item_count;
     int32_t kv_pair_count;
     int32_t kv_queue;
-    int32_t pad[57];
+    int32_t wait_limit_us;   // bounded device waits give up after this (0: 1 s)
+    int32_t pad[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -111,12 +112,19 @@ struct AttnArgs {
     void* dk;
     void* dv;
     float* dq_acc;
+    // bias gradient (NULL: not requested).  RELPOS: fp32 [H][relpos_len],
+    // zeroed before the backward kernels, which add into it; DENSE_JAGGED:
+    // element type, the bias layout, one ds per visited pair
+    void* dbias;
     // tensor-core path, relative-position bias: each head's table scaled by
     // log2(e) as runs of four (float4 entry t = entries t .. t+3), so that any
     // run of table entries can be read with 16-byte-aligned vector loads;
     // entry t of head h is bias4[4 * (h * bias4_stride + t) + 0..3]
     const float* bias4;
     int bias4_stride;  // float4 entries per head (at least 384)
+    // test hook (jfa_test_inject): CTA 0 of the tensor-core forward skips its
+    // first key-tile load, so that the bounded waits run out
+    int test_skip_load;
 };
 
 // ---------------------------------------------------------------------------
@@ -170,6 +178,8 @@ enum KernelId {
     K_TC_DQ_FINALIZE,
     K_TC_FWD_MXFP8,
     K_TC_BIAS_PREP,
+    K_DBIAS_ZERO,
+    K_NORM_QUANT,
     K_COUNT
 };
 void prof_begin(cudaStream_t st);

@@ -62,14 +62,17 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
               int max_q, int max_kv, int64_t total_q, int64_t total_kv, int causal, int backward,
               int tile, int64_t pairs_cap, int want_dense, WsHeader* hdr, int64_t* dense_off,
               int2* pair_bt, int64_t* pair_cost, int32_t* pair_count_out, int reset_err,
-              int64_t* seq_tmp, int64_t* seq_start) {
+              int64_t* seq_tmp, int64_t* seq_start, int wait_limit_us) {
     __shared__ int s_bad;
     __shared__ int64_t s_scan[kPrepThreads];
     __shared__ int64_t s_dscan[kPrepThreads];
     const int tid = threadIdx.x;
     if (tid == 0) {
         s_bad = 0;
-        if (reset_err) hdr->err = 0;
+        if (reset_err) {
+            hdr->err = 0;
+            hdr->wait_limit_us = wait_limit_us;
+        }
     }
     __syncthreads();
     // 1. validation of both offset arrays
@@ -238,13 +241,14 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int causal, int backward, int tile, WsHeader* hdr, int64_t* dense_off,
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
-                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream) {
+                           int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream,
+                           int wait_limit_us) {
     int want_dense = (pb.bias_kind == JFA_BIAS_DENSE_JAGGED && dense_off != nullptr) ? 1 : 0;
     prof_begin(stream);
     sched_prepare<<<1, kPrepThreads, 0, stream>>>(
         q_off, kv_off, pb.batch, pb.heads, pb.max_q_len, pb.max_kv_len, pb.total_q, pb.total_kv,
         causal, backward, tile, pairs_cap, want_dense, hdr, dense_off, pair_bt, pair_cost,
-        pair_count, reset_err, seq_tmp, seq_start);
+        pair_count, reset_err, seq_tmp, seq_start, wait_limit_us);
     prof_end(stream, K_SCHED_PREPARE);
     int64_t bound = pairs_bound(pb.batch, backward ? pb.max_kv_len : pb.max_q_len,
                                 backward ? pb.total_kv : pb.total_q, tile);

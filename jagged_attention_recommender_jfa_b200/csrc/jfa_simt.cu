@@ -258,6 +258,17 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq(AttnArgs a) {
                 weight_and_dscore(a.act, x, lse_i, d_i, inv_n, dp[jj], w, ds);
             }
             dSs[r * LP + c + 4 * jj] = ds;
+            // bias gradient: d beta = ds (this pass visits every pair once)
+            if (a.dbias) {
+                if (a.bias_kind == JFA_BIAS_DENSE_JAGGED) {
+                    if (i < nq && j < nkv)
+                        reinterpret_cast<T*>(a.dbias)[a.dense_off[b] + ((int64_t)h * nq + i) * nkv + j] = from_f<T>(ds);
+                } else if (ok) {
+                    const int C = (a.relpos_len - 1) >> 1;
+                    const int rr = min(max(i - j, -C), C) + C;
+                    atomicAdd(reinterpret_cast<float*>(a.dbias) + (int64_t)h * a.relpos_len + rr, ds);
+                }
+            }
         }
         __syncthreads();
         const int jn = min(BN, kv_end - j0);

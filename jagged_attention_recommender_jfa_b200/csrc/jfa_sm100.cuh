@@ -82,14 +82,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// ~1 s of wall-clock time (or as soon as another warp of the CTA, or another
-// CTA, has given up), recording JFA_ERR_TIMEOUT; returns false in that case.
+// ~1 s of wall-clock time (the workspace header's wait_limit_us when set), or
+// as soon as another warp of the CTA, or another CTA, has given up, recording
+// JFA_ERR_TIMEOUT; returns false in that case.
 // The spin polls only the barrier and the CTA's shared abort flag; the
 // grid's error word (an L2 round trip) and the clock are read every
 // kPollEvery spins, so that a completed phase is seen within one
 // shared-memory round trip rather than one global-memory round trip.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr uint32_t kPollEvery = 1024;
+
+__device__ __forceinline__ uint64_t wait_limit_ns(WsHeader* hdr) {
+    const int us = *reinterpret_cast<volatile int32_t*>(&hdr->wait_limit_us);
+    return us > 0 ? (uint64_t)us * 1000ull : kWaitLimitNs;
+}
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           WsHeader* hdr) {
@@ -104,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                 *abort_flag = 1;
                 return false;
             }
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > wait_limit_ns(hdr)) {
                 *abort_flag = 1;
                 set_error(hdr, JFA_ERR_TIMEOUT);
                 return false;
@@ -121,7 +127,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (it % kPollEvery == 0 && globaltimer() - t0 > kWaitLimitNs) {
+        if (it % kPollEvery == 0 && globaltimer() - t0 > wait_limit_ns(hdr)) {
             set_error(hdr, JFA_ERR_TIMEOUT);
             return false;
         }

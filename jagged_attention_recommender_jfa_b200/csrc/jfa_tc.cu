@@ -2,10 +2,12 @@
 // how they are launched.
 //
 // MXFP8 (dtype JFA_MXFP8): Q and K are quantised along d, V along 32-row
-// blocks of each sequence (OCP MX: E4M3 elements, one E8M0 scale per 32), and
-// the attention runs on the exact dequantised operands, with P quantised the
-// same way per 32 keys inside the forward kernel.  The backward computes bf16
-// gradients on the dequantised Q/K/V (straight-through quantiser).
+// blocks of each sequence (OCP MX: E4M3 elements, one E8M0 scale per 32) into
+// the workspace, once, and the forward runs block-scaled E4M3 MMAs on them
+// (P quantised per 32 keys inside the kernel); jfa_forward_mxfp8 takes
+// operands quantised by their producer and skips that pass.  The backward
+// computes bf16 gradients on the dequantised Q/K/V (straight-through
+// quantiser).
 #include "jfa_common.cuh"
 
 namespace jfa {
@@ -16,6 +18,13 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
 cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
                               int64_t total_q, int64_t total_kv, int heads, int d, int batch,
                               int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st);
+cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
+                        int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,
+                        uint8_t* scales, cudaStream_t st);
+cudaError_t tc_forward_mx_launch(const jfa_problem& p, const AttnArgs& a, const void* q8,
+                                 const uint8_t* qs, const void* k8, const uint8_t* ks,
+                                 const void* v8, const uint8_t* vs, int64_t n_vblocks,
+                                 int32_t* vbase, cudaStream_t st);
 
 // bf16 storage with head_dim 128 (any activation and bias kind); MXFP8 with
 // head_dim 128 and softmax.
@@ -29,7 +38,9 @@ bool tc_supported(const jfa_problem& p, int act, int backward) {
 namespace {
 struct Extra {
     size_t dq_acc, qf, kf, vf, bias4, total;
+    size_t q8, qs, k8, ks, v8, vs, vbase;   // MXFP8 forward: quantised operands
 };
+int64_t mx_vblocks(const jfa_problem& p) { return p.total_kv / 32 + p.batch; }
 // entries per head of the prepared table: the table, and at least the
 // 384-entry window the forward stages per key tile
 int bias4_stride(const jfa_problem& p) { return p.relpos_len < 384 ? 384 : p.relpos_len; }
@@ -44,10 +55,20 @@ Extra extra_layout(const jfa_problem& p, int backward) {
         e.dq_acc = off;
         off = align256(off + sizeof(float) * (size_t)p.total_q * p.heads * p.head_dim);
     }
-    if (p.dtype == JFA_MXFP8) {
+    if (p.dtype == JFA_MXFP8 && backward) {
         e.qf = off; off = align256(off + 2 * (size_t)p.total_q * p.heads * p.head_dim);
         e.kf = off; off = align256(off + 2 * (size_t)p.total_kv * p.heads * p.head_dim);
         e.vf = off; off = align256(off + 2 * (size_t)p.total_kv * p.heads * p.head_dim);
+    }
+    if (p.dtype == JFA_MXFP8 && !backward) {
+        const size_t hd = (size_t)p.heads * p.head_dim;
+        e.q8 = off; off = align256(off + (size_t)p.total_q * hd);
+        e.qs = off; off = align256(off + (size_t)p.total_q * hd / 32);
+        e.k8 = off; off = align256(off + (size_t)p.total_kv * hd);
+        e.ks = off; off = align256(off + (size_t)p.total_kv * hd / 32);
+        e.v8 = off; off = align256(off + (size_t)p.total_kv * hd);
+        e.vs = off; off = align256(off + (size_t)mx_vblocks(p) * hd);
+        e.vbase = off; off = align256(off + sizeof(int32_t) * (size_t)(p.batch > 0 ? p.batch : 1));
     }
     e.total = off;
     return e;
@@ -94,8 +115,9 @@ cudaError_t prep_bias(const jfa_problem& p, AttnArgs& a, char* ws, const Extra& 
 }
 }  // namespace
 
-// The backward keeps an fp32 dQ accumulator [total_q][heads][128]; MXFP8
-// adds the three dequantised operands; a relative-position bias adds its
+// The backward keeps an fp32 dQ accumulator [total_q][heads][128] and, for
+// MXFP8, the three dequantised operands; the MXFP8 forward keeps the E4M3
+// codes and E8M0 scales of Q, K and V; a relative-position bias adds its
 // log2(e)-scaled table of runs of four.
 size_t tc_workspace_extra(const jfa_problem& p, int backward) {
     return extra_layout(p, backward).total;
@@ -108,11 +130,38 @@ cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, 
         if (e != cudaSuccess) return e;
     }
     if (p.dtype == JFA_MXFP8) {
-        cudaError_t e = fake_quant(p, aa, reinterpret_cast<char*>(ws_extra), extra_layout(p, 0), st);
+        // quantise Q, K along d and V along 32-key blocks once, then the
+        // block-scaled kernel
+        char* ws = reinterpret_cast<char*>(ws_extra);
+        const Extra L = extra_layout(p, 0);
+        uint8_t *q8 = reinterpret_cast<uint8_t*>(ws + L.q8), *k8 = reinterpret_cast<uint8_t*>(ws + L.k8);
+        uint8_t *v8 = reinterpret_cast<uint8_t*>(ws + L.v8);
+        uint8_t *qs = reinterpret_cast<uint8_t*>(ws + L.qs), *ks = reinterpret_cast<uint8_t*>(ws + L.ks);
+        uint8_t *vs = reinterpret_cast<uint8_t*>(ws + L.vs);
+        cudaError_t e = quantize_mx(a.q, p.total_q, p.heads, p.head_dim, nullptr, 0, 0, 0, q8, qs, st);
+        if (e == cudaSuccess)
+            e = quantize_mx(a.k, p.total_kv, p.heads, p.head_dim, nullptr, 0, 0, 0, k8, ks, st);
+        if (e == cudaSuccess)
+            e = quantize_mx(a.v, p.total_kv, p.heads, p.head_dim, a.kv_off, p.batch, p.max_kv_len, 1,
+                            v8, vs, st);
         if (e != cudaSuccess) return e;
-        return tc_forward_launch(p, aa, true, st);
+        return tc_forward_mx_launch(p, aa, q8, qs, k8, ks, v8, vs, mx_vblocks(p),
+                                    reinterpret_cast<int32_t*>(ws + L.vbase), st);
     }
     return tc_forward_launch(p, aa, false, st);
+}
+
+// Forward on operands quantised by their producer (jfa_forward_mxfp8).
+cudaError_t tc_forward_mx_prequant(const jfa_problem& p, const AttnArgs& a, const void* q8,
+                                   const uint8_t* qs, const void* k8, const uint8_t* ks,
+                                   const void* v8, const uint8_t* vs, void* ws_extra,
+                                   cudaStream_t st) {
+    AttnArgs aa = a;
+    const Extra L = extra_layout(p, 0);
+    cudaError_t e = prep_bias(p, aa, reinterpret_cast<char*>(ws_extra), L, st);
+    if (e != cudaSuccess) return e;
+    return tc_forward_mx_launch(p, aa, q8, qs, k8, ks, v8, vs, mx_vblocks(p),
+                                reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws_extra) + L.vbase), st);
 }
 
 cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,

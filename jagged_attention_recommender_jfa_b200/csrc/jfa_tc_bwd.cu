@@ -73,7 +73,12 @@ constexpr uint32_t kOffRow = kOffBar + 256;       // lse2[2][128], D[2][128] (do
 constexpr int kWin = 272;
 constexpr uint32_t kWinBytes = kWin * 16;          // 4352
 constexpr uint32_t kOffWin = kOffRow + 2048;
-constexpr uint32_t kOffEnd = kOffWin + 2 * kWinBytes;
+// Relative-position bias gradient of a query tile, 2 buffers: the 255
+// diagonals i - j of a 128 x 128 tile, entry e = (i - qb0) - (j - j0) + 127,
+// summed in shared memory and added to the table once per tile.
+constexpr int kDbWin = 256;
+constexpr uint32_t kOffDb = kOffWin + 2 * kWinBytes;
+constexpr uint32_t kOffEnd = kOffDb + 2 * kDbWin * 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
@@ -87,6 +92,8 @@ struct Bars {
     uint64_t rows_full[2];  // LSE / D of a query tile staged (4 warps of group 0)
     uint64_t rows_free[2];  // ... and read by every score warp (16)
     uint64_t bias_full[2];  // bias window of a query tile loaded
+    uint64_t db_done[2];    // 16 score warps: their bias-gradient sums of a tile are in
+    uint64_t db_free[2];    // the tile's flusher warp added the buffer to the table and cleared it
     uint64_t fin;
     uint64_t drain;
     uint32_t tmem_base;
@@ -150,8 +157,11 @@ __device__ __forceinline__ void zero_row(uint8_t* tile, int r) {
 }
 
 // BIAS: 0 none, 1 relative-position, 2 dense jagged.  SOFTMAX: softmax (true)
-// or GDPA.
-template <int BIAS, bool SOFTMAX>
+// or GDPA.  DBIAS: also the bias gradient -- ds of every pair written to the
+// dense bias gradient, or summed along the diagonals of each tile in shared
+// memory and added to the relative-position table gradient by one warp
+// (score warp t % 16 for tile t, at the start of tile t + 1).
+template <int BIAS, bool SOFTMAX, bool DBIAS>
 __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
@@ -189,9 +199,17 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
         mbar_init(&bars->dq_empty, NG * 4);
         mbar_init(&bars->fin, 1);
         mbar_init(&bars->drain, 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&bars->db_done[s2], NG * 4);
+            mbar_init(&bars->db_free[s2], 1);
+        }
         bars->abort_flag = 0;
         fence_barrier_init();
     }
+    constexpr bool kDbRel = DBIAS && BIAS == 1, kDbDense = DBIAS && BIAS == 2;
+    float* db_win = reinterpret_cast<float*>(smem + kOffDb);   // [2][kDbWin]
+    if (kDbRel)
+        for (int e = threadIdx.x; e < 2 * kDbWin; e += blockDim.x) db_win[e] = 0.f;
     if (warp == 1) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
@@ -397,6 +415,23 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
             fetch_rowstats(0, l2, dv);
             stage_rowstats(0, l2, dv);
         }
+        // relative-position bias gradient: the flusher of tile tt (score warp
+        // tt % 16) adds the tile's diagonal sums to the table and clears them
+        const int sw = warp - 2;
+        float* dtab = kDbRel ? reinterpret_cast<float*>(a.dbias) + (int64_t)h * a.relpos_len : nullptr;
+        auto flush_db = [&](int tt) -> bool {
+            if (!wwait(&bars->db_done[tt & 1], (tt >> 1) & 1)) return false;
+            float* dw = db_win + (tt & 1) * kDbWin;
+            const int d0 = (i_start + tt * BM) - j0 - (BN - 1);   // diagonal i - j of entry 0
+            for (int e = lane; e < 2 * BN - 1; e += 32) {
+                const float val = dw[e];
+                if (val != 0.f) atomicAdd(dtab + (min(max(d0 + e, -C), C) + C), val);
+                dw[e] = 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->db_free[tt & 1]);
+            return true;
+        };
         const int tslot = (warp == 2 && lane == 0) ? 2 : ((warp == kThreads / 32 - 1 && lane == 0) ? 3 : -1);
 #define SC_EV(ev)                                     \
     do {                                              \
@@ -423,6 +458,12 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
             if (t == 0 && grp == 0 && !jvalid) zero_row(smem + kOffK, r);
             if (!wwait(&bars->rows_full[buf], (t >> 1) & 1)) { ok = false; break; }
             if (BIAS == 1 && !wwait(&bars->bias_full[buf], (t >> 1) & 1)) { ok = false; break; }
+            if (kDbRel) {
+                // the previous tile's sums are complete once S^T of this tile exists
+                if (t >= 1 && sw == (t - 1) % (NG * 4) && !flush_db(t - 1)) { ok = false; break; }
+                // this tile's buffer was flushed after tile t - 2
+                if (t >= 2 && !wwait(&bars->db_free[buf], ((t >> 1) - 1) & 1)) { ok = false; break; }
+            }
             SC_EV(2);
             // bias(qc0 + v, j) = table[qc0 - j + C + v]: window entries
             // qc0 - j + C - w0 + 4q hold table[... + 4q + 0..3]
@@ -519,6 +560,20 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
                         g[v] = vis ? g[v] : 0u;
                     }
                 }
+                // bias gradient: d beta(i, j) = ds_ij (g, masked pairs 0)
+                if (kDbDense && jvalid) {
+                    __nv_bfloat16* col = reinterpret_cast<__nv_bfloat16*>(a.dbias) + dense_base + j;
+#pragma unroll
+                    for (int v = 0; v < 16; ++v)
+                        if (qc0 + v < nq) col[(int64_t)(qc0 + v) * nkv] = __float2bfloat16_rn(__uint_as_float(g[v]));
+                }
+                if (kDbRel) {
+                    // diagonal entry (qc0 + v - qb0) - r + 127; for a fixed v the
+                    // lanes (consecutive r) hit consecutive entries
+                    float* dw = db_win + buf * kDbWin + (c16 * 16 - r + (BN - 1));
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) atomicAdd(dw + v, __uint_as_float(g[v]));
+                }
             };
             // Two 16-column halves: half hh of group grp is query chunk
             // c16 = 4 hh + grp (columns 16 c16 ..), so that every group's first
@@ -561,6 +616,7 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
             if (lane == 0) {
                 mbar_arrive(&bars->rows_free[buf]);
                 mbar_arrive(&bars->ds_full);
+                if (kDbRel) mbar_arrive(&bars->db_done[buf]);
             }
             // LSE / D of tile t+1 into the other buffer, whose readers (tile t-1)
             // have all released it
@@ -594,6 +650,7 @@ __global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams
             SC_EV(6);
         }
 #undef SC_EV
+        if (kDbRel && ok && nt > 0 && sw == (nt - 1) % (NG * 4)) ok = flush_db(nt - 1);
         // ------------------------------------------------------ epilogue
         if (ok && nt > 0) ok = __all_sync(0xffffffffu, wwait(&bars->fin, 0));
         if (ok && !*abort_flag) {
@@ -699,10 +756,15 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
     const int smem = 1024 + (int)kOffEnd;
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
     const bool sm = a.act == JFA_ACT_SOFTMAX;
+    const bool db = a.dbias != nullptr;
     void (*kern)(BwdParams) = nullptr;
-    if (bias == 0) kern = sm ? tc_bwd_kernel<0, true> : tc_bwd_kernel<0, false>;
-    else if (bias == 1) kern = sm ? tc_bwd_kernel<1, true> : tc_bwd_kernel<1, false>;
-    else kern = sm ? tc_bwd_kernel<2, true> : tc_bwd_kernel<2, false>;
+    if (bias == 0) kern = sm ? tc_bwd_kernel<0, true, false> : tc_bwd_kernel<0, false, false>;
+    else if (bias == 1)
+        kern = db ? (sm ? tc_bwd_kernel<1, true, true> : tc_bwd_kernel<1, false, true>)
+                  : (sm ? tc_bwd_kernel<1, true, false> : tc_bwd_kernel<1, false, false>);
+    else
+        kern = db ? (sm ? tc_bwd_kernel<2, true, true> : tc_bwd_kernel<2, false, true>)
+                  : (sm ? tc_bwd_kernel<2, true, false> : tc_bwd_kernel<2, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int64_t grid = pairs_bound(p.batch, p.max_kv_len, p.total_kv, BN) * p.heads;

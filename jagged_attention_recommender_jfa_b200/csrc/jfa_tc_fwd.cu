@@ -263,9 +263,14 @@ __global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams
                     const int z = w.k0 + j * BN;
                     if (g >= 2 && !mbar_wait(&bars->k_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
                     JFA_TRACE_EV(fwd, 0, g, 0);
-                    mbar_arrive_expect_tx(&bars->k_full[s], kTile);
-                    tma_load_3d(smem + kOffK + s * kTile, &P.tm_k, &bars->k_full[s], 0, w.h, z);
-                    tma_load_3d(smem + kOffK + s * kTile + kBox, &P.tm_k, &bars->k_full[s], 64, w.h, z);
+                    // test hook: CTA 0 leaves out its first key tile (load and
+                    // expected bytes), so that the waits on it run out
+                    const bool skip = a.test_skip_load && cta == 0 && g == 0;
+                    if (!skip) {
+                        mbar_arrive_expect_tx(&bars->k_full[s], kTile);
+                        tma_load_3d(smem + kOffK + s * kTile, &P.tm_k, &bars->k_full[s], 0, w.h, z);
+                        tma_load_3d(smem + kOffK + s * kTile + kBox, &P.tm_k, &bars->k_full[s], 64, w.h, z);
+                    }
                     if (g >= 2 && !mbar_wait(&bars->v_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
                     JFA_TRACE_EV(fwd, 0, g, 1);
                     mbar_arrive_expect_tx(&bars->v_full[s], kTile);

@@ -39,7 +39,10 @@ STATUS_NAMES = {0: "JFA_OK", 1: "JFA_ERR_INVALID_ARGUMENT", 2: "JFA_ERR_UNSUPPOR
 EXPORTS = ("jfa_workspace_bytes", "jfa_forward", "jfa_backward", "jfa_quantize_mxfp8",
            "jfa_schedule", "jfa_check_error", "jfa_last_error", "jfa_path",
            "jfa_profile_enable", "jfa_profile_read", "jfa_kernel_name",
-           "jfa_forward_fixed_scratch", "jfa_partition")
+           "jfa_forward_fixed_scratch", "jfa_partition", "jfa_backward_dbias",
+           "jfa_block_offsets", "jfa_test_inject", "jfa_forward_mxfp8",
+           "jfa_norm_quantize_mxfp8")
+JFA_TEST_FWD_SKIP_LOAD = 1
 PARTITION = {"lpt": 0, "bbs": 1}
 
 
@@ -96,6 +99,17 @@ def load():
         lib.jfa_kernel_name.restype = ctypes.c_char_p
         lib.jfa_forward_fixed_scratch.argtypes = [PP, P, P, P, P, P, P, i32, i32, P, P, P]
         lib.jfa_forward_fixed_scratch.restype = i32
+        lib.jfa_backward_dbias.argtypes = [PP, P, P, P, P, P, P, P, P, P, i32, i32, P, P, P, P, P,
+                                           sz, P]
+        lib.jfa_backward_dbias.restype = i32
+        lib.jfa_forward_mxfp8.argtypes = [PP, P, P, P, P, P, P, P, P, P, i32, P, P, P, sz, P]
+        lib.jfa_forward_mxfp8.restype = i32
+        lib.jfa_norm_quantize_mxfp8.argtypes = [P, i64, i32, P, P, ctypes.c_float, i32, P, P, P]
+        lib.jfa_norm_quantize_mxfp8.restype = i32
+        lib.jfa_test_inject.argtypes = [i32]
+        lib.jfa_test_inject.restype = i32
+        lib.jfa_block_offsets.argtypes = [P, i32, i64, i32, P, P]
+        lib.jfa_block_offsets.restype = i32
         lib.jfa_partition.argtypes = [i32, P, P, i32, i32, i32, i32, P, P]
         lib.jfa_partition.restype = i32
         _LIB = lib
@@ -160,6 +174,16 @@ def jfa_forward(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out,
                               _addr(workspace), int(ws_bytes), _stream(stream)))
 
 
+def jfa_forward_mxfp8(problem, q8, q_scales, k8, k_scales, v8, v_scales, q_offsets, kv_offsets,
+                      bias, causal, out, lse, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().jfa_forward_mxfp8(ctypes.byref(problem), _addr(q8), _addr(q_scales), _addr(k8),
+                                    _addr(k_scales), _addr(v8), _addr(v_scales), _addr(q_offsets),
+                                    _addr(kv_offsets), _addr(bias), int(bool(causal)), _addr(out),
+                                    _addr(lse), _addr(workspace), int(ws_bytes), _stream(stream)))
+
+
 def jfa_forward_fixed_scratch(problem, q, k, v, q_offsets, kv_offsets, bias, act, causal, out,
                               lse, stream=None):
     """Forward without a workspace: for callers that cannot allocate device
@@ -181,6 +205,18 @@ def jfa_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, 
                                _stream(stream)))
 
 
+def jfa_backward_dbias(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act,
+                       causal, dq, dk, dv, dbias, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().jfa_backward_dbias(ctypes.byref(problem), _addr(q), _addr(k), _addr(v),
+                                     _addr(out), _addr(lse), _addr(dout), _addr(q_offsets),
+                                     _addr(kv_offsets), _addr(bias), ACT.get(act, act),
+                                     int(bool(causal)), _addr(dq), _addr(dk), _addr(dv),
+                                     _addr(dbias), _addr(workspace), int(ws_bytes),
+                                     _stream(stream)))
+
+
 def jfa_quantize_mxfp8(x, rows, heads, d, offsets, batch, max_len, along_rows, codes, scales,
                        stream=None):
     _check(load().jfa_quantize_mxfp8(_addr(x), int(rows), int(heads), int(d), _addr(offsets),
@@ -198,6 +234,25 @@ def jfa_schedule(problem, q_offsets, kv_offsets, causal, backward, tile, items, 
                                _stream(stream)))
 
 
+def jfa_block_offsets(offsets, batch, total, block, block_offsets, stream=None):
+    _check(load().jfa_block_offsets(_addr(offsets), int(batch), int(total), int(block),
+                                    _addr(block_offsets), _stream(stream)))
+
+
+def block_attention(problem: jfa_problem, offsets, block: int, stream=None):
+    """BlockAttention with block length ``block`` as a jagged problem over the
+    blocks: returns (descriptor, block offsets) to pass to jfa_forward /
+    jfa_backward as both q and kv offsets (self-attention)."""
+    n_out = problem.batch + problem.total_q // block
+    boff = torch.empty(n_out + 1, dtype=torch.int32, device=offsets.device)
+    jfa_block_offsets(offsets, problem.batch, problem.total_q, block, boff, stream)
+    p2 = jfa_problem.from_buffer_copy(problem)
+    p2.batch = n_out
+    p2.max_q_len = min(block, problem.max_q_len)
+    p2.max_kv_len = min(block, problem.max_kv_len)
+    return p2, boff
+
+
 def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
     """Host-side split of a global batch across ``ranks``: returns (rank_of
     int32 [batch], rank_cost int64 [ranks]) as numpy arrays."""
@@ -212,6 +267,16 @@ def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
                                 PARTITION.get(method, method), int(sub_batch), c(rank_of),
                                 c(rank_cost)))
     return rank_of, rank_cost
+
+
+def jfa_norm_quantize_mxfp8(x, rows, D, gamma, beta, eps, layernorm, codes, scales, stream=None):
+    _check(load().jfa_norm_quantize_mxfp8(_addr(x), int(rows), int(D), _addr(gamma), _addr(beta),
+                                          float(eps), int(bool(layernorm)), _addr(codes),
+                                          _addr(scales), _stream(stream)))
+
+
+def jfa_test_inject(what: int):
+    _check(load().jfa_test_inject(int(what)))
 
 
 def jfa_profile_enable(enable: bool):
@@ -272,14 +337,22 @@ def attention_forward(problem, q, k, v, q_offsets, kv_offsets, bias=None, act="s
 
 
 def attention_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias=None,
-                       act="softmax", causal=False, ws=None, stream=None, check=True):
+                       act="softmax", causal=False, ws=None, stream=None, check=True,
+                       want_dbias=False):
     """Allocates dq / dk / dv (and the workspace unless ``ws`` is given) and
-    runs jfa_backward; ``check`` as in :func:`attention_forward`."""
+    runs jfa_backward; ``check`` as in :func:`attention_forward`.  With
+    ``want_dbias`` it runs jfa_backward_dbias and also returns the bias
+    gradient (shaped like ``bias``)."""
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if ws is None:
         ws = workspace(problem, True, q.device)
-    jfa_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act, causal,
-                 dq, dk, dv, ws, stream=stream)
+    if want_dbias:
+        dbias = torch.empty_like(bias)
+        jfa_backward_dbias(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act,
+                           causal, dq, dk, dv, dbias, ws, stream=stream)
+    else:
+        jfa_backward(problem, q, k, v, out, lse, dout, q_offsets, kv_offsets, bias, act, causal,
+                     dq, dk, dv, ws, stream=stream)
     if check:
         jfa_check_error(ws, stream)
-    return dq, dk, dv
+    return (dq, dk, dv, dbias) if want_dbias else (dq, dk, dv)

@@ -383,3 +383,26 @@ def partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
     for b in range(B):
         rank_cost[rank_of[b]] += cost[b]
     return rank_of, rank_cost
+
+
+# ---------------------------------------------------------------------------
+# Normalisation ahead of MX quantisation (plain fp64 definitions).
+#   RMSNorm  : y = x * gamma / sqrt(mean(x^2) + eps)
+#   LayerNorm: y = (x - mean(x)) * gamma / sqrt(mean((x - mean)^2) + eps) + beta
+# "Meta Enhances GEM Training Efficiency ...", "Implementing Ultra-Low-Precision
+# Methods": the quantisation is fused into the normalisation that produces the
+# low-precision operand; the result is then quantised like quantize_mx.
+# ---------------------------------------------------------------------------
+
+def norm(x, gamma=None, beta=None, eps=1e-6, layernorm=False) -> np.ndarray:
+    """x [rows, D] -> y [rows, D] in fp64."""
+    x64 = _f64(x)
+    mean = x64.mean(axis=-1, keepdims=True) if layernorm else 0.0
+    c = x64 - mean
+    var = (c * c).mean(axis=-1, keepdims=True)
+    y = c / np.sqrt(var + eps)
+    if gamma is not None:
+        y = y * _f64(gamma)
+    if layernorm and beta is not None:
+        y = y + _f64(beta)
+    return y

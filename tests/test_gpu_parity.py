@@ -453,3 +453,69 @@ def test_full_size_mxfp8_sampled(cuda_device):
         assert np.all(np.abs(gg - rr) <= MX_MAX + half_ulp_bf16(rr)), name
     gl = lse.cpu().numpy()[rows, 0]
     assert np.all(np.abs(gl - rl[:, 0]) <= LSE_MAX)
+
+
+# ---------------------------------------------------------------------------
+# bounded device waits: a left-out load makes them give up with
+# JFA_ERR_TIMEOUT (no fault, nothing left in flight), and the next call on the
+# same workspace is clean
+# ---------------------------------------------------------------------------
+def test_bounded_wait_times_out_and_recovers(cuda_device):
+    import time
+    p = make_problem("self_bf16", 60, B=4, max_len=300)
+    d = _dev(p, cuda_device)
+    prob = jfa.problem_of(p)
+    assert jfa.jfa_path(prob, "softmax", 0) == 1
+    ws = jfa.workspace(prob, False, cuda_device)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(p.total_q, p.H, device=cuda_device)
+    jfa.jfa_test_inject(jfa.JFA_TEST_FWD_SKIP_LOAD)
+    t0 = time.perf_counter()
+    jfa.jfa_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"], d["bias"], "softmax",
+                    True, out, lse, ws)
+    with pytest.raises(jfa.JfaError) as ei:
+        jfa.jfa_check_error(ws)
+    assert ei.value.status == jfa.JFA_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 0.5   # the injected 5 ms limit, not the default 1 s
+    # the context is usable and the next call on the same workspace is exact
+    out2, lse2 = jfa.attention_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"],
+                                       d["bias"], "softmax", True, ws=ws)
+    ro, rl, _ = run_oracle(p, backward=False)
+    compare("O", out2, ro, slice(None), BF16_MAX, BF16_MEAN)
+    compare("LSE", lse2, rl, slice(None), LSE_MAX)
+    with pytest.raises(jfa.JfaError):
+        jfa.jfa_test_inject(7)
+
+
+def test_mxfp8_prequantised_entry_matches(cuda_device):
+    # jfa_forward_mxfp8 on operands quantised beforehand (by the public
+    # quantiser, standing in for a producer kernel) runs the same block-scaled
+    # kernel as jfa_forward with dtype MXFP8: bitwise equal outputs
+    p = make_problem("self_mxfp8", 33, B=6, max_len=330)
+    d = _dev(p, cuda_device)
+    prob = jfa.problem_of(p)
+    rows_q, H, dd = p.q.shape
+    rows_k = p.k.shape[0]
+    q8 = torch.empty(rows_q, H, dd, dtype=torch.uint8, device=cuda_device)
+    k8 = torch.empty(rows_k, H, dd, dtype=torch.uint8, device=cuda_device)
+    v8 = torch.empty_like(k8)
+    qs = torch.empty(rows_q, H, dd // 32, dtype=torch.uint8, device=cuda_device)
+    ks = torch.empty(rows_k, H, dd // 32, dtype=torch.uint8, device=cuda_device)
+    vs = torch.zeros(rows_k // 32 + p.B, H, dd, dtype=torch.uint8, device=cuda_device)
+    jfa.jfa_quantize_mxfp8(d["q"], rows_q, H, dd, None, 0, 0, False, q8, qs)
+    jfa.jfa_quantize_mxfp8(d["k"], rows_k, H, dd, None, 0, 0, False, k8, ks)
+    jfa.jfa_quantize_mxfp8(d["v"], rows_k, H, dd, d["kv_off"], p.B, p.max_kv_len, True, v8, vs)
+    ws = jfa.workspace(prob, False, cuda_device)
+    out = torch.full_like(d["q"], float("nan"))
+    lse = torch.full((p.total_q, H), float("nan"), device=cuda_device)
+    jfa.jfa_forward_mxfp8(prob, q8, qs, k8, ks, v8, vs, d["q_off"], d["kv_off"], d["bias"], True,
+                          out, lse, ws)
+    jfa.jfa_check_error(ws)
+    ref_out, ref_lse = jfa.attention_forward(prob, d["q"], d["k"], d["v"], d["q_off"],
+                                             d["kv_off"], d["bias"], "softmax", True)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    # a bf16 problem is refused by the MXFP8 entry point
+    with pytest.raises(jfa.JfaError) as ei:
+        jfa.jfa_forward_mxfp8(jfa.problem_of(p, dtype="bf16"), q8, qs, k8, ks, v8, vs, d["q_off"],
+                              d["kv_off"], d["bias"], True, out, lse, ws)
+    assert ei.value.status == jfa.JFA_ERR_UNSUPPORTED

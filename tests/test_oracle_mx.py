@@ -305,3 +305,29 @@ def test_dequantize_along_rows_round_trip():
                     assert np.array_equal(back[lo:hi, h, col], ref[:hi - lo])
         blk0 += nb
     assert blk0 == scales.shape[0]
+
+
+# ---------------------------------------------------------------------------
+# normalisation that feeds the MX quantiser: the oracle's plain definitions
+# against torch's library routines in float64
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("layernorm", [False, True])
+def test_norm_matches_torch(layernorm):
+    rng = np.random.default_rng(20)
+    x = rng.standard_normal((37, 256)) * 3 + 0.5
+    g = rng.standard_normal(256)
+    b = rng.standard_normal(256)
+    y = oracle.norm(x, g, b, 1e-5, layernorm)
+    xt = torch.from_numpy(x)
+    if layernorm:
+        ref = torch.nn.functional.layer_norm(xt, (256,), torch.from_numpy(g), torch.from_numpy(b), 1e-5)
+    else:
+        ref = torch.nn.functional.rms_norm(xt, (256,), torch.from_numpy(g), 1e-5)
+    np.testing.assert_allclose(y, ref.numpy(), rtol=0, atol=1e-12)
+    # without gamma / beta: unit RMS (RMSNorm) or zero mean, unit variance
+    y0 = oracle.norm(x, None, None, 0.0 + 1e-300, layernorm)
+    if layernorm:
+        np.testing.assert_allclose(y0.mean(1), 0.0, atol=1e-12)
+        np.testing.assert_allclose((y0 ** 2).mean(1), 1.0, atol=1e-12)
+    else:
+        np.testing.assert_allclose((y0 ** 2).mean(1), 1.0, atol=1e-12)
