@@ -29,6 +29,7 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
                         void* ws_extra, cudaStream_t st);
 int tc_fwd_tile();
 int tc_bwd_tile();
+bool tc_backward_short_q(const jfa_problem& p);
 cudaError_t dbias_zero_masked(const AttnArgs& a, int elem_bytes, cudaStream_t st);
 cudaError_t tc_forward_mx_prequant(const jfa_problem& p, const AttnArgs& a, const void* q8,
                                    const uint8_t* qs, const void* k8, const uint8_t* ks,
@@ -66,7 +67,7 @@ constexpr int kTestWaitLimitUs = 5000;  // the injected failure's wait limit
 const char* const kKernelNames[K_COUNT] = {
     "sched_prepare", "sched_rank", "simt_fwd", "simt_bwd_pre", "simt_bwd_dq", "simt_bwd_dkdv",
     "quant_along_d", "quant_along_rows", "tc_fwd", "tc_bwd_pre", "tc_bwd", "tc_dq_finalize",
-    "tc_fwd_mxfp8", "tc_bias_prep", "dbias_zero_masked", "norm_quantize_mxfp8"};
+    "tc_fwd_mxfp8", "tc_bias_prep", "dbias_zero_masked", "norm_quantize_mxfp8", "tc_bwd_sq"};
 
 }  // namespace
 
@@ -305,13 +306,16 @@ jfa_status backward_impl(const jfa_problem* problem, const void* q, const void* 
     WsLayout L = ws_layout(p, true, false);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     const bool tc = use_tc(p, act, 1);
+    // short queries on the tensor cores: one item per (sequence, head)
+    const bool sq = tc && tc_backward_short_q(p);
     const int qtile = tc ? tc_fwd_tile() : kSimtFwdTile;
     const int ktile = tc ? tc_bwd_tile() : kSimtBwdTile;
-    // the CUDA-core backward walks both schedules; the tensor-core backward only
-    // the key-tile one (its first build resets the error word and, for a dense
-    // bias, writes the sequences' bias offsets)
+    // the CUDA-core backward walks both schedules, the query-stationary one
+    // only the query-block one, the key-stationary one only the key-tile one
+    // (the first build resets the error word and, for a dense bias, writes
+    // the sequences' bias offsets)
     cudaError_t e = cudaSuccess;
-    if (!tc) {
+    if (!tc || sq) {
         e = build_schedule(p, q_offsets, kv_offsets, causal, 0, qtile, hdr,
                            reinterpret_cast<int64_t*>(ws + L.dense_off),
                            reinterpret_cast<int2*>(ws + L.pair_bt),
@@ -320,14 +324,16 @@ jfa_status backward_impl(const jfa_problem* problem, const void* q, const void* 
                            &hdr->pair_count, 1, nullptr, nullptr, st);
         if (e != cudaSuccess) return cuda_fail(e, "schedule");
     }
-    e = build_schedule(p, q_offsets, kv_offsets, causal, 1, ktile, hdr,
-                       tc ? reinterpret_cast<int64_t*>(ws + L.dense_off) : nullptr,
-                       reinterpret_cast<int2*>(ws + L.kv_pair_bt),
-                       reinterpret_cast<int64_t*>(ws + L.kv_pair_cost), L.pairs_max_kv,
-                       reinterpret_cast<int4*>(ws + L.kv_items), &hdr->kv_item_count,
-                       &hdr->kv_pair_count, tc ? 1 : 0, reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp),
-                       reinterpret_cast<int64_t*>(ws + L.kv_seq_start), st);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule");
+    if (!sq) {
+        e = build_schedule(p, q_offsets, kv_offsets, causal, 1, ktile, hdr,
+                           tc ? reinterpret_cast<int64_t*>(ws + L.dense_off) : nullptr,
+                           reinterpret_cast<int2*>(ws + L.kv_pair_bt),
+                           reinterpret_cast<int64_t*>(ws + L.kv_pair_cost), L.pairs_max_kv,
+                           reinterpret_cast<int4*>(ws + L.kv_items), &hdr->kv_item_count,
+                           &hdr->kv_pair_count, tc ? 1 : 0, reinterpret_cast<int64_t*>(ws + L.kv_seq_tmp),
+                           reinterpret_cast<int64_t*>(ws + L.kv_seq_start), st);
+        if (e != cudaSuccess) return cuda_fail(e, "schedule");
+    }
     AttnArgs a{};
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
     a.bias = bias; a.dense_off = reinterpret_cast<const int64_t*>(ws + L.dense_off);

@@ -180,6 +180,7 @@ enum KernelId {
     K_TC_BIAS_PREP,
     K_DBIAS_ZERO,
     K_NORM_QUANT,
+    K_TC_BWD_SQ,
     K_COUNT
 };
 void prof_begin(cudaStream_t st);

@@ -15,6 +15,9 @@ namespace jfa {
 cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quant_p, cudaStream_t st);
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                                cudaStream_t st);
+cudaError_t tc_bwd_pre_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
+cudaError_t tc_backward_sq_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
+bool tc_backward_short_q(const jfa_problem& p);
 cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
                               int64_t total_q, int64_t total_kv, int heads, int d, int batch,
                               int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st);
@@ -184,8 +187,18 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
         akv.k = aq.k;
         akv.v = aq.v;
     }
+    if (tc_backward_short_q(p)) {
+        // query-stationary: one CTA per (sequence, head), items from the
+        // query-block schedule in `a`
+        cudaError_t e = tc_bwd_pre_launch(p, aq, st);
+        if (e != cudaSuccess) return e;
+        return tc_backward_sq_launch(p, aq, st);
+    }
     return tc_backward_launch(p, aq, akv, st);
 }
+
+// Short query sequences (every n_q <= 64) take the query-stationary backward.
+bool tc_backward_short_q(const jfa_problem& p) { return p.max_q_len <= 64; }
 
 int tc_fwd_tile() { return 256; }   // a forward work item is a 256-row query block
 int tc_bwd_tile() { return 128; }

@@ -736,8 +736,8 @@ __global__ void __launch_bounds__(256) tc_bwd_dq_finalize(const float* __restric
 
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per block
 
-cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
-                               cudaStream_t st) {
+// D = rowsum(dO * O) and the zeroed dQ accumulator
+cudaError_t tc_bwd_pre_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st) {
     const int64_t rows = p.total_q * p.heads;
     if (rows > 0) {
         prof_begin(st);
@@ -745,6 +745,16 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
             reinterpret_cast<const __nv_bfloat16*>(a.out), reinterpret_cast<const __nv_bfloat16*>(a.dout),
             a.dterm, a.dq_acc, rows, a.act == JFA_ACT_SOFTMAX ? 1 : 0);
         prof_end(st, K_TC_BWD_PRE);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
+                               cudaStream_t st) {
+    const int64_t rows = p.total_q * p.heads;
+    {
+        cudaError_t e0 = tc_bwd_pre_launch(p, a, st);
+        if (e0 != cudaSuccess) return e0;
     }
     BwdParams P{};
     if (!make_tmap_rows_heads_d(&P.tm_q, a.q, p.total_q, p.heads) ||

@@ -745,18 +745,23 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 // [rows][heads][128] bf16 viewed as a 3-D tensor (d, head, row); boxes of
-// 64 d x 1 head x 128 rows with the 128-byte swizzle.
-bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads) {
+// 64 d x 1 head x box_rows rows with the 128-byte swizzle.
+bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows, int heads,
+                                int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
     cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)heads * HD * 2};
-    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads) {
+    return make_tmap_rows_heads_d_box(map, base, rows, heads, 128);
 }
 
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per CTA

@@ -175,6 +175,10 @@ def test_other_head_dims(cuda_device, d, dtype):
 
 EDGE_LENS = [
     # (q_lens, kv_lens, causal)
+    # every n_q <= 64 (the query-stationary backward): rows without keys,
+    # empty sequences on either side, long key ranges
+    ([40, 64, 1, 33, 0, 5], [10, 300, 0, 33, 17, 1000], True),
+    ([40, 64, 1, 33, 0, 5], [10, 300, 0, 33, 17, 1000], False),
     ([1, 64, 65, 127, 128, 129, 0, 2], None, True),
     ([1, 64, 65, 127, 128, 129, 0, 2], None, False),
     ([5, 40, 200, 1], [1, 1, 1, 1], False),           # single key
