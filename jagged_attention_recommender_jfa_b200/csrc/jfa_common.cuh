@@ -181,6 +181,7 @@ enum KernelId {
     K_DBIAS_ZERO,
     K_NORM_QUANT,
     K_TC_BWD_SQ,
+    K_TC_FWD_SQ,
     K_COUNT
 };
 void prof_begin(cudaStream_t st);

@@ -18,6 +18,7 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
 cudaError_t tc_bwd_pre_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
 cudaError_t tc_backward_sq_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
 bool tc_backward_short_q(const jfa_problem& p);
+cudaError_t tc_forward_sq_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
 cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
                               int64_t total_q, int64_t total_kv, int heads, int d, int batch,
                               int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st);
@@ -151,6 +152,8 @@ cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, 
         return tc_forward_mx_launch(p, aa, q8, qs, k8, ks, v8, vs, mx_vblocks(p),
                                     reinterpret_cast<int32_t*>(ws + L.vbase), st);
     }
+    // short query sequences: two (sequence, head) items per CTA step
+    if (tc_backward_short_q(p)) return tc_forward_sq_launch(p, aa, st);
     return tc_forward_launch(p, aa, false, st);
 }
 
@@ -197,7 +200,8 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
     return tc_backward_launch(p, aq, akv, st);
 }
 
-// Short query sequences (every n_q <= 64) take the query-stationary backward.
+// Short query sequences (every n_q <= 64) take the paired-item forward and
+// the query-stationary backward.
 bool tc_backward_short_q(const jfa_problem& p) { return p.max_q_len <= 64; }
 
 int tc_fwd_tile() { return 256; }   // a forward work item is a 256-row query block
