@@ -12,7 +12,7 @@
 
 namespace jfa {
 
-cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quant_p, cudaStream_t st);
+cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
 cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const AttnArgs& kv,
                                cudaStream_t st);
 cudaError_t tc_bwd_pre_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st);
@@ -154,7 +154,7 @@ cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, 
     }
     // short query sequences: two (sequence, head) items per CTA step
     if (tc_backward_short_q(p)) return tc_forward_sq_launch(p, aa, st);
-    return tc_forward_launch(p, aa, false, st);
+    return tc_forward_launch(p, aa, st);
 }
 
 // Forward on operands quantised by their producer (jfa_forward_mxfp8).

@@ -39,7 +39,6 @@
 // exchange.
 #include <math_constants.h>
 
-#include "jfa_mx.cuh"
 #include "jfa_sm100.cuh"
 
 namespace jfa {
@@ -184,9 +183,7 @@ __device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int st
 }
 
 // BIAS: 0 none, 1 relative-position (log2(e)-scaled table staged per key tile),
-// 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.  QP: MXFP8 attention -- P
-// is quantised to E4M3 with one E8M0 scale per 32 keys (counted from the
-// sequence's first key) before P.V; l uses the unquantised weights.
+// 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.
 //
 // Tensor-core order per item (n key tiles; tile T has n_T <= n of them):
 //   QK_A(0), QK_B(0), then for each j: [P_A(j)] PV_A(j), QK_A(j+1),
@@ -194,7 +191,7 @@ __device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int st
 // Barrier phases follow per-CTA counters: g (key tiles so far, for the K/V
 // ring), gt[T] (steps of tile T so far), mt[T] (items with steps for T so
 // far), nk (items so far, for Q).
-template <int BIAS, bool SOFTMAX, bool QP>
+template <int BIAS, bool SOFTMAX>
 __global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
@@ -550,15 +547,13 @@ __global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams
                     if (!pair_sync()) { ok = false; break; }
                     pm = fmaxf(pm, rp[(hf ^ 1) * 128 + r_]);
                     // lazy rescale: keep the reference unless the row maximum grew by
-                    // more than 8 (a factor 2^8).  With MXFP8 P the reference is an
-                    // integer (ceil of the maximum, log2 units), so rescales are exact
-                    // powers of two and the block quantisation of P does not depend on
-                    // it; otherwise the maximum itself, so the largest weight is 1.
-                    // Both halves of a row take the same decision.
+                    // more than 8 (a factor 2^8); the reference is then the maximum
+                    // itself, so the largest weight is 1.  Both halves of a row take
+                    // the same decision.
                     float alpha = 1.f;
                     bool rescale = false;
                     const bool need = pm > m_used + kRescaleThreshold;
-                    const float m_new = need ? (QP ? ceilf(pm) : pm) : m_used;
+                    const float m_new = need ? pm : m_used;
                     if (need && m_used != -CUDART_INF_F) {
                         alpha = ex2(m_used - m_new);
                         rescale = true;
@@ -599,8 +594,6 @@ __global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams
                 {
                     const float2 ref2 = make_float2(ref, ref);
                     float2 ps = make_float2(0.f, 0.f), ps2 = make_float2(0.f, 0.f);
-                    float qbuf[QP ? 32 : 1];   // MXFP8: one 32-key block
-                    (void)qbuf;
                     uint32_t ub[2][16];
                     tmem_ld16(tS + cb, ub[0]);
 #pragma unroll
@@ -625,27 +618,10 @@ __global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams
                                 x[v] = cc + v < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
                             }
                         }
-                        if (QP) {
-                            // the 32 keys of an MX block span two chunks: quantise once
-                            // both halves are in (pairs of chunks, even then odd)
-                            if ((c & 1) == 0) {
+                        uint32_t pw[8];
 #pragma unroll
-                                for (int v = 0; v < 16; ++v) qbuf[v] = x[v];
-                                continue;
-                            }
-#pragma unroll
-                            for (int v = 0; v < 16; ++v) qbuf[16 + v] = x[v];
-                            mx::fake_quant32(qbuf);
-                            uint32_t pw[16];
-#pragma unroll
-                            for (int t = 0; t < 16; ++t) pw[t] = pack_bf16(qbuf[2 * t], qbuf[2 * t + 1]);
-                            tmem_st16(tS + cb + (c - 1) * 8, pw);
-                        } else {
-                            uint32_t pw[8];
-#pragma unroll
-                            for (int t = 0; t < 8; ++t) pw[t] = pack_bf16(x[2 * t], x[2 * t + 1]);
-                            tmem_st8(tS + cb + c * 8, pw);
-                        }
+                        for (int t = 0; t < 8; ++t) pw[t] = pack_bf16(x[2 * t], x[2 * t + 1]);
+                        tmem_st8(tS + cb + c * 8, pw);
                     }
                     tmem_wait_st();
                     const float2 s4 = add2(ps, ps2);
@@ -766,7 +742,7 @@ bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, in
 
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per CTA
 
-cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quant_p, cudaStream_t st) {
+cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st) {
     FwdParams P{};
     if (!make_tmap_rows_heads_d(&P.tm_q, a.q, p.total_q, p.heads) ||
         !make_tmap_rows_heads_d(&P.tm_k, a.k, p.total_kv, p.heads) ||
@@ -782,22 +758,18 @@ cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, bool quan
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
     const bool sm = a.act == JFA_ACT_SOFTMAX;
     void (*kern)(FwdParams) = nullptr;
-    if (quant_p) {
-        if (!sm) return cudaErrorInvalidValue;
-        kern = bias == 0 ? tc_fwd_kernel<0, true, true>
-                         : (bias == 1 ? tc_fwd_kernel<1, true, true> : tc_fwd_kernel<2, true, true>);
-    } else if (bias == 0) {
-        kern = sm ? tc_fwd_kernel<0, true, false> : tc_fwd_kernel<0, false, false>;
+    if (bias == 0) {
+        kern = sm ? tc_fwd_kernel<0, true> : tc_fwd_kernel<0, false>;
     } else if (bias == 1) {
-        kern = sm ? tc_fwd_kernel<1, true, false> : tc_fwd_kernel<1, false, false>;
+        kern = sm ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
     } else {
-        kern = sm ? tc_fwd_kernel<2, true, false> : tc_fwd_kernel<2, false, false>;
+        kern = sm ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;
     prof_begin(st);
     kern<<<grid, kThreads, smem, st>>>(P);
-    prof_end(st, quant_p ? K_TC_FWD_MXFP8 : K_TC_FWD);
+    prof_end(st, K_TC_FWD);
     return cudaGetLastError();
 }
 
