@@ -162,7 +162,7 @@ __device__ __forceinline__ void zero_row(uint8_t* tile, int r) {
 // memory and added to the relative-position table gradient by one warp
 // (score warp t % 16 for tile t, at the start of tile t + 1).
 template <int BIAS, bool SOFTMAX, bool DBIAS>
-__global__ void __maxnreg__(112) tc_bwd_kernel(const __grid_constant__ BwdParams P) {
+__global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_constant__ BwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
     extern __shared__ uint8_t smem_dyn[];

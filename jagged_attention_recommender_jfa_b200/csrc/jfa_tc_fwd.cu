@@ -192,7 +192,7 @@ __device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int st
 // ring), gt[T] (steps of tile T so far), mt[T] (items with steps for T so
 // far), nk (items so far, for Q).
 template <int BIAS, bool SOFTMAX>
-__global__ void __maxnreg__(112) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
+__global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
     if (a.hdr->err != 0 || (int)blockIdx.x >= n_items) return;

@@ -262,7 +262,7 @@ __device__ __forceinline__ uint4 sf_v(const uint8_t* vs, int64_t blk0, int nblk,
 }
 
 template <int BIAS>
-__global__ void __maxnreg__(112) tc_fwd_mx_kernel(const __grid_constant__ MxParams P) {
+__global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_constant__ MxParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
     if (a.hdr->err != 0 || (int)blockIdx.x >= n_items) return;

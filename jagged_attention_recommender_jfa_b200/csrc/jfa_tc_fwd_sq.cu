@@ -136,7 +136,7 @@ __device__ __forceinline__ void dense_bias16(const __nv_bfloat16* p, float (&bb)
 }
 
 template <int BIAS, bool SOFTMAX>
-__global__ void __maxnreg__(144) tc_fwd_sq_kernel(const __grid_constant__ FwdSqParams P) {
+__global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_constant__ FwdSqParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
     const int n_pairs = (n_items + 1) >> 1;

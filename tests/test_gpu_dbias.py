@@ -77,8 +77,23 @@ def check_relpos(name, db, ref, n_c, max_tol, mean_tol):
     assert w.mean() <= mean_tol, f"{name}: mean |err|/sqrt(n) {w.mean():.3e}"
 
 
-def check_dense(name, db, ref, max_tol, mean_tol, rows_mask=None):
+def dense_mask(p):
+    """True at the valid (query, key) pairs of the dense bias layout."""
+    parts = []
+    for nq, nk in zip(p.q_lens, p.kv_lens):
+        nq, nk = int(nq), int(nk)
+        i = np.arange(nq)[:, None]
+        j = np.arange(nk)[None, :]
+        ok = np.ones((nq, nk), bool) if not p.causal else (j <= i + nk - nq)
+        parts.append(np.broadcast_to(ok, (p.H, nq, nk)).reshape(-1))
+    return np.concatenate(parts) if parts else np.zeros(0, bool)
+
+
+def check_dense(name, db, ref, max_tol, mean_tol, rows_mask=None, valid=None):
     g = db.double().cpu().numpy()
+    if valid is not None:
+        # masked pairs are exactly zero
+        assert np.all(g[~valid] == 0.0), f"{name}: masked pairs not zero"
     if rows_mask is not None:
         g, ref = g[rows_mask], ref[rows_mask]
     assert np.all(np.isfinite(ref))
@@ -88,8 +103,6 @@ def check_dense(name, db, ref, max_tol, mean_tol, rows_mask=None):
     assert np.all(err <= bound), f"{name}: max |err| {err.max():.3e}"
     refm = torch.from_numpy(ref).to(torch.bfloat16).double().numpy() if bf16 else ref
     assert np.abs(g - refm).mean() <= mean_tol, f"{name}: mean |err|"
-    # masked pairs are exactly zero
-    assert np.all(g[ref == 0.0] == 0.0), f"{name}: masked pairs not zero"
 
 
 def oracle_dbias(p, act, seq_mask=None):
@@ -125,7 +138,7 @@ def test_dbias_small(cuda_device, workload, seed, kw, act):
     if p.bias_kind == "relpos":
         check_relpos("dtable", db, ref, pairs_per_entry(p), BF16_MAX, BF16_MEAN)
     else:
-        check_dense("dbias", db, ref, BF16_MAX, BF16_MEAN)
+        check_dense("dbias", db, ref, BF16_MAX, BF16_MEAN, valid=dense_mask(p))
 
 
 @pytest.mark.parametrize("d,bias", [(32, "relpos"), (64, "dense")])
@@ -137,7 +150,7 @@ def test_dbias_cuda_core_path(cuda_device, d, bias):
     if bias == "relpos":
         check_relpos("dtable", db, ref, pairs_per_entry(p), F32_MAX, F32_MAX)
     else:
-        check_dense("dbias", db, ref, F32_MAX, F32_MAX)
+        check_dense("dbias", db, ref, F32_MAX, F32_MAX, valid=dense_mask(p))
 
 
 def test_dbias_tiny_f32(cuda_device):
