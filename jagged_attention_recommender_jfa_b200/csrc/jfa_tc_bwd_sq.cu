@@ -23,7 +23,8 @@
 // S^T / dP^T of tile j+1 are issued as soon as the score warps have read
 // those of tile j, so they run during tile j's score phase.
 // TMEM: S^T [0,64), dP^T [64,128), dK [128,256), dV [256,384), dQ^T [384,448).
-// Warps: 0 TMA, 1 MMA, 2..17 score (lane quarter x 16-query group).
+// Warps: 0 TMA, 1 MMA, 2..17 score: warp w reads TMEM lane quarter w % 4, and
+// the four consecutive warps 2 + 4g .. 5 + 4g take queries 16 g .. 16 g + 15.
 #include <math_constants.h>
 
 #include "jfa_sm100.cuh"
@@ -252,8 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.hdr));
         };
         const int sw = warp - 2;
-        const int wq = sw & 3;                 // TMEM lane quarter: keys / d rows 32 wq ..
-        const int grp = sw >> 2;               // queries 16 grp .. +15
+        const int wq = warp & 3;               // TMEM lane quarter (a warp reaches lanes 32 (warp % 4) ..)
+        const int grp = sw >> 2;               // queries 16 grp .. +15 (warps 2..5, 6..9, ...)
         const int r = wq * 32 + lane;          // key row (S^T, dK, dV) / d row (dQ^T)
         const int qc0 = grp * 16;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;

@@ -1,5 +1,13 @@
 """GPU parity of the bias gradient (jfa_backward_dbias) against the oracle.
 
+The backward takes the forward's output O and LSE as inputs, and D =
+rowsum(dO * O) comes from that O.  A bf16 O carries its final rounding (2^-9
+relative), which moves D -- and with it every score gradient ds of the row --
+by up to |dO| |O| 2^-9: harmless in dQ / dK (sums over many pairs) but of the
+order of the bound in a single ds.  So both sides here get the same O and LSE:
+the oracle's forward, rounded to the stored types, is passed to the GPU
+backward and, as out_for_d, to the oracle's backward.
+
 Bounds, written here:
   dense jagged bias (one ds per entry): max |err| <= 2e-2 + half a bf16 ulp of
       the reference and mean |err| <= 2e-3, the benchmark spec's bounds for bf16
@@ -32,12 +40,22 @@ def _dev(p, dev):
     return {n: t(getattr(p, n)) for n in ("q", "k", "v", "dout", "bias", "q_off", "kv_off")}
 
 
+def oracle_forward_inputs(p, act, dev):
+    """The oracle's O (rounded to the stored type) and LSE (fp32), as the
+    backward's inputs on both sides."""
+    ro, rl = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, bias=p.bias,
+                            bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
+                            causal=p.causal)
+    out = torch.from_numpy(ro).to(p.q.dtype).to(dev)
+    lse = torch.from_numpy(rl).float().to(dev) if rl is not None else None
+    return out, lse
+
+
 def run_gpu(p, dev, act=None):
     act = act or p.act
     d = _dev(p, dev)
     prob = jfa.problem_of(p)
-    out, lse = jfa.attention_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"],
-                                     d["bias"], act, p.causal)
+    out, lse = oracle_forward_inputs(p, act, dev)
     dq, dk, dv, db = jfa.attention_backward(prob, d["q"], d["k"], d["v"], out, lse, d["dout"],
                                             d["q_off"], d["kv_off"], d["bias"], act, p.causal,
                                             want_dbias=True)
@@ -106,9 +124,11 @@ def check_dense(name, db, ref, max_tol, mean_tol, rows_mask=None, valid=None):
 
 
 def oracle_dbias(p, act, seq_mask=None):
+    out, _ = oracle_forward_inputs(p, act, "cpu")
     return oracle.backward(p.q_off, p.kv_off, p.q, p.k, p.v, p.dout, bias=p.bias,
                            bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
-                           causal=p.causal, seq_mask=seq_mask, dbias=True)[3]
+                           causal=p.causal, seq_mask=seq_mask, dbias=True,
+                           out_for_d=out if act == "softmax" else None)[3]
 
 
 CASES = [
