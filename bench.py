@@ -107,6 +107,21 @@ def visible_pairs(q_lens, kv_lens, causal, block=0):
     return out
 
 
+def sq_bytes(p, backward: bool, softmax: bool) -> float:
+    """Algorithmic HBM bytes of one short-query kernel launch: every operand
+    read once and every result written once.  Forward: Q, K, V, the dense
+    bias, O (and the fp32 LSE).  Backward: Q, K, V, dO, the dense bias, LSE
+    and D (fp32), written dQ, dK, dV."""
+    el = 2 if p.dtype != "f32" else 4
+    tq = float(p.total_q) * p.H * p.d * el
+    tkv = float(p.kv_off[-1]) * p.H * p.d * el
+    bias = float(p.bias.numel()) * el if p.bias_kind == "dense" else 0.0
+    rows = float(p.total_q) * p.H * 4
+    if not backward:
+        return tq + 2 * tkv + bias + tq + (rows if softmax else 0.0)
+    return 2 * tq + 2 * tkv + bias + (2 * rows if softmax else 0.0) + tq + 2 * tkv
+
+
 def flops_of(p, pairs_per_seq=None, block=0):
     pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block) if pairs_per_seq is None else pairs_per_seq
     f_fwd = 4.0 * p.d * p.H * float(pairs.sum())
@@ -449,7 +464,15 @@ def main():
         pairs = f_fwd / (4.0 * d_)
         algo = {"tc_fwd": f_fwd, "tc_fwd_mxfp8": f_fwd, "tc_bwd": f_bwd, "simt_fwd": f_fwd,
                 "simt_bwd_dq": 6.0 * d_ * pairs, "simt_bwd_dkdv": 8.0 * d_ * pairs}.get(dom)
-        if dom == "tc_fwd_mxfp8":
+        if dom in ("tc_fwd_sq", "tc_bwd_sq"):
+            # short query sequences: the pair work is small against the bytes
+            # every operand costs once, so HBM bounds these kernels
+            algo = sq_bytes(p, dom == "tc_bwd_sq", act == "softmax")
+            peak = peaks["hbm_gbs"]
+            bound, unit = "hbm", "GB/s"
+            note = f"HBM copy bandwidth of {peak_src}"
+            achieved = algo / avg_s / 1e9
+        elif dom == "tc_fwd_mxfp8":
             # E4M3 block-scaled MMAs: the measured bf16 peak x the nominal
             # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
             peak = 2.0 * peaks["bf16_tflops"]
@@ -466,12 +489,15 @@ def main():
             peak = SM_COUNT * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
             bound, unit = "alu", "TFLOP/s"
             note = f"fp32 FMA: {SM_COUNT} SMs x {FP32_LANES_PER_SM} lanes x 2 x {mhz:.0f} MHz"
-        achieved = algo / avg_s / 1e12 if algo else None
+        if bound != "hbm":
+            achieved = algo / avg_s / 1e12 if algo else None
         traffic = recorded_traffic(dom, args.workload)
         roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": unit, "frac": achieved / peak if achieved else None,
                     "traffic": traffic, "peak_source": note,
-                    "algorithmic_flops_per_launch": algo, "avg_launch_ms": avg_s * 1e3}
+                    ("algorithmic_bytes_per_launch" if bound == "hbm"
+                     else "algorithmic_flops_per_launch"): algo,
+                    "avg_launch_ms": avg_s * 1e3}
 
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,

@@ -206,6 +206,27 @@ def test_no_bias(cuda_device):
     check_problem(p, cuda_device)
 
 
+@pytest.mark.parametrize("bias", ["relpos", "none"])
+def test_forward_reference_moves(cuda_device, bias):
+    """Scores whose row maximum moves across key tiles: the forward keeps a
+    row's softmax reference until the maximum outgrows it by 2^8, then rescales
+    O.  Keys of sequence 0 grow in norm tile by tile (the maximum jumps past
+    the threshold at every tile), those of sequence 1 shrink (the first tile
+    holds the maximum), those of sequence 2 grow slowly (weights above 1, no
+    rescale), sequence 3 is unscaled; gradients are checked relative to their
+    RMS, as the key norms reach ~10."""
+    import dataclasses
+    p = make_problem("self_bf16", 17, q_lens=[700, 520, 640, 300], bias=bias)
+    k = p.k.float().clone()
+    for b, (slope, sign) in enumerate([(2.5, 1), (2.5, -1), (0.4, 1), (0.0, 1)]):
+        lo, hi = int(p.kv_off[b]), int(p.kv_off[b + 1])
+        t = torch.arange(hi - lo, dtype=torch.float32) // 128
+        ramp = 1.0 + slope * (t if sign > 0 else t.max() - t)
+        k[lo:hi] *= ramp[:, None, None]
+    p = dataclasses.replace(p, k=k.to(p.k.dtype))
+    check_problem(p, cuda_device, rms_scaled=True)
+
+
 # ---------------------------------------------------------------------------
 # properties: neighbours do not leak, guards untouched, V = 1 gives O = 1
 # ---------------------------------------------------------------------------
