@@ -24,7 +24,11 @@
 // those of tile j, so they run during tile j's score phase.
 // TMEM: S^T [0,64), dP^T [64,128), dK [128,256), dV [256,384), dQ^T [384,448).
 // Warps: 0 TMA, 1 MMA, 2..17 score: warp w reads TMEM lane quarter w % 4, and
-// the four consecutive warps 2 + 4g .. 5 + 4g take queries 16 g .. 16 g + 15.
+// the four consecutive warps 2 + 4g .. 5 + 4g take queries 16 g .. 16 g + 15;
+// 18, 19 stage a dense bias (one query row per lane: the 16-byte blocks that
+// cover the row's keys of the tile, one bulk copy) into shared memory once
+// the score warps have read the previous tile's.  Twenty warps still leave
+// 96 registers per thread (five warps per SM sub-partition).
 #include <math_constants.h>
 
 #include "jfa_sm100.cuh"
@@ -39,7 +43,7 @@ bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows
 namespace {
 
 constexpr int BQ = 64, BN = 128, HD = 128;
-constexpr int kThreads = 64 + 16 * 32;
+constexpr int kThreads = 64 + 16 * 32 + 64;
 constexpr uint32_t kKBox = 128 * 128;            // [128 rows][64 bf16]
 constexpr uint32_t kKTile = 2 * kKBox;           // 128 x 128 bf16
 constexpr uint32_t kQBox = 64 * 128;             // [64 rows][64 bf16]
@@ -51,7 +55,11 @@ constexpr uint32_t kOffV = kOffK + 2 * kKTile;   // 2 stages
 constexpr uint32_t kOffPT = kOffV + 2 * kKTile;  // P^T  [128 keys][64 queries] bf16 (128-byte rows)
 constexpr uint32_t kOffDST = kOffPT + 128 * 128; // dS^T [128 keys][64 queries]
 constexpr uint32_t kOffRow = kOffDST + 128 * 128; // LSE (log2) [64], D [64]
-constexpr uint32_t kOffBar = kOffRow + 512;
+// dense bias rows of a key tile: 64 query rows x 272 bytes (the 16-byte
+// blocks that cover 128 bf16 at any 2-byte alignment)
+constexpr uint32_t kDRow = 272;
+constexpr uint32_t kOffDense = kOffRow + 512;
+constexpr uint32_t kOffBar = kOffDense + BQ * kDRow;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -64,6 +72,7 @@ struct Bars {
     uint64_t dkv_full;   // dK, dV, dQ^T of the key tile done
     uint64_t dkv_free;   // 16 score warps read dK / dV
     uint64_t rows_full;  // LSE / D staged (2 warps)
+    uint64_t dense_full, dense_empty;   // dense bias rows staged (2 warps) / read (16)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -145,6 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
         mbar_init(&bars->dkv_full, 1);
         mbar_init(&bars->dkv_free, 16);
         mbar_init(&bars->rows_full, 2);
+        mbar_init(&bars->dense_full, 2);
+        mbar_init(&bars->dense_empty, 16);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_barrier_init();
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             mma_commit(&bars->drain);
             mbar_wait_drain(&bars->drain, 0, a.hdr);
         }
-    } else {
+    } else if (warp < 18) {
         // ------------------------------------------------ score warps
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.hdr));
@@ -267,6 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
         const float* tab = (BIAS == 1) ? reinterpret_cast<const float*>(a.bias) + (int64_t)h * a.relpos_len : nullptr;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
         const int64_t dense_base = (BIAS == 2) ? a.dense_off[b] + (int64_t)h * nq * nkv : 0;
+        // staged bias: query row q's keys of a tile start at element
+        // (row start index) mod 8 of its row buffer
+        const uintptr_t dense_e0 = reinterpret_cast<uintptr_t>(dense + dense_base) >> 1;
         bool ok = nt > 0;
         // LSE (log2 units) and D of the <= 64 queries: two warps stage them
         if (ok && sw < 2) {
@@ -294,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             const int jk = j * BN + r;          // key index within the sequence
             const bool jvalid = jk < nkv;
             if (!wwait(&bars->s_full, j & 1)) { ok = false; break; }
+            if (BIAS == 2 && !wwait(&bars->dense_full, j & 1)) { ok = false; break; }
             tc_fence_after();
             uint32_t u[16], g[16];
             tmem_ld16(tS, u);
@@ -319,10 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                         x[v] = fmaf(__uint_as_float(u[v]), sc,
                                     __ldg(tab + min(max(qc0 + v - jk, -C), C) + C) * kLog2e);
                 } else if (BIAS == 2) {
-                    const __nv_bfloat16* col = dense + dense_base + min(jk, nkv - 1);
                     __nv_bfloat16 bh[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) bh[v] = col[(int64_t)min(qc0 + v, nq - 1) * nkv];
+                    for (int v = 0; v < 16; ++v) {
+                        const int qq = min(qc0 + v, nq - 1);
+                        const int e = (int)((dense_e0 + (uintptr_t)qq * (uintptr_t)nkv) & 7u) + r;
+                        bh[v] = reinterpret_cast<const __nv_bfloat16*>(smem + kOffDense + qq * kDRow)[e];
+                    }
 #pragma unroll
                     for (int v = 0; v < 16; ++v)
                         x[v] = fmaf(__uint_as_float(u[v]), sc, __bfloat162float(bh[v]) * kLog2e);
@@ -367,6 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                     for (int v = 0; v < 16; ++v)
                         if (g[v] != 0u) atomicAdd(dtab + min(max(qc0 + v - jk, -C), C) + C, __uint_as_float(g[v]));
                 }
+            }
+            if (BIAS == 2) {   // this tile's staged bias rows are read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->dense_empty);
             }
             // P^T and dS^T to shared memory; the MMAs of the previous tile that
             // read them have completed (this warp saw their commit below)
@@ -422,6 +444,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(a.dq) + ((int64_t)q0 * a.H + h) * HD + r;
             for (int qi = 0; qi < nq; ++qi) dq[(int64_t)qi * a.H * HD] = __float2bfloat16_rn(0.f);
         }
+    } else if (BIAS == 2 && nt > 0) {
+        // ------------------------------------------------ dense bias stagers
+        const int row = (warp - 18) * 32 + lane;   // query row of this lane
+        const bool has_row = row < nq;
+        const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+        const int64_t row_off = has_row ? a.dense_off[b] + ((int64_t)h * nq + row) * nkv : 0;
+        uint8_t* dst = smem + kOffDense + row * kDRow;
+        int staged = 0;
+        for (int j = 0; j < nt; ++j) {
+            // the buffer is free once the score warps have read tile j - 1
+            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->dense_empty, (j - 1) & 1, abort_flag, a.hdr)))
+                break;
+            const int jc = j * BN;
+            const int nk = min(BN, nkv - jc);   // keys of this tile (>= 1)
+            // the 16-byte blocks covering the row's nk bias values: every block
+            // holds a value of the bias tensor, so the copy stays in its allocation
+            uintptr_t src = 0;
+            uint32_t bytes = 0;
+            if (has_row) {
+                const uintptr_t first = reinterpret_cast<uintptr_t>(dense + row_off + jc);
+                src = first & ~static_cast<uintptr_t>(15);
+                bytes = (uint32_t)(((first + 2u * (uint32_t)nk + 15u) & ~static_cast<uintptr_t>(15)) - src);
+            }
+            const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&bars->dense_full, total);
+            __syncwarp();
+            if (bytes) bulk_load(dst, reinterpret_cast<const void*>(src), bytes, &bars->dense_full);
+            if (has_row && j + 1 < nt) {   // warm L2 for the next tile's rows
+                prefetch_l2(dense + row_off + jc + BN);
+                prefetch_l2(dense + row_off + min(jc + 2 * BN, nkv) - 1);
+            }
+            staged = j + 1;
+        }
+        // never leave the CTA with copies in flight
+        if (staged > 0 && lane == 0) mbar_wait_drain(&bars->dense_full, (staged - 1) & 1, a.hdr);
     }
     tc_fence_before();
     __syncthreads();

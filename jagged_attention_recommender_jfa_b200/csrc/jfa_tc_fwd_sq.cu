@@ -20,7 +20,13 @@
 //
 // Warps: softmax warps 0, 1, 4, 5 (tile A) and 8, 9, 12, 13 (tile B): lane
 // quarter w % 4 in {0, 1} (rows 0..63), half row (w >> 2) & 1 (64 columns);
-// warp 2 MMA issuer and TMEM allocator, warp 3 TMA; warps 6, 7, 10, 11 idle.
+// warp 2 MMA issuer and TMEM allocator, warp 3 TMA; warps 6, 7 (tile A) and
+// 10, 11 (tile B) stage a dense bias: each lane copies one query row's
+// segment of the key tile (the covering 16-byte blocks, one bulk copy) into a
+// per-tile shared buffer as soon as the softmax warps have read the previous
+// tile's, so the bias of a step is on chip when its scores arrive.
+// The Q tile is a 64-row box: the upper 64 rows of the M = 128 operand read
+// whatever follows it in shared memory, and their S / O rows are ignored.
 // With 448 threads a softmax thread keeps its 64 scores in registers between
 // the maximum and the exponentials (one TMEM read per step).
 #include <math_constants.h>
@@ -32,6 +38,7 @@ namespace jfa {
 using namespace sm100;
 
 bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads);
+bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_rows);
 
 namespace {
 
@@ -41,13 +48,19 @@ constexpr int kThreads = 32 * 14;
 constexpr int CW = 64;
 constexpr uint32_t kBox = 128 * 128;
 constexpr uint32_t kTile = 2 * kBox;
+constexpr uint32_t kQBox = BQ * 128;              // one [64 rows][64 bf16] box
+constexpr uint32_t kQTile = 2 * kQBox;
 constexpr uint32_t kOffQ = 0;                     // Q_A, Q_B
-constexpr uint32_t kOffK = kOffQ + 2 * kTile;     // K_A, K_B
+constexpr uint32_t kOffK = kOffQ + 2 * kQTile;    // K_A, K_B
 constexpr uint32_t kOffV = kOffK + 2 * kTile;     // V_A, V_B
 constexpr int kWin = 384;
 constexpr uint32_t kWinBytes = kWin * 16;
 constexpr uint32_t kOffBias = kOffV + 2 * kTile;  // per tile
-constexpr uint32_t kOffRed = kOffBias + 2 * kWinBytes;    // [parity][tile][half][64] row maxima
+// dense bias rows of a key tile, per tile: 64 rows x 272 bytes (the 16-byte
+// blocks that cover 128 bf16 at any 2-byte alignment)
+constexpr uint32_t kDRow = 272;
+constexpr uint32_t kOffDense = kOffBias + 2 * kWinBytes;
+constexpr uint32_t kOffRed = kOffDense + 2 * BQ * kDRow;  // [parity][tile][half][64] row maxima
 constexpr uint32_t kOffLred = kOffRed + 2 * 2 * 2 * 64 * 4;
 constexpr uint32_t kOffBar = kOffLred + 2 * 2 * 2 * 64 * 4;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;
@@ -60,6 +73,7 @@ struct Bars {
     uint64_t v_full[2], v_empty[2];
     uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
     uint64_t bias_full[2];
+    uint64_t dense_full[2], dense_empty[2];   // per tile: dense bias rows staged / read
     uint64_t pair[4];     // [tile][lane quarter]
     uint64_t drain;
     uint32_t tmem_base;
@@ -79,6 +93,9 @@ __device__ __forceinline__ uint32_t kmajor_lo(uint32_t tile_base) { return sw128
 __device__ __forceinline__ uint32_t mnmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, kBox); }
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t lo, int k) {
     return sw128_desc(lo + (uint32_t)(k >> 2) * (kBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
+}
+__device__ __forceinline__ uint64_t qmajor_desc(uint32_t lo, int k) {
+    return sw128_desc(lo + (uint32_t)(k >> 2) * (kQBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
 }
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t lo, int k) {
     return sw128_desc(lo + (uint32_t)k * 128u, kDescHi);
@@ -135,6 +152,27 @@ __device__ __forceinline__ void dense_bias16(const __nv_bfloat16* p, float (&bb)
     }
 }
 
+// 16 consecutive bf16 of a staged bias row as floats: element e of the row
+// buffer (its first element at e0 < 8 of the first 16-byte block); the three
+// blocks that cover them are in the buffer for every e <= e0 + 112.
+__device__ __forceinline__ void staged_bias16(const uint8_t* rowbuf, int e, float (&bb)[16]) {
+    const uint4* blk = reinterpret_cast<const uint4*>(rowbuf) + (e >> 3);
+    const uint4 b0 = blk[0], b1 = blk[1], b2 = blk[2];
+    const uint32_t W[12] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w, b2.x, b2.y, b2.z, b2.w};
+    const int e0 = e & 7, s = e0 >> 1, sh = (e0 & 1) * 16;
+    uint32_t V1[10], V2[9];
+#pragma unroll
+    for (int k = 0; k < 10; ++k) V1[k] = (s & 2) ? W[k + 2] : W[k];
+#pragma unroll
+    for (int k = 0; k < 9; ++k) V2[k] = (s & 1) ? V1[k + 1] : V1[k];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t pr = __funnelshift_r(V2[k], V2[k + 1], sh);
+        bb[2 * k] = __uint_as_float(pr << 16);
+        bb[2 * k + 1] = __uint_as_float(pr & 0xffff0000u);
+    }
+}
+
 template <int BIAS, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_constant__ FwdSqParams P) {
     const AttnArgs& a = P.a;
@@ -161,6 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             mbar_init(&bars->pv_done[t], 1);
             mbar_init(&bars->o_free[t], 4);
             mbar_init(&bars->bias_full[t], 1);
+            mbar_init(&bars->dense_full[t], 2);
+            mbar_init(&bars->dense_empty[t], 4);
         }
         for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 2);
         mbar_init(&bars->drain, 1);
@@ -195,9 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 const Item w = load_item(a, 2 * pr + t, n_items);
                 if (w.n == 0) continue;
                 if (qc > 0 && !mbar_wait(&bars->q_free[t], (qc - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars->q_full[t], kTile);
-                tma_load_3d(smem + kOffQ + t * kTile, &P.tm_q, &bars->q_full[t], 0, w.h, w.q0);
-                tma_load_3d(smem + kOffQ + t * kTile + kBox, &P.tm_q, &bars->q_full[t], 64, w.h, w.q0);
+                mbar_arrive_expect_tx(&bars->q_full[t], kQTile);
+                tma_load_3d(smem + kOffQ + t * kQTile, &P.tm_q, &bars->q_full[t], 0, w.h, w.q0);
+                tma_load_3d(smem + kOffQ + t * kQTile + kQBox, &P.tm_q, &bars->q_full[t], 64, w.h, w.q0);
                 ++qc;
                 for (int j = 0; j < w.n; ++j) {
                     const int z = w.k0 + j * BN;
@@ -243,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
             int qc[2] = {0, 0}, kc[2] = {0, 0}, gt[2] = {0, 0}, mt[2] = {0, 0};
             bool ok = true;
-            const uint32_t qK[2] = {kmajor_lo(sbase + kOffQ), kmajor_lo(sbase + kOffQ + kTile)};
+            const uint32_t qK[2] = {kmajor_lo(sbase + kOffQ), kmajor_lo(sbase + kOffQ + kQTile)};
             const uint32_t kK[2] = {kmajor_lo(sbase + kOffK), kmajor_lo(sbase + kOffK + kTile)};
             const uint32_t vM[2] = {mnmajor_lo(sbase + kOffV), mnmajor_lo(sbase + kOffV + kTile)};
             for (int r = 0; ok; ++r) {
@@ -256,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < HD / 16; ++k)
-                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qK[t], k), kmajor_desc(kK[t], k), idesc_qk, k > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem + t * 128, qmajor_desc(qK[t], k), kmajor_desc(kK[t], k), idesc_qk, k > 0 ? 1u : 0u);
                     mma_commit(&bars->s_full[t]);
                     mma_commit(&bars->k_empty[t]);
                     if (j == w[t].n - 1) mma_commit(&bars->q_free[t]);
@@ -344,12 +384,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
                                           ? a.dense_off[w.b] + ((int64_t)w.h * w.nq + i) * w.nkv : 0;
+            // this row's staged bias: element k of key tile j at element e0 + k
+            // of the row buffer (e0: the 2-byte offset of the tile's first key
+            // in its 16-byte block; a key tile starts 128 elements on, so e0
+            // is the same for every tile of the row)
+            const uint8_t* drow = smem + kOffDense + (tt * BQ + r_) * kDRow;
+            const int e0 = (int)((reinterpret_cast<uintptr_t>(dense + dense_row) & 15) >> 1);
             float m_used = -CUDART_INF_F, l = 0.f;
             for (int j = 0; j < n; ++j, ++gt) {
                 if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
                 tc_fence_after();
                 const int jc = j * BN;
                 if (BIAS == 1 && !wwait(&bars->bias_full[tt], gt & 1)) { ok = false; break; }
+                if (BIAS == 2 && !wwait(&bars->dense_full[tt], gt & 1)) { ok = false; break; }
                 const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;
                 const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW);
                 const int lo = i - jc - (BN - 1) + C;
@@ -387,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                     } else if (BIAS == 2) {
                         if (cc + 16 <= nvis) {
                             float bb[16];
-                            dense_bias16(dense + dense_row + jc + cc, bb);
+                            staged_bias16(drow, e0 + cc, bb);
 #pragma unroll
                             for (int v = 0; v < 16; v += 2) {
                                 const float2 r2 = fma2(make_float2(x[v], x[v + 1]), sc2,
@@ -397,7 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                         } else {
 #pragma unroll
                             for (int v = 0; v < 16; ++v)
-                                x[v] = fmaf(x[v], sc, cc + v < nvis ? __bfloat162float(dense[dense_row + jc + cc + v]) * kLog2e : 0.f);
+                                x[v] = fmaf(x[v], sc,
+                                            cc + v < nvis
+                                                ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(drow)[e0 + cc + v]) * kLog2e
+                                                : 0.f);
                         }
                     } else {
 #pragma unroll
@@ -416,6 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                         const float m4 = max3(x[12], x[13], x[14]);
                         pm = max3(pm, max3(m0, m1, m2), max3(m3, m4, x[15]));
                     }
+                }
+                if (BIAS == 2) {   // the staged rows of this step are read
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->dense_empty[tt]);
                 }
                 float ref = 0.f;
                 if (softmax) {
@@ -545,6 +599,53 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 a.lse[(int64_t)(w.q0 + i) * a.H + w.h] =
                     l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
         }
+    } else if (BIAS == 2 && warp >= 4) {
+        // ------------------------------------------------ dense bias stagers
+        // warps 6, 7 (tile A) and 10, 11 (tile B); lane -> query row
+        const int tt = warp >> 3;
+        const int row = (warp & 1) * 32 + lane;
+        uint8_t* dst = smem + kOffDense + (tt * BQ + row) * kDRow;
+        uint64_t* full = &bars->dense_full[tt];
+        const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
+        int g = 0;   // steps staged for this tile (the softmax warps' step count)
+        bool ok = true;
+        for (int rr = 0; ok; ++rr) {
+            const int pr = pair_of_turn(rr, cta, G);
+            if (pr >= n_pairs) break;
+            const Item w = load_item(a, 2 * pr + tt, n_items);
+            if (!w.live || w.n == 0) continue;
+            const bool has_row = row < w.nq;
+            const int64_t row_off = has_row ? a.dense_off[w.b] + ((int64_t)w.h * w.nq + row) * w.nkv : 0;
+            for (int j = 0; j < w.n; ++j, ++g) {
+                // the buffer is free once the softmax warps have read step g - 1
+                if (g > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->dense_empty[tt], (g - 1) & 1, abort_flag, a.hdr))) {
+                    ok = false;
+                    break;
+                }
+                const int jc = j * BN;
+                const int nk = min(BN, w.nkv - jc);   // keys of this tile (>= 1)
+                // the 16-byte blocks covering the row's nk bias values: every
+                // block holds a value of the bias tensor, so the copy stays in
+                // its allocation
+                uintptr_t src = 0;
+                uint32_t bytes = 0;
+                if (has_row) {
+                    const uintptr_t first = reinterpret_cast<uintptr_t>(dense + row_off + jc);
+                    src = first & ~static_cast<uintptr_t>(15);
+                    bytes = (uint32_t)(((first + 2u * (uint32_t)nk + 15u) & ~static_cast<uintptr_t>(15)) - src);
+                }
+                const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+                if (lane == 0) mbar_arrive_expect_tx(full, total);
+                __syncwarp();
+                if (bytes) bulk_load(dst, reinterpret_cast<const void*>(src), bytes, full);
+                if (has_row && j + 1 < w.n) {   // warm L2 for the next step's rows
+                    prefetch_l2(dense + row_off + jc + BN);
+                    prefetch_l2(dense + row_off + min(jc + 2 * BN, w.nkv) - 1);
+                }
+            }
+        }
+        // never leave the CTA with copies in flight
+        if (g > 0 && lane == 0) mbar_wait_drain(full, (g - 1) & 1, a.hdr);
     }
     tc_fence_before();
     __syncthreads();
@@ -562,7 +663,7 @@ constexpr int kSmemLimitFsq = 232448;
 // when every n_q <= 64), taken two at a time.
 cudaError_t tc_forward_sq_launch(const jfa_problem& p, const AttnArgs& a, cudaStream_t st) {
     FwdSqParams P{};
-    if (!make_tmap_rows_heads_d(&P.tm_q, a.q, p.total_q, p.heads) ||
+    if (!make_tmap_rows_heads_d_box(&P.tm_q, a.q, p.total_q, p.heads, BQ) ||
         !make_tmap_rows_heads_d(&P.tm_k, a.k, p.total_kv, p.heads) ||
         !make_tmap_rows_heads_d(&P.tm_v, a.v, p.total_kv, p.heads))
         return cudaErrorInvalidValue;
