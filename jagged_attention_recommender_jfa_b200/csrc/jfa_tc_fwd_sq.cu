@@ -15,18 +15,21 @@
 // Q K^T), and the tensor core alternates between them:
 //   QK_A(0), QK_B(0), then per step j: [P_A(j)] PV_A(j), QK_A(j+1),
 //   [P_B(j)] PV_B(j), QK_B(j+1).
-// A tile's rows 64..127 are never used (the MMAs run M = 128 on a 128-row
-// box whose upper half belongs to other rows; those S/O rows are ignored).
+// The queries of both items share one 128-row Q tile: item A's <= 64 rows in
+// rows 0..63, item B's in rows 64..127.  Both Q K^T run M = 128 on the whole
+// tile (each against its own item's keys), so item A's scores are valid in
+// TMEM lanes 0..63 of S_A and item B's in lanes 64..127 of S_B (the other
+// lanes pair a query with the other item's keys and are never read); P.V
+// keeps the same lanes in O_A / O_B.  The softmax work of the two items thus
+// falls on all four lane quarters, i.e. on all four SM sub-partitions.
 //
-// Warps: softmax warps 0, 1, 4, 5 (tile A) and 8, 9, 12, 13 (tile B): lane
-// quarter w % 4 in {0, 1} (rows 0..63), half row (w >> 2) & 1 (64 columns);
-// warp 2 MMA issuer and TMEM allocator, warp 3 TMA; warps 6, 7 (tile A) and
-// 10, 11 (tile B) stage a dense bias: each lane copies one query row's
-// segment of the key tile (the covering 16-byte blocks, one bulk copy) into a
-// per-tile shared buffer as soon as the softmax warps have read the previous
-// tile's, so the bias of a step is on chip when its scores arrive.
-// The Q tile is a 64-row box: the upper 64 rows of the M = 128 operand read
-// whatever follows it in shared memory, and their S / O rows are ignored.
+// Warps: softmax warps 0, 1, 4, 5 (item A: lane quarters 0, 1) and 2, 3, 6, 7
+// (item B: quarters 2, 3), half row (w >> 2) & 1 (64 columns); warp 8 MMA
+// issuer and TMEM allocator, warp 9 TMA; warps 10, 11 (item A) and 12, 13
+// (item B) stage a dense bias: each lane copies one query row's segment of
+// the key tile (the covering 16-byte blocks, one bulk copy) into a per-item
+// shared buffer as soon as the softmax warps have read the previous tile's,
+// so the bias of a step is on chip when its scores arrive.
 // With 448 threads a softmax thread keeps its 64 scores in registers between
 // the maximum and the exponentials (one TMEM read per step).
 #include <math_constants.h>
@@ -43,15 +46,14 @@ bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128, BQ = 64;
-constexpr int kMmaWarp = 2, kTmaWarp = 3;
+constexpr int kMmaWarp = 8, kTmaWarp = 9;
 constexpr int kThreads = 32 * 14;
 constexpr int CW = 64;
 constexpr uint32_t kBox = 128 * 128;
 constexpr uint32_t kTile = 2 * kBox;
-constexpr uint32_t kQBox = BQ * 128;              // one [64 rows][64 bf16] box
-constexpr uint32_t kQTile = 2 * kQBox;
-constexpr uint32_t kOffQ = 0;                     // Q_A, Q_B
-constexpr uint32_t kOffK = kOffQ + 2 * kQTile;    // K_A, K_B
+constexpr uint32_t kQHalf = BQ * 128;             // one item's [64 rows][64 bf16] in a box
+constexpr uint32_t kOffQ = 0;                     // [Q_A; Q_B]: one 128-row tile
+constexpr uint32_t kOffK = kOffQ + kTile;         // K_A, K_B
 constexpr uint32_t kOffV = kOffK + 2 * kTile;     // V_A, V_B
 constexpr int kWin = 384;
 constexpr uint32_t kWinBytes = kWin * 16;
@@ -93,9 +95,6 @@ __device__ __forceinline__ uint32_t kmajor_lo(uint32_t tile_base) { return sw128
 __device__ __forceinline__ uint32_t mnmajor_lo(uint32_t tile_base) { return sw128_desc_lo(tile_base, kBox); }
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t lo, int k) {
     return sw128_desc(lo + (uint32_t)(k >> 2) * (kBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
-}
-__device__ __forceinline__ uint64_t qmajor_desc(uint32_t lo, int k) {
-    return sw128_desc(lo + (uint32_t)(k >> 2) * (kQBox >> 4) + (uint32_t)(k & 3) * 2u, kDescHi);
 }
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t lo, int k) {
     return sw128_desc(lo + (uint32_t)k * 128u, kDescHi);
@@ -235,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 const Item w = load_item(a, 2 * pr + t, n_items);
                 if (w.n == 0) continue;
                 if (qc > 0 && !mbar_wait(&bars->q_free[t], (qc - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars->q_full[t], kQTile);
-                tma_load_3d(smem + kOffQ + t * kQTile, &P.tm_q, &bars->q_full[t], 0, w.h, w.q0);
-                tma_load_3d(smem + kOffQ + t * kQTile + kQBox, &P.tm_q, &bars->q_full[t], 64, w.h, w.q0);
+                mbar_arrive_expect_tx(&bars->q_full[t], 2 * kQHalf);
+                tma_load_3d(smem + kOffQ + t * kQHalf, &P.tm_q, &bars->q_full[t], 0, w.h, w.q0);
+                tma_load_3d(smem + kOffQ + kBox + t * kQHalf, &P.tm_q, &bars->q_full[t], 64, w.h, w.q0);
                 ++qc;
                 for (int j = 0; j < w.n; ++j) {
                     const int z = w.k0 + j * BN;
@@ -283,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
             int qc[2] = {0, 0}, kc[2] = {0, 0}, gt[2] = {0, 0}, mt[2] = {0, 0};
             bool ok = true;
-            const uint32_t qK[2] = {kmajor_lo(sbase + kOffQ), kmajor_lo(sbase + kOffQ + kQTile)};
+            const uint32_t qK = kmajor_lo(sbase + kOffQ);   // both items' queries
             const uint32_t kK[2] = {kmajor_lo(sbase + kOffK), kmajor_lo(sbase + kOffK + kTile)};
             const uint32_t vM[2] = {mnmajor_lo(sbase + kOffV), mnmajor_lo(sbase + kOffV + kTile)};
             for (int r = 0; ok; ++r) {
@@ -296,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < HD / 16; ++k)
-                        mma_bf16_ss(tmem + t * 128, qmajor_desc(qK[t], k), kmajor_desc(kK[t], k), idesc_qk, k > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qK, k), kmajor_desc(kK[t], k), idesc_qk, k > 0 ? 1u : 0u);
                     mma_commit(&bars->s_full[t]);
                     mma_commit(&bars->k_empty[t]);
                     if (j == w[t].n - 1) mma_commit(&bars->q_free[t]);
@@ -334,22 +333,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             mma_commit(&bars->drain);
             mbar_wait_drain(&bars->drain, 0, a.hdr);
         }
-    } else if ((warp & 3) < 2) {
+    } else if (warp < 8) {
         // ------------------------------------------------ softmax warps
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, a.hdr));
         };
-        const int tt = warp >> 3;
+        const int wq = warp & 3;                 // TMEM lane quarter
+        const int tt = wq >> 1;                  // item A: quarters 0, 1; item B: 2, 3
         const int hf = (warp >> 2) & 1;
-        const int wq = warp & 3;                 // 0 or 1
-        const int r_ = wq * 32 + lane;           // row 0..63
+        const int r_ = (wq & 1) * 32 + lane;     // row 0..63 of the item
         const int cb = hf * CW;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tmem + lane_addr + tt * 128;
         const uint32_t tO = tmem + lane_addr + 256 + tt * 128 + cb;
         float* red = reinterpret_cast<float*>(smem + kOffRed);
         float* lred = reinterpret_cast<float*>(smem + kOffLred);
-        uint64_t* pair_bar = &bars->pair[tt * 2 + wq];
+        uint64_t* pair_bar = &bars->pair[tt * 2 + (wq & 1)];
         int n_pair = 0;
         auto pair_sync = [&]() -> bool {
             __syncwarp();
@@ -599,10 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 a.lse[(int64_t)(w.q0 + i) * a.H + w.h] =
                     l_row > 0.f ? m_used * (1.0f / kLog2e) + logf(l_row) : -CUDART_INF_F;
         }
-    } else if (BIAS == 2 && warp >= 4) {
+    } else if (BIAS == 2 && warp >= 10) {
         // ------------------------------------------------ dense bias stagers
-        // warps 6, 7 (tile A) and 10, 11 (tile B); lane -> query row
-        const int tt = warp >> 3;
+        // warps 10, 11 (item A) and 12, 13 (item B); lane -> query row
+        const int tt = (warp - 10) >> 1;
         const int row = (warp & 1) * 32 + lane;
         uint8_t* dst = smem + kOffDense + (tt * BQ + row) * kDRow;
         uint64_t* full = &bars->dense_full[tt];
