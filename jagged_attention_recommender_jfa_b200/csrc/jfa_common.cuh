@@ -214,6 +214,31 @@ __device__ __forceinline__ float act_arg(int act, float x) {
 
 __device__ __forceinline__ float act_f(int act, float x) { return x * sigmoid_fast(act_arg(act, x)); }
 
+// The forward's GDPA weight act(s) * c from x = s log2(e) (scores kept in
+// log2 units), with one hardware tanh (relative error ~2^-11) instead of an
+// exponential and a reciprocal:
+//   SiLU(s)      = s/2 (1 + tanh(s / 2))
+//   GELU_tanh(s) = s/2 (1 + tanh(sqrt(2/pi) (s + 0.044715 s^3)))
+// half_c = c / (2 log2(e)), so that x * half_c = c s / 2.  x = -inf gives NaN:
+// callers select 0 for masked keys.
+__device__ __forceinline__ float tanh_hw(float z) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(z));
+    return t;
+}
+template <int ACT>
+__device__ __forceinline__ float gdpa_weight_log2(float x, float half_c) {
+    const float y = x * half_c;
+    float z;
+    if (ACT == JFA_ACT_SILU) {
+        z = x * (0.5f / 1.4426950408889634f);
+    } else {
+        const float s = x * (1.0f / 1.4426950408889634f);
+        z = 0.7978845608028654f * fmaf(0.044715f * s, s * s, s);
+    }
+    return fmaf(y, tanh_hw(z), y);
+}
+
 // Derivatives, from s = sigmoid(k(x)):
 //   SiLU'(x)      = s (1 + x (1 - s))
 //   GELU_tanh'(x) = 0.5 (1 + t) + 0.5 x (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 x^2)

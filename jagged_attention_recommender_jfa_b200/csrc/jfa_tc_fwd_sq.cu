@@ -378,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             }
             const int shift = w.nkv - w.nq;
             const float inv_n = w.nkv > 0 ? 1.0f / (float)w.nkv : 0.f;
+            const float half_c = inv_n * (0.5f / kLog2e);   // GDPA: act(s) / n_kv = x half_c (1 + tanh)
             const int jmax_vis = a.causal ? min(w.nkv - 1, i + shift) : w.nkv - 1;
             const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)w.h * 4 * a.bias4_stride : nullptr;
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
@@ -526,12 +527,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                                 if (v & 2) ps2 = add2(ps2, make_float2(x[v], x[v + 1]));
                                 else ps = add2(ps, make_float2(x[v], x[v + 1]));
                             }
+                        } else if (a.act == JFA_ACT_SILU) {
+#pragma unroll
+                            for (int v = 0; v < 16; ++v)
+                                x[v] = cc + v < nvis ? gdpa_weight_log2<JFA_ACT_SILU>(x[v], half_c) : 0.f;
                         } else {
 #pragma unroll
-                            for (int v = 0; v < 16; ++v) {
-                                const float s_nat = x[v] * (1.0f / kLog2e);
-                                x[v] = cc + v < nvis ? act_f(a.act, s_nat) * inv_n : 0.f;
-                            }
+                            for (int v = 0; v < 16; ++v)
+                                x[v] = cc + v < nvis ? gdpa_weight_log2<JFA_ACT_GELU_TANH>(x[v], half_c) : 0.f;
                         }
                         uint32_t pw[8];
 #pragma unroll
