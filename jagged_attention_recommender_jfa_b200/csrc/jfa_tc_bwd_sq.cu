@@ -21,8 +21,15 @@
 //   dK_j = dS^T Q,   dV_j = P^T dO                     (M 128 keys, N 128 d, K 64)
 //   dQ^T += K_j^T dS^T                                 (M 128 d, N 64 queries, K 128)
 // S^T / dP^T of tile j+1 are issued as soon as the score warps have read
-// those of tile j, so they run during tile j's score phase.
-// TMEM: S^T [0,64), dP^T [64,128), dK [128,256), dV [256,384), dQ^T [384,448).
+// those of tile j, so they run during tile j's score phase.  K and V tiles
+// stream through two-stage rings (a K stage is free once dQ^T of its tile has
+// run, a V stage once dP^T has).  dK and dV of a tile leave through a 32 KB
+// staging tile in turn: the score warps write their (key row, 32 d) pieces,
+// meet on an mbarrier, and each warp then stores eight whole 256-byte rows
+// (one row per half warp and instruction) instead of 16-byte pieces of 32
+// rows 1 KB apart, which the L2 takes as half-sector writes.
+// TMEM: S^T [0,64), dP^T [64,128), dK [128,256), dV [256,384), dQ^T [384,448),
+// P^T (bf16 pairs, the A operand of dV) [448,480).
 // Warps: 0 TMA, 1 MMA, 2..17 score: warp w reads TMEM lane quarter w % 4, and
 // the four consecutive warps 2 + 4g .. 5 + 4g take queries 16 g .. 16 g + 15;
 // 18, 19 stage a dense bias (one query row per lane: the 16-byte blocks that
@@ -40,6 +47,8 @@ using namespace sm100;
 bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads);
 bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_rows);
 
+JFA_TRACE_DEFINE(bwdsq)
+
 namespace {
 
 constexpr int BQ = 64, BN = 128, HD = 128;
@@ -50,11 +59,12 @@ constexpr uint32_t kQBox = 64 * 128;             // [64 rows][64 bf16]
 constexpr uint32_t kQTile = 2 * kQBox;           // 64 x 128 bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffDO = kOffQ + kQTile;
-constexpr uint32_t kOffK = kOffDO + kQTile;      // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kKTile;   // 2 stages
-constexpr uint32_t kOffPT = kOffV + 2 * kKTile;  // P^T  [128 keys][64 queries] bf16 (128-byte rows)
-constexpr uint32_t kOffDST = kOffPT + 128 * 128; // dS^T [128 keys][64 queries]
-constexpr uint32_t kOffRow = kOffDST + 128 * 128; // LSE (log2) [64], D [64]
+constexpr int kKStages = 2, kVStages = 2;
+constexpr uint32_t kOffK = kOffDO + kQTile;                // K ring
+constexpr uint32_t kOffV = kOffK + kKStages * kKTile;      // V ring
+constexpr uint32_t kOffDST = kOffV + kVStages * kKTile;    // dS^T [128 keys][64 queries] bf16 (128-byte rows)
+constexpr uint32_t kOffOut = kOffDST + 128 * 128;          // dK or dV staging [128 keys][256 bytes]
+constexpr uint32_t kOffRow = kOffOut + 128 * 256; // LSE (log2) [64], D [64]
 // dense bias rows of a key tile: 64 query rows x 272 bytes (the 16-byte
 // blocks that cover 128 bf16 at any 2-byte alignment)
 constexpr uint32_t kDRow = 272;
@@ -65,7 +75,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
     uint64_t q_full;
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t k_full[kKStages], k_empty[kKStages];
+    uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full;
     uint64_t sp_free;    // 16 score warps read S^T / dP^T
     uint64_t ds_full;    // 16 score warps wrote P^T / dS^T
@@ -73,6 +84,7 @@ struct Bars {
     uint64_t dkv_free;   // 16 score warps read dK / dV
     uint64_t rows_full;  // LSE / D staged (2 warps)
     uint64_t dense_full, dense_empty;   // dense bias rows staged (2 warps) / read (16)
+    uint64_t out_full, out_read;        // staging tile written / read back (16 score warps each)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -144,9 +156,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->sp_free, 16);
@@ -155,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
         mbar_init(&bars->dkv_free, 16);
         mbar_init(&bars->rows_full, 2);
         mbar_init(&bars->dense_full, 2);
+        mbar_init(&bars->out_full, 16);
+        mbar_init(&bars->out_read, 16);
         mbar_init(&bars->dense_empty, 16);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -183,27 +201,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             tma_load_3d(smem + kOffQ + kQBox, &P.tm_q, &bars->q_full, 64, h, q0);
             tma_load_3d(smem + kOffDO, &P.tm_do, &bars->q_full, 0, h, q0);
             tma_load_3d(smem + kOffDO + kQBox, &P.tm_do, &bars->q_full, 64, h, q0);
-            int issued = 0;
+            // V(j) once dP^T(j - 2) has run, K(j) once dQ^T(j - 3) has run (the
+            // order in which those complete)
+            int v_issued = 0, k_issued = 0;
             for (int j = 0; j < nt; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait(&bars->kv_empty[s], ((j >> 1) - 1) & 1, abort_flag, a.hdr)) break;
                 const int z = k0 + j * BN;
-                mbar_arrive_expect_tx(&bars->kv_full[s], 2 * kKTile);
-                tma_load_3d(smem + kOffK + s * kKTile, &P.tm_k, &bars->kv_full[s], 0, h, z);
-                tma_load_3d(smem + kOffK + s * kKTile + kKBox, &P.tm_k, &bars->kv_full[s], 64, h, z);
-                tma_load_3d(smem + kOffV + s * kKTile, &P.tm_v, &bars->kv_full[s], 0, h, z);
-                tma_load_3d(smem + kOffV + s * kKTile + kKBox, &P.tm_v, &bars->kv_full[s], 64, h, z);
-                if (j + 2 < nt) {
-                    tma_prefetch_l2_3d(&P.tm_k, 0, h, z + 2 * BN);
-                    tma_prefetch_l2_3d(&P.tm_k, 64, h, z + 2 * BN);
-                    tma_prefetch_l2_3d(&P.tm_v, 0, h, z + 2 * BN);
-                    tma_prefetch_l2_3d(&P.tm_v, 64, h, z + 2 * BN);
+                const int sv = j % kVStages, sk = j % kKStages;
+                if (j >= kVStages &&
+                    !mbar_wait(&bars->v_empty[sv], ((j / kVStages) - 1) & 1, abort_flag, a.hdr))
+                    break;
+                mbar_arrive_expect_tx(&bars->v_full[sv], kKTile);
+                tma_load_3d(smem + kOffV + sv * kKTile, &P.tm_v, &bars->v_full[sv], 0, h, z);
+                tma_load_3d(smem + kOffV + sv * kKTile + kKBox, &P.tm_v, &bars->v_full[sv], 64, h, z);
+                v_issued = j + 1;
+                if (j >= kKStages &&
+                    !mbar_wait(&bars->k_empty[sk], ((j / kKStages) - 1) & 1, abort_flag, a.hdr))
+                    break;
+                mbar_arrive_expect_tx(&bars->k_full[sk], kKTile);
+                tma_load_3d(smem + kOffK + sk * kKTile, &P.tm_k, &bars->k_full[sk], 0, h, z);
+                tma_load_3d(smem + kOffK + sk * kKTile + kKBox, &P.tm_k, &bars->k_full[sk], 64, h, z);
+                k_issued = j + 1;
+                if (j + 3 < nt) {   // warm L2 for the tiles loaded three steps on
+                    tma_prefetch_l2_3d(&P.tm_k, 0, h, z + 3 * BN);
+                    tma_prefetch_l2_3d(&P.tm_k, 64, h, z + 3 * BN);
+                    tma_prefetch_l2_3d(&P.tm_v, 0, h, z + 3 * BN);
+                    tma_prefetch_l2_3d(&P.tm_v, 64, h, z + 3 * BN);
                 }
-                issued = j + 1;
             }
             mbar_wait_drain(&bars->q_full, 0, a.hdr);
-            for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
-                mbar_wait_drain(&bars->kv_full[j & 1], (j >> 1) & 1, a.hdr);
+            for (int j = v_issued > kVStages ? v_issued - kVStages : 0; j < v_issued; ++j)
+                mbar_wait_drain(&bars->v_full[j % kVStages], (j / kVStages) & 1, a.hdr);
+            for (int j = k_issued > kKStages ? k_issued - kKStages : 0; j < k_issued; ++j)
+                mbar_wait_drain(&bars->k_full[j % kKStages], (j / kKStages) & 1, a.hdr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -214,16 +243,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             const uint32_t tS = tmem, tdP = tmem + 64, tdK = tmem + 128, tdV = tmem + 256, tdQ = tmem + 384;
             const uint32_t qK = sw128_desc_lo(sbase + kOffQ, 16u), doK = sw128_desc_lo(sbase + kOffDO, 16u);
             const uint32_t qM = sw128_desc_lo(sbase + kOffQ, kQBox), doM = sw128_desc_lo(sbase + kOffDO, kQBox);
-            const uint32_t ptK = sw128_desc_lo(sbase + kOffPT, 16u), dsK = sw128_desc_lo(sbase + kOffDST, 16u);
+            const uint32_t dsK = sw128_desc_lo(sbase + kOffDST, 16u);
+            const uint32_t tP = tmem + 448;   // P^T: queries 16k .. 16k + 15 at columns 8k .. 8k + 7
             const uint32_t dsM = sw128_desc_lo(sbase + kOffDST, 16u);
             bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.hdr);
             auto issue_sp = [&](int j) -> bool {   // S^T, dP^T of key tile j
-                const int s = j & 1;
-                if (!mbar_wait(&bars->kv_full[s], (j >> 1) & 1, abort_flag, a.hdr)) return false;
+                const int sk = j % kKStages, sv = j % kVStages;
+                if (!mbar_wait(&bars->k_full[sk], (j / kKStages) & 1, abort_flag, a.hdr)) return false;
+                if (!mbar_wait(&bars->v_full[sv], (j / kVStages) & 1, abort_flag, a.hdr)) return false;
                 if (j > 0 && !mbar_wait(&bars->sp_free, (j - 1) & 1, abort_flag, a.hdr)) return false;
+                JFA_TRACE_EV(bwdsq, 1, j, 0);
                 tc_fence_after();
-                const uint32_t kK = sw128_desc_lo(sbase + kOffK + s * kKTile, 16u);
-                const uint32_t vK = sw128_desc_lo(sbase + kOffV + s * kKTile, 16u);
+                const uint32_t kK = sw128_desc_lo(sbase + kOffK + sk * kKTile, 16u);
+                const uint32_t vK = sw128_desc_lo(sbase + kOffV + sv * kKTile, 16u);
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tS, kdesc(kK, k, kKBox), kdesc(qK, k, kQBox), id_s, k > 0 ? 1u : 0u);
@@ -231,14 +263,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                 for (int k = 0; k < HD / 16; ++k)
                     mma_bf16_ss(tdP, kdesc(vK, k, kKBox), kdesc(doK, k, kQBox), id_s, k > 0 ? 1u : 0u);
                 mma_commit(&bars->s_full);
+                mma_commit(&bars->v_empty[sv]);   // V(j) is read by dP^T(j) only
                 return true;
             };
             if (ok) ok = issue_sp(0);
             for (int j = 0; ok && j < nt; ++j) {
-                const int s = j & 1;
+                const int s = j % kKStages;
                 if (j + 1 < nt && !issue_sp(j + 1)) { ok = false; break; }
+                JFA_TRACE_EV(bwdsq, 1, j, 1);
                 if (!mbar_wait(&bars->ds_full, j & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwdsq, 1, j, 2);
                 if (j > 0 && !mbar_wait(&bars->dkv_free, (j - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                JFA_TRACE_EV(bwdsq, 1, j, 3);
                 tc_fence_after();
                 // dK = dS^T Q, dV = P^T dO: K = the 64 queries (4 steps)
 #pragma unroll
@@ -246,14 +282,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                     mma_bf16_ss(tdK, kdesc(dsK, k, 0), mdesc(qM, k), id_kv, k > 0 ? 1u : 0u);
 #pragma unroll
                 for (int k = 0; k < BQ / 16; ++k)
-                    mma_bf16_ss(tdV, kdesc(ptK, k, 0), mdesc(doM, k), id_kv, k > 0 ? 1u : 0u);
+                    mma_bf16_ts(tdV, tP + k * 8, mdesc(doM, k), id_kv, k > 0 ? 1u : 0u);
                 // dQ^T += K^T dS^T: A = K MN-major (d halves a box apart), K = 128 keys
                 const uint32_t kM = sw128_desc_lo(sbase + kOffK + s * kKTile, kKBox);
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tdQ, mdesc(kM, k), mdesc(dsM, k), id_q, (j > 0 || k > 0) ? 1u : 0u);
                 mma_commit(&bars->dkv_full);
-                mma_commit(&bars->kv_empty[s]);
+                mma_commit(&bars->k_empty[s]);
+                JFA_TRACE_EV(bwdsq, 1, j, 4);
             }
             mma_commit(&bars->drain);
             mbar_wait_drain(&bars->drain, 0, a.hdr);
@@ -304,11 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             zero_row(smem + kOffDO, r, 2, kQBox);
         }
         for (int j = 0; ok && j < nt; ++j) {
-            const int s = j & 1;
+            const int s = j % kKStages;
             const int jk = j * BN + r;          // key index within the sequence
             const bool jvalid = jk < nkv;
+            const bool tr = warp == 2 && lane == 0;
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 0);
             if (!wwait(&bars->s_full, j & 1)) { ok = false; break; }
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 1);
             if (BIAS == 2 && !wwait(&bars->dense_full, j & 1)) { ok = false; break; }
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 2);
             tc_fence_after();
             uint32_t u[16], g[16];
             tmem_ld16(tS, u);
@@ -390,16 +431,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->dense_empty);
             }
-            // P^T and dS^T to shared memory; the MMAs of the previous tile that
-            // read them have completed (this warp saw their commit below)
-            store16_bf16(smem + kOffPT, r, grp, u);
+            // P^T to TMEM and dS^T to shared memory; the MMAs of the previous tile
+            // that read them have completed (this warp saw their commit below)
+            {   // P^T (bf16 pairs): queries qc0 .. qc0 + 15 at columns 448 + 8 grp ..
+                uint32_t pw[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) pw[t] = pack_bf16(__uint_as_float(u[2 * t]), __uint_as_float(u[2 * t + 1]));
+                tmem_st8(tmem + lane_addr + 448 + grp * 8, pw);
+            }
             store16_bf16(smem + kOffDST, r, grp, g);
             fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->ds_full);
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 3);
             // dK and dV of this key tile are complete: write them out
             if (!wwait(&bars->dkv_full, j & 1)) { ok = false; break; }
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 4);
             tc_fence_after();
             uint32_t uk[32], uv[32];
             tmem_ld32(tdK, uk);
@@ -408,24 +457,45 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dkv_free);
-            if (jvalid) {
-                __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + ((int64_t)(k0 + jk) * a.H + h) * HD + grp * 32;
-                __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(a.dv) + ((int64_t)(k0 + jk) * a.H + h) * HD + grp * 32;
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 5);
+            // dK (scaled) then dV through the staging tile: row r, 16-byte chunk c
+            // of its 256 bytes at chunk c ^ (r % 16) (a warp's 32 rows then fall
+            // on distinct banks in each quarter warp)
+            uint8_t* stg = smem + kOffOut;
+            const int sw_rows = (warp - 2) * 8;   // rows this warp stores
 #pragma unroll
-                for (int t = 0; t < 32; t += 8) {
-                    uint4 wk, wv;
-                    wk.x = pack_bf16(__uint_as_float(uk[t + 0]) * a.scale, __uint_as_float(uk[t + 1]) * a.scale);
-                    wk.y = pack_bf16(__uint_as_float(uk[t + 2]) * a.scale, __uint_as_float(uk[t + 3]) * a.scale);
-                    wk.z = pack_bf16(__uint_as_float(uk[t + 4]) * a.scale, __uint_as_float(uk[t + 5]) * a.scale);
-                    wk.w = pack_bf16(__uint_as_float(uk[t + 6]) * a.scale, __uint_as_float(uk[t + 7]) * a.scale);
-                    wv.x = pack_bf16(__uint_as_float(uv[t + 0]), __uint_as_float(uv[t + 1]));
-                    wv.y = pack_bf16(__uint_as_float(uv[t + 2]), __uint_as_float(uv[t + 3]));
-                    wv.z = pack_bf16(__uint_as_float(uv[t + 4]), __uint_as_float(uv[t + 5]));
-                    wv.w = pack_bf16(__uint_as_float(uv[t + 6]), __uint_as_float(uv[t + 7]));
-                    *reinterpret_cast<uint4*>(dkrow + t) = wk;
-                    *reinterpret_cast<uint4*>(dvrow + t) = wv;
+            for (int tsr = 0; tsr < 2; ++tsr) {
+                const int use = 2 * j + tsr;
+                if (use > 0 && !wwait(&bars->out_read, (use - 1) & 1)) { ok = false; break; }
+                const uint32_t (&vals)[32] = tsr ? uv : uk;
+                const float mul = tsr ? 1.0f : a.scale;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w4;
+                    w4.x = pack_bf16(__uint_as_float(vals[8 * q + 0]) * mul, __uint_as_float(vals[8 * q + 1]) * mul);
+                    w4.y = pack_bf16(__uint_as_float(vals[8 * q + 2]) * mul, __uint_as_float(vals[8 * q + 3]) * mul);
+                    w4.z = pack_bf16(__uint_as_float(vals[8 * q + 4]) * mul, __uint_as_float(vals[8 * q + 5]) * mul);
+                    w4.w = pack_bf16(__uint_as_float(vals[8 * q + 6]) * mul, __uint_as_float(vals[8 * q + 7]) * mul);
+                    const int c = 4 * grp + q;
+                    *reinterpret_cast<uint4*>(stg + r * 256 + ((c ^ (r & 15)) << 4)) = w4;
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->out_full);
+                if (!wwait(&bars->out_full, use & 1)) { ok = false; break; }
+                __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(tsr ? a.dv : a.dk);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int row = sw_rows + 2 * i + (lane >> 4), c = lane & 15;
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(stg + row * 256 + ((c ^ (row & 15)) << 4));
+                    const int key = j * BN + row;
+                    if (key < nkv)
+                        *reinterpret_cast<uint4*>(base + ((int64_t)(k0 + key) * a.H + h) * HD + c * 8) = w4;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->out_read);
             }
+            if (!ok) break;
+            if (tr) JFA_TRACE_EV(bwdsq, 2, j, 6);
         }
         // dQ = scale * (dQ^T)^T: d row r, queries qc0 .. +15; every dQ^T MMA
         // retired with the last dkv_full
