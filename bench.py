@@ -198,7 +198,8 @@ class ClockSampler:
 
 
 def kernel_source_hash(name):
-    src = {"tc_fwd": "jfa_tc_fwd.cu", "tc_bwd": "jfa_tc_bwd.cu", "simt_fwd": "jfa_simt.cu",
+    src = {"tc_fwd": "jfa_tc_fwd.cu", "tc_bwd": "jfa_tc_bwd.cu", "tc_fwd_sq": "jfa_tc_fwd_sq.cu",
+           "tc_bwd_sq": "jfa_tc_bwd_sq.cu", "tc_fwd_mxfp8": "jfa_tc_fwd_mx.cu", "simt_fwd": "jfa_simt.cu",
            "simt_bwd_dq": "jfa_simt.cu", "simt_bwd_dkdv": "jfa_simt.cu"}.get(name)
     if src is None:
         return None

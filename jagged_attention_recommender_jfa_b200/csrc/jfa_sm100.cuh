@@ -388,5 +388,23 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 16 fp32 (bits) v[0..15] times m, as 16 bf16 (32 bytes) at p.  Rows of an
+// output are written one piece per thread, consecutive threads on different
+// rows: with a 32-byte aligned p (aligned32) the piece is one 256-bit store,
+// a whole L2 sector; otherwise two 16-byte stores, two half sectors.
+__device__ __forceinline__ void store_bf16x16(void* p, const uint32_t* v, float m, bool aligned32) {
+    uint32_t w[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) w[t] = pack_bf16(__uint_as_float(v[2 * t]) * m, __uint_as_float(v[2 * t + 1]) * m);
+    if (aligned32) {
+        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                     "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    } else {
+        reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
 }  // namespace sm100
 }  // namespace jfa

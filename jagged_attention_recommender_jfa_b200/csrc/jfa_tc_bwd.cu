@@ -667,19 +667,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 for (int t = 0; t < 32; ++t) uk[t] = 0u, uv[t] = 0u;
             }
             if (jvalid) {
+                const bool kv32 = ((reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) & 31) == 0;
 #pragma unroll
-                for (int t = 0; t < 32; t += 8) {
-                    uint4 wk, wv;
-                    wk.x = pack_bf16(__uint_as_float(uk[t + 0]) * a.scale, __uint_as_float(uk[t + 1]) * a.scale);
-                    wk.y = pack_bf16(__uint_as_float(uk[t + 2]) * a.scale, __uint_as_float(uk[t + 3]) * a.scale);
-                    wk.z = pack_bf16(__uint_as_float(uk[t + 4]) * a.scale, __uint_as_float(uk[t + 5]) * a.scale);
-                    wk.w = pack_bf16(__uint_as_float(uk[t + 6]) * a.scale, __uint_as_float(uk[t + 7]) * a.scale);
-                    wv.x = pack_bf16(__uint_as_float(uv[t + 0]), __uint_as_float(uv[t + 1]));
-                    wv.y = pack_bf16(__uint_as_float(uv[t + 2]), __uint_as_float(uv[t + 3]));
-                    wv.z = pack_bf16(__uint_as_float(uv[t + 4]), __uint_as_float(uv[t + 5]));
-                    wv.w = pack_bf16(__uint_as_float(uv[t + 6]), __uint_as_float(uv[t + 7]));
-                    *reinterpret_cast<uint4*>(dkrow + t) = wk;
-                    *reinterpret_cast<uint4*>(dvrow + t) = wv;
+                for (int t = 0; t < 32; t += 16) {
+                    store_bf16x16(dkrow + t, uk + t, a.scale, kv32);
+                    store_bf16x16(dvrow + t, uv + t, 1.0f, kv32);
                 }
             }
         }

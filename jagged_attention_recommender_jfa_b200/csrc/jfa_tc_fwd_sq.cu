@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
     const int n_items = *a.item_count;
     const int n_pairs = (n_items + 1) >> 1;
     if (a.hdr->err != 0 || (int)blockIdx.x >= n_pairs) return;
+    const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t* smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
@@ -584,14 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 tmem_wait_ld();
                 if (i < w.nq) {
 #pragma unroll
-                    for (int t = 0; t < 32; t += 8) {
-                        uint4 wv;
-                        wv.x = pack_bf16(__uint_as_float(u[t + 0]) * inv, __uint_as_float(u[t + 1]) * inv);
-                        wv.y = pack_bf16(__uint_as_float(u[t + 2]) * inv, __uint_as_float(u[t + 3]) * inv);
-                        wv.z = pack_bf16(__uint_as_float(u[t + 4]) * inv, __uint_as_float(u[t + 5]) * inv);
-                        wv.w = pack_bf16(__uint_as_float(u[t + 6]) * inv, __uint_as_float(u[t + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + c * 32 + t) = wv;
-                    }
+                    for (int t = 0; t < 32; t += 16) store_bf16x16(orow + c * 32 + t, u + t, inv, out32);
                 }
             }
             tc_fence_before();
