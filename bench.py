@@ -147,6 +147,67 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML (read-only queries)
+    every 5 ms on a host thread, so that a timed region of a few tens of
+    milliseconds still gets samples."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device_index):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self.stop_evt.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                mask = get_reasons(self.handle) if get_reasons else 0
+                self.samples.append((sm, mask))
+            except Exception:
+                pass
+            self.stop_evt.wait(0.005)
+
+    def start(self):
+        self.thread.start()
+
+    def stop(self):
+        self.stop_evt.set()
+        self.thread.join(timeout=2)
+        nv = self.nv
+        try:
+            smax = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        except Exception:
+            smax = None
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"], "source": "nvml"}
+        reasons = sorted({name for _, m in self.samples for name, attr in self.REASONS
+                          if hasattr(nv, attr) and (m & getattr(nv, attr))})
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
+
+
+def clock_sampler(device_index):
+    """NVML sampler when the binding is there, else nvidia-smi."""
+    try:
+        return NvmlClockSampler(device_index)
+    except Exception:
+        return ClockSampler(device_index)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons (every 200 ms)."""
 
@@ -418,9 +479,10 @@ def main():
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(local)
+    clocks = clock_sampler(local)
     clocks.start()
-    time.sleep(0.3)
+    if isinstance(clocks, ClockSampler):
+        time.sleep(0.3)   # nvidia-smi needs a moment before its first sample
     marks = [[ev(), ev(), ev()] for _ in range(args.steps)]
     t_start, t_end = ev(), ev()
     if world > 1:
