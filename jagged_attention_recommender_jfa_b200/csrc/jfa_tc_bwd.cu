@@ -22,9 +22,10 @@
 //                             accumulator with coalesced reductions (a warp
 //                             covers 32 consecutive d of one query row)
 //                    dK and dV run over the tile's two query halves, the
-//                    first while the score warps form the second; then dQ^T
-//                    of tile t and S^T, dP^T of tile t+1 follow back to back:
-//                    dQ^T(t) is read out while S^T(t+1) runs, and Q / dO
+//                    first while the score warps form the second; once the
+//                    whole dS^T is formed, dQ^T of tile t goes ahead of the
+//                    second halves, then S^T, dP^T of tile t+1 follow:
+//                    dQ^T(t) is read out while those run, and Q / dO
 //                    come from a three-buffer ring that fetches Q(t+1) two
 //                    tiles ahead and dO(t+1) once dK(t) has retired (both
 //                    warmed in L2 a tile earlier).
@@ -332,15 +333,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, a.hdr)) { ok = false; break; }
                 JFA_TRACE_EV(bwd, 1, t, 0);
                 tc_fence_after();
-                issue_dk(t, 4);
-                mma_commit(&bars->buf_empty[(2 * t) % 3]);
-                issue_dv(t, 4);
-                mma_commit(&bars->buf_empty[(2 * t + 1) % 3]);
-                // dQ^T = K^T dS^T over the dP^T columns (A = K, B = dS^T, both MN-major)
+                // dQ^T = K^T dS^T over the dP^T columns (A = K, B = dS^T, both
+                // MN-major), ahead of the second halves of dK and dV, so that its
+                // read-out and reductions start while those run
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
                     mma_bf16_ss(tdP, mnmajor_desc(kM, k), mnmajor_desc(dsM, k), idesc_tn, k > 0 ? 1u : 0u);
                 mma_commit(&bars->dq_full);
+                issue_dk(t, 4);
+                mma_commit(&bars->buf_empty[(2 * t) % 3]);
+                issue_dv(t, 4);
+                mma_commit(&bars->buf_empty[(2 * t + 1) % 3]);
                 JFA_TRACE_EV(bwd, 1, t, 1);
                 if (t + 1 < nt) {
                     // S^T(t+1) overwrites P^T(t): issued after dV, which reads it
