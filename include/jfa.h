@@ -177,7 +177,12 @@ jfa_status jfa_backward_dbias(const jfa_problem* problem, const void* q, const v
                               jfa_stream_t stream);
 
 /* MX (OCP v1.0) quantisation of a bf16 tensor x [rows][heads][d] to E4M3
- * codes [rows][heads][d] (same layout, one byte each) and E8M0 scales.
+ * codes [rows][heads][d] (same layout, one byte each) and E8M0 scales: the
+ * MXFP8 attention operands ("GEM Training: How Meta Doubled the Efficiency of
+ * Its LLM-Scale Ads Foundation Model", opening summary: MXFP8 attention;
+ * "Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a Different
+ * Stack", "Bottleneck move 2": block-scaled low precision with the scales
+ * generated on the device).
  * Shared exponent X = floor(log2(amax of the block)) - 8, clamped to
  * [-127, 127] (-127 for an all-zero block); codes = RNE(x * 2^-X) saturated
  * to +-448; scale byte = X + 127.
@@ -216,7 +221,11 @@ jfa_status jfa_norm_quantize_mxfp8(const void* x, int64_t rows, int32_t D, const
                                    uint8_t* scales, jfa_stream_t stream);
 
 /* The longest-first tile schedule that jfa_forward (backward = 0: items are
- * query tiles) or jfa_backward (backward = 1: items are key/value tiles) runs,
+ * query tiles) or jfa_backward (backward = 1: items are key/value tiles) runs
+ * over the jagged batch, so that short and long samples balance across SMs
+ * ("GEM Training: How Meta Doubled the Efficiency of Its LLM-Scale Ads
+ * Foundation Model", "Challenge 1: Achieving High Per-GPU Utilization": work
+ * per sample varies with its sequence length),
  * written to items (device int32 [capacity][4] = {sequence, head, tile,
  * cost}) and its length to *count (device int32).  cost = number of (query,
  * key) pairs the tile computes; order = cost descending, then sequence, tile,

@@ -43,6 +43,8 @@ using namespace sm100;
 bool make_tmap_rows_heads_d(CUtensorMap* map, const void* base, int64_t rows, int heads);
 bool make_tmap_rows_heads_d_box(CUtensorMap* map, const void* base, int64_t rows, int heads, int box_rows);
 
+JFA_TRACE_DEFINE(fwdsq)
+
 namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128, BQ = 64;
@@ -292,7 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 Item w[2] = {load_item(a, 2 * pr, n_items), load_item(a, 2 * pr + 1, n_items)};
                 // S_T = Q_T K_T(j)^T; K is released after it, Q after the item's last
                 auto issue_qk = [&](int t, int j) -> bool {
+                    JFA_TRACE_EV(fwdsq, 1, kc[t], 2 * t);
                     if (!mbar_wait(&bars->k_full[t], kc[t] & 1, abort_flag, a.hdr)) return false;
+                    JFA_TRACE_EV(fwdsq, 1, kc[t], 2 * t + 1);
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < HD / 16; ++k)
@@ -315,7 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                         if (!mbar_wait(&bars->p_full[t], gt[t] & 1, abort_flag, a.hdr)) { ok = false; break; }
                         if (j == 0 && mt[t] > 0 &&
                             !mbar_wait(&bars->o_free[t], (mt[t] - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
+                        JFA_TRACE_EV(fwdsq, 1, kc[t], 4 + 2 * t);
                         if (!mbar_wait(&bars->v_full[t], kc[t] & 1, abort_flag, a.hdr)) { ok = false; break; }
+                        JFA_TRACE_EV(fwdsq, 1, kc[t], 5 + 2 * t);
                         tc_fence_after();
                         const uint32_t tP = tmem + t * 128, tO = tmem + 256 + t * 128;
 #pragma unroll
@@ -392,12 +398,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
             const uint8_t* drow = smem + kOffDense + (tt * BQ + r_) * kDRow;
             const int e0 = (int)((reinterpret_cast<uintptr_t>(dense + dense_row) & 15) >> 1);
             float m_used = -CUDART_INF_F, l = 0.f;
+            const bool tr = lane == 0 && (warp == 0 || warp == 2);
             for (int j = 0; j < n; ++j, ++gt) {
+                if (tr) JFA_TRACE_EV(fwdsq, 2 + tt, gt, 0);
                 if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
+                if (tr) JFA_TRACE_EV(fwdsq, 2 + tt, gt, 1);
                 tc_fence_after();
                 const int jc = j * BN;
                 if (BIAS == 1 && !wwait(&bars->bias_full[tt], gt & 1)) { ok = false; break; }
                 if (BIAS == 2 && !wwait(&bars->dense_full[tt], gt & 1)) { ok = false; break; }
+                if (tr) JFA_TRACE_EV(fwdsq, 2 + tt, gt, 2);
                 const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;
                 const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW);
                 const int lo = i - jc - (BN - 1) + C;
@@ -472,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->dense_empty[tt]);
                 }
+                if (tr) JFA_TRACE_EV(fwdsq, 2 + tt, gt, 3);
                 float ref = 0.f;
                 if (softmax) {
                     float* rp = red + ((gt & 1) * 4 + tt * 2) * 64;
@@ -562,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_sq_kernel(const __grid_con
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
+                if (tr) JFA_TRACE_EV(fwdsq, 2 + tt, gt, 4);
                 if (lane == 0) mbar_arrive(&bars->p_full[tt]);
             }
             if (!ok) break;
