@@ -24,10 +24,11 @@
 // those of tile j, so they run during tile j's score phase.  K and V tiles
 // stream through two-stage rings (a K stage is free once dQ^T of its tile has
 // run, a V stage once dP^T has).  dK and dV of a tile leave through a 32 KB
-// staging tile in turn: the score warps write their (key row, 32 d) pieces,
-// meet on an mbarrier, and each warp then stores eight whole 256-byte rows
-// (one row per half warp and instruction) instead of 16-byte pieces of 32
-// rows 1 KB apart, which the L2 takes as half-sector writes.
+// staging tile in turn: the four score warps of a lane quarter write their
+// (key row, 32 d) pieces of its 32 rows, meet on the quarter's mbarrier, and
+// each warp then stores eight whole 256-byte rows (one row per half warp and
+// instruction) instead of 16-byte pieces of 32 rows 1 KB apart, which the L2
+// takes as half-sector writes.
 // TMEM: S^T [0,64), dP^T [64,128), dK [128,256), dV [256,384), dQ^T [384,448),
 // P^T (bf16 pairs, the A operand of dV) [448,480).
 // Warps: 0 TMA, 1 MMA, 2..17 score: warp w reads TMEM lane quarter w % 4, and
@@ -84,7 +85,7 @@ struct Bars {
     uint64_t dkv_free;   // 16 score warps read dK / dV
     uint64_t rows_full;  // LSE / D staged (2 warps)
     uint64_t dense_full, dense_empty;   // dense bias rows staged (2 warps) / read (16)
-    uint64_t out_full, out_read;        // staging tile written / read back (16 score warps each)
+    uint64_t out_full[4], out_read[4];  // per lane quarter: its staging rows written / read back (4 warps)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -171,8 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
         mbar_init(&bars->dkv_free, 16);
         mbar_init(&bars->rows_full, 2);
         mbar_init(&bars->dense_full, 2);
-        mbar_init(&bars->out_full, 16);
-        mbar_init(&bars->out_read, 16);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&bars->out_full[q], 4);
+            mbar_init(&bars->out_read[q], 4);
+        }
         mbar_init(&bars->dense_empty, 16);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
@@ -458,15 +461,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dkv_free);
             if (tr) JFA_TRACE_EV(bwdsq, 2, j, 5);
-            // dK (scaled) then dV through the staging tile: row r, 16-byte chunk c
-            // of its 256 bytes at chunk c ^ (r % 16) (a warp's 32 rows then fall
-            // on distinct banks in each quarter warp)
-            uint8_t* stg = smem + kOffOut;
-            const int sw_rows = (warp - 2) * 8;   // rows this warp stores
+            // dK (scaled) then dV through the staging tile, one 8 KB part per lane
+            // quarter: the four warps of a quarter hold its 32 key rows (32 d each)
+            // and meet on their own barrier.  Local row lr, 16-byte chunk c of its
+            // 256 bytes at chunk c ^ (lr % 16) (a warp's rows then fall on
+            // distinct banks in each quarter warp); warp grp stores rows
+            // 8 grp .. 8 grp + 7 of the part.
+            uint8_t* stg = smem + kOffOut + wq * (32 * 256);
+            const int lr = lane;
 #pragma unroll
             for (int tsr = 0; tsr < 2; ++tsr) {
                 const int use = 2 * j + tsr;
-                if (use > 0 && !wwait(&bars->out_read, (use - 1) & 1)) { ok = false; break; }
+                if (use > 0 && !wwait(&bars->out_read[wq], (use - 1) & 1)) { ok = false; break; }
                 const uint32_t (&vals)[32] = tsr ? uv : uk;
                 const float mul = tsr ? 1.0f : a.scale;
 #pragma unroll
@@ -477,22 +483,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_sq_kernel(const __grid_con
                     w4.z = pack_bf16(__uint_as_float(vals[8 * q + 4]) * mul, __uint_as_float(vals[8 * q + 5]) * mul);
                     w4.w = pack_bf16(__uint_as_float(vals[8 * q + 6]) * mul, __uint_as_float(vals[8 * q + 7]) * mul);
                     const int c = 4 * grp + q;
-                    *reinterpret_cast<uint4*>(stg + r * 256 + ((c ^ (r & 15)) << 4)) = w4;
+                    *reinterpret_cast<uint4*>(stg + lr * 256 + ((c ^ (lr & 15)) << 4)) = w4;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->out_full);
-                if (!wwait(&bars->out_full, use & 1)) { ok = false; break; }
+                if (lane == 0) mbar_arrive(&bars->out_full[wq]);
+                if (!wwait(&bars->out_full[wq], use & 1)) { ok = false; break; }
                 __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(tsr ? a.dv : a.dk);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int row = sw_rows + 2 * i + (lane >> 4), c = lane & 15;
+                    const int row = 8 * grp + 2 * i + (lane >> 4), c = lane & 15;   // local row
                     const uint4 w4 = *reinterpret_cast<const uint4*>(stg + row * 256 + ((c ^ (row & 15)) << 4));
-                    const int key = j * BN + row;
+                    const int key = j * BN + wq * 32 + row;
                     if (key < nkv)
                         *reinterpret_cast<uint4*>(base + ((int64_t)(k0 + key) * a.H + h) * HD + c * 8) = w4;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->out_read);
+                if (lane == 0) mbar_arrive(&bars->out_read[wq]);
             }
             if (!ok) break;
             if (tr) JFA_TRACE_EV(bwdsq, 2, j, 6);
