@@ -15,7 +15,7 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
                            int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream,
-                           int wait_limit_us = 0);
+                           int wait_limit_us = 0, int cost_tiles = 0);
 cudaError_t simt_forward(const AttnArgs& a, int head_dim, bool bf16, int grid, cudaStream_t st);
 cudaError_t simt_backward(const AttnArgs& a, const AttnArgs& kv_args, int head_dim, bool bf16,
                           int grid_q, int grid_kv, int64_t rows, cudaStream_t st);
@@ -215,7 +215,8 @@ jfa_status forward_impl(const jfa_problem* problem, const void* q, const void* k
                                    reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
                                    reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
                                    &hdr->pair_count, 1, nullptr, nullptr, st,
-                                   inject ? kTestWaitLimitUs : 0);
+                                   inject ? kTestWaitLimitUs : 0,
+                                   (tc && p.dtype != JFA_MXFP8 && tc_backward_short_q(p)) ? 1 : 0);
     if (e != cudaSuccess) return cuda_fail(e, "schedule");
     AttnArgs a{};
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
@@ -321,7 +322,7 @@ jfa_status backward_impl(const jfa_problem* problem, const void* q, const void* 
                            reinterpret_cast<int2*>(ws + L.pair_bt),
                            reinterpret_cast<int64_t*>(ws + L.pair_cost), L.pairs_max_q,
                            reinterpret_cast<int4*>(ws + L.items), &hdr->item_count,
-                           &hdr->pair_count, 1, nullptr, nullptr, st);
+                           &hdr->pair_count, 1, nullptr, nullptr, st, 0, sq ? 1 : 0);
         if (e != cudaSuccess) return cuda_fail(e, "schedule");
     }
     if (!sq) {

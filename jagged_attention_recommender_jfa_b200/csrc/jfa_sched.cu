@@ -11,6 +11,12 @@
 // takes items in order runs the long causal tiles first and fills the tail
 // with short ones.
 //
+// Short query sequences (every n_q <= 64, one item per (sequence, head)):
+// the kernels stream the item's key/value tiles, each costing the same HBM
+// bytes whatever n_q is, so these items are ranked by their 128-key tiles
+// first (pairs only break ties): ranking them by pairs alone spreads the key
+// tiles unevenly over the CTAs.
+//
 // Key-tile schedule (backward): the items of one (sequence, head) are kept
 // together, so that the key tiles that read the same query / dO tiles and add
 // into the same dQ rows run at the same time and share them through L2.
@@ -62,7 +68,7 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
               int max_q, int max_kv, int64_t total_q, int64_t total_kv, int causal, int backward,
               int tile, int64_t pairs_cap, int want_dense, WsHeader* hdr, int64_t* dense_off,
               int2* pair_bt, int64_t* pair_cost, int32_t* pair_count_out, int reset_err,
-              int64_t* seq_tmp, int64_t* seq_start, int wait_limit_us) {
+              int64_t* seq_tmp, int64_t* seq_start, int wait_limit_us, int cost_tiles) {
     __shared__ int s_bad;
     __shared__ int64_t s_scan[kPrepThreads];
     __shared__ int64_t s_dscan[kPrepThreads];
@@ -142,8 +148,14 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
         int nq = q_off[bt.x + 1] - q_off[bt.x], nkv = kv_off[bt.x + 1] - kv_off[bt.x];
         int rows = backward ? nkv : nq;
         int lo = bt.y * tile, hi = min(rows, lo + tile);
-        pair_cost[p] = backward ? key_tile_cost(lo, hi, nq, nkv, causal)
-                                : query_tile_cost(lo, hi, nq, nkv, causal);
+        int64_t c = backward ? key_tile_cost(lo, hi, nq, nkv, causal) : query_tile_cost(lo, hi, nq, nkv, causal);
+        if (cost_tiles) {
+            // 128-key tiles of the item's visible key range, then its pairs
+            int kv_end = causal ? min(nkv, hi + (nkv - nq)) : nkv;
+            kv_end = kv_end < 0 ? 0 : kv_end;
+            c = ((int64_t)((kv_end + 127) / 128) << 32) | (c < 0xffffffffll ? c : 0xffffffffll);
+        }
+        pair_cost[p] = c;
     }
     if (seq_start == nullptr) return;
     // 4. sequence order of the grouped (key-tile) schedule: seq_start[b] =
@@ -242,13 +254,13 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
                            int2* pair_bt, int64_t* pair_cost, int64_t pairs_cap, int4* items,
                            int32_t* item_count, int32_t* pair_count, int reset_err,
                            int64_t* seq_tmp, int64_t* seq_start, cudaStream_t stream,
-                           int wait_limit_us) {
+                           int wait_limit_us, int cost_tiles) {
     int want_dense = (pb.bias_kind == JFA_BIAS_DENSE_JAGGED && dense_off != nullptr) ? 1 : 0;
     prof_begin(stream);
     sched_prepare<<<1, kPrepThreads, 0, stream>>>(
         q_off, kv_off, pb.batch, pb.heads, pb.max_q_len, pb.max_kv_len, pb.total_q, pb.total_kv,
         causal, backward, tile, pairs_cap, want_dense, hdr, dense_off, pair_bt, pair_cost,
-        pair_count, reset_err, seq_tmp, seq_start, wait_limit_us);
+        pair_count, reset_err, seq_tmp, seq_start, wait_limit_us, cost_tiles);
     prof_end(stream, K_SCHED_PREPARE);
     int64_t bound = pairs_bound(pb.batch, backward ? pb.max_kv_len : pb.max_q_len,
                                 backward ? pb.total_kv : pb.total_q, tile);
