@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["jfa", "reference"], default="jfa")
     ap.add_argument("--workload", default="self_bf16")
     ap.add_argument("--act", default=None, help="override the workload's activation")
+    ap.add_argument("--bias", default=None, choices=["none", "relpos", "dense"],
+                    help="override the workload's bias kind (a what-if: the metric's workload keeps its own)")
     ap.add_argument("--seed", type=int, default=1)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's number of sequences (profiling captures)")
@@ -339,7 +341,7 @@ def reference_arm(args, rank, world):
         return
     from jagged_attention_recommender_jfa_b200.inputs import make_problem
     import oracle
-    p = make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len)
+    p = make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len, bias=args.bias)
     act = args.act or p.act
     target = args.cpu_sample_pairs / 4
     mask, pairs = cpu_sample_mask(p, target, args.block)
@@ -639,7 +641,7 @@ def rank_problem(args, rank, world, jfa):
     of its own sequences only (seed args.seed + 1 + rank)."""
     from jagged_attention_recommender_jfa_b200.inputs import WORKLOADS, draw_lengths, make_problem
     if world == 1:
-        return make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len), None
+        return make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len, bias=args.bias), None
     B = args.batch or WORKLOADS[args.workload]["B"]
     q_lens, kv_lens = draw_lengths(args.workload, args.seed, B=B * world, max_len=args.max_len)
     causal = WORKLOADS[args.workload]["causal"]
@@ -647,7 +649,7 @@ def rank_problem(args, rank, world, jfa):
                                    args.sub_batch, jfa)
     mine = np.nonzero(rank_of == rank)[0]
     p = make_problem(args.workload, args.seed + 1 + rank, q_lens=q_lens[mine],
-                     kv_lens=kv_lens[mine], max_len=args.max_len)
+                     kv_lens=kv_lens[mine], max_len=args.max_len, bias=args.bias)
     return p, report
 
 
