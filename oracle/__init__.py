@@ -57,9 +57,9 @@ def _lib():
             P = ctypes.c_void_p
             i32, f64 = ctypes.c_int, ctypes.c_double
             lib.jfa_oracle_forward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                               i32, f64, i32, i32, P, P, P, i32]
+                                               i32, f64, i32, i32, i32, P, P, P, i32]
             lib.jfa_oracle_backward.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P, i32, i32,
-                                                i32, f64, i32, P, P, P, P, P, P, P, i32]
+                                                i32, f64, i32, i32, P, P, P, P, P, P, P, i32]
             lib.jfa_oracle_quantize_mx.argtypes = [P, ctypes.c_int64, P, P]
             lib.jfa_oracle_dequantize_mx.argtypes = [P, P, ctypes.c_int64, P]
             lib.jfa_oracle_e4m3_encode.argtypes = [f64]
@@ -113,14 +113,16 @@ def _item_mask(seq_mask, B, H):
 
 def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0,
             act="softmax", causal=False, scale=0.0, quant_p=False, seq_mask=None,
-            block=0, nthreads=0):
+            block=0, window=0, nthreads=0):
     """fp64 forward.  Returns (out [total_q,H,d], lse [total_q,H] or None).
 
     ``seq_mask`` ([B] per sequence or [B*H] per (sequence, head)) selects what
     is computed; everything else is NaN in the result.  ``block`` > 0:
     BlockAttention, each query sees only the keys of its own block of
     ``block`` consecutive positions (GDPA then divides by the block's key
-    count)."""
+    count).  ``window`` > 0: sliding window, query i (aligned position
+    p = i + n_kv - n_q) sees key j only when p - j < window, and without the
+    causal rule also when j - p < window (GDPA still divides by n_kv)."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     q64, k64, v64 = _f64(q), _f64(k), _f64(v)
     B = len(q_off) - 1
@@ -132,13 +134,14 @@ def forward(q_off, kv_off, q, k, v, *, bias=None, bias_kind="none", relpos_len=0
     _lib().jfa_oracle_forward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                               _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                               ACT[act], int(bool(causal)), float(scale), int(bool(quant_p)),
-                              int(block), _ptr(mask), _ptr(out), _ptr(lse), int(nthreads))
+                              int(block), int(window), _ptr(mask), _ptr(out), _ptr(lse),
+                              int(nthreads))
     return out, (lse if act == "softmax" else None)
 
 
 def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpos_len=0,
              act="softmax", causal=False, scale=0.0, seq_mask=None, out_for_d=None,
-             dbias=False, block=0, nthreads=0):
+             dbias=False, block=0, window=0, nthreads=0):
     """fp64 analytic gradients (dq, dk, dv), and with ``dbias`` also the bias
     gradient as a fourth result: for a dense bias an array like ``bias``
     (ds of each valid pair, 0 at masked pairs, NaN in items not computed),
@@ -166,7 +169,7 @@ def backward(q_off, kv_off, q, k, v, dout, *, bias=None, bias_kind="none", relpo
     _lib().jfa_oracle_backward(B, H, d, _ptr(q_off), _ptr(kv_off), _ptr(q64), _ptr(k64),
                                _ptr(v64), BIAS[bias_kind], _ptr(b64), int(relpos_len),
                                ACT[act], int(bool(causal)), float(scale), int(block),
-                               _ptr(mask), _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv),
+                               int(window), _ptr(mask), _ptr(do64), _ptr(o64), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(db), int(nthreads))
     if dbias:
         return dq, dk, dv, db
@@ -285,19 +288,21 @@ def dequantize_along_rows(codes, scales, offsets):
 # descending, ties by b -- with the key tiles of a group in ascending order.
 # ---------------------------------------------------------------------------
 
-def _visible_keys(i, nq, nkv, causal):
-    if not causal:
-        return nkv
-    return max(0, min(nkv, i + 1 + nkv - nq))
+def _visible_keys(i, nq, nkv, causal, window=0):
+    p = i + nkv - nq                      # bottom-right aligned position
+    hi = min(nkv - 1, p) if causal else (min(nkv - 1, p + window - 1) if window else nkv - 1)
+    lo = max(0, p - window + 1) if window else 0
+    return max(0, hi - lo + 1)
 
 
-def _seeing_queries(j, nq, nkv, causal):
-    if not causal:
-        return nq
-    return max(0, nq - max(0, j - (nkv - nq)))
+def _seeing_queries(j, nq, nkv, causal, window=0):
+    shift = nkv - nq                      # query i sits at position i + shift
+    lo = max(0, j - shift) if causal else (max(0, j - window + 1 - shift) if window else 0)
+    hi = min(nq - 1, j + window - 1 - shift) if window else nq - 1
+    return max(0, hi - lo + 1)
 
 
-def schedule(q_off, kv_off, H, tile, causal, backward=False):
+def schedule(q_off, kv_off, H, tile, causal, backward=False, window=0):
     """Returns int32 [N, 4] rows (b, h, t, cost) in execution order."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     pairs = []
@@ -309,9 +314,9 @@ def schedule(q_off, kv_off, H, tile, causal, backward=False):
         for t in range(n_tiles):
             lo, hi = t * tile, min(n_rows, (t + 1) * tile)
             if backward:
-                cost = sum(_seeing_queries(j, nq, nkv, causal) for j in range(lo, hi))
+                cost = sum(_seeing_queries(j, nq, nkv, causal, window) for j in range(lo, hi))
             else:
-                cost = sum(_visible_keys(i, nq, nkv, causal) for i in range(lo, hi))
+                cost = sum(_visible_keys(i, nq, nkv, causal, window) for i in range(lo, hi))
             pairs.append((cost, b, t))
     if not backward:
         pairs.sort(key=lambda p: (-p[0], p[1], p[2]))
@@ -328,14 +333,14 @@ def schedule(q_off, kv_off, H, tile, causal, backward=False):
     return np.asarray(out, dtype=np.int32).reshape(-1, 4)
 
 
-def valid_pairs(q_off, kv_off, causal):
+def valid_pairs(q_off, kv_off, causal, window=0):
     """Number of (query, key) pairs that attention computes, per head."""
     q_off, kv_off = _i32(q_off), _i32(kv_off)
     total = 0
     for b in range(len(q_off) - 1):
         nq = int(q_off[b + 1] - q_off[b])
         nkv = int(kv_off[b + 1] - kv_off[b])
-        total += sum(_visible_keys(i, nq, nkv, causal) for i in range(nq))
+        total += sum(_visible_keys(i, nq, nkv, causal, window) for i in range(nq))
     return total
 
 

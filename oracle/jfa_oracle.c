@@ -94,6 +94,21 @@ static int block_of(int W, int i, int nq, int nkv) {
     return p < 0 ? -1 : (int)(p / W);
 }
 
+/* Windowed (sliding-window) attention ("Meta Enhances GEM Training Efficiency
+ * ...", "Exploring the Customized Kernel Library" -> "BlockAttention":
+ * windows instead of full attention over long user histories).  With window
+ * w > 0 query i, at the bottom-right aligned position p = i + n_kv - n_q,
+ * sees key j only when p - j < w (the w most recent positions up to p under
+ * the causal rule) and, without the causal rule, also j - p < w (a band of
+ * half-width w - 1 around p). */
+static int window_ok(int w, int causal, int i, int j, int nq, int nkv) {
+    if (w <= 0) return 1;
+    long p = (long)i + (long)(nkv - nq);
+    if (p - (long)j >= (long)w) return 0;
+    if (!causal && (long)j - p >= (long)w) return 0;
+    return 1;
+}
+
 
 
 /* Additive bias beta_h(i, j).
@@ -209,11 +224,13 @@ typedef struct {
     double scale;
     int quant_p; /* MXFP8: quantise exp(s - m) per 32 keys before P.V */
     int block;   /* BlockAttention block length; 0 = full attention */
+    int window;  /* sliding-window width; 0 = no window */
 } orc_problem;
 
 static int is_valid(const orc_problem* P, int i, int j, int nq, int nkv) {
     if (!causal_ok(P->causal, i, j, nq, nkv)) return 0;
     if (P->block > 0 && block_of(P->block, i, nq, nkv) != j / P->block) return 0;
+    if (!window_ok(P->window, P->causal, i, j, nq, nkv)) return 0;
     return 1;
 }
 
@@ -418,7 +435,7 @@ static void backward_item(const orc_problem* P, int b, int h, const double* dout
 static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_off,
                          const int32_t* kv_off, const double* q, const double* k, const double* v,
                          int bias_kind, const double* bias, int relpos_len, int act, int causal,
-                         double scale, int quant_p, int block) {
+                         double scale, int quant_p, int block, int window) {
     P->B = B; P->H = H; P->d = d;
     P->q_off = q_off; P->kv_off = kv_off;
     P->q = q; P->k = k; P->v = v;
@@ -428,6 +445,7 @@ static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_o
     P->scale = scale > 0.0 ? scale : 1.0 / sqrt((double)d);
     P->quant_p = quant_p;
     P->block = block;
+    P->window = window;
 }
 
 /* Forward over all (sequence b, head h) items with item_mask == NULL or
@@ -435,11 +453,11 @@ static void fill_problem(orc_problem* P, int B, int H, int d, const int32_t* q_o
 int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                        const double* q, const double* k, const double* v, int bias_kind,
                        const double* bias, int relpos_len, int act, int causal, double scale,
-                       int quant_p, int block, const int32_t* item_mask, double* out,
+                       int quant_p, int block, int window, const int32_t* item_mask, double* out,
                        double* lse, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
-                 scale, quant_p, block);
+                 scale, quant_p, block, window);
     long n_items = (long)B * H;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -460,12 +478,12 @@ int jfa_oracle_forward(int B, int H, int d, const int32_t* q_off, const int32_t*
 int jfa_oracle_backward(int B, int H, int d, const int32_t* q_off, const int32_t* kv_off,
                         const double* q, const double* k, const double* v, int bias_kind,
                         const double* bias, int relpos_len, int act, int causal, double scale,
-                        int block, const int32_t* item_mask, const double* dout,
+                        int block, int window, const int32_t* item_mask, const double* dout,
                         const double* out_for_d, double* dq, double* dk, double* dv,
                         double* dbias, int nthreads) {
     orc_problem P;
     fill_problem(&P, B, H, d, q_off, kv_off, q, k, v, bias_kind, bias, relpos_len, act, causal,
-                 scale, 0, block);
+                 scale, 0, block, window);
     long n_items = (long)B * H;
     const int want_tab = dbias && bias_kind == ORC_BIAS_RELPOS;
     double** parts = want_tab ? (double**)calloc((size_t)(n_items > 0 ? n_items : 1), sizeof(double*)) : NULL;

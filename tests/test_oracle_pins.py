@@ -566,3 +566,106 @@ def test_block_attention_is_attention_on_the_blocks(act):
     # and it differs from full attention whenever a sequence spans blocks
     full, _ = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
     assert not np.allclose(full, out)
+
+
+# ---------------------------------------------------------------------------
+# Sliding-window attention: query i (aligned position p = i + n_kv - n_q)
+# sees key j only when p - j < w, and without the causal rule also when
+# j - p < w
+# ---------------------------------------------------------------------------
+def _window_mask(P, Lq, Lk, causal, w):
+    B = len(P["q_lens"])
+    m = torch.zeros(B, 1, Lq, Lk, dtype=torch.bool)
+    for b in range(B):
+        nq, nk = P["q_lens"][b], P["kv_lens"][b]
+        if nq == 0 or nk == 0:
+            continue
+        p = torch.arange(nq)[:, None] + (nk - nq)
+        j = torch.arange(nk)[None, :]
+        blk = (p - j) < w
+        blk &= (j <= p) if causal else ((j - p) < w)
+        m[b, 0, :nq, :nk] = blk
+    return m
+
+
+WINDOW_CASES = [
+    # (q_lens, kv_lens, causal, bias_kind, w)
+    ([5, 1, 9, 12], [5, 1, 9, 12], True, "relpos", 3),
+    ([5, 1, 9, 12], [5, 1, 9, 12], True, "relpos", 1),
+    ([7, 3, 12], [7, 3, 12], False, "relpos", 4),
+    ([3, 8, 1], [11, 5, 6], False, "dense", 2),     # short q / long kv, band around p
+    ([9, 6, 2], [4, 6, 7], True, "dense", 3),       # n_q > n_kv: rows with p < 0 see nothing
+]
+
+
+@pytest.mark.parametrize("act", ["softmax", "silu", "gelu_tanh"])
+@pytest.mark.parametrize("q_lens,kv_lens,causal,bias_kind,w", WINDOW_CASES)
+def test_window_equals_band_masked_attention_and_autograd(act, q_lens, kv_lens, causal, bias_kind, w):
+    P = _jagged(21, q_lens, kv_lens, bias_kind=bias_kind)
+    kw = dict(bias=P["bias"], bias_kind=bias_kind, relpos_len=P["relpos_len"], causal=causal,
+              act=act, window=w)
+    out, lse = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
+    dq, dk, dv, db = oracle.backward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], P["do"],
+                                     dbias=True, **kw)
+    Lq, Lk = max(q_lens), max(kv_lens)
+    q = P["q"].clone().requires_grad_()
+    k = P["k"].clone().requires_grad_()
+    v = P["v"].clone().requires_grad_()
+    Pb = dict(P)
+    Pb["bias"] = P["bias"].clone().requires_grad_()
+    qp = _pad(q, P["q_off"], Lq).transpose(1, 2)
+    kp = _pad(k, P["kv_off"], Lk).transpose(1, 2)
+    vp = _pad(v, P["kv_off"], Lk).transpose(1, 2)
+    valid = _window_mask(P, Lq, Lk, causal, w)
+    row_ok = valid.any(-1, keepdim=True)
+    bias = _padded_bias(Pb, Lq, Lk)
+    s = qp @ kp.transpose(-1, -2) / math.sqrt(P["d"]) + bias
+    if act == "softmax":
+        mask = torch.where(valid, torch.zeros_like(s), torch.full_like(s, float("-inf")))
+        mask = torch.where(row_ok, mask, torch.zeros_like(mask))
+        ref = F.scaled_dot_product_attention(qp, kp, vp, attn_mask=bias + mask)
+        ref = torch.where(row_ok, ref, torch.zeros_like(ref))
+        ref_lse = _unpad(torch.logsumexp(s.masked_fill(~valid, float("-inf")), -1)[..., None],
+                         P["q_off"])[..., 0]
+        keep = np.isfinite(ref_lse.detach().numpy())
+        np.testing.assert_allclose(lse[keep], ref_lse.detach().numpy()[keep], atol=1e-12, rtol=0)
+        assert np.all(np.isneginf(lse[~keep]))
+    else:
+        a = F.silu(s) if act == "silu" else F.gelu(s, approximate="tanh")
+        nkv = torch.tensor(P["kv_lens"], dtype=torch.float64)[:, None, None, None]
+        ref = (a * valid / nkv) @ vp          # GDPA divides by n_kv, window or not
+        assert lse is None
+    o = _unpad(ref, P["q_off"])
+    np.testing.assert_allclose(out, o.detach().numpy(), atol=1e-12, rtol=0)
+    (o * P["do"]).sum().backward()
+    np.testing.assert_allclose(dq, q.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, k.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dv, v.grad.numpy(), atol=1e-12, rtol=0)
+    # masked pairs get 0 in the dense gradient, as in autograd
+    np.testing.assert_allclose(db, Pb["bias"].grad.numpy(), atol=1e-12, rtol=0)
+
+
+def test_window_special_cases():
+    lens = [6, 1, 11]
+    P = _jagged(22, lens, lens, bias_kind="relpos")
+    kw = dict(bias=P["bias"], bias_kind="relpos", relpos_len=P["relpos_len"], causal=True)
+    # w = 1 under the causal rule: each query sees only its own position, so
+    # the softmax output is that row of V and LSE its score
+    out, lse = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], window=1, **kw)
+    np.testing.assert_allclose(out, P["v"].numpy(), atol=1e-15, rtol=0)
+    C = (P["relpos_len"] - 1) // 2
+    s_ii = (P["q"] * P["k"]).sum(-1).numpy() / math.sqrt(P["d"]) + P["bias"][:, C].numpy()[None, :]
+    np.testing.assert_allclose(lse, s_ii, atol=1e-12, rtol=0)
+    # a window that covers every sequence is no window at all (bit for bit);
+    # one less changes the longest sequence's last row only
+    full, lse_f = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], **kw)
+    cov, lse_c = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], window=11, **kw)
+    assert np.array_equal(full, cov) and np.array_equal(lse_f, lse_c)
+    short, _ = oracle.forward(P["q_off"], P["kv_off"], P["q"], P["k"], P["v"], window=10, **kw)
+    diff = np.abs(short - full).max(axis=(1, 2)) > 0
+    assert list(np.nonzero(diff)[0]) == [int(P["q_off"][3]) - 1]
+    # the schedule costs count exactly the window's pairs
+    for causal in (False, True):
+        for w in (1, 3, 7):
+            mask = _window_mask(P, 11, 11, causal, w)
+            assert oracle.valid_pairs(P["q_off"], P["kv_off"], causal, w) == int(mask.sum())
