@@ -76,6 +76,8 @@ def parse_args():
                     help="override the workload's length clip (profiling captures)")
     ap.add_argument("--block", type=int, default=0,
                     help="BlockAttention block length (self-attention workloads); 0 = full")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding-window width (query at position p sees keys p - w < j); 0 = none")
     ap.add_argument("--partition", choices=["bbs", "lpt"], default="bbs",
                     help="split of the global batch across ranks (N > 1)")
     ap.add_argument("--sub-batch", type=int, default=8,
@@ -92,15 +94,22 @@ def parse_args():
 # ---------------------------------------------------------------------------
 # work accounting
 # ---------------------------------------------------------------------------
-def visible_pairs(q_lens, kv_lens, causal, block=0):
+def visible_pairs(q_lens, kv_lens, causal, block=0, window=0):
     """Per-sequence number of (query, key) pairs attention computes; with
-    BlockAttention (block > 0, self-attention) only pairs inside a block."""
+    BlockAttention (block > 0, self-attention) only pairs inside a block, with
+    a sliding window (window > 0) only pairs with p - j < window (and, without
+    the causal rule, j - p < window), p = i + n_kv - n_q."""
     out = np.zeros(len(q_lens), np.int64)
     for b, (nq, nk) in enumerate(zip(q_lens, kv_lens)):
         nq, nk = int(nq), int(nk)
         if block > 0:
             m = np.minimum(block, nq - np.arange(0, nq, block)).astype(np.int64)
             out[b] = int((m * (m + 1) // 2).sum() if causal else (m * m).sum())
+        elif window > 0:
+            pos = np.arange(nq, dtype=np.int64) + nk - nq
+            hi = np.minimum(nk - 1, pos if causal else pos + window - 1)
+            lo = np.maximum(0, pos - window + 1)
+            out[b] = int(np.maximum(hi - lo + 1, 0).sum())
         elif not causal:
             out[b] = nq * nk
         else:
@@ -124,8 +133,9 @@ def sq_bytes(p, backward: bool, softmax: bool) -> float:
     return 2 * tq + 2 * tkv + bias + (2 * rows if softmax else 0.0) + tq + 2 * tkv
 
 
-def flops_of(p, pairs_per_seq=None, block=0):
-    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block) if pairs_per_seq is None else pairs_per_seq
+def flops_of(p, pairs_per_seq=None, block=0, window=0):
+    pairs = (visible_pairs(p.q_lens, p.kv_lens, p.causal, block, window) if pairs_per_seq is None
+             else pairs_per_seq)
     f_fwd = 4.0 * p.d * p.H * float(pairs.sum())
     return f_fwd, 2.5 * f_fwd
 
@@ -294,10 +304,10 @@ def recorded_traffic(kernel, workload):
 # ---------------------------------------------------------------------------
 # reference arm / CPU baseline: the fp64 oracle on a bounded stratified sample
 # ---------------------------------------------------------------------------
-def cpu_sample_mask(p, target_pairs_heads, block=0):
+def cpu_sample_mask(p, target_pairs_heads, block=0, window=0):
     """Sequences picked evenly over the length-sorted batch (shortest first)
     until the sample holds ~target (pairs x heads)."""
-    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block) * p.H
+    pairs = visible_pairs(p.q_lens, p.kv_lens, p.causal, block, window) * p.H
     order = np.argsort(pairs, kind="stable")
     mask = np.zeros(p.B, np.int32)
     total = 0
@@ -314,20 +324,20 @@ def cpu_sample_mask(p, target_pairs_heads, block=0):
     return mask, pairs
 
 
-def run_oracle_step(p, mask, act, block=0):
+def run_oracle_step(p, mask, act, block=0, window=0):
     import oracle
     kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act=act,
-              causal=p.causal, seq_mask=mask, block=block)
+              causal=p.causal, seq_mask=mask, block=block, window=window)
     o, l = oracle.forward(p.q_off, p.kv_off, p.q, p.k, p.v, **kw)
     oracle.backward(p.q_off, p.kv_off, p.q, p.k, p.v, p.dout, **kw)
 
 
-def cpu_baseline(p, act, target, block=0):
+def cpu_baseline(p, act, target, block=0, window=0):
     import oracle
-    mask, pairs = cpu_sample_mask(p, target, block)
+    mask, pairs = cpu_sample_mask(p, target, block, window)
     f_fwd = 4.0 * p.d * float((pairs * mask).sum())
     t0 = time.perf_counter()
-    run_oracle_step(p, mask, act, block)
+    run_oracle_step(p, mask, act, block, window)
     dt = time.perf_counter() - t0
     n = int(mask.sum())
     return {"value": 3.5 * f_fwd / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
@@ -344,13 +354,13 @@ def reference_arm(args, rank, world):
     p = make_problem(args.workload, args.seed, B=args.batch, max_len=args.max_len, bias=args.bias)
     act = args.act or p.act
     target = args.cpu_sample_pairs / 4
-    mask, pairs = cpu_sample_mask(p, target, args.block)
+    mask, pairs = cpu_sample_mask(p, target, args.block, args.window)
     f_sample = 3.5 * 4.0 * p.d * float((pairs * mask).sum())
     for _ in range(args.warmup):
-        run_oracle_step(p, mask, act, args.block)
+        run_oracle_step(p, mask, act, args.block, args.window)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        run_oracle_step(p, mask, act, args.block)
+        run_oracle_step(p, mask, act, args.block, args.window)
     dt = (time.perf_counter() - t0) / max(1, args.steps)
     value = f_sample / dt / 1e12
     n = int(mask.sum())
@@ -361,7 +371,7 @@ def reference_arm(args, rank, world):
         "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "global_batch": p.B, "heads": p.H,
                    "head_dim": p.d, "act": act, "causal": p.causal, "block": args.block or None,
-                   "sample_sequences": n, "l2": "inputs larger than L2"},
+                   "window": args.window or None, "sample_sequences": n, "l2": "inputs larger than L2"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
                          "sample": f"each step: {n} of {p.B} sequences (stratified by length), "
@@ -438,9 +448,11 @@ def main():
 
     p, split = rank_problem(args, rank, world, jfa)
     act = args.act or p.act
-    prob = jfa.problem_of(p)
+    if args.block and args.window:
+        raise SystemExit("--block and --window are alternatives")
+    prob = jfa.problem_of(p, window=args.window)
     path = jfa.jfa_path(prob, act, 0), jfa.jfa_path(prob, act, 1)
-    f_fwd, f_bwd = flops_of(p, block=args.block)
+    f_fwd, f_bwd = flops_of(p, block=args.block, window=args.window)
     d = {n: getattr(p, n).to(dev).contiguous() for n in ("q", "k", "v", "dout", "q_off", "kv_off")}
     seq_off = d["q_off"]
     if args.block:
@@ -576,7 +588,7 @@ def main():
                    "heads": p.H,
                    "head_dim": p.d, "act": act, "causal": p.causal, "bias": p.bias_kind,
                    "total_tokens": p.total_q, "max_len": p.max_q_len,
-                   "block": args.block or None,
+                   "block": args.block or None, "window": args.window or None,
                    "parallelism": (f"dp{world} ({args.partition} split of one global batch)"
                                    if world > 1 else "dp1"),
                    "l2": "inputs larger than L2 (each of Q/K/V/dO > 126 MB); no flush",
@@ -608,10 +620,11 @@ def main():
     # end to end through the C ABI with host buffers
     if not args.no_e2e:
         result["e2e"] = e2e_leg(args, p, prob, act, dev, stream, jfa, f_fwd + f_bwd, world)
-    if rank == 0 and world == 1 and not args.no_padded and not args.block:
+    if rank == 0 and world == 1 and not args.no_padded and not args.block and not args.window:
         result["padded_dense_baseline"] = padded_dense_baseline(p, dev, f_fwd + f_bwd)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(p, act, args.cpu_sample_pairs, args.block)
+        result["cpu_baseline"] = cpu_baseline(p, act, args.cpu_sample_pairs, args.block,
+                                              args.window)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:

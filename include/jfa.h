@@ -102,7 +102,21 @@ typedef struct {
     float scale;         /* tau; <= 0 selects 1/sqrt(head_dim) */
     jfa_bias_kind bias_kind;
     int32_t relpos_len;  /* odd table length for JFA_BIAS_RELPOS, else ignored */
+    int32_t window;      /* sliding-window width w >= 0; 0 = no window (below) */
 } jfa_problem;
+
+/* Masks.  Query i of a sequence sits at the bottom-right aligned key position
+ * p = i + n_kv - n_q (p = i for self-attention).  causal = 1: key j is
+ * visible only when j <= p.  Sliding window (windowed attention: "Meta
+ * Enhances GEM Training Efficiency with Advanced LLM-Scale Innovations",
+ * "Exploring the Customized Kernel Library" -> "BlockAttention", windows
+ * instead of full attention over long user histories): with window = w > 0
+ * key j is visible only when p - j < w, and, without the causal rule, also
+ * when j - p < w (a band of 2w - 1 keys around p).  Causal with w keeps the
+ * w most recent positions up to p.  Only the key tiles inside the band are
+ * computed; GDPA still divides by n_kv.  A query row that sees no key gets a
+ * zero output and LSE = -inf.  A negative window is
+ * JFA_ERR_INVALID_ARGUMENT. */
 
 /* Bytes of device workspace that jfa_forward (backward = 0) or jfa_backward
  * (backward = 1) needs for this problem; 0 if the descriptor is invalid.

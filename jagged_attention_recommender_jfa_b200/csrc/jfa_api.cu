@@ -127,6 +127,7 @@ jfa_status check_problem(const jfa_problem* p) {
     if (p->bias_kind == JFA_BIAS_RELPOS && (p->relpos_len < 1 || (p->relpos_len & 1) == 0))
         return fail(JFA_ERR_INVALID_ARGUMENT, "relpos_len must be odd and >= 1");
     if (!(p->scale == p->scale)) return fail(JFA_ERR_INVALID_ARGUMENT, "scale is NaN");
+    if (p->window < 0) return fail(JFA_ERR_INVALID_ARGUMENT, "negative window %d", p->window);
     return JFA_OK;
 }
 
@@ -222,7 +223,7 @@ jfa_status forward_impl(const jfa_problem* problem, const void* q, const void* k
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
     a.bias = bias; a.dense_off = reinterpret_cast<const int64_t*>(ws + L.dense_off);
     a.bias_kind = p.bias_kind; a.relpos_len = p.relpos_len; a.B = p.batch; a.H = p.heads;
-    a.causal = causal ? 1 : 0; a.act = act; a.scale = eff_scale(p);
+    a.causal = causal ? 1 : 0; a.window = p.window; a.act = act; a.scale = eff_scale(p);
     a.out = out; a.lse = (act == JFA_ACT_SOFTMAX) ? lse : nullptr;
     a.items = reinterpret_cast<const int4*>(ws + L.items); a.item_count = &hdr->item_count;
     a.hdr = hdr;
@@ -339,15 +340,15 @@ jfa_status backward_impl(const jfa_problem* problem, const void* q, const void* 
     a.q = q; a.k = k; a.v = v; a.q_off = q_offsets; a.kv_off = kv_offsets;
     a.bias = bias; a.dense_off = reinterpret_cast<const int64_t*>(ws + L.dense_off);
     a.bias_kind = p.bias_kind; a.relpos_len = p.relpos_len; a.B = p.batch; a.H = p.heads;
-    a.causal = causal ? 1 : 0; a.act = act; a.scale = eff_scale(p);
+    a.causal = causal ? 1 : 0; a.window = p.window; a.act = act; a.scale = eff_scale(p);
     a.out = const_cast<void*>(out); a.lse = const_cast<float*>(lse);
     a.items = reinterpret_cast<const int4*>(ws + L.items); a.item_count = &hdr->item_count;
     a.hdr = hdr;
     a.dout = dout; a.dterm = reinterpret_cast<float*>(ws + L.dterm);
     a.dq = dq; a.dk = dk; a.dv = dv;
     a.dbias = dbias;
-    if (dbias && p.bias_kind == JFA_BIAS_DENSE_JAGGED && causal) {
-        // masked pairs of a causal block get 0; the kernels write the rest
+    if (dbias && p.bias_kind == JFA_BIAS_DENSE_JAGGED && (causal || p.window > 0)) {
+        // masked pairs of a causal or windowed block get 0; the kernels write the rest
         e = dbias_zero_masked(a, p.dtype == JFA_F32 ? 4 : 2, st);
         if (e != cudaSuccess) return cuda_fail(e, "dbias zero");
     }

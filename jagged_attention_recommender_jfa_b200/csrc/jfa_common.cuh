@@ -97,6 +97,7 @@ struct AttnArgs {
     int relpos_len;
     int B, H;
     int causal;
+    int window;   // sliding-window width w (0: none), see vis_key_lo / vis_key_hi
     int act;
     float scale;
     void* out;
@@ -265,9 +266,36 @@ __device__ __forceinline__ float bias_at(const AttnArgs& a, int b, int h, int nq
     return 0.0f;
 }
 
-// Bottom-right causal validity.
-__device__ __forceinline__ bool key_visible(int causal, int i, int j, int nq, int nkv) {
-    return !causal || j <= i + (nkv - nq);
+// Validity with bottom-right alignment: query i sits at key position
+// p = i + (n_kv - n_q).  Causal: key j is visible iff j <= p.  Sliding window
+// w > 0 (windowed attention, "Meta Enhances GEM Training Efficiency with
+// Advanced LLM-Scale Innovations", "Exploring the Customized Kernel Library"
+// -> "BlockAttention": windows instead of full attention over long user
+// histories): additionally p - j < w, and without the causal rule also
+// j - p < w.  The visible keys of a query row and the queries that see a key
+// are contiguous ranges, returned clamped to the sequence (empty: lo > hi).
+__device__ __forceinline__ int vis_key_lo(int window, int i, int nq, int nkv) {
+    if (window <= 0) return 0;
+    const int64_t lo = (int64_t)i + (nkv - nq) - window + 1;
+    return lo < 0 ? 0 : (int)lo;
+}
+__device__ __forceinline__ int vis_key_hi(int causal, int window, int i, int nq, int nkv) {
+    const int64_t p = (int64_t)i + (nkv - nq);
+    const int64_t hi = causal ? p : (window > 0 ? p + window - 1 : (int64_t)nkv - 1);
+    return (int)(hi < (int64_t)nkv - 1 ? (hi < -1 ? -1 : hi) : (int64_t)nkv - 1);
+}
+__device__ __forceinline__ int vis_query_lo(int causal, int window, int j, int nq, int nkv) {
+    const int64_t shift = (int64_t)nkv - nq;
+    const int64_t lo = causal ? j - shift : (window > 0 ? j - window + 1 - shift : 0);
+    return lo < 0 ? 0 : (lo > nq ? nq : (int)lo);
+}
+__device__ __forceinline__ int vis_query_hi(int window, int j, int nq, int nkv) {
+    if (window <= 0) return nq - 1;
+    const int64_t hi = (int64_t)j + window - 1 - ((int64_t)nkv - nq);
+    return (int)(hi < (int64_t)nq - 1 ? (hi < -1 ? -1 : hi) : (int64_t)nq - 1);
+}
+__device__ __forceinline__ bool key_visible(int causal, int window, int i, int j, int nq, int nkv) {
+    return j >= vis_key_lo(window, i, nq, nkv) && j <= vis_key_hi(causal, window, i, nq, nkv);
 }
 
 }  // namespace jfa

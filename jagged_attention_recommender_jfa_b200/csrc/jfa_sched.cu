@@ -39,25 +39,22 @@ namespace {
 constexpr int kPrepThreads = 1024;
 
 // Pairs (query, key) computed by rows [lo, hi) of a query tile.
-__device__ int64_t query_tile_cost(int lo, int hi, int nq, int nkv, int causal) {
-    if (!causal) return (int64_t)(hi - lo) * nkv;
+__device__ int64_t query_tile_cost(int lo, int hi, int nq, int nkv, int causal, int window) {
+    if (!causal && window <= 0) return (int64_t)(hi - lo) * nkv;
     int64_t c = 0;
     for (int i = lo; i < hi; ++i) {
-        int vis = i + 1 + (nkv - nq);
-        vis = vis < 0 ? 0 : (vis > nkv ? nkv : vis);
-        c += vis;
+        const int vis = vis_key_hi(causal, window, i, nq, nkv) - vis_key_lo(window, i, nq, nkv) + 1;
+        c += vis > 0 ? vis : 0;
     }
     return c;
 }
 
 // Pairs computed by key rows [lo, hi) of a key/value tile.
-__device__ int64_t key_tile_cost(int lo, int hi, int nq, int nkv, int causal) {
-    if (!causal) return (int64_t)(hi - lo) * nq;
+__device__ int64_t key_tile_cost(int lo, int hi, int nq, int nkv, int causal, int window) {
+    if (!causal && window <= 0) return (int64_t)(hi - lo) * nq;
     int64_t c = 0;
     for (int j = lo; j < hi; ++j) {
-        int first = j - (nkv - nq);
-        first = first < 0 ? 0 : first;
-        int cnt = nq - first;
+        const int cnt = vis_query_hi(window, j, nq, nkv) - vis_query_lo(causal, window, j, nq, nkv) + 1;
         c += cnt > 0 ? cnt : 0;
     }
     return c;
@@ -65,7 +62,8 @@ __device__ int64_t key_tile_cost(int lo, int hi, int nq, int nkv, int causal) {
 
 __global__ void __launch_bounds__(kPrepThreads)
 sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_off, int B, int H,
-              int max_q, int max_kv, int64_t total_q, int64_t total_kv, int causal, int backward,
+              int max_q, int max_kv, int64_t total_q, int64_t total_kv, int causal, int window,
+              int backward,
               int tile, int64_t pairs_cap, int want_dense, WsHeader* hdr, int64_t* dense_off,
               int2* pair_bt, int64_t* pair_cost, int32_t* pair_count_out, int reset_err,
               int64_t* seq_tmp, int64_t* seq_start, int wait_limit_us, int cost_tiles) {
@@ -128,6 +126,7 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
         int64_t first = carry + s_scan[tid] - nt;
         if (b < B) {
             if (want_dense) dense_off[b] = dcarry + s_dscan[tid] - dn;
+            if (seq_start != nullptr) seq_start[b] = first;   // the sequence's first pair (step 4)
             for (int64_t t = 0; t < nt && first + t < pairs_cap; ++t)
                 pair_bt[first + t] = make_int2(b, (int)t);
         }
@@ -148,9 +147,11 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
         int nq = q_off[bt.x + 1] - q_off[bt.x], nkv = kv_off[bt.x + 1] - kv_off[bt.x];
         int rows = backward ? nkv : nq;
         int lo = bt.y * tile, hi = min(rows, lo + tile);
-        int64_t c = backward ? key_tile_cost(lo, hi, nq, nkv, causal) : query_tile_cost(lo, hi, nq, nkv, causal);
+        int64_t c = backward ? key_tile_cost(lo, hi, nq, nkv, causal, window)
+                             : query_tile_cost(lo, hi, nq, nkv, causal, window);
         if (cost_tiles) {
             // 128-key tiles of the item's visible key range, then its pairs
+            // (the short-query kernels run only without a window)
             int kv_end = causal ? min(nkv, hi + (nkv - nq)) : nkv;
             kv_end = kv_end < 0 ? 0 : kv_end;
             c = ((int64_t)((kv_end + 127) / 128) << 32) | (c < 0xffffffffll ? c : 0xffffffffll);
@@ -159,10 +160,16 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
     }
     if (seq_start == nullptr) return;
     // 4. sequence order of the grouped (key-tile) schedule: seq_start[b] =
-    //    tiles of the sequences ranked before b (cost descending, then b)
+    //    tiles of the sequences ranked before b (cost descending, then b);
+    //    a sequence's cost is the sum of its pairs' costs from step 3
+    __syncthreads();
     for (int b = tid; b < B; b += kPrepThreads) {
-        const int nq = q_off[b + 1] - q_off[b], nkv = kv_off[b + 1] - kv_off[b];
-        seq_tmp[b] = key_tile_cost(0, nkv, nq, nkv, causal);
+        const int rows = backward ? kv_off[b + 1] - kv_off[b] : q_off[b + 1] - q_off[b];
+        const int64_t first = seq_start[b];
+        const int64_t last = min(first + (rows + tile - 1) / tile, npairs);
+        int64_t c = 0;
+        for (int64_t p = first; p < last; ++p) c += pair_cost[p];
+        seq_tmp[b] = c;
     }
     __syncthreads();
     for (int b = tid; b < B; b += kPrepThreads) {
@@ -259,7 +266,7 @@ cudaError_t build_schedule(const jfa_problem& pb, const int32_t* q_off, const in
     prof_begin(stream);
     sched_prepare<<<1, kPrepThreads, 0, stream>>>(
         q_off, kv_off, pb.batch, pb.heads, pb.max_q_len, pb.max_kv_len, pb.total_q, pb.total_kv,
-        causal, backward, tile, pairs_cap, want_dense, hdr, dense_off, pair_bt, pair_cost,
+        causal, pb.window, backward, tile, pairs_cap, want_dense, hdr, dense_off, pair_bt, pair_cost,
         pair_count, reset_err, seq_tmp, seq_start, wait_limit_us, cost_tiles);
     prof_end(stream, K_SCHED_PREPARE);
     int64_t bound = pairs_bound(pb.batch, backward ? pb.max_kv_len : pb.max_q_len,

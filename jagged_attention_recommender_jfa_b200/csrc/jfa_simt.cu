@@ -67,14 +67,15 @@ __global__ void __launch_bounds__(kThreads) simt_fwd(AttnArgs a) {
     const T* V = reinterpret_cast<const T*>(a.v) + (int64_t)h * D;
     const int rows_hi = min(row0 + BM, nq);
     load_rows<D, T>(Qs, Q, (int64_t)H * D, q0 + row0, rows_hi - row0, BM);
-    int kv_end = a.causal ? min(nkv, rows_hi + (nkv - nq)) : nkv;
-    kv_end = max(kv_end, 0);
+    // keys seen by rows [row0, rows_hi): the first row's first to the last row's last
+    const int kv_begin = vis_key_lo(a.window, row0, nq, nkv);
+    const int kv_end = max(vis_key_hi(a.causal, a.window, rows_hi - 1, nq, nkv) + 1, 0);
     const bool softmax = a.act == JFA_ACT_SOFTMAX;
     float m = -CUDART_INF_F, l = 0.f;
     float4 o[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) o[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < kv_end; j0 += BN) {
+    for (int j0 = kv_begin; j0 < kv_end; j0 += BN) {
         __syncthreads();
         const int nvalid = min(BN, nkv - j0);
         load_rows<D, T>(Ks, K, (int64_t)H * D, k0 + j0, nvalid, BN);
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) simt_fwd(AttnArgs a) {
 #pragma unroll
         for (int jj = 0; jj < BN / 4; ++jj) {
             const int j = j0 + c + 4 * jj;
-            const bool ok = i < nq && j < nkv && key_visible(a.causal, i, j, nq, nkv);
+            const bool ok = i < nq && j < nkv && key_visible(a.causal, a.window, i, j, nq, nkv);
             float x = ok ? s[jj] * a.scale + bias_at<T>(a, b, h, nq, nkv, i, j) : -CUDART_INF_F;
             s[jj] = x;
             tmax = fmaxf(tmax, x);
@@ -221,12 +222,13 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq(AttnArgs a) {
         d_i = a.dterm[(int64_t)(q0 + i) * H + h];
     }
     const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
-    int kv_end = a.causal ? min(nkv, rows_hi + (nkv - nq)) : nkv;
-    kv_end = max(kv_end, 0);
+    // keys seen by rows [row0, rows_hi): the first row's first to the last row's last
+    const int kv_begin = vis_key_lo(a.window, row0, nq, nkv);
+    const int kv_end = max(vis_key_hi(a.causal, a.window, rows_hi - 1, nq, nkv) + 1, 0);
     float4 acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < kv_end; j0 += BN) {
+    for (int j0 = kv_begin; j0 < kv_end; j0 += BN) {
         __syncthreads();
         const int nvalid = min(BN, nkv - j0);
         load_rows<D, T>(Ks, K, (int64_t)H * D, k0 + j0, nvalid, BN);
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dq(AttnArgs a) {
 #pragma unroll
         for (int jj = 0; jj < BN / 4; ++jj) {
             const int j = j0 + c + 4 * jj;
-            const bool ok = i < nq && j < nkv && key_visible(a.causal, i, j, nq, nkv);
+            const bool ok = i < nq && j < nkv && key_visible(a.causal, a.window, i, j, nq, nkv);
             float ds = 0.f;
             if (ok) {
                 float x = s[jj] * a.scale + bias_at<T>(a, b, h, nq, nkv, i, j);
@@ -322,12 +324,13 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv(AttnArgs a) {
     load_rows<D, T>(Vs, V, (int64_t)H * D, k0 + col0, cols_hi - col0, BN);
     const bool softmax = a.act == JFA_ACT_SOFTMAX;
     const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
-    // first query row that sees key col0: i >= col0 - (nkv - nq)
-    int i_start = a.causal ? max(0, col0 - (nkv - nq)) : 0;
+    // queries that see keys [col0, cols_hi): the first key's first to the last key's last
+    const int i_start = vis_query_lo(a.causal, a.window, col0, nq, nkv);
+    const int i_end = vis_query_hi(a.window, cols_hi - 1, nq, nkv) + 1;
     float4 dk[G], dv[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) dk[g] = make_float4(0.f, 0.f, 0.f, 0.f), dv[g] = dk[g];
-    for (int i0 = i_start; i0 < nq; i0 += BM) {
+    for (int i0 = i_start; i0 < i_end; i0 += BM) {
         __syncthreads();
         const int nvalid = min(BM, nq - i0);
         load_rows<D, T>(Qs, Q, (int64_t)H * D, q0 + i0, nvalid, BM);
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(kThreads) simt_bwd_dkdv(AttnArgs a) {
 #pragma unroll
         for (int ii = 0; ii < BM / 4; ++ii) {
             const int il = c + 4 * ii, i = i0 + il;
-            const bool ok = i < nq && j < nkv && key_visible(a.causal, i, j, nq, nkv);
+            const bool ok = i < nq && j < nkv && key_visible(a.causal, a.window, i, j, nq, nkv);
             float w = 0.f, ds = 0.f;
             if (ok) {
                 float x = s[ii] * a.scale + bias_at<T>(a, b, h, nq, nkv, i, j);

@@ -201,8 +201,9 @@ cudaError_t tc_backward(const jfa_problem& p, const AttnArgs& a, const AttnArgs&
 }
 
 // Short query sequences (every n_q <= 64) take the paired-item forward and
-// the query-stationary backward.
-bool tc_backward_short_q(const jfa_problem& p) { return p.max_q_len <= 64; }
+// the query-stationary backward; with a sliding window the general kernels,
+// which compute only the key tiles inside the band, run instead.
+bool tc_backward_short_q(const jfa_problem& p) { return p.max_q_len <= 64 && p.window == 0; }
 
 int tc_fwd_tile() { return 256; }   // a forward work item is a 256-row query block
 int tc_bwd_tile() { return 128; }

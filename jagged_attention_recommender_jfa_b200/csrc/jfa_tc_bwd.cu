@@ -162,7 +162,7 @@ __device__ __forceinline__ void zero_row(uint8_t* tile, int r) {
 // dense bias gradient, or summed along the diagonals of each tile in shared
 // memory and added to the relative-position table gradient by one warp
 // (score warp t % 16 for tile t, at the start of tile t + 1).
-template <int BIAS, bool SOFTMAX, bool DBIAS>
+template <int BIAS, bool SOFTMAX, bool DBIAS, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_constant__ BwdParams P) {
     const AttnArgs& a = P.a;
     if ((int)blockIdx.x >= *a.item_count || a.hdr->err != 0) return;
@@ -176,9 +176,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     const int b = it.x, h = it.y, j0 = it.z * BN;
     const int q0 = a.q_off[b], nq = a.q_off[b + 1] - q0;
     const int k0 = a.kv_off[b], nkv = a.kv_off[b + 1] - k0;
+    // the queries that see keys [j0, j0 + BN): from the first key's first to
+    // the last key's last (all of them without a causal rule or window)
     const int shift = nkv - nq;  // causal: key j visible from query i iff j <= i + shift
-    const int i_start = a.causal ? max(0, j0 - shift) : 0;
-    const int nt = nq > i_start ? (nq - i_start + BM - 1) / BM : 0;
+    const int i_start = WINDOW ? vis_query_lo(a.causal, a.window, j0, nq, nkv)
+                               : (a.causal ? max(0, j0 - shift) : 0);
+    const int i_end = WINDOW ? vis_query_hi(a.window, min(j0 + BN, nkv) - 1, nq, nkv) + 1 : nq;
+    const int nt = i_end > i_start ? (i_end - i_start + BM - 1) / BM : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool softmax = SOFTMAX;
 
@@ -472,12 +476,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             // qc0 - j + C - w0 + 4q hold table[... + 4q + 0..3]
             const int wbase = BIAS == 1 ? (qb0 - j + C) - bias_window_start(qb0, j0, C, a.bias4_stride) : 0;
             const float4* win = reinterpret_cast<const float4*>(smem + kOffWin + buf * kWinBytes);
-            const int imin_vis = a.causal ? j - shift : 0;  // queries i >= imin_vis see key j
+            // queries imin_vis .. imax_vis see key j
+            const int imin_vis = WINDOW ? vis_query_lo(a.causal, a.window, j, nq, nkv)
+                                        : (a.causal ? j - shift : 0);
+            const int imax_vis = WINDOW ? vis_query_hi(a.window, j, nq, nkv) : nq - 1;
             // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
             auto process = [&](uint32_t (&u)[16], uint32_t (&g)[16], int c16) {
                 const int qc0 = qb0 + c16 * 16;      // query index of the part's column 0
-                const bool all_vis = jvalid && (qc0 + 15 < nq) && (qc0 >= imin_vis);
-                const bool none_vis = !jvalid || qc0 >= nq || (qc0 + 15 < imin_vis);
+                const bool all_vis = jvalid && (qc0 + 15 <= imax_vis) && (qc0 >= imin_vis);
+                const bool none_vis = !jvalid || qc0 > imax_vis || (qc0 + 15 < imin_vis);
                 if (none_vis) {
 #pragma unroll
                     for (int v = 0; v < 16; ++v) u[v] = 0u, g[v] = 0u;
@@ -558,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
 #pragma unroll
                     for (int v = 0; v < 16; ++v) {
                         const int qi = qc0 + v;
-                        const bool vis = jvalid && qi < nq && qi >= imin_vis;
+                        const bool vis = jvalid && qi <= imax_vis && qi >= imin_vis;
                         u[v] = vis ? u[v] : 0u;
                         g[v] = vis ? g[v] : 0u;
                     }
@@ -763,13 +770,23 @@ cudaError_t tc_backward_launch(const jfa_problem& p, const AttnArgs& a, const At
     const bool sm = a.act == JFA_ACT_SOFTMAX;
     const bool db = a.dbias != nullptr;
     void (*kern)(BwdParams) = nullptr;
-    if (bias == 0) kern = sm ? tc_bwd_kernel<0, true, false> : tc_bwd_kernel<0, false, false>;
-    else if (bias == 1)
-        kern = db ? (sm ? tc_bwd_kernel<1, true, true> : tc_bwd_kernel<1, false, true>)
-                  : (sm ? tc_bwd_kernel<1, true, false> : tc_bwd_kernel<1, false, false>);
-    else
-        kern = db ? (sm ? tc_bwd_kernel<2, true, true> : tc_bwd_kernel<2, false, true>)
-                  : (sm ? tc_bwd_kernel<2, true, false> : tc_bwd_kernel<2, false, false>);
+    if (a.window > 0) {
+        if (bias == 0) kern = sm ? tc_bwd_kernel<0, true, false, true> : tc_bwd_kernel<0, false, false, true>;
+        else if (bias == 1)
+            kern = db ? (sm ? tc_bwd_kernel<1, true, true, true> : tc_bwd_kernel<1, false, true, true>)
+                      : (sm ? tc_bwd_kernel<1, true, false, true> : tc_bwd_kernel<1, false, false, true>);
+        else
+            kern = db ? (sm ? tc_bwd_kernel<2, true, true, true> : tc_bwd_kernel<2, false, true, true>)
+                      : (sm ? tc_bwd_kernel<2, true, false, true> : tc_bwd_kernel<2, false, false, true>);
+    } else {
+        if (bias == 0) kern = sm ? tc_bwd_kernel<0, true, false, false> : tc_bwd_kernel<0, false, false, false>;
+        else if (bias == 1)
+            kern = db ? (sm ? tc_bwd_kernel<1, true, true, false> : tc_bwd_kernel<1, false, true, false>)
+                      : (sm ? tc_bwd_kernel<1, true, false, false> : tc_bwd_kernel<1, false, false, false>);
+        else
+            kern = db ? (sm ? tc_bwd_kernel<2, true, true, false> : tc_bwd_kernel<2, false, true, false>)
+                      : (sm ? tc_bwd_kernel<2, true, false, false> : tc_bwd_kernel<2, false, false, false>);
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int64_t grid = pairs_bound(p.batch, p.max_kv_len, p.total_kv, BN) * p.heads;

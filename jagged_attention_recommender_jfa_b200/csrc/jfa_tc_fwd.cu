@@ -146,10 +146,12 @@ __device__ __forceinline__ void dense_bias16(const __nv_bfloat16* p, float (&bb)
 
 struct Item {
     int b, h, row0, q0, nq, k0, nkv;
-    int n_t[2];   // key tiles of tile A and tile B (0: the tile has no rows or sees no key)
+    int jb;       // first key tile of the block (0 unless a sliding window starts later)
+    int n_t[2];   // key tiles of tile A and tile B from jb (0: the tile has no rows or sees no key)
     int n;        // key tiles of the block
 };
 
+template <bool WINDOW>
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     const int4 it = a.items[idx];
     Item w;
@@ -160,6 +162,10 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     w.nq = a.q_off[w.b + 1] - w.q0;
     w.k0 = a.kv_off[w.b];
     w.nkv = a.kv_off[w.b + 1] - w.k0;
+    // both tiles stream the key tiles from the one tile A's first row needs
+    // (tile B's rows see the same or later keys; a key tile of the band that
+    // B does not see is masked for it)
+    w.jb = WINDOW ? vis_key_lo(a.window, w.row0, w.nq, w.nkv) / BN : 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int lo = w.row0 + t * BM, hi = min(lo + BM, w.nq);
@@ -167,9 +173,13 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
             w.n_t[t] = 0;
             continue;
         }
-        int kv_end = a.causal ? min(w.nkv, hi + (w.nkv - w.nq)) : w.nkv;
-        kv_end = max(kv_end, 0);
-        w.n_t[t] = (kv_end + BN - 1) / BN;
+        if (WINDOW) {
+            const int kv_end = vis_key_hi(a.causal, a.window, hi - 1, w.nq, w.nkv) + 1;
+            w.n_t[t] = max((kv_end + BN - 1) / BN - w.jb, 0);
+        } else {
+            const int kv_end = max(a.causal ? min(w.nkv, hi + (w.nkv - w.nq)) : w.nkv, 0);
+            w.n_t[t] = (kv_end + BN - 1) / BN;
+        }
     }
     w.n = max(w.n_t[0], w.n_t[1]);
     return w;
@@ -183,7 +193,8 @@ __device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int st
 }
 
 // BIAS: 0 none, 1 relative-position (log2(e)-scaled table staged per key tile),
-// 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.
+// 2 dense jagged.  SOFTMAX: softmax (true) or GDPA.  WINDOW: a sliding window
+// (a lower key bound per row and a first key tile per item).
 //
 // Tensor-core order per item (n key tiles; tile T has n_T <= n of them):
 //   QK_A(0), QK_B(0), then for each j: [P_A(j)] PV_A(j), QK_A(j+1),
@@ -191,7 +202,7 @@ __device__ __forceinline__ int bias_window_start(int row0, int jc, int C, int st
 // Barrier phases follow per-CTA counters: g (key tiles so far, for the K/V
 // ring), gt[T] (steps of tile T so far), mt[T] (items with steps for T so
 // far), nk (items so far, for Q).
-template <int BIAS, bool SOFTMAX>
+template <int BIAS, bool SOFTMAX, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_constant__ FwdParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
@@ -245,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
-                const Item w = load_item(a, idx);
+                const Item w = load_item<WINDOW>(a, idx);
                 if (w.n == 0) continue;
                 if (nk > 0 && !mbar_wait(&bars->q_free, (nk - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
                 mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
@@ -258,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 for (int j = 0; j < w.n; ++j, ++g) {
                     const int s = g & 1;
                     const uint32_t par = ((g >> 1) - 1) & 1;
-                    const int z = w.k0 + j * BN;
+                    const int z = w.k0 + (w.jb + j) * BN;
                     if (g >= 2 && !mbar_wait(&bars->k_empty[s], par, abort_flag, a.hdr)) { ok = false; break; }
                     JFA_TRACE_EV(fwd, 0, g, 0);
                     // test hook: CTA 0 leaves out its first key tile (load and
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         // the stage's previous window was read by the softmax warps of
                         // both tiles before its P.V, hence before v_empty above
                         const int C = (a.relpos_len - 1) >> 1;
-                        const int w0 = bias_window_start(w.row0, j * BN, C, a.bias4_stride);
+                        const int w0 = bias_window_start(w.row0, (w.jb + j) * BN, C, a.bias4_stride);
                         const float* src = a.bias4 + 4 * ((int64_t)w.h * a.bias4_stride + w0);
                         mbar_arrive_expect_tx(&bars->bias_full[s], kWinBytes);
                         bulk_load(smem + kOffBias + s * kWinBytes, src, kWinBytes, &bars->bias_full[s]);
@@ -314,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
-                const Item w = load_item(a, idx);
+                const Item w = load_item<WINDOW>(a, idx);
                 if (w.n == 0) continue;
                 if (!mbar_wait(&bars->q_full, nk & 1, abort_flag, a.hdr)) { ok = false; break; }
                 ++nk;
@@ -416,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         for (int rr = 0; ok; ++rr) {
             const int idx = item_of_turn(rr, cta, G);
             if (idx >= n_items) break;
-            const Item w = load_item(a, idx);
+            const Item w = load_item<WINDOW>(a, idx);
             const int n = w.n_t[tt];
             const int gkv_item = gkv;
             gkv += w.n;
@@ -432,10 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 }
                 continue;
             }
-            const int shift = w.nkv - w.nq;        // causal: key j visible iff j <= i + shift
             const float inv_n = w.nkv > 0 ? 1.0f / (float)w.nkv : 0.f;
             const float half_c = inv_n * (0.5f / kLog2e);   // GDPA: act(s) / n_kv = x half_c (1 + tanh)
-            const int jmax_vis = a.causal ? min(w.nkv - 1, i + shift) : w.nkv - 1;
+            const int jmax_vis = WINDOW ? vis_key_hi(a.causal, a.window, i, w.nq, w.nkv)
+                                        : (a.causal ? min(w.nkv - 1, i + (w.nkv - w.nq)) : w.nkv - 1);
+            const int jmin_vis = WINDOW ? vis_key_lo(a.window, i, w.nq, w.nkv) : 0;
             const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)w.h * 4 * a.bias4_stride : nullptr;
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
@@ -445,7 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             // once from HBM) is brought into L2 a key tile ahead
             auto prefetch_bias_seg = [&](int jt) {
                 if (BIAS == 2 && i < w.nq && jt < n) {
-                    const int k_lo = min(jt * BN + cb, w.nkv - 1), k_hi = min(jt * BN + cb + CW - 1, w.nkv - 1);
+                    const int kj = (w.jb + jt) * BN + cb;
+                    const int k_lo = min(kj, w.nkv - 1), k_hi = min(kj + CW - 1, w.nkv - 1);
                     prefetch_l2(dense + dense_row + k_lo);
                     prefetch_l2(dense + dense_row + k_hi);
                 }
@@ -456,11 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                 if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
                 SM_EV(1);
                 tc_fence_after();
-                const int jc = j * BN;               // key index of column 0
+                const int jc = (w.jb + j) * BN;      // key index of column 0
                 const int gk = gkv_item + j, sk = gk & 1;   // key / value / bias stage
                 if (BIAS == 1 && !wwait(&bars->bias_full[sk], (gk >> 1) & 1)) { ok = false; break; }
-                const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;   // visible: [0, nvis)
-                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW);
+                const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;   // visible: [nlo, nvis)
+                const int nlo = WINDOW ? jmin_vis - jc : 0;
+                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW || (WINDOW && nlo > cb));
                 // bias(i, jc + c) = table[lo + 127 - c], lo = i - jc - 127 + C: the run
                 // table[lo .. lo+127] as the window entries lo - w0 + 4q, or clamped
                 // reads of the table when the run leaves the table or the window
@@ -529,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                     }
                     if (masked_half) {
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) x[v] = cc + v < nvis ? x[v] : -CUDART_INF_F;
+                        for (int v = 0; v < 16; ++v) x[v] = (cc + v < nvis && (!WINDOW || cc + v >= nlo)) ? x[v] : -CUDART_INF_F;
                     }
                     if (softmax) {
                         const float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
@@ -616,11 +630,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         } else if (a.act == JFA_ACT_SILU) {
 #pragma unroll
                             for (int v = 0; v < 16; ++v)
-                                x[v] = cc + v < nvis ? gdpa_weight_log2<JFA_ACT_SILU>(x[v], half_c) : 0.f;
+                                x[v] = (cc + v < nvis && (!WINDOW || cc + v >= nlo)) ? gdpa_weight_log2<JFA_ACT_SILU>(x[v], half_c) : 0.f;
                         } else {
 #pragma unroll
                             for (int v = 0; v < 16; ++v)
-                                x[v] = cc + v < nvis ? gdpa_weight_log2<JFA_ACT_GELU_TANH>(x[v], half_c) : 0.f;
+                                x[v] = (cc + v < nvis && (!WINDOW || cc + v >= nlo)) ? gdpa_weight_log2<JFA_ACT_GELU_TANH>(x[v], half_c) : 0.f;
                         }
                         uint32_t pw[8];
 #pragma unroll
@@ -754,13 +768,17 @@ cudaError_t tc_forward_launch(const jfa_problem& p, const AttnArgs& a, cudaStrea
     const int grid = (int)(items_bound < sms ? items_bound : sms);
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
     const bool sm = a.act == JFA_ACT_SOFTMAX;
+    const bool win = a.window > 0;
     void (*kern)(FwdParams) = nullptr;
     if (bias == 0) {
-        kern = sm ? tc_fwd_kernel<0, true> : tc_fwd_kernel<0, false>;
+        kern = win ? (sm ? tc_fwd_kernel<0, true, true> : tc_fwd_kernel<0, false, true>)
+                   : (sm ? tc_fwd_kernel<0, true, false> : tc_fwd_kernel<0, false, false>);
     } else if (bias == 1) {
-        kern = sm ? tc_fwd_kernel<1, true> : tc_fwd_kernel<1, false>;
+        kern = win ? (sm ? tc_fwd_kernel<1, true, true> : tc_fwd_kernel<1, false, true>)
+                   : (sm ? tc_fwd_kernel<1, true, false> : tc_fwd_kernel<1, false, false>);
     } else {
-        kern = sm ? tc_fwd_kernel<2, true> : tc_fwd_kernel<2, false>;
+        kern = win ? (sm ? tc_fwd_kernel<2, true, true> : tc_fwd_kernel<2, false, true>)
+                   : (sm ? tc_fwd_kernel<2, true, false> : tc_fwd_kernel<2, false, false>);
     }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return e;

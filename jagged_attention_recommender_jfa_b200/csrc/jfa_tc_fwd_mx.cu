@@ -169,7 +169,8 @@ __device__ __forceinline__ int item_of_turn(int r, int c, int G) {
 
 struct Item {
     int b, h, row0, q0, nq, k0, nkv;
-    int n_t[2];
+    int jb;       // first key tile of the block (0 unless a sliding window starts later)
+    int n_t[2];   // key tiles of tile A and tile B from jb
     int n;
 };
 
@@ -183,6 +184,9 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     w.nq = a.q_off[w.b + 1] - w.q0;
     w.k0 = a.kv_off[w.b];
     w.nkv = a.kv_off[w.b + 1] - w.k0;
+    // both tiles stream the key tiles from the one tile A's first row needs
+    // (96-key tiles keep the MX blocks of V aligned to the sequence start)
+    w.jb = vis_key_lo(a.window, w.row0, w.nq, w.nkv) / BN;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int lo = w.row0 + t * BM, hi = min(lo + BM, w.nq);
@@ -190,9 +194,8 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
             w.n_t[t] = 0;
             continue;
         }
-        int kv_end = a.causal ? min(w.nkv, hi + (w.nkv - w.nq)) : w.nkv;
-        kv_end = max(kv_end, 0);
-        w.n_t[t] = (kv_end + BN - 1) / BN;
+        const int kv_end = vis_key_hi(a.causal, a.window, hi - 1, w.nq, w.nkv) + 1;
+        w.n_t[t] = max((kv_end + BN - 1) / BN - w.jb, 0);
     }
     w.n = max(w.n_t[0], w.n_t[1]);
     return w;
@@ -342,14 +345,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
             for (int j = 0; j < w.n; ++j, ++g) {
                 const int s = g % NS;
                 const uint32_t par = ((g / NS) - 1) & 1;
-                const int z = w.k0 + j * BN;
+                const int jt = w.jb + j;   // key tile of the sequence
+                const int z = w.k0 + jt * BN;
                 if (g >= NS && !wwait(&bars->k_empty[s], par)) { ok = false; break; }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars->k_full[s], kKVTile);
                     tma_load_3d(smem + kOffK + s * kKVTile, &P.tm_k, &bars->k_full[s], 0, w.h, z);
                 }
                 {
-                    const uint4 sf = sf_rows4(P.ks, z, max(0, min(BN, w.nkv - j * BN)), P.total_kv, a.H, w.h, lane);
+                    const uint4 sf = sf_rows4(P.ks, z, max(0, min(BN, w.nkv - jt * BN)), P.total_kv, a.H, w.h, lane);
                     *reinterpret_cast<uint4*>(smem + kOffSfK + s * kSfChunk + lane * 16) = sf;
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -361,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                     tma_load_3d(smem + kOffV + s * kKVTile, &P.tm_v, &bars->v_full[s], 0, w.h, z);
                     if (BIAS == 1) {
                         const int C = (a.relpos_len - 1) >> 1;
-                        const int w0 = bias_window_start(w.row0, j * BN, C, a.bias4_stride);
+                        const int w0 = bias_window_start(w.row0, jt * BN, C, a.bias4_stride);
                         const float* src = a.bias4 + 4 * ((int64_t)w.h * a.bias4_stride + w0);
                         mbar_arrive_expect_tx(&bars->bias_full[s], kWinBytes);
                         bulk_load(smem + kOffBias + s * kWinBytes, src, kWinBytes, &bars->bias_full[s]);
@@ -372,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                     }
                 }
                 {
-                    const uint4 sf = sf_v(P.vs, (int64_t)P.vbase[w.b] + 3 * j, nblk - 3 * j, a.H, w.h, lane);
+                    const uint4 sf = sf_v(P.vs, (int64_t)P.vbase[w.b] + 3 * jt, nblk - 3 * jt, a.H, w.h, lane);
                     *reinterpret_cast<uint4*>(smem + kOffSfV + s * kSfChunk + lane * 16) = sf;
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -515,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                 }
                 continue;
             }
-            const int shift = w.nkv - w.nq;
-            const int jmax_vis = a.causal ? min(w.nkv - 1, i + shift) : w.nkv - 1;
+            const int jmax_vis = vis_key_hi(a.causal, a.window, i, w.nq, w.nkv);
+            const int jmin_vis = vis_key_lo(a.window, i, w.nq, w.nkv);
             const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)w.h * 4 * a.bias4_stride : nullptr;
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
@@ -525,11 +529,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
             for (int j = 0; j < n; ++j, ++gt) {
                 if (!wwait(&bars->s_full[tt], gt & 1)) { ok = false; break; }
                 tc_fence_after();
-                const int jc = j * BN;
+                const int jc = (w.jb + j) * BN;
                 const int gk = gkv_item + j, sk = gk % NS;
                 if (BIAS == 1 && !wwait(&bars->bias_full[sk], (gk / NS) & 1)) { ok = false; break; }
-                const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;
-                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW);
+                const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;   // visible: [nlo, nvis)
+                const int nlo = jmin_vis - jc;
+                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW || nlo > cb);
                 const int lo = i - jc - (BN - 1) + C;
                 const int wrel = BIAS == 1 ? lo - bias_window_start(w.row0, jc, C, a.bias4_stride) : 0;
                 const bool win_ok = BIAS == 1 && lo >= 0 && lo + (BN - 1) <= 2 * C && wrel >= 0 && wrel + BN - 4 < kWin;
@@ -587,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                     }
                     if (masked_half) {
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) x[v] = cc + v < nvis ? x[v] : -CUDART_INF_F;
+                        for (int v = 0; v < 16; ++v) x[v] = (cc + v < nvis && cc + v >= nlo) ? x[v] : -CUDART_INF_F;
                     }
                     const float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
                     const float m2 = max3(x[6], x[7], x[8]), m3 = max3(x[9], x[10], x[11]);

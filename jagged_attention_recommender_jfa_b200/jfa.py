@@ -57,7 +57,8 @@ class jfa_problem(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("max_q_len", ctypes.c_int32),
                 ("max_kv_len", ctypes.c_int32), ("total_q", ctypes.c_int64),
                 ("total_kv", ctypes.c_int64), ("dtype", ctypes.c_int), ("scale", ctypes.c_float),
-                ("bias_kind", ctypes.c_int), ("relpos_len", ctypes.c_int32)]
+                ("bias_kind", ctypes.c_int), ("relpos_len", ctypes.c_int32),
+                ("window", ctypes.c_int32)]
 
 
 def lib_path() -> str:
@@ -138,18 +139,20 @@ def _check(status: int):
 
 
 def make_problem(*, batch, heads, head_dim, max_q_len, max_kv_len, total_q, total_kv,
-                 dtype="bf16", scale=0.0, bias_kind="none", relpos_len=0) -> jfa_problem:
+                 dtype="bf16", scale=0.0, bias_kind="none", relpos_len=0, window=0) -> jfa_problem:
+    """``window`` > 0: sliding window of that width (0: none)."""
     return jfa_problem(int(batch), int(heads), int(head_dim), int(max_q_len), int(max_kv_len),
                        int(total_q), int(total_kv), DTYPE[dtype] if isinstance(dtype, str) else int(dtype),
                        float(scale), BIAS[bias_kind] if isinstance(bias_kind, str) else int(bias_kind),
-                       int(relpos_len))
+                       int(relpos_len), int(window))
 
 
-def problem_of(p, dtype: Optional[str] = None) -> jfa_problem:
+def problem_of(p, dtype: Optional[str] = None, window: int = 0) -> jfa_problem:
     """Descriptor of an ``inputs.Problem`` batch."""
     return make_problem(batch=p.B, heads=p.H, head_dim=p.d, max_q_len=p.max_q_len,
                         max_kv_len=p.max_kv_len, total_q=p.total_q, total_kv=p.total_kv,
-                        dtype=dtype or p.dtype, bias_kind=p.bias_kind, relpos_len=p.relpos_len)
+                        dtype=dtype or p.dtype, bias_kind=p.bias_kind, relpos_len=p.relpos_len,
+                        window=window)
 
 
 # ---------------------------------------------------------------------------
