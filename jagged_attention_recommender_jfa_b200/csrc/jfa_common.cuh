@@ -31,7 +31,7 @@ struct WsHeader {
     int32_t queue;
     int32_t kv_item_count;
     int32_t kv_pair_count;
-    int32_t kv_queue;
+    int32_t kv_queue;        // next work item of the persistent key-tile backward
     int32_t wait_limit_us;   // bounded device waits give up after this (0: 1 s)
     int32_t pad[56];
 };

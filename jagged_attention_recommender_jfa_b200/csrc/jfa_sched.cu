@@ -73,6 +73,7 @@ sched_prepare(const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_
     const int tid = threadIdx.x;
     if (tid == 0) {
         s_bad = 0;
+        if (backward) hdr->kv_queue = 0;   // work-item counter of the persistent backward
         if (reset_err) {
             hdr->err = 0;
             hdr->wait_limit_us = wait_limit_us;

@@ -549,3 +549,25 @@ def test_mxfp8_prequantised_entry_matches(cuda_device):
         jfa.jfa_forward_mxfp8(jfa.problem_of(p, dtype="bf16"), q8, qs, k8, ks, v8, vs, d["q_off"],
                               d["kv_off"], d["bias"], True, out, lse, ws)
     assert ei.value.status == jfa.JFA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# the general backward's query tiles start at the first query that sees a key
+# tile: on 128-row block boundaries for self-attention and for n_kv - n_q a
+# multiple of 128, anywhere otherwise
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("q_lens,kv_lens,causal", [
+    ([300, 128, 1, 700, 129], [300, 128, 1, 700, 129], True),     # self-attention
+    ([300, 100, 3], [428, 356, 259], True),                        # n_kv - n_q = 128, 256
+    ([300, 100], [305, 100], True),                                # n_kv - n_q = 5
+    ([90, 200], [400, 30], False),
+    ([50, 0, 100], [50, 0, 0], True),                              # a sequence without keys
+])
+def test_backward_query_tile_offsets(cuda_device, q_lens, kv_lens, causal):
+    p = make_problem("self_bf16", 70, q_lens=q_lens, kv_lens=kv_lens, causal=causal)
+    out, lse, (dq, dk, dv) = run_gpu(p, cuda_device, "softmax")
+    ro, rl, (rdq, rdk, rdv) = run_oracle(p, "softmax")
+    compare("O", out, ro, slice(None), BF16_MAX, BF16_MEAN)
+    compare("dQ", dq, rdq, slice(None), BF16_MAX, BF16_MEAN)
+    compare("dK", dk, rdk, slice(None), BF16_MAX, BF16_MEAN)
+    compare("dV", dv, rdv, slice(None), BF16_MAX, BF16_MEAN)
