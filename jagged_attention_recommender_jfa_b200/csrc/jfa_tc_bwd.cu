@@ -84,7 +84,8 @@ constexpr uint32_t kOffEnd = kOffDb + 2 * kDbWin * 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Bars {
-    uint64_t kv_full;
+    uint64_t k_full, v_full;   // the item's K / V tile loaded
+    uint64_t k_free, v_free;   // the item's last MMA reading K (dQ^T) / V (dP^T) retired
     uint64_t buf_full[3], buf_empty[3];   // the Q / dO ring
     uint64_t s_full;
     uint64_t ds_half;       // 16 score warps: queries 0..63 of the tile done
@@ -220,7 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
     constexpr bool softmax = SOFTMAX;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->kv_full, 1);
+        mbar_init(&bars->k_full, 1);
+        mbar_init(&bars->v_full, 1);
+        mbar_init(&bars->k_free, 1);
+        mbar_init(&bars->v_free, 1);
         for (int s3 = 0; s3 < 3; ++s3) {
             mbar_init(&bars->buf_full[s3], 1);
             mbar_init(&bars->buf_empty[s3], 1);
@@ -297,13 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     tma_prefetch_l2_3d(&P.tm_do, 0, w.h, zq);
                     tma_prefetch_l2_3d(&P.tm_do, 64, w.h, zq);
                 }
-                // K and V replace the previous item's once its MMAs have retired
-                if (kf > 0 && !mbar_wait(&bars->fin, (kf - 1) & 1, abort_flag, a.hdr)) break;
-                mbar_arrive_expect_tx(&bars->kv_full, 2 * kTile);
-                tma_load_3d(smem + kOffK, &P.tm_k, &bars->kv_full, 0, w.h, w.k0 + w.j0);
-                tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->kv_full, 64, w.h, w.k0 + w.j0);
-                tma_load_3d(smem + kOffV, &P.tm_v, &bars->kv_full, 0, w.h, w.k0 + w.j0);
-                tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->kv_full, 64, w.h, w.k0 + w.j0);
+                // V replaces the previous item's once its last dP^T has retired,
+                // K once its last dQ^T has (both ahead of the item's last dK, dV)
+                if (kf > 0 && !mbar_wait(&bars->v_free, (kf - 1) & 1, abort_flag, a.hdr)) break;
+                mbar_arrive_expect_tx(&bars->v_full, kTile);
+                tma_load_3d(smem + kOffV, &P.tm_v, &bars->v_full, 0, w.h, w.k0 + w.j0);
+                tma_load_3d(smem + kOffV + kBox, &P.tm_v, &bars->v_full, 64, w.h, w.k0 + w.j0);
+                if (kf > 0 && !mbar_wait(&bars->k_free, (kf - 1) & 1, abort_flag, a.hdr)) break;
+                mbar_arrive_expect_tx(&bars->k_full, kTile);
+                tma_load_3d(smem + kOffK, &P.tm_k, &bars->k_full, 0, w.h, w.k0 + w.j0);
+                tma_load_3d(smem + kOffK + kBox, &P.tm_k, &bars->k_full, 64, w.h, w.k0 + w.j0);
                 ++kf;
                 // load n of the item is ring load N = issued: Q(n/2) (with a
                 // relative-position bias also the tile's bias window) or dO(n/2);
@@ -341,7 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 gtile += w.nt;
             }
             // never leave the CTA with copies in flight
-            if (kf > 0) mbar_wait_drain(&bars->kv_full, (kf - 1) & 1, a.hdr);
+            if (kf > 0) {
+                mbar_wait_drain(&bars->v_full, (kf - 1) & 1, a.hdr);
+                mbar_wait_drain(&bars->k_full, (kf - 1) & 1, a.hdr);
+            }
             for (int n = issued > 3 ? issued - 3 : 0; n < issued; ++n)
                 mbar_wait_drain(&bars->buf_full[n % 3], (n / 3) & 1, a.hdr);
             if (BIAS == 1) {
@@ -406,13 +416,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const BItem w = load_bitem<WINDOW>(a, idx);
                 if (w.nt == 0) continue;
                 // dP^T of the first tile overwrites the previous item's last dQ^T
-                ok = mbar_wait(&bars->kv_full, kf & 1, abort_flag, a.hdr) && wait_load(2 * gtile) &&
-                     wait_load(2 * gtile + 1) &&
-                     (gtile == 0 || mbar_wait(&bars->dq_empty, (gtile - 1) & 1, abort_flag, a.hdr));
+                ok = mbar_wait(&bars->k_full, kf & 1, abort_flag, a.hdr) && wait_load(2 * gtile);
                 if (!ok) break;
                 tc_fence_after();
                 issue_s(gtile);
+                ok = mbar_wait(&bars->v_full, kf & 1, abort_flag, a.hdr) && wait_load(2 * gtile + 1) &&
+                     (gtile == 0 || mbar_wait(&bars->dq_empty, (gtile - 1) & 1, abort_flag, a.hdr));
+                if (!ok) break;
+                tc_fence_after();
                 issue_dp(gtile);
+                if (w.nt == 1) mma_commit(&bars->v_free);
                 mma_commit(&bars->s_full);
                 for (int t = 0; ok && t < w.nt; ++t) {
                     const int gt = gtile + t;
@@ -436,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     for (int k = 0; k < BN / 16; ++k)
                         mma_bf16_ss(tdP, mnmajor_desc(kM, k), mnmajor_desc(dsM, k), idesc_tn, k > 0 ? 1u : 0u);
                     mma_commit(&bars->dq_full);
+                    if (t + 1 == w.nt) mma_commit(&bars->k_free);   // the item's last use of K
                     issue_dk(gt, t, 4);
                     mma_commit(&bars->buf_empty[(2 * gt) % 3]);
                     issue_dv(gt, t, 4);
@@ -454,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                         JFA_TRACE_EV(bwd, 1, gt, 3);
                         tc_fence_after();
                         issue_dp(gt + 1);
+                        if (t + 2 == w.nt) mma_commit(&bars->v_free);   // the item's last use of V
                         mma_commit(&bars->s_full);
                     }
                 }
@@ -482,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
         const float sc = a.scale * kLog2e;
         const int C = (a.relpos_len - 1) >> 1;
         const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
-        const bool kv32 = ((reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) & 31) == 0;
         const int sw = warp - 2;
         bool ok = true;
         int kf = 0, gtile = 0;
@@ -494,12 +508,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
             if (lane == 0) mbar_arrive(&bars->item_empty[slot]);
             if (idx < 0) break;
             const BItem w = load_bitem<WINDOW>(a, idx);
-            const int h = w.h, j0 = w.j0, q0 = w.q0, nq = w.nq, nkv = w.nkv, shift = w.shift;
+            const int h = w.h, j0 = w.j0, q0 = w.q0, nq = w.nq, nkv = w.nkv;
             const int i_start = w.i_start, nt = w.nt;
             const int j = j0 + r;                    // key index within the sequence
             const bool jvalid = j < nkv;
             const int k0 = w.k0;
             // this thread's 32 columns of its dK and dV rows
+            auto kv32 = [&]() {
+                return ((reinterpret_cast<uintptr_t>(a.dk) | reinterpret_cast<uintptr_t>(a.dv)) & 31) == 0;
+            };
             auto grad_rows = [&](__nv_bfloat16*& dkrow, __nv_bfloat16*& dvrow) {
                 const int64_t o = ((int64_t)(k0 + j) * a.H + h) * HD + cofs;
                 dkrow = reinterpret_cast<__nv_bfloat16*>(a.dk) + o;
@@ -515,17 +532,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                     for (int e = 0; e < 16; ++e) z[e] = 0u;
 #pragma unroll
                     for (int e = 0; e < 32; e += 16) {
-                        store_bf16x16(dkrow + e, z, 1.0f, kv32);
-                        store_bf16x16(dvrow + e, z, 1.0f, kv32);
+                        store_bf16x16(dkrow + e, z, 1.0f, kv32());
+                        store_bf16x16(dvrow + e, z, 1.0f, kv32());
                     }
                 }
                 continue;
             }
             const float inv_n = nkv > 0 ? 1.0f / (float)nkv : 0.f;
-            // log2(e)-scaled table: entry t at tab4[4 t]
-            const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)h * 4 * a.bias4_stride : nullptr;
             const int64_t dense_base = (BIAS == 2) ? a.dense_off[w.b] + (int64_t)h * nq * nkv : 0;
-            float* dq_col = a.dq_acc + ((int64_t)q0 * a.H + h) * HD + r;   // + qi * H * HD
             // LSE (log2 units) and D of a query tile: group 0 stages them into one
             // of two buffers a tile ahead (rows_full), every warp releases the
             // buffer after reading it (rows_free); buffers by the CTA's tile gt
@@ -613,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 const float4* win = reinterpret_cast<const float4*>(smem + kOffWin + buf * kWinBytes);
                 // queries imin_vis .. imax_vis see key j
                 const int imin_vis = WINDOW ? vis_query_lo(a.causal, a.window, j, nq, nkv)
-                                            : (a.causal ? j - shift : 0);
+                                            : (a.causal ? j - (nkv - nq) : 0);
                 const int imax_vis = WINDOW ? vis_query_hi(a.window, j, nq, nkv) : nq - 1;
                 // one 16-column part: scores u (TMEM bits) -> P in place, dP g -> dS in place
                 auto process = [&](uint32_t (&u)[16], uint32_t (&g)[16], int c16) {
@@ -639,6 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                             }
                         } else {
     #pragma unroll
+                            // log2(e)-scaled table of head h: entry t at tab4[4 t]
+                            const float* tab4 = a.bias4 + (int64_t)h * 4 * a.bias4_stride;
                             for (int v = 0; v < 16; ++v) bb[v] = __ldg(tab4 + 4 * min(max(s0 + v, 0), 2 * C));
                         }
     #pragma unroll
@@ -782,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 SC_EV(5);
                 {
                     const int qc = qb0 + grp * 32;
-                    float* dst = dq_col + (int64_t)qc * a.H * HD;
+                    float* dst = a.dq_acc + ((int64_t)(q0 + qc) * a.H + h) * HD + r;
                     const int64_t stride = (int64_t)a.H * HD;
                     const int nvalid = min(32, nq - qc);   // warp-uniform
     #pragma unroll
@@ -810,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_bwd_kernel(const __grid_consta
                 grad_rows(dkrow, dvrow);
 #pragma unroll
                 for (int e = 0; e < 32; e += 16) {
-                    store_bf16x16(dkrow + e, uk + e, a.scale, kv32);
-                    store_bf16x16(dvrow + e, uv + e, 1.0f, kv32);
+                    store_bf16x16(dkrow + e, uk + e, a.scale, kv32());
+                    store_bf16x16(dvrow + e, uv + e, 1.0f, kv32());
                 }
             }
             gtile += nt;
