@@ -75,7 +75,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
 
 struct Bars {
-    uint64_t q_full, q_free;
+    uint64_t q_full[2], q_free[2];   // per tile slot
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
     uint64_t s_full[2];    // per tile
@@ -146,13 +146,18 @@ __device__ __forceinline__ void dense_bias16(const __nv_bfloat16* p, float (&bb)
 
 struct Item {
     int b, h, row0, q0, nq, k0, nkv;
+    int sw;       // tile slot t holds the rows row0 + (t ^ sw) * 128 .. +127
     int jb;       // first key tile of the block (0 unless a sliding window starts later)
-    int n_t[2];   // key tiles of tile A and tile B from jb (0: the tile has no rows or sees no key)
+    int n_t[2];   // key tiles of slots A and B from jb (0: the slot has no rows or sees no key)
     int n;        // key tiles of the block
 };
 
+// The CTA's odd items swap the slots' rows: under the causal rule the lower
+// 128 rows take one key tile more than the upper ones, and alternating which
+// slot has the extra key tile lets each slot start its next item a key tile
+// early every other item (see the MMA thread).
 template <bool WINDOW>
-__device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
+__device__ __forceinline__ Item load_item(const AttnArgs& a, int idx, int sw) {
     const int4 it = a.items[idx];
     Item w;
     w.b = it.x;
@@ -165,10 +170,11 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     // both tiles stream the key tiles from the one tile A's first row needs
     // (tile B's rows see the same or later keys; a key tile of the band that
     // B does not see is masked for it)
+    w.sw = sw;
     w.jb = WINDOW ? vis_key_lo(a.window, w.row0, w.nq, w.nkv) / BN : 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const int lo = w.row0 + t * BM, hi = min(lo + BM, w.nq);
+        const int lo = w.row0 + (t ^ sw) * BM, hi = min(lo + BM, w.nq);
         if (hi <= lo) {
             w.n_t[t] = 0;
             continue;
@@ -216,8 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
     constexpr bool softmax = SOFTMAX;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars->q_full, 1);
-        mbar_init(&bars->q_free, 1);
+        mbar_init(&bars->q_full[0], 1);
+        mbar_init(&bars->q_free[0], 1);
+        mbar_init(&bars->q_full[1], 1);
+        mbar_init(&bars->q_free[1], 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
@@ -251,22 +259,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
             tma_prefetch_desc(&P.tm_q);
             tma_prefetch_desc(&P.tm_k);
             tma_prefetch_desc(&P.tm_v);
-            int g = 0, nk = 0;        // key tiles issued, items with keys
+            int g = 0;                // key tiles issued
+            int nq[2] = {0, 0};       // Q tiles issued per slot (items where the slot sees keys)
             bool ok = true;
+            // Q of a slot replaces the slot's previous one once that item's last
+            // Q K^T of the slot has retired.  The slot that ended the previous
+            // item a key tile early (its first score MMA of this item goes out
+            // then) gets its Q before the item's first key tile, the other one
+            // after it.
+            auto load_q = [&](const Item& w, int t) -> bool {
+                if (w.n_t[t] == 0) return true;
+                if (nq[t] > 0 && !mbar_wait(&bars->q_free[t], (nq[t] - 1) & 1, abort_flag, a.hdr)) return false;
+                const int z = w.q0 + w.row0 + (t ^ w.sw) * BM;
+                mbar_arrive_expect_tx(&bars->q_full[t], kTile);
+                tma_load_3d(smem + kOffQ + t * kTile, &P.tm_q, &bars->q_full[t], 0, w.h, z);
+                tma_load_3d(smem + kOffQ + t * kTile + kBox, &P.tm_q, &bars->q_full[t], 64, w.h, z);
+                ++nq[t];
+                return true;
+            };
+            int early = 0;
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
-                const Item w = load_item<WINDOW>(a, idx);
+                const Item w = load_item<WINDOW>(a, idx, r & 1);
                 if (w.n == 0) continue;
-                if (nk > 0 && !mbar_wait(&bars->q_free, (nk - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                mbar_arrive_expect_tx(&bars->q_full, 2 * kTile);
-                for (int t = 0; t < 2; ++t) {
-                    const int z = w.q0 + w.row0 + t * BM;
-                    tma_load_3d(smem + kOffQ + t * kTile, &P.tm_q, &bars->q_full, 0, w.h, z);
-                    tma_load_3d(smem + kOffQ + t * kTile + kBox, &P.tm_q, &bars->q_full, 64, w.h, z);
-                }
-                ++nk;
+                if (!load_q(w, early)) { ok = false; break; }
                 for (int j = 0; j < w.n; ++j, ++g) {
+                    if (j == 1 && !load_q(w, early ^ 1)) { ok = false; break; }
                     const int s = g & 1;
                     const uint32_t par = ((g >> 1) - 1) & 1;
                     const int z = w.k0 + (w.jb + j) * BN;
@@ -301,9 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                         tma_prefetch_l2_3d(&P.tm_v, 64, w.h, z + 2 * BN);
                     }
                 }
+                if (ok && w.n == 1 && !load_q(w, early ^ 1)) { ok = false; break; }
+                early = (w.n_t[1] == w.n - 1 && w.n_t[0] == w.n) ? 1 : 0;
             }
             // never leave the CTA with copies in flight: wait for the last loads
-            if (nk > 0) mbar_wait_drain(&bars->q_full, (nk - 1) & 1, a.hdr);
+            for (int t = 0; t < 2; ++t)
+                if (nq[t] > 0) mbar_wait_drain(&bars->q_full[t], (nq[t] - 1) & 1, a.hdr);
             for (int t = (g > 2 ? g - 2 : 0); t < g; ++t) {
                 mbar_wait_drain(&bars->k_full[t & 1], (t >> 1) & 1, a.hdr);
                 mbar_wait_drain(&bars->v_full[t & 1], (t >> 1) & 1, a.hdr);
@@ -315,54 +337,67 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(BM, HD, 0, 1);
-            int g = 0, nk = 0;
-            int gt[2] = {0, 0}, mt[2] = {0, 0};
+            int g = 0;
+            int gt[2] = {0, 0}, mt[2] = {0, 0}, nq[2] = {0, 0};   // steps, items, Q tiles per slot
             bool ok = true;
             // descriptor lower words of every operand tile, computed once
             const uint32_t qK0 = kmajor_lo(sbase + kOffQ), qK1 = kmajor_lo(sbase + kOffQ + kTile);
             const uint32_t kK0 = kmajor_lo(sbase + kOffK), kK1 = kmajor_lo(sbase + kOffK + kTile);
             const uint32_t vM0 = mnmajor_lo(sbase + kOffV), vM1 = mnmajor_lo(sbase + kOffV + kTile);
+            // user of key/value step j of an item: slot A while j < n_A, slot B while j < n_B
+            auto first_user = [](const Item& w, int j) { return j < w.n_t[0] ? 0 : 1; };
+            auto last_user = [](const Item& w, int j) { return j < w.n_t[1] ? 1 : 0; };
+            // S_T = Q_T K_j^T into S_T for step j of item w (first key tile g0).
+            // The first score MMA on a key tile waits for its load and the last
+            // releases the stage (wait_k / release_k); Q_T is released by the
+            // slot's last score MMA of the item (its first waits for Q_T).
+            auto issue_qk = [&](const Item& w, int g0, int t, int j, bool wait_k, bool release_k) -> bool {
+                const int gg = g0 + j, s = gg & 1;
+                if (j == 0) {
+                    if (!mbar_wait(&bars->q_full[t], nq[t] & 1, abort_flag, a.hdr)) return false;
+                    ++nq[t];
+                }
+                if (wait_k) {
+                    if (!mbar_wait(&bars->k_full[s], (gg >> 1) & 1, abort_flag, a.hdr)) return false;
+                    JFA_TRACE_EV(fwd, 1, gg, 0);
+                }
+                tc_fence_after();
+                const uint32_t qd = t ? qK1 : qK0, kd = s ? kK1 : kK0;
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    mma_bf16_ss(tmem + t * 128, kmajor_desc(qd, k), kmajor_desc(kd, k), idesc_qk, k > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full[t]);
+                if (release_k) mma_commit(&bars->k_empty[s]);
+                if (j == w.n_t[t] - 1) mma_commit(&bars->q_free[t]);
+                return true;
+            };
+            // in item order the first user issues first and the last releases
+            auto issue_qk_ordered = [&](const Item& w, int g0, int t, int j) -> bool {
+                return issue_qk(w, g0, t, j, t == first_user(w, j), t == last_user(w, j));
+            };
+            int early = -1;   // slot whose first score MMA of this item went out during the previous one
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
-                const Item w = load_item<WINDOW>(a, idx);
+                const Item w = load_item<WINDOW>(a, idx, r & 1);
                 if (w.n == 0) continue;
-                if (!mbar_wait(&bars->q_full, nk & 1, abort_flag, a.hdr)) { ok = false; break; }
-                ++nk;
-                // user of key/value step j: tile A while j < n_A, tile B while j < n_B
-                auto first_user = [&](int j) { return j < w.n_t[0] ? 0 : 1; };
-                auto last_user = [&](int j) { return j < w.n_t[1] ? 1 : 0; };
                 const int g0 = g;
-                // S_T = Q_T K_j^T into S_T; the K stage is released by its last user,
-                // Q by the item's last score MMA
-                auto issue_qk = [&](int t, int j) -> bool {
-                    const int gg = g0 + j, s = gg & 1;
-                    if (t == first_user(j)) {
-                        if (!mbar_wait(&bars->k_full[s], (gg >> 1) & 1, abort_flag, a.hdr)) return false;
-                        JFA_TRACE_EV(fwd, 1, gg, 0);
-                    }
-                    tc_fence_after();
-                    const uint32_t qd = t ? qK1 : qK0, kd = s ? kK1 : kK0;
-#pragma unroll
-                    for (int k = 0; k < HD / 16; ++k)
-                        mma_bf16_ss(tmem + t * 128, kmajor_desc(qd, k), kmajor_desc(kd, k), idesc_qk, k > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full[t]);
-                    if (t == last_user(j)) mma_commit(&bars->k_empty[s]);
-                    if (j == w.n - 1 && t == last_user(j)) mma_commit(&bars->q_free);
-                    return true;
-                };
+                // after an early slot's score MMA on the item's first key tile the
+                // other slot's comes second: it releases the stage
                 for (int t = 0; t < 2 && ok; ++t)
-                    if (w.n_t[t] > 0) ok = issue_qk(t, 0);
+                    if (w.n_t[t] > 0 && t != early)
+                        ok = early >= 0 ? issue_qk(w, g0, t, 0, true, true) : issue_qk_ordered(w, g0, t, 0);
+                early = -1;
                 for (int j = 0; ok && j < w.n; ++j, ++g) {
                     const int s = g & 1;
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (j >= w.n_t[t]) continue;
                         if (!mbar_wait(&bars->p_full[t], gt[t] & 1, abort_flag, a.hdr)) { ok = false; break; }
                         JFA_TRACE_EV(fwd, 1, g, 1 + 2 * t);
-                        // the epilogue of this tile's previous item must be done with O_T
+                        // the epilogue of this slot's previous item must be done with O_T
                         if (j == 0 && mt[t] > 0 &&
                             !mbar_wait(&bars->o_free[t], (mt[t] - 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
-                        if (t == first_user(j) &&
+                        if (t == first_user(w, j) &&
                             !mbar_wait(&bars->v_full[s], (g >> 1) & 1, abort_flag, a.hdr)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t vd = s ? vM1 : vM0;
@@ -373,12 +408,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
                             mma_bf16_ts(tO, tP + k * 8 + (k >= 4 ? 32 : 0), mnmajor_desc(vd, k), idesc_pv,
                                         (j > 0 || k > 0) ? 1u : 0u);
                         mma_commit(&bars->pv_done[t]);
-                        if (t == last_user(j)) mma_commit(&bars->v_empty[s]);
+                        if (t == last_user(w, j)) mma_commit(&bars->v_empty[s]);
                         JFA_TRACE_EV(fwd, 1, g, 2 + 2 * t);
                         ++gt[t];
                         if (j == 0) ++mt[t];
                         // S_T(j+1) overwrites P_T(j): issued after the P.V that reads it
-                        if (j + 1 < w.n_t[t]) ok = issue_qk(t, j + 1);
+                        if (j + 1 < w.n_t[t]) ok = issue_qk_ordered(w, g0, t, j + 1);
+                    }
+                    // A slot with one key tile fewer than the other ends the item a
+                    // step early: its first score MMA of the next item goes out now,
+                    // while the other slot works on the item's last key tile.  Its
+                    // Q and key tile need only releases issued above (the slot's Q by
+                    // its last score MMA a step earlier, the key stage by both
+                    // slots' score MMAs a step earlier and their P.V just now).
+                    for (int es = 0; es < 2 && ok; ++es) {
+                        if (j != w.n_t[es] - 1 || j + 2 != w.n || w.n_t[es ^ 1] != w.n) continue;
+                        for (int r2 = r + 1;; ++r2) {
+                            const int idx2 = item_of_turn(r2, cta, G);
+                            if (idx2 >= n_items) break;
+                            const Item w2 = load_item<WINDOW>(a, idx2, r2 & 1);
+                            if (w2.n == 0) continue;
+                            if (w2.n_t[es] > 0) {
+                                // issued before the other slot's: it waits for the
+                                // load, and releases the stage only as sole user
+                                ok = issue_qk(w2, g0 + w.n, es, 0, true, w2.n_t[es ^ 1] == 0);
+                                early = es;
+                            }
+                            break;
+                        }
                     }
                 }
             }
@@ -427,11 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_kernel(const __grid_consta
         for (int rr = 0; ok; ++rr) {
             const int idx = item_of_turn(rr, cta, G);
             if (idx >= n_items) break;
-            const Item w = load_item<WINDOW>(a, idx);
+            const Item w = load_item<WINDOW>(a, idx, rr & 1);
             const int n = w.n_t[tt];
             const int gkv_item = gkv;
             gkv += w.n;
-            const int i = w.row0 + tt * BM + r_;   // query index within the sequence
+            const int i = w.row0 + (tt ^ w.sw) * BM + r_;   // query index within the sequence
             if (n == 0) {
                 // rows that see no key (no keys at all, or causal with n_q > n_kv):
                 // zero output, LSE = -inf; the tensor core never touches this tile
