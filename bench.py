@@ -615,7 +615,7 @@ def main():
     else:
         gq, gk = draw_lengths(args.workload, args.seed, B=8 * p.B, max_len=args.max_len)
         result["partition_8_ranks"] = {
-            m: split_report(gq, gk, p.causal, 8, m, args.sub_batch, jfa)[1] for m in ("bbs", "lpt")}
+            m: split_report(gq, gk, p.causal, 8, m, args.sub_batch, jfa, args.window)[1] for m in ("bbs", "lpt")}
 
     # end to end through the C ABI with host buffers
     if not args.no_e2e:
@@ -632,13 +632,13 @@ def main():
         dist.destroy_process_group()
 
 
-def split_report(q_lens, kv_lens, causal, ranks, method, sub_batch, jfa):
+def split_report(q_lens, kv_lens, causal, ranks, method, sub_batch, jfa, window=0):
     """Rank imbalance (heaviest rank's visible pairs / mean) of the chosen
     split and of a contiguous split (rank r takes the r-th run of B/N)."""
-    rank_of, cost = jfa.jfa_partition(q_lens, kv_lens, causal, ranks, method, sub_batch)
+    rank_of, cost = jfa.jfa_partition(q_lens, kv_lens, causal, ranks, method, sub_batch, window)
     per = len(q_lens) // ranks
     contiguous = np.minimum(np.arange(len(q_lens)) // max(per, 1), ranks - 1).astype(np.int32)
-    pairs = visible_pairs(q_lens, kv_lens, causal)
+    pairs = visible_pairs(q_lens, kv_lens, causal, 0, window)
     c_cost = np.bincount(contiguous, weights=pairs, minlength=ranks)
     imb = lambda c: float(np.max(c) / np.mean(c)) if np.mean(c) > 0 else 1.0
     return rank_of, {"method": method, "sub_batch": sub_batch if method == "bbs" else None,
@@ -659,7 +659,7 @@ def rank_problem(args, rank, world, jfa):
     q_lens, kv_lens = draw_lengths(args.workload, args.seed, B=B * world, max_len=args.max_len)
     causal = WORKLOADS[args.workload]["causal"]
     rank_of, report = split_report(q_lens, kv_lens, causal, world, args.partition,
-                                   args.sub_batch, jfa)
+                                   args.sub_batch, jfa, args.window)
     mine = np.nonzero(rank_of == rank)[0]
     p = make_problem(args.workload, args.seed + 1 + rank, q_lens=q_lens[mine],
                      kv_lens=kv_lens[mine], max_len=args.max_len, bias=args.bias)

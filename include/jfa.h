@@ -301,8 +301,8 @@ jfa_status jfa_block_offsets(const int32_t* offsets, int32_t batch, int64_t tota
  * Returns JFA_ERR_INVALID_ARGUMENT for a bad size, pointer or method. */
 typedef enum { JFA_PARTITION_LPT = 0, JFA_PARTITION_BBS = 1 } jfa_partition_method;
 jfa_status jfa_partition(int32_t batch, const int32_t* q_lens, const int32_t* kv_lens, int causal,
-                         int32_t ranks, int method, int32_t sub_batch, int32_t* rank_of,
-                         int64_t* rank_cost);
+                         int32_t window, int32_t ranks, int method, int32_t sub_batch,
+                         int32_t* rank_of, int64_t* rank_cost);
 
 /* Synchronises `stream`, then reads and clears the workspace's device error
  * word: JFA_OK, JFA_ERR_BAD_OFFSETS or JFA_ERR_TIMEOUT. */

@@ -33,9 +33,20 @@
 namespace {
 
 // Visible (query, key) pairs of one sequence; bottom-right causal: query i
-// sees keys j <= i + n_kv - n_q.
-int64_t visible_pairs(int64_t nq, int64_t nkv, int causal) {
+// sees keys j <= i + n_kv - n_q; a sliding window w > 0 keeps the keys with
+// p - j < w (and, without the causal rule, j - p < w), p = i + n_kv - n_q.
+int64_t visible_pairs(int64_t nq, int64_t nkv, int causal, int32_t window) {
     if (nq <= 0 || nkv <= 0) return 0;
+    if (window > 0) {
+        int64_t c = 0;
+        for (int64_t i = 0; i < nq; ++i) {
+            const int64_t p = i + nkv - nq;
+            const int64_t hi = std::min(nkv - 1, causal ? p : p + window - 1);
+            const int64_t lo = std::max<int64_t>(0, p - window + 1);
+            c += hi >= lo ? hi - lo + 1 : 0;
+        }
+        return c;
+    }
     if (!causal) return nq * nkv;
     const int64_t s = nkv - nq;
     if (s >= 0) return nq * (nq + 1) / 2 + nq * s;
@@ -45,10 +56,10 @@ int64_t visible_pairs(int64_t nq, int64_t nkv, int causal) {
 }  // namespace
 
 extern "C" jfa_status jfa_partition(int32_t batch, const int32_t* q_lens, const int32_t* kv_lens,
-                                    int causal, int32_t ranks, int method, int32_t sub_batch,
-                                    int32_t* rank_of, int64_t* rank_cost) {
-    if (batch < 0 || ranks < 1)
-        return jfa::set_last_error(JFA_ERR_INVALID_ARGUMENT, "batch must be >= 0 and ranks >= 1");
+                                    int causal, int32_t window, int32_t ranks, int method,
+                                    int32_t sub_batch, int32_t* rank_of, int64_t* rank_cost) {
+    if (batch < 0 || ranks < 1 || window < 0)
+        return jfa::set_last_error(JFA_ERR_INVALID_ARGUMENT, "batch, window must be >= 0 and ranks >= 1");
     if (batch > 0 && (!q_lens || !kv_lens || !rank_of))
         return jfa::set_last_error(JFA_ERR_INVALID_ARGUMENT, "NULL lengths or rank_of");
     if (method != JFA_PARTITION_LPT && method != JFA_PARTITION_BBS)
@@ -59,7 +70,7 @@ extern "C" jfa_status jfa_partition(int32_t batch, const int32_t* q_lens, const 
     for (int32_t b = 0; b < batch; ++b) {
         if (q_lens[b] < 0 || kv_lens[b] < 0)
             return jfa::set_last_error(JFA_ERR_INVALID_ARGUMENT, "negative length at %d", b);
-        cost[b] = visible_pairs(q_lens[b], kv_lens[b], causal);
+        cost[b] = visible_pairs(q_lens[b], kv_lens[b], causal, window);
     }
     std::vector<int64_t> load(ranks, 0);
     if (method == JFA_PARTITION_LPT) {

@@ -111,7 +111,7 @@ def load():
         lib.jfa_test_inject.restype = i32
         lib.jfa_block_offsets.argtypes = [P, i32, i64, i32, P, P]
         lib.jfa_block_offsets.restype = i32
-        lib.jfa_partition.argtypes = [i32, P, P, i32, i32, i32, i32, P, P]
+        lib.jfa_partition.argtypes = [i32, P, P, i32, i32, i32, i32, i32, P, P]
         lib.jfa_partition.restype = i32
         _LIB = lib
         return lib
@@ -256,9 +256,10 @@ def block_attention(problem: jfa_problem, offsets, block: int, stream=None):
     return p2, boff
 
 
-def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
+def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1, window=0):
     """Host-side split of a global batch across ``ranks``: returns (rank_of
-    int32 [batch], rank_cost int64 [ranks]) as numpy arrays."""
+    int32 [batch], rank_cost int64 [ranks]) as numpy arrays.  ``window`` > 0
+    counts a sliding window's pairs."""
     import numpy as np
     ql = np.ascontiguousarray(np.asarray(q_lens, np.int32))
     kl = np.ascontiguousarray(np.asarray(kv_lens, np.int32))
@@ -266,7 +267,7 @@ def jfa_partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
     rank_of = np.zeros(len(ql), np.int32)
     rank_cost = np.zeros(int(ranks), np.int64)
     c = lambda a: a.ctypes.data_as(ctypes.c_void_p)
-    _check(load().jfa_partition(len(ql), c(ql), c(kl), int(bool(causal)), int(ranks),
+    _check(load().jfa_partition(len(ql), c(ql), c(kl), int(bool(causal)), int(window), int(ranks),
                                 PARTITION.get(method, method), int(sub_batch), c(rank_of),
                                 c(rank_cost)))
     return rank_of, rank_cost

@@ -358,16 +358,16 @@ def valid_pairs(q_off, kv_off, causal, window=0):
 # (query, key) pairs, counted row by row.
 # ---------------------------------------------------------------------------
 
-def sequence_pairs(nq, nkv, causal):
-    return sum(_visible_keys(i, nq, nkv, causal) for i in range(nq))
+def sequence_pairs(nq, nkv, causal, window=0):
+    return sum(_visible_keys(i, nq, nkv, causal, window) for i in range(nq))
 
 
-def partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1):
+def partition(q_lens, kv_lens, causal, ranks, method="lpt", sub_batch=1, window=0):
     """Returns (rank_of [B], rank_cost [ranks]) as int lists."""
     q_lens = [int(x) for x in q_lens]
     kv_lens = [int(x) for x in kv_lens]
     B = len(q_lens)
-    cost = [sequence_pairs(q_lens[b], kv_lens[b], causal) for b in range(B)]
+    cost = [sequence_pairs(q_lens[b], kv_lens[b], causal, window) for b in range(B)]
     rank_of = [0] * B
     if method == "lpt":
         load = [0] * ranks

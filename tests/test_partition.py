@@ -35,17 +35,18 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("window", [0, 300])
 @pytest.mark.parametrize("workload,seed,B,ranks,method,sub", CASES)
-def test_partition_matches_oracle(workload, seed, B, ranks, method, sub):
+def test_partition_matches_oracle(workload, seed, B, ranks, method, sub, window):
     ql, kl = draw_lengths(workload, seed, B=B) if B else (np.zeros(0, int), np.zeros(0, int))
     causal = workload == "self_bf16"
-    rank_of, cost = jfa.jfa_partition(ql, kl, causal, ranks, method, sub)
-    r_rank, r_cost = oracle.partition(ql, kl, causal, ranks, method, sub)
+    rank_of, cost = jfa.jfa_partition(ql, kl, causal, ranks, method, sub, window)
+    r_rank, r_cost = oracle.partition(ql, kl, causal, ranks, method, sub, window)
     assert rank_of.tolist() == r_rank
     assert cost.tolist() == r_cost
     # every sequence exactly once, on a valid rank; costs add up
     assert np.all((rank_of >= 0) & (rank_of < ranks))
-    pairs = [oracle.sequence_pairs(int(a), int(b), causal) for a, b in zip(ql, kl)]
+    pairs = [oracle.sequence_pairs(int(a), int(b), causal, window) for a, b in zip(ql, kl)]
     assert int(cost.sum()) == sum(pairs)
     if B and method == "lpt":
         # list scheduling: the heaviest rank exceeds the mean by at most one item
