@@ -4,7 +4,8 @@
 // Efficiency: Why LLM-Scale Recommenders Need a Different Stack", section
 // "Bottleneck move 1"): a work item is (sequence, head, 256-row query block),
 // taken from the longest-first schedule.  The block is two 128-row query
-// tiles A and B that share one stream of 128-row key/value tiles (a
+// tiles held in slots A and B (the CTA's odd items swap which slot holds the
+// upper rows) that share one stream of 128-row key/value tiles (a
 // two-stage ring fetched by TMA); rows of a key tile past the sequence end
 // belong to the neighbouring sequence and are masked out of the scores (and
 // zeroed in the value tile) before they can contribute.
@@ -29,7 +30,9 @@
 //   0..31, keys 64..127 to columns 64..95)
 //   O_T += P_T V_j                   (tcgen05, A = P from TMEM, B = V MN-major)
 // The tensor core alternates between the tiles: while the softmax warps of
-// one tile work, it runs P.V and the next Q K^T of the other.  The rescale of
+// one tile work, it runs P.V and the next Q K^T of the other; a slot whose
+// rows end one key tile before the other's starts its next item during that
+// last key tile.  The rescale of
 // O by exp2(m_old - m_new) is lazy: it happens only when a row's running
 // maximum grows by more than 8 (a factor 256), otherwise the old maximum stays
 // the reference; the final O / l is exact either way.
