@@ -174,6 +174,7 @@ struct Item {
     int n;
 };
 
+template <bool WINDOW>
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     const int4 it = a.items[idx];
     Item w;
@@ -186,7 +187,7 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
     w.nkv = a.kv_off[w.b + 1] - w.k0;
     // both tiles stream the key tiles from the one tile A's first row needs
     // (96-key tiles keep the MX blocks of V aligned to the sequence start)
-    w.jb = vis_key_lo(a.window, w.row0, w.nq, w.nkv) / BN;
+    w.jb = WINDOW ? vis_key_lo(a.window, w.row0, w.nq, w.nkv) / BN : 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int lo = w.row0 + t * BM, hi = min(lo + BM, w.nq);
@@ -194,8 +195,13 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int idx) {
             w.n_t[t] = 0;
             continue;
         }
-        const int kv_end = vis_key_hi(a.causal, a.window, hi - 1, w.nq, w.nkv) + 1;
-        w.n_t[t] = max((kv_end + BN - 1) / BN - w.jb, 0);
+        if (WINDOW) {
+            const int kv_end = vis_key_hi(a.causal, a.window, hi - 1, w.nq, w.nkv) + 1;
+            w.n_t[t] = max((kv_end + BN - 1) / BN - w.jb, 0);
+        } else {
+            const int kv_end = max(a.causal ? min(w.nkv, hi + (w.nkv - w.nq)) : w.nkv, 0);
+            w.n_t[t] = (kv_end + BN - 1) / BN;
+        }
     }
     w.n = max(w.n_t[0], w.n_t[1]);
     return w;
@@ -264,7 +270,7 @@ __device__ __forceinline__ uint4 sf_v(const uint8_t* vs, int64_t blk0, int nblk,
     return make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-template <int BIAS>
+template <int BIAS, bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_constant__ MxParams P) {
     const AttnArgs& a = P.a;
     const int n_items = *a.item_count;
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
         for (int r = 0; ok; ++r) {
             const int idx = item_of_turn(r, cta, G);
             if (idx >= n_items) break;
-            const Item w = load_item(a, idx);
+            const Item w = load_item<WINDOW>(a, idx);
             if (w.n == 0) continue;
             if (nk > 0 && !wwait(&bars->q_free, (nk - 1) & 1)) { ok = false; break; }
             if (lane == 0) {
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
             for (int r = 0; ok; ++r) {
                 const int idx = item_of_turn(r, cta, G);
                 if (idx >= n_items) break;
-                const Item w = load_item(a, idx);
+                const Item w = load_item<WINDOW>(a, idx);
                 if (w.n == 0) continue;
                 if (!mbar_wait(&bars->q_full, nk & 1, abort_flag, a.hdr)) { ok = false; break; }
                 tc_fence_after();
@@ -505,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
         for (int rr = 0; ok; ++rr) {
             const int idx = item_of_turn(rr, cta, G);
             if (idx >= n_items) break;
-            const Item w = load_item(a, idx);
+            const Item w = load_item<WINDOW>(a, idx);
             const int n = w.n_t[tt];
             const int gkv_item = gkv;
             gkv += w.n;
@@ -519,8 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                 }
                 continue;
             }
-            const int jmax_vis = vis_key_hi(a.causal, a.window, i, w.nq, w.nkv);
-            const int jmin_vis = vis_key_lo(a.window, i, w.nq, w.nkv);
+            const int jmax_vis = WINDOW ? vis_key_hi(a.causal, a.window, i, w.nq, w.nkv)
+                                        : (a.causal ? min(w.nkv - 1, i + (w.nkv - w.nq)) : w.nkv - 1);
+            const int jmin_vis = WINDOW ? vis_key_lo(a.window, i, w.nq, w.nkv) : 0;
             const float* tab4 = (BIAS == 1) ? a.bias4 + (int64_t)w.h * 4 * a.bias4_stride : nullptr;
             const __nv_bfloat16* dense = reinterpret_cast<const __nv_bfloat16*>(a.bias);
             const int64_t dense_row = (BIAS == 2 && i < w.nq)
@@ -533,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                 const int gk = gkv_item + j, sk = gk % NS;
                 if (BIAS == 1 && !wwait(&bars->bias_full[sk], (gk / NS) & 1)) { ok = false; break; }
                 const int nvis = i < w.nq ? max(0, min(BN, jmax_vis - jc + 1)) : 0;   // visible: [nlo, nvis)
-                const int nlo = jmin_vis - jc;
-                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW || nlo > cb);
+                const int nlo = WINDOW ? jmin_vis - jc : 0;
+                const bool masked_half = __any_sync(0xffffffffu, nvis < cb + CW || (WINDOW && nlo > cb));
                 const int lo = i - jc - (BN - 1) + C;
                 const int wrel = BIAS == 1 ? lo - bias_window_start(w.row0, jc, C, a.bias4_stride) : 0;
                 const bool win_ok = BIAS == 1 && lo >= 0 && lo + (BN - 1) <= 2 * C && wrel >= 0 && wrel + BN - 4 < kWin;
@@ -592,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fwd_mx_kernel(const __grid_con
                     }
                     if (masked_half) {
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) x[v] = (cc + v < nvis && cc + v >= nlo) ? x[v] : -CUDART_INF_F;
+                        for (int v = 0; v < 16; ++v) x[v] = (cc + v < nvis && (!WINDOW || cc + v >= nlo)) ? x[v] : -CUDART_INF_F;
                     }
                     const float m0 = max3(x[0], x[1], x[2]), m1 = max3(x[3], x[4], x[5]);
                     const float m2 = max3(x[6], x[7], x[8]), m3 = max3(x[9], x[10], x[11]);
@@ -849,7 +856,9 @@ cudaError_t tc_forward_mx_launch(const jfa_problem& p, const AttnArgs& a, const 
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = (int)(items_bound < sms ? items_bound : sms);
     const int bias = p.bias_kind == JFA_BIAS_RELPOS ? 1 : (p.bias_kind == JFA_BIAS_DENSE_JAGGED ? 2 : 0);
-    void (*kern)(MxParams) = bias == 0 ? tc_fwd_mx_kernel<0> : (bias == 1 ? tc_fwd_mx_kernel<1> : tc_fwd_mx_kernel<2>);
+    void (*kern)(MxParams) =
+        a.window > 0 ? (bias == 0 ? tc_fwd_mx_kernel<0, true> : (bias == 1 ? tc_fwd_mx_kernel<1, true> : tc_fwd_mx_kernel<2, true>))
+                     : (bias == 0 ? tc_fwd_mx_kernel<0, false> : (bias == 1 ? tc_fwd_mx_kernel<1, false> : tc_fwd_mx_kernel<2, false>));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimitMx);
     if (e != cudaSuccess) return e;
     static_assert(kSmemBytes <= (uint32_t)kSmemLimitMx, "shared memory");
