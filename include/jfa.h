@@ -288,7 +288,9 @@ jfa_status jfa_block_offsets(const int32_t* offsets, int32_t batch, int64_t tota
  * pairs heavy and light sub-batches without cross-rank communication).
  * Every rank computes the same split from the lengths alone.
  *   q_lens, kv_lens : int32 [batch] sequence lengths (>= 0)
- *   causal          : cost = visible (query, key) pairs, bottom-right causal
+ *   causal, window  : cost = visible (query, key) pairs under the masks of
+ *                     jfa_problem (bottom-right causal; sliding window w > 0,
+ *                     0 = none; negative is JFA_ERR_INVALID_ARGUMENT)
  *   method          : JFA_PARTITION_LPT -- sequences by cost descending (ties
  *                     by index), each to the least-loaded rank (ties: lowest);
  *                     JFA_PARTITION_BBS -- sub-batches of `sub_batch`
