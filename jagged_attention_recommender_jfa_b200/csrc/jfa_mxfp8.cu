@@ -64,48 +64,94 @@ __global__ void __launch_bounds__(256) quant_along_d(const __nv_bfloat16* __rest
     scales[blk] = (uint8_t)(X + 127);
 }
 
-// Blocks of 32 consecutive rows of one sequence: grid (sequence, row block),
-// threads over the heads * d columns (coalesced along the row).
-__global__ void __launch_bounds__(256) quant_along_rows(const __nv_bfloat16* __restrict__ x,
-                                                        const int32_t* __restrict__ off, int B,
-                                                        int64_t total_rows, int cols,
-                                                        uint8_t* __restrict__ codes,
-                                                        uint8_t* __restrict__ scales) {
-    const int b = blockIdx.x, blk = blockIdx.y;
-    const int r0 = off[b], n = off[b + 1] - r0;
-    // rows outside [0, total_rows) are never touched, whatever the offsets say
-    if (blk * 32 >= n || r0 < 0 || (int64_t)r0 + n > total_rows) return;
-    // first block index of sequence b = sum_{b' < b} ceil(n(b') / 32)
-    __shared__ int64_t s_part[256];
+// Blocks of 32 consecutive rows of one sequence.  Grid (sequence, slot): a
+// CTA takes its sequence's row blocks slot, slot + gridDim.y, ... (at most
+// kRowSlots CTAs per sequence, so a short batch of long sequences launches
+// no idle CTAs); a thread takes two adjacent columns, so a warp reads 128
+// contiguous bytes of each row, and all 32 loads of a block are in flight
+// before the first conversion.
+constexpr int kRowSlots = 16;
+
+// first block index of sequence b = sum_{b' < b} ceil(n(b') / 32)
+__device__ int64_t seq_block_base(const int32_t* __restrict__ off, int b) {
+    __shared__ int64_t s_warp[8];
     int64_t part = 0;
     for (int bb = threadIdx.x; bb < b; bb += blockDim.x) part += (off[bb + 1] - off[bb] + 31) / 32;
-    s_part[threadIdx.x] = part;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = part;
     __syncthreads();
-    for (int st = 128; st > 0; st >>= 1) {
-        if ((int)threadIdx.x < st) s_part[threadIdx.x] += s_part[threadIdx.x + st];
-        __syncthreads();
-    }
-    const int64_t gblk = s_part[0] + blk;
-    const int rows = min(32, n - blk * 32);
-    const __nv_bfloat16* base = x + (int64_t)(r0 + blk * 32) * cols;
-    uint8_t* cbase = codes + (int64_t)(r0 + blk * 32) * cols;
-    for (int col = threadIdx.x; col < cols; col += blockDim.x) {
-        float f[32];
-        float amax = 0.f;
+    int64_t total = 0;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            f[t] = t < rows ? __bfloat162float(base[(int64_t)t * cols + col]) : 0.f;
-            amax = fmaxf(amax, fabsf(f[t]));
-        }
-        const int X = shared_exponent(amax);
-        const float s = pow2_neg(X);
+    for (int w = 0; w < 8; ++w) total += s_warp[w];
+    return total;
+}
+
+// FAKE = false: E4M3 codes and E8M0 scales; FAKE = true: the dequantised
+// value E4M3(x * 2^-X) * 2^X in bf16 (exact), no scales.
+template <bool FAKE>
+__global__ void __launch_bounds__(256, 4) mx_along_rows(const __nv_bfloat16* __restrict__ x,
+                                                     const int32_t* __restrict__ off,
+                                                     int64_t total_rows, int cols,
+                                                     uint8_t* __restrict__ codes,
+                                                     uint8_t* __restrict__ scales,
+                                                     __nv_bfloat16* __restrict__ y) {
+    const int b = blockIdx.x;
+    const int r0 = off[b], n = off[b + 1] - r0;
+    // rows outside [0, total_rows) are never touched, whatever the offsets say
+    if (n <= 0 || r0 < 0 || (int64_t)r0 + n > total_rows) return;
+    const int nblk = (n + 31) / 32;
+    if ((int)blockIdx.y >= nblk) return;
+    const int64_t blk0 = FAKE ? 0 : seq_block_base(off, b);
+    const bool scale_pairs = ((reinterpret_cast<uintptr_t>(scales) & 1) == 0);
+    for (int blk = blockIdx.y; blk < nblk; blk += gridDim.y) {
+        const int rows = min(32, n - blk * 32);
+        const int64_t row0 = (int64_t)r0 + (int64_t)blk * 32;
+        for (int c = threadIdx.x * 2; c < cols; c += blockDim.x * 2) {
+            // one running address per pass (not 32 precomputed ones); rows
+            // past a short last block repeat its last row, which leaves the
+            // block maximum as zero padding would
+            const __nv_bfloat16* src = x + row0 * cols + c;
+            uint32_t raw[32];
 #pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-            uint16_t two = pack_e4m3x2(f[t] * s, f[t + 1] * s);
-            if (t < rows) cbase[(int64_t)t * cols + col] = (uint8_t)(two & 0xFF);
-            if (t + 1 < rows) cbase[(int64_t)(t + 1) * cols + col] = (uint8_t)(two >> 8);
+            for (int t = 0; t < 32; ++t) {
+                raw[t] = __ldg(reinterpret_cast<const unsigned int*>(src));
+                if (t + 1 < rows) src += cols;
+            }
+            // block maxima of |x| in bf16 (exact: a maximum rounds nothing)
+            __nv_bfloat162 m = __float2bfloat162_rn(0.f);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&raw[t])));
+            const float2 am = __bfloat1622float2(m);
+            const int X0 = shared_exponent(am.x), X1 = shared_exponent(am.y);
+            const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
+            const float b0 = pow2(X0), b1 = pow2(X1);
+            uint8_t* cdst = FAKE ? nullptr : codes + row0 * cols + c;
+            __nv_bfloat16* ydst = FAKE ? y + row0 * cols + c : nullptr;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[t]));
+                const uint16_t two = pack_e4m3x2(v.x * s0, v.y * s1);
+                if (t < rows) {
+                    if (FAKE) {
+                        const float2 d = decode_e4m3x2(two);
+                        *reinterpret_cast<__nv_bfloat162*>(ydst) = __floats2bfloat162_rn(d.x * b0, d.y * b1);
+                    } else {
+                        *reinterpret_cast<uint16_t*>(cdst) = two;
+                    }
+                }
+                if (FAKE) ydst += cols; else cdst += cols;
+            }
+            if (!FAKE) {
+                uint8_t* sp = scales + (blk0 + blk) * cols + c;
+                if (scale_pairs) {
+                    *reinterpret_cast<uint16_t*>(sp) = (uint16_t)((X0 + 127) | ((X1 + 127) << 8));
+                } else {
+                    sp[0] = (uint8_t)(X0 + 127);
+                    sp[1] = (uint8_t)(X1 + 127);
+                }
+            }
         }
-        scales[gblk * cols + col] = (uint8_t)(X + 127);
     }
 }
 
@@ -150,36 +196,6 @@ __global__ void __launch_bounds__(256) fake_quant_along_d(const __nv_bfloat16* _
     for (int t = 0; t < 4; ++t) dst[t] = out[t];
 }
 
-// Quantise-dequantise along 32-row blocks of each sequence.
-__global__ void __launch_bounds__(256) fake_quant_along_rows(const __nv_bfloat16* __restrict__ x,
-                                                             const int32_t* __restrict__ off,
-                                                             int64_t total_rows, int cols,
-                                                             __nv_bfloat16* __restrict__ y) {
-    const int b = blockIdx.x, blk = blockIdx.y;
-    const int r0 = off[b], n = off[b + 1] - r0;
-    if (blk * 32 >= n || r0 < 0 || (int64_t)r0 + n > total_rows) return;
-    const int rows = min(32, n - blk * 32);
-    const __nv_bfloat16* base = x + (int64_t)(r0 + blk * 32) * cols;
-    __nv_bfloat16* obase = y + (int64_t)(r0 + blk * 32) * cols;
-    for (int col = threadIdx.x; col < cols; col += blockDim.x) {
-        float f[32];
-        float amax = 0.f;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            f[t] = t < rows ? __bfloat162float(base[(int64_t)t * cols + col]) : 0.f;
-            amax = fmaxf(amax, fabsf(f[t]));
-        }
-        const int X = shared_exponent(amax);
-        const float s = pow2_neg(X), back = pow2(X);
-#pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-            const float2 d2 = decode_e4m3x2(pack_e4m3x2(f[t] * s, f[t + 1] * s));
-            if (t < rows) obase[(int64_t)t * cols + col] = __float2bfloat16_rn(d2.x * back);
-            if (t + 1 < rows) obase[(int64_t)(t + 1) * cols + col] = __float2bfloat16_rn(d2.y * back);
-        }
-    }
-}
-
 }  // namespace
 
 // MXFP8 operands for the attention passes: Q and K quantised along d, V along
@@ -197,10 +213,12 @@ cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const
             reinterpret_cast<const __nv_bfloat16*>(k), nk_blocks, reinterpret_cast<__nv_bfloat16*>(kf));
     prof_end(st, K_QUANT_ALONG_D);
     if (batch > 0 && max_kv_len > 0) {
-        dim3 grid(batch, (max_kv_len + 31) / 32);
+        const int slots = (max_kv_len + 31) / 32 < kRowSlots ? (max_kv_len + 31) / 32 : kRowSlots;
+        dim3 grid(batch, slots);
         prof_begin(st);
-        fake_quant_along_rows<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), kv_off,
-                                                    total_kv, heads * d, reinterpret_cast<__nv_bfloat16*>(vf));
+        mx_along_rows<true><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), kv_off,
+                                                  total_kv, heads * d, nullptr, nullptr,
+                                                  reinterpret_cast<__nv_bfloat16*>(vf));
         prof_end(st, K_QUANT_ALONG_ROWS);
     }
     return cudaGetLastError();
@@ -219,9 +237,10 @@ cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int
         prof_end(st, K_QUANT_ALONG_D);
     } else {
         if (batch == 0 || max_rows_per_seq == 0) return cudaSuccess;
-        dim3 grid(batch, (max_rows_per_seq + 31) / 32);
+        const int slots = (max_rows_per_seq + 31) / 32 < kRowSlots ? (max_rows_per_seq + 31) / 32 : kRowSlots;
+        dim3 grid(batch, slots);
         prof_begin(st);
-        quant_along_rows<<<grid, 256, 0, st>>>(xb, offsets, batch, rows, heads * d, codes, scales);
+        mx_along_rows<false><<<grid, 256, 0, st>>>(xb, offsets, rows, heads * d, codes, scales, nullptr);
         prof_end(st, K_QUANT_ALONG_ROWS);
     }
     return cudaGetLastError();

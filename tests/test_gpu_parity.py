@@ -341,6 +341,29 @@ def test_quantize_mxfp8_bit_exact(cuda_device):
     assert np.array_equal(scales[:rs.shape[0]].cpu().numpy(), rs)
 
 
+def test_quantize_mxfp8_along_rows_long_sequences(cuda_device):
+    # sequences of many 32-row blocks (more than the CTAs a sequence gets, so
+    # a CTA takes several blocks), ragged last blocks, and scales written at
+    # an odd address (byte stores instead of pairs)
+    lens = [1100, 37, 700, 32, 1]
+    off = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    rows, H, d = int(off[-1]), 3, 64
+    g = torch.Generator().manual_seed(5)
+    v = (torch.randn(rows, H, d, generator=g) * torch.exp(torch.randn(rows, 1, 1, generator=g))).to(torch.bfloat16)
+    v[40:72] = 0.0
+    v[1100 + 5] = -600.0
+    nblk = rows // 32 + len(lens)
+    rc, rs = oracle.quantize_mx_along_rows(v, off)
+    for shift in (0, 1):
+        codes = torch.empty(rows, H, d, dtype=torch.uint8, device=cuda_device)
+        store = torch.zeros(nblk * H * d + 16, dtype=torch.uint8, device=cuda_device)
+        scales = store[shift:shift + nblk * H * d].view(nblk, H, d)
+        jfa.jfa_quantize_mxfp8(v.to(cuda_device), rows, H, d, off.to(cuda_device), len(lens),
+                               max(lens), True, codes, scales)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+        assert np.array_equal(scales[:rs.shape[0]].cpu().numpy(), rs)
+
+
 # ---------------------------------------------------------------------------
 # MXFP8: Q/K quantised along d, V along 32-row blocks, P per 32 keys
 # ---------------------------------------------------------------------------
