@@ -86,6 +86,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-peak-probe", action="store_true",
+                    help="time the library FP8 GEMM (E4M3, and MX-scaled where supported) at 8192^3 "
+                         "as the fp8 roofline denominator, print one JSON line and exit")
     ap.add_argument("--cpu-sample-pairs", type=float, default=8e6,
                     help="(query, key) pairs x heads in the CPU oracle's sample")
     return ap.parse_args()
@@ -424,6 +427,46 @@ def padded_dense_baseline(p, dev, f_valid, iters=3):
 # ---------------------------------------------------------------------------
 # main arm
 # ---------------------------------------------------------------------------
+def fp8_peak_probe(dev, n=8192, warmup=5, iters=20):
+    """Dense FP8 tensor-core throughput of the library GEMM (cuBLASLt through
+    torch._scaled_mm) at n^3, E4M3 x E4M3 -> bf16: with per-tensor scales, and
+    with MX block scales (one E8M0 per 32 elements along K, all 2^0, so their
+    layout does not matter) where this build supports them.  Timed with CUDA
+    events after warm-up; the MXFP8 attention kernel's fp8 roofline."""
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)   # [N][K]: b.t() is K x N column-major
+    one = torch.ones((), device=dev)
+
+    def tflops(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(iters):
+            fn()
+        t1.record()
+        torch.cuda.synchronize()
+        return 2.0 * n ** 3 / (t0.elapsed_time(t1) / iters * 1e-3) / 1e12
+
+    out = {"probe": "fp8_peak", "n": n, "iters": iters,
+           "fp8_e4m3_tflops": tflops(lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one,
+                                                              out_dtype=torch.bfloat16))}
+    try:
+        def rup(x, m):
+            return (x + m - 1) // m * m
+        ns = rup(n, 128) * rup(n // 32, 4)
+        sa = torch.full((ns,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+        sb = torch.full((ns,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+        out["mxfp8_tflops"] = tflops(lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb,
+                                                              out_dtype=torch.bfloat16))
+    except Exception as e:   # noqa: BLE001 -- reported, not fatal
+        out["mxfp8_tflops"] = None
+        out["mxfp8_unavailable"] = str(e).splitlines()[0][:200]
+    out["device"] = torch.cuda.get_device_name(dev)
+    return out
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -443,6 +486,10 @@ def main():
         raise SystemExit("bench.py --impl jfa needs a CUDA device")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.fp8_peak_probe:
+        if rank == 0:
+            print(json.dumps(fp8_peak_probe(dev)))
+        return
     from jagged_attention_recommender_jfa_b200 import jfa
     from jagged_attention_recommender_jfa_b200.inputs import WORKLOADS, draw_lengths
 
