@@ -86,6 +86,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mx-internal", action="store_true",
+                    help="MXFP8: run jfa_forward / jfa_backward with dtype MXFP8 (quantising inside "
+                         "each call) instead of the producer form of the step")
     ap.add_argument("--fp8-peak-probe", action="store_true",
                     help="time the library FP8 GEMM (E4M3, and MX-scaled where supported) at 8192^3 "
                          "as the fp8 roofline denominator, print one JSON line and exit")
@@ -513,8 +516,8 @@ def main():
     out = torch.empty_like(d["q"])
     lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
     dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
-    ws_f = jfa.workspace(prob, False, dev)
-    ws_b = jfa.workspace(prob, True, dev)
+    apass = AttentionPass(jfa, prob, p, act, dev, internal=args.mx_internal)
+    ws_f, ws_b = apass.workspaces
     stream = torch.cuda.current_stream(dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
@@ -523,12 +526,10 @@ def main():
             marks[0].record(stream)
         if args.block:
             jfa.jfa_block_offsets(seq_off, p.B, p.total_q, args.block, d["q_off"], stream=stream)
-        jfa.jfa_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"], bias, act,
-                        p.causal, out, lse, ws_f, stream=stream)
+        apass.forward(d, d["q_off"], d["kv_off"], bias, out, lse, stream)
         if marks is not None:
             marks[1].record(stream)
-        jfa.jfa_backward(prob, d["q"], d["k"], d["v"], out, lse, d["dout"], d["q_off"],
-                         d["kv_off"], bias, act, p.causal, dq, dk, dv, ws_b, stream=stream)
+        apass.backward(d, d["q_off"], d["kv_off"], bias, out, lse, dq, dk, dv, stream)
         if marks is not None:
             marks[2].record(stream)
 
@@ -727,6 +728,60 @@ def aggregate_over_ranks(ms_per_step, flops, device, world):
     return float(t.item()), float(fl.item())
 
 
+class AttentionPass:
+    """One forward + backward of the library on device inputs.  MXFP8 runs in
+    its producer form: one quantisation pass per operand writes the E4M3 codes
+    for jfa_forward_mxfp8 and the dequantised operands for a bf16
+    jfa_backward, which is then the MXFP8 backward (bf16 gradients on the
+    values the forward's block-scaled MMAs saw), so nothing is quantised
+    twice; ``internal`` runs jfa_forward / jfa_backward with dtype MXFP8
+    instead, which quantise inside the call."""
+
+    def __init__(self, jfa, prob, p, act, dev, internal=False):
+        self.jfa, self.prob, self.p, self.act = jfa, prob, p, act
+        self.mx = p.dtype == "mxfp8" and not internal
+        self.ws_f = jfa.workspace(prob, False, dev)
+        self.bprob = prob
+        if self.mx:
+            self.bprob = jfa.jfa_problem.from_buffer_copy(prob)
+            self.bprob.dtype = jfa.JFA_BF16
+            H, dd = prob.heads, prob.head_dim
+            u8 = dict(dtype=torch.uint8, device=dev)
+            self.q8 = torch.empty(prob.total_q, H, dd, **u8)
+            self.k8 = torch.empty(prob.total_kv, H, dd, **u8)
+            self.v8 = torch.empty(prob.total_kv, H, dd, **u8)
+            self.qs = torch.empty(prob.total_q, H, dd // 32, **u8)
+            self.ks = torch.empty(prob.total_kv, H, dd // 32, **u8)
+            self.vs = torch.empty(prob.total_kv // 32 + prob.batch, H, dd, **u8)
+            bf = dict(dtype=torch.bfloat16, device=dev)
+            self.qd = torch.empty(prob.total_q, H, dd, **bf)
+            self.kd = torch.empty(prob.total_kv, H, dd, **bf)
+            self.vd = torch.empty(prob.total_kv, H, dd, **bf)
+        self.ws_b = jfa.workspace(self.bprob, True, dev)
+        self.workspaces = (self.ws_f, self.ws_b)
+
+    def forward(self, inp, qo, ko, bias, out, lse, stream):
+        j, pr, causal = self.jfa, self.prob, self.p.causal
+        if not self.mx:
+            j.jfa_forward(pr, inp["q"], inp["k"], inp["v"], qo, ko, bias, self.act, causal, out, lse,
+                          self.ws_f, stream=stream)
+            return
+        H, dd = pr.heads, pr.head_dim
+        j.jfa_quantize_mxfp8_dequant(inp["q"], pr.total_q, H, dd, None, 0, 0, False, self.q8, self.qs,
+                                     self.qd, stream=stream)
+        j.jfa_quantize_mxfp8_dequant(inp["k"], pr.total_kv, H, dd, None, 0, 0, False, self.k8, self.ks,
+                                     self.kd, stream=stream)
+        j.jfa_quantize_mxfp8_dequant(inp["v"], pr.total_kv, H, dd, ko, pr.batch, pr.max_kv_len, True,
+                                     self.v8, self.vs, self.vd, stream=stream)
+        j.jfa_forward_mxfp8(pr, self.q8, self.qs, self.k8, self.ks, self.v8, self.vs, qo, ko, bias,
+                            causal, out, lse, self.ws_f, stream=stream)
+
+    def backward(self, inp, qo, ko, bias, out, lse, dq, dk, dv, stream):
+        q, k, v = (self.qd, self.kd, self.vd) if self.mx else (inp["q"], inp["k"], inp["v"])
+        self.jfa.jfa_backward(self.bprob, q, k, v, out, lse, inp["dout"], qo, ko, bias, self.act,
+                              self.p.causal, dq, dk, dv, self.ws_b, stream=stream)
+
+
 def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
     """Same metric with pinned host inputs copied in and every result copied
     out inside the timed region, pipelined the way a training input loop is:
@@ -745,8 +800,7 @@ def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
         lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=dev) if act == "softmax" else None
         dq, dk, dv = torch.empty_like(dev_in["q"]), torch.empty_like(dev_in["k"]), torch.empty_like(dev_in["v"])
         sets.append((dev_in, out, lse, dq, dk, dv))
-    ws_f = jfa.workspace(prob, False, dev)
-    ws_b = jfa.workspace(prob, True, dev)
+    apass = AttentionPass(jfa, prob, p, act, dev, internal=args.mx_internal)
     # BlockAttention: block offsets rebuilt from each step's sequence offsets
     boffs = [torch.empty(prob.batch + 1, dtype=torch.int32, device=dev) for _ in range(2)]
 
@@ -778,11 +832,8 @@ def e2e_leg(args, p, prob, act, dev, stream, jfa, flops_rank, world):
             if args.block:
                 jfa.jfa_block_offsets(qo, p.B, p.total_q, args.block, boffs[b], stream=stream)
                 qo = ko = boffs[b]
-            jfa.jfa_forward(prob, dev_in["q"], dev_in["k"], dev_in["v"], qo, ko,
-                            dev_in.get("bias"), act, p.causal, out, lse, ws_f, stream=stream)
-            jfa.jfa_backward(prob, dev_in["q"], dev_in["k"], dev_in["v"], out, lse, dev_in["dout"],
-                             qo, ko, dev_in.get("bias"), act, p.causal, dq, dk, dv, ws_b,
-                             stream=stream)
+            apass.forward(dev_in, qo, ko, dev_in.get("bias"), out, lse, stream)
+            apass.backward(dev_in, qo, ko, dev_in.get("bias"), out, lse, dq, dk, dv, stream)
             comp_done[b].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(comp_done[b])

@@ -215,6 +215,23 @@ jfa_status jfa_quantize_mxfp8(const void* x_bf16, int64_t rows, int32_t heads, i
                               int along_rows, uint8_t* codes, uint8_t* scales,
                               jfa_stream_t stream);
 
+/* jfa_quantize_mxfp8 that, in the same pass, also writes every element's
+ * dequantised value code * 2^X (exact in bf16: three mantissa bits times a
+ * power of two) to dequant_bf16, a device tensor [rows][heads][d], 16-byte
+ * aligned, owned by the caller.  For the producer of an MXFP8 training step
+ * ("Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a Different
+ * Stack", "Bottleneck move 2": casting belongs in the kernel that makes the
+ * tensor, not in extra passes): the codes feed jfa_forward_mxfp8 and the
+ * dequantised tensors a bf16 jfa_backward, which is then the MXFP8 backward
+ * (bf16 gradients on the operands the forward's block-scaled MMAs saw, the
+ * quantiser passed straight through) without a second quantisation pass.
+ * Arguments, layouts and errors otherwise as jfa_quantize_mxfp8; a NULL
+ * dequant_bf16 with rows > 0 is JFA_ERR_INVALID_ARGUMENT. */
+jfa_status jfa_quantize_mxfp8_dequant(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
+                                      const int32_t* offsets, int32_t batch, int32_t max_len,
+                                      int along_rows, uint8_t* codes, uint8_t* scales,
+                                      void* dequant_bf16, jfa_stream_t stream);
+
 /* Normalisation fused with MX quantisation, for the producer of MXFP8
  * operands ("Meta Enhances GEM Training Efficiency with Advanced LLM-Scale
  * Innovations", "Implementing Ultra-Low-Precision Methods"; "Meta GEM

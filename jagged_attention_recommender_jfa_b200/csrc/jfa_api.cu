@@ -21,7 +21,7 @@ cudaError_t simt_backward(const AttnArgs& a, const AttnArgs& kv_args, int head_d
                           int grid_q, int grid_kv, int64_t rows, cudaStream_t st);
 cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
                         int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,
-                        uint8_t* scales, cudaStream_t st);
+                        uint8_t* scales, void* dequant, cudaStream_t st);
 bool tc_supported(const jfa_problem& p, int act, int backward);
 size_t tc_workspace_extra(const jfa_problem& p, int backward);
 cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, cudaStream_t st);
@@ -391,20 +391,39 @@ jfa_status jfa_backward_dbias(const jfa_problem* problem, const void* q, const v
                          causal, dq, dk, dv, dbias, workspace, ws_bytes, stream);
 }
 
+namespace {
+jfa_status quantize_entry(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
+                          const int32_t* offsets, int32_t batch, int32_t max_len, int along_rows,
+                          uint8_t* codes, uint8_t* scales, void* dequant, jfa_stream_t stream) {
+    if (rows < 0 || heads < 1 || d < 32 || (d % 32) != 0)
+        return fail(JFA_ERR_INVALID_ARGUMENT, "bad quantiser sizes");
+    if (rows > 0 && (!x_bf16 || !codes || !scales)) return fail(JFA_ERR_INVALID_ARGUMENT, "NULL tensor");
+    if (!ALIGNED16(x_bf16) || !ALIGNED16(codes) || !ALIGNED16(dequant))
+        return fail(JFA_ERR_INVALID_ARGUMENT, "x, codes and dequant must be 16-byte aligned");
+    if (along_rows && (!offsets || batch < 0 || max_len < 0))
+        return fail(JFA_ERR_INVALID_ARGUMENT, "along_rows needs offsets, batch and max_len");
+    cudaError_t e = quantize_mx(x_bf16, rows, heads, d, offsets, batch, max_len, along_rows, codes,
+                                scales, dequant, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quantize");
+    return JFA_OK;
+}
+}  // namespace
+
 jfa_status jfa_quantize_mxfp8(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
                               const int32_t* offsets, int32_t batch, int32_t max_len,
                               int along_rows, uint8_t* codes, uint8_t* scales,
                               jfa_stream_t stream) {
-    if (rows < 0 || heads < 1 || d < 32 || (d % 32) != 0)
-        return fail(JFA_ERR_INVALID_ARGUMENT, "bad quantiser sizes");
-    if (rows > 0 && (!x_bf16 || !codes || !scales)) return fail(JFA_ERR_INVALID_ARGUMENT, "NULL tensor");
-    if (!ALIGNED16(x_bf16) || !ALIGNED16(codes)) return fail(JFA_ERR_INVALID_ARGUMENT, "x and codes must be 16-byte aligned");
-    if (along_rows && (!offsets || batch < 0 || max_len < 0))
-        return fail(JFA_ERR_INVALID_ARGUMENT, "along_rows needs offsets, batch and max_len");
-    cudaError_t e = quantize_mx(x_bf16, rows, heads, d, offsets, batch, max_len, along_rows, codes,
-                                scales, reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "quantize");
-    return JFA_OK;
+    return quantize_entry(x_bf16, rows, heads, d, offsets, batch, max_len, along_rows, codes, scales,
+                          nullptr, stream);
+}
+
+jfa_status jfa_quantize_mxfp8_dequant(const void* x_bf16, int64_t rows, int32_t heads, int32_t d,
+                                      const int32_t* offsets, int32_t batch, int32_t max_len,
+                                      int along_rows, uint8_t* codes, uint8_t* scales,
+                                      void* dequant_bf16, jfa_stream_t stream) {
+    if (rows > 0 && !dequant_bf16) return fail(JFA_ERR_INVALID_ARGUMENT, "NULL dequant");
+    return quantize_entry(x_bf16, rows, heads, d, offsets, batch, max_len, along_rows, codes, scales,
+                          dequant_bf16, stream);
 }
 
 jfa_status jfa_schedule(const jfa_problem* problem, const int32_t* q_offsets,

@@ -25,10 +25,14 @@ using mx::pow2;
 using mx::pack_e4m3x2;
 using mx::decode_e4m3x2;
 
-// Blocks of 32 consecutive elements along d: one thread per block.
-__global__ void __launch_bounds__(256) quant_along_d(const __nv_bfloat16* __restrict__ x,
-                                                     int64_t n_blocks, uint8_t* __restrict__ codes,
-                                                     uint8_t* __restrict__ scales) {
+// Blocks of 32 consecutive elements along d: one thread per block (64-byte
+// loads).  CODES: E4M3 codes and the E8M0 scale; DEQ: the dequantised value
+// E4M3(x * 2^-X) * 2^X in bf16 (exact: 3 mantissa bits times a power of two).
+template <bool CODES, bool DEQ>
+__global__ void __launch_bounds__(256) mx_along_d(const __nv_bfloat16* __restrict__ x,
+                                                  int64_t n_blocks, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ scales,
+                                                  __nv_bfloat16* __restrict__ y) {
     int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (blk >= n_blocks) return;
     const uint4* src = reinterpret_cast<const uint4*>(x + blk * 32);
@@ -50,18 +54,32 @@ __global__ void __launch_bounds__(256) quant_along_d(const __nv_bfloat16* __rest
 #pragma unroll
     for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(f[t]));
     const int X = shared_exponent(amax);
-    const float s = pow2_neg(X);
-    uint32_t w[8];
+    const float s = pow2_neg(X), back = pow2(X);
+    uint16_t two[16];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-        uint32_t lo = pack_e4m3x2(f[4 * t] * s, f[4 * t + 1] * s);
-        uint32_t hi = pack_e4m3x2(f[4 * t + 2] * s, f[4 * t + 3] * s);
-        w[t] = lo | (hi << 16);
+    for (int t = 0; t < 16; ++t) two[t] = pack_e4m3x2(f[2 * t] * s, f[2 * t + 1] * s);
+    if (CODES) {
+        uint32_t w[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) w[t] = (uint32_t)two[2 * t] | ((uint32_t)two[2 * t + 1] << 16);
+        uint4* dst = reinterpret_cast<uint4*>(codes + blk * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        scales[blk] = (uint8_t)(X + 127);
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes + blk * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    scales[blk] = (uint8_t)(X + 127);
+    if (DEQ) {
+        uint4 out[4];
+        uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const float2 d2 = decode_e4m3x2(two[t]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(d2.x * back, d2.y * back);
+            o32[t] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(y + blk * 32);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) dst[t] = out[t];
+    }
 }
 
 // Blocks of 32 consecutive rows of one sequence.  Grid (sequence, slot): a
@@ -87,9 +105,9 @@ __device__ int64_t seq_block_base(const int32_t* __restrict__ off, int b) {
     return total;
 }
 
-// FAKE = false: E4M3 codes and E8M0 scales; FAKE = true: the dequantised
-// value E4M3(x * 2^-X) * 2^X in bf16 (exact), no scales.
-template <bool FAKE>
+// CODES: E4M3 codes and E8M0 scales; DEQ: the dequantised value
+// E4M3(x * 2^-X) * 2^X in bf16 (exact).
+template <bool CODES, bool DEQ>
 __global__ void __launch_bounds__(256, 4) mx_along_rows(const __nv_bfloat16* __restrict__ x,
                                                      const int32_t* __restrict__ off,
                                                      int64_t total_rows, int cols,
@@ -102,7 +120,7 @@ __global__ void __launch_bounds__(256, 4) mx_along_rows(const __nv_bfloat16* __r
     if (n <= 0 || r0 < 0 || (int64_t)r0 + n > total_rows) return;
     const int nblk = (n + 31) / 32;
     if ((int)blockIdx.y >= nblk) return;
-    const int64_t blk0 = FAKE ? 0 : seq_block_base(off, b);
+    const int64_t blk0 = CODES ? seq_block_base(off, b) : 0;
     const bool scale_pairs = ((reinterpret_cast<uintptr_t>(scales) & 1) == 0);
     for (int blk = blockIdx.y; blk < nblk; blk += gridDim.y) {
         const int rows = min(32, n - blk * 32);
@@ -126,23 +144,23 @@ __global__ void __launch_bounds__(256, 4) mx_along_rows(const __nv_bfloat16* __r
             const int X0 = shared_exponent(am.x), X1 = shared_exponent(am.y);
             const float s0 = pow2_neg(X0), s1 = pow2_neg(X1);
             const float b0 = pow2(X0), b1 = pow2(X1);
-            uint8_t* cdst = FAKE ? nullptr : codes + row0 * cols + c;
-            __nv_bfloat16* ydst = FAKE ? y + row0 * cols + c : nullptr;
+            uint8_t* cdst = CODES ? codes + row0 * cols + c : nullptr;
+            __nv_bfloat16* ydst = DEQ ? y + row0 * cols + c : nullptr;
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[t]));
                 const uint16_t two = pack_e4m3x2(v.x * s0, v.y * s1);
                 if (t < rows) {
-                    if (FAKE) {
+                    if (DEQ) {
                         const float2 d = decode_e4m3x2(two);
                         *reinterpret_cast<__nv_bfloat162*>(ydst) = __floats2bfloat162_rn(d.x * b0, d.y * b1);
-                    } else {
-                        *reinterpret_cast<uint16_t*>(cdst) = two;
                     }
+                    if (CODES) *reinterpret_cast<uint16_t*>(cdst) = two;
                 }
-                if (FAKE) ydst += cols; else cdst += cols;
+                if (DEQ) ydst += cols;
+                if (CODES) cdst += cols;
             }
-            if (!FAKE) {
+            if (CODES) {
                 uint8_t* sp = scales + (blk0 + blk) * cols + c;
                 if (scale_pairs) {
                     *reinterpret_cast<uint16_t*>(sp) = (uint16_t)((X0 + 127) | ((X1 + 127) << 8));
@@ -155,95 +173,50 @@ __global__ void __launch_bounds__(256, 4) mx_along_rows(const __nv_bfloat16* __r
     }
 }
 
-// Quantise-dequantise ("fake quantisation") along d: the output holds, in
-// bf16, exactly the value E4M3(x * 2^-X) * 2^X that an MXFP8 operand
-// represents (3 mantissa bits times a power of two fit bf16 exactly).
-__global__ void __launch_bounds__(256) fake_quant_along_d(const __nv_bfloat16* __restrict__ x,
-                                                          int64_t n_blocks,
-                                                          __nv_bfloat16* __restrict__ y) {
-    int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (blk >= n_blocks) return;
-    const uint4* src = reinterpret_cast<const uint4*>(x + blk * 32);
-    uint4 raw[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) raw[t] = src[t];
-    float f[32];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[t]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            float2 v = __bfloat1622float2(p2[u]);
-            f[8 * t + 2 * u] = v.x;
-            f[8 * t + 2 * u + 1] = v.y;
-        }
+}  // namespace
+
+// codes / scales (both or neither) and / or the dequantised bf16 `dequant`.
+cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
+                        int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,
+                        uint8_t* scales, void* dequant, cudaStream_t st) {
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(dequant);
+    const bool cd = codes != nullptr, dq = dequant != nullptr;
+    if (!cd && !dq) return cudaSuccess;
+    if (!along_rows) {
+        int64_t n_blocks = rows * heads * (d / 32);
+        if (n_blocks == 0) return cudaSuccess;
+        const unsigned grid = (unsigned)((n_blocks + 255) / 256);
+        prof_begin(st);
+        if (cd && dq) mx_along_d<true, true><<<grid, 256, 0, st>>>(xb, n_blocks, codes, scales, y);
+        else if (cd) mx_along_d<true, false><<<grid, 256, 0, st>>>(xb, n_blocks, codes, scales, y);
+        else mx_along_d<false, true><<<grid, 256, 0, st>>>(xb, n_blocks, codes, scales, y);
+        prof_end(st, K_QUANT_ALONG_D);
+    } else {
+        if (batch == 0 || max_rows_per_seq == 0) return cudaSuccess;
+        const int slots = (max_rows_per_seq + 31) / 32 < kRowSlots ? (max_rows_per_seq + 31) / 32 : kRowSlots;
+        dim3 grid(batch, slots);
+        const int cols = heads * d;
+        prof_begin(st);
+        if (cd && dq) mx_along_rows<true, true><<<grid, 256, 0, st>>>(xb, offsets, rows, cols, codes, scales, y);
+        else if (cd) mx_along_rows<true, false><<<grid, 256, 0, st>>>(xb, offsets, rows, cols, codes, scales, y);
+        else mx_along_rows<false, true><<<grid, 256, 0, st>>>(xb, offsets, rows, cols, codes, scales, y);
+        prof_end(st, K_QUANT_ALONG_ROWS);
     }
-    float amax = 0.f;
-#pragma unroll
-    for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(f[t]));
-    const int X = shared_exponent(amax);
-    const float s = pow2_neg(X), back = pow2(X);
-    uint4 out[4];
-    uint32_t* o32 = reinterpret_cast<uint32_t*>(out);
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-        const float2 d2 = decode_e4m3x2(pack_e4m3x2(f[2 * t] * s, f[2 * t + 1] * s));
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(d2.x * back, d2.y * back);
-        o32[t] = *reinterpret_cast<uint32_t*>(&b2);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(y + blk * 32);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) dst[t] = out[t];
+    return cudaGetLastError();
 }
 
-}  // namespace
 
 // MXFP8 operands for the attention passes: Q and K quantised along d, V along
 // 32-row blocks of each sequence, each returned dequantised in bf16.
 cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const int32_t* kv_off,
                               int64_t total_q, int64_t total_kv, int heads, int d, int batch,
                               int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st) {
-    const int64_t nq_blocks = total_q * heads * (d / 32), nk_blocks = total_kv * heads * (d / 32);
-    prof_begin(st);
-    if (nq_blocks > 0)
-        fake_quant_along_d<<<(unsigned)((nq_blocks + 255) / 256), 256, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(q), nq_blocks, reinterpret_cast<__nv_bfloat16*>(qf));
-    if (nk_blocks > 0)
-        fake_quant_along_d<<<(unsigned)((nk_blocks + 255) / 256), 256, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(k), nk_blocks, reinterpret_cast<__nv_bfloat16*>(kf));
-    prof_end(st, K_QUANT_ALONG_D);
-    if (batch > 0 && max_kv_len > 0) {
-        const int slots = (max_kv_len + 31) / 32 < kRowSlots ? (max_kv_len + 31) / 32 : kRowSlots;
-        dim3 grid(batch, slots);
-        prof_begin(st);
-        mx_along_rows<true><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), kv_off,
-                                                  total_kv, heads * d, nullptr, nullptr,
-                                                  reinterpret_cast<__nv_bfloat16*>(vf));
-        prof_end(st, K_QUANT_ALONG_ROWS);
-    }
-    return cudaGetLastError();
-}
-
-cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
-                        int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,
-                        uint8_t* scales, cudaStream_t st) {
-    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (!along_rows) {
-        int64_t n_blocks = rows * heads * (d / 32);
-        if (n_blocks == 0) return cudaSuccess;
-        int64_t grid = (n_blocks + 255) / 256;
-        prof_begin(st);
-        quant_along_d<<<(unsigned)grid, 256, 0, st>>>(xb, n_blocks, codes, scales);
-        prof_end(st, K_QUANT_ALONG_D);
-    } else {
-        if (batch == 0 || max_rows_per_seq == 0) return cudaSuccess;
-        const int slots = (max_rows_per_seq + 31) / 32 < kRowSlots ? (max_rows_per_seq + 31) / 32 : kRowSlots;
-        dim3 grid(batch, slots);
-        prof_begin(st);
-        mx_along_rows<false><<<grid, 256, 0, st>>>(xb, offsets, rows, heads * d, codes, scales, nullptr);
-        prof_end(st, K_QUANT_ALONG_ROWS);
-    }
-    return cudaGetLastError();
+    cudaError_t e = quantize_mx(q, total_q, heads, d, nullptr, 0, 0, 0, nullptr, nullptr, qf, st);
+    if (e == cudaSuccess) e = quantize_mx(k, total_kv, heads, d, nullptr, 0, 0, 0, nullptr, nullptr, kf, st);
+    if (e == cudaSuccess)
+        e = quantize_mx(v, total_kv, heads, d, kv_off, batch, max_kv_len, 1, nullptr, nullptr, vf, st);
+    return e;
 }
 
 }  // namespace jfa

@@ -24,7 +24,7 @@ cudaError_t mx_fake_quant_qkv(const void* q, const void* k, const void* v, const
                               int max_kv_len, void* qf, void* kf, void* vf, cudaStream_t st);
 cudaError_t quantize_mx(const void* x, int64_t rows, int heads, int d, const int32_t* offsets,
                         int batch, int max_rows_per_seq, int along_rows, uint8_t* codes,
-                        uint8_t* scales, cudaStream_t st);
+                        uint8_t* scales, void* dequant, cudaStream_t st);
 cudaError_t tc_forward_mx_launch(const jfa_problem& p, const AttnArgs& a, const void* q8,
                                  const uint8_t* qs, const void* k8, const uint8_t* ks,
                                  const void* v8, const uint8_t* vs, int64_t n_vblocks,
@@ -142,12 +142,12 @@ cudaError_t tc_forward(const jfa_problem& p, const AttnArgs& a, void* ws_extra, 
         uint8_t *v8 = reinterpret_cast<uint8_t*>(ws + L.v8);
         uint8_t *qs = reinterpret_cast<uint8_t*>(ws + L.qs), *ks = reinterpret_cast<uint8_t*>(ws + L.ks);
         uint8_t *vs = reinterpret_cast<uint8_t*>(ws + L.vs);
-        cudaError_t e = quantize_mx(a.q, p.total_q, p.heads, p.head_dim, nullptr, 0, 0, 0, q8, qs, st);
+        cudaError_t e = quantize_mx(a.q, p.total_q, p.heads, p.head_dim, nullptr, 0, 0, 0, q8, qs, nullptr, st);
         if (e == cudaSuccess)
-            e = quantize_mx(a.k, p.total_kv, p.heads, p.head_dim, nullptr, 0, 0, 0, k8, ks, st);
+            e = quantize_mx(a.k, p.total_kv, p.heads, p.head_dim, nullptr, 0, 0, 0, k8, ks, nullptr, st);
         if (e == cudaSuccess)
             e = quantize_mx(a.v, p.total_kv, p.heads, p.head_dim, a.kv_off, p.batch, p.max_kv_len, 1,
-                            v8, vs, st);
+                            v8, vs, nullptr, st);
         if (e != cudaSuccess) return e;
         return tc_forward_mx_launch(p, aa, q8, qs, k8, ks, v8, vs, mx_vblocks(p),
                                     reinterpret_cast<int32_t*>(ws + L.vbase), st);

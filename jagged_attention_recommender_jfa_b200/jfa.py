@@ -37,6 +37,7 @@ STATUS_NAMES = {0: "JFA_OK", 1: "JFA_ERR_INVALID_ARGUMENT", 2: "JFA_ERR_UNSUPPOR
 
 # Every symbol include/jfa.h declares.
 EXPORTS = ("jfa_workspace_bytes", "jfa_forward", "jfa_backward", "jfa_quantize_mxfp8",
+           "jfa_quantize_mxfp8_dequant",
            "jfa_schedule", "jfa_check_error", "jfa_last_error", "jfa_path",
            "jfa_profile_enable", "jfa_profile_read", "jfa_kernel_name",
            "jfa_forward_fixed_scratch", "jfa_partition", "jfa_backward_dbias",
@@ -85,6 +86,8 @@ def load():
         lib.jfa_backward.restype = i32
         lib.jfa_quantize_mxfp8.argtypes = [P, i64, i32, i32, P, i32, i32, i32, P, P, P]
         lib.jfa_quantize_mxfp8.restype = i32
+        lib.jfa_quantize_mxfp8_dequant.argtypes = [P, i64, i32, i32, P, i32, i32, i32, P, P, P, P]
+        lib.jfa_quantize_mxfp8_dequant.restype = i32
         lib.jfa_schedule.argtypes = [PP, P, P, i32, i32, i32, P, i64, P, P, sz, P]
         lib.jfa_schedule.restype = i32
         lib.jfa_check_error.argtypes = [P, P]
@@ -225,6 +228,14 @@ def jfa_quantize_mxfp8(x, rows, heads, d, offsets, batch, max_len, along_rows, c
     _check(load().jfa_quantize_mxfp8(_addr(x), int(rows), int(heads), int(d), _addr(offsets),
                                      int(batch), int(max_len), int(bool(along_rows)),
                                      _addr(codes), _addr(scales), _stream(stream)))
+
+
+def jfa_quantize_mxfp8_dequant(x, rows, heads, d, offsets, batch, max_len, along_rows, codes,
+                               scales, dequant, stream=None):
+    _check(load().jfa_quantize_mxfp8_dequant(_addr(x), int(rows), int(heads), int(d), _addr(offsets),
+                                             int(batch), int(max_len), int(bool(along_rows)),
+                                             _addr(codes), _addr(scales), _addr(dequant),
+                                             _stream(stream)))
 
 
 def jfa_schedule(problem, q_offsets, kv_offsets, causal, backward, tile, items, capacity, count,

@@ -574,6 +574,58 @@ def test_mxfp8_prequantised_entry_matches(cuda_device):
     assert ei.value.status == jfa.JFA_ERR_UNSUPPORTED
 
 
+def test_mxfp8_training_step_from_producer(cuda_device):
+    # the producer writes the codes and the dequantised operands in one pass
+    # (jfa_quantize_mxfp8_dequant); jfa_forward_mxfp8 takes the codes and a
+    # bf16 jfa_backward the dequantised operands: the dequantised values are
+    # the oracle's exactly, the forward is the MXFP8 forward's bitwise, dK and
+    # dV are the MXFP8 backward's bitwise (same kernel, same values; dQ adds
+    # key tiles in an arbitrary order), and all match the oracle
+    p = make_problem("self_mxfp8", 34, B=6, max_len=330)
+    d = _dev(p, cuda_device)
+    prob = jfa.problem_of(p)
+    rows_q, H, dd = p.q.shape
+    rows_k = p.k.shape[0]
+    u8 = dict(dtype=torch.uint8, device=cuda_device)
+    q8, k8, v8 = torch.empty(rows_q, H, dd, **u8), torch.empty(rows_k, H, dd, **u8), torch.empty(rows_k, H, dd, **u8)
+    qs, ks = torch.empty(rows_q, H, dd // 32, **u8), torch.empty(rows_k, H, dd // 32, **u8)
+    vs = torch.zeros(rows_k // 32 + p.B, H, dd, **u8)
+    qd, kd, vd = (torch.full_like(d[n], float("nan")) for n in ("q", "k", "v"))
+    jfa.jfa_quantize_mxfp8_dequant(d["q"], rows_q, H, dd, None, 0, 0, False, q8, qs, qd)
+    jfa.jfa_quantize_mxfp8_dequant(d["k"], rows_k, H, dd, None, 0, 0, False, k8, ks, kd)
+    jfa.jfa_quantize_mxfp8_dequant(d["v"], rows_k, H, dd, d["kv_off"], p.B, p.max_kv_len, True, v8, vs, vd)
+    rq, rk, rv = mx_dequantised_inputs(p)
+    for name, got, ref in (("Q", qd, rq), ("K", kd, rk), ("V", vd, rv)):
+        assert np.array_equal(got.double().cpu().numpy(), ref), name
+    rc, rs = oracle.quantize_mx_along_rows(p.v, p.kv_off)
+    assert np.array_equal(v8.cpu().numpy(), rc)
+    assert np.array_equal(vs[:rs.shape[0]].cpu().numpy(), rs)
+    ws = jfa.workspace(prob, False, cuda_device)
+    out = torch.full_like(d["q"], float("nan"))
+    lse = torch.full((p.total_q, H), float("nan"), device=cuda_device)
+    jfa.jfa_forward_mxfp8(prob, q8, qs, k8, ks, v8, vs, d["q_off"], d["kv_off"], d["bias"], True,
+                          out, lse, ws)
+    jfa.jfa_check_error(ws)
+    bprob = jfa.problem_of(p, dtype="bf16")
+    dq, dk, dv = jfa.attention_backward(bprob, qd, kd, vd, out, lse, d["dout"], d["q_off"],
+                                        d["kv_off"], d["bias"], "softmax", True)
+    ref_out, ref_lse = jfa.attention_forward(prob, d["q"], d["k"], d["v"], d["q_off"],
+                                             d["kv_off"], d["bias"], "softmax", True)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    mdq, mdk, mdv = jfa.attention_backward(prob, d["q"], d["k"], d["v"], out, lse, d["dout"],
+                                           d["q_off"], d["kv_off"], d["bias"], "softmax", True)
+    torch.cuda.synchronize()
+    assert torch.equal(dk, mdk) and torch.equal(dv, mdv)
+    kw = dict(bias=p.bias, bias_kind=p.bias_kind, relpos_len=p.relpos_len, act="softmax", causal=True)
+    ro, rl = oracle.forward(p.q_off, p.kv_off, rq, rk, rv, quant_p=True, **kw)
+    rdq, rdk, rdv = oracle.backward(p.q_off, p.kv_off, rq, rk, rv, p.dout, out_for_d=ro, **kw)
+    compare("O", out, ro, slice(None), MX_MAX)
+    compare("LSE", lse, rl, slice(None), LSE_MAX)
+    compare("dQ", dq, rdq, slice(None), MX_MAX)
+    compare("dK", dk, rdk, slice(None), MX_MAX)
+    compare("dV", dv, rdv, slice(None), MX_MAX)
+
+
 # ---------------------------------------------------------------------------
 # the general backward's query tiles start at the first query that sees a key
 # tile: on 128-row block boundaries for self-attention and for n_kv - n_q a
