@@ -82,13 +82,17 @@ def parse_args():
                     help="split of the global batch across ranks (N > 1)")
     ap.add_argument("--sub-batch", type=int, default=8,
                     help="sequences per sub-batch for --partition bbs")
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=16,
+                    help="timed steps of the end-to-end leg (its pipeline fills and drains once)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-padded", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mx-internal", action="store_true",
                     help="MXFP8: run jfa_forward / jfa_backward with dtype MXFP8 (quantising inside "
                          "each call) instead of the producer form of the step")
+    ap.add_argument("--copy-probe", action="store_true",
+                    help="time pinned host<->device copies of the e2e leg's size (in alone, out "
+                         "alone, both at once on two streams), print one JSON line and exit")
     ap.add_argument("--fp8-peak-probe", action="store_true",
                     help="time the library FP8 GEMM (E4M3, and MX-scaled where supported) at 8192^3 "
                          "as the fp8 roofline denominator, print one JSON line and exit")
@@ -470,6 +474,47 @@ def fp8_peak_probe(dev, n=8192, warmup=5, iters=20):
     return out
 
 
+def copy_probe(dev, nbytes=1_821_206_568, reps=5):
+    """Host link bandwidth for the end-to-end leg: pinned host memory to the
+    device, back, and both directions at once on two streams, timed with
+    CUDA events; nbytes is one self_bf16 step's input (Q, K, V, dO, offsets,
+    bias table)."""
+    h_in = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    h_out = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_out = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def timed(do_in, do_out):
+        ms = []
+        for _ in range(reps + 1):
+            torch.cuda.synchronize(dev)
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            up.wait_event(t0)
+            down.wait_event(t0)
+            if do_in:
+                with torch.cuda.stream(up):
+                    d_in.copy_(h_in, non_blocking=True)
+            if do_out:
+                with torch.cuda.stream(down):
+                    h_out.copy_(d_out, non_blocking=True)
+            cur = torch.cuda.current_stream(dev)
+            cur.wait_stream(up)
+            cur.wait_stream(down)
+            t1.record()
+            torch.cuda.synchronize(dev)
+            ms.append(t0.elapsed_time(t1))
+        return statistics.median(ms[1:])
+
+    res = {"probe": "host_copies", "bytes_per_direction": nbytes}
+    for name, a, b in (("h2d", True, False), ("d2h", False, True), ("both", True, True)):
+        ms = timed(a, b)
+        res[name + "_ms"] = ms
+        res[name + "_gbs_per_direction"] = nbytes / (ms * 1e-3) / 1e9
+    return res
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -492,6 +537,10 @@ def main():
     if args.fp8_peak_probe:
         if rank == 0:
             print(json.dumps(fp8_peak_probe(dev)))
+        return
+    if args.copy_probe:
+        if rank == 0:
+            print(json.dumps(copy_probe(dev)))
         return
     from jagged_attention_recommender_jfa_b200 import jfa
     from jagged_attention_recommender_jfa_b200.inputs import WORKLOADS, draw_lengths
