@@ -48,6 +48,10 @@
  *  - Streams: all work is enqueued on `stream` (NULL = legacy default stream);
  *    there is no host synchronisation.  max_q_len / max_kv_len / total_* come
  *    from the host so that no device->host copy is needed to size grids.
+ *    So the compute calls (forward, backward, quantisers, schedule) can be
+ *    captured in a CUDA graph and replayed on new data written into the same
+ *    buffers (the work-item counters and the error word are reset by each
+ *    call's schedule); jfa_check_error() synchronises and is not for capture.
  *  - Alignment: tensors 16-byte aligned.
  *  - Errors are returned, never thrown; nothing aborts or traps.  Argument
  *    errors are detected on the host before anything is enqueued.  Offsets

@@ -626,6 +626,63 @@ def test_mxfp8_training_step_from_producer(cuda_device):
     compare("dV", dv, rdv, slice(None), MX_MAX)
 
 
+@pytest.mark.parametrize("workload", ["self_bf16", "cross_bf16"])
+def test_step_replays_from_a_cuda_graph(cuda_device, workload):
+    # the calls allocate nothing and never wait on the host, so a training
+    # step (schedules, bias preparation, forward, backward) can be captured
+    # once in a CUDA graph and replayed on new inputs copied into the
+    # captured buffers: the forward and dK / dV equal eager calls bitwise
+    # (dQ adds key tiles in an arbitrary order), and all match the oracle
+    p = make_problem(workload, 41, B=5, max_len=600)
+    d = _dev(p, cuda_device)
+    prob = jfa.problem_of(p)
+    act = p.act
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(p.total_q, p.H, dtype=torch.float32, device=cuda_device)
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+    ws_f, ws_b = jfa.workspace(prob, False, cuda_device), jfa.workspace(prob, True, cuda_device)
+    side = torch.cuda.Stream(cuda_device)
+
+    def step(stream):
+        jfa.jfa_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"], d["bias"], act,
+                        p.causal, out, lse, ws_f, stream=stream)
+        jfa.jfa_backward(prob, d["q"], d["k"], d["v"], out, lse, d["dout"], d["q_off"], d["kv_off"],
+                         d["bias"], act, p.causal, dq, dk, dv, ws_b, stream=stream)
+
+    side.wait_stream(torch.cuda.current_stream(cuda_device))
+    with torch.cuda.stream(side):
+        step(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step(side)
+    for seed in (42, 43):
+        fresh = make_problem(workload, seed, B=5, max_len=600, q_lens=np.diff(p.q_off.numpy()),
+                             kv_lens=np.diff(p.kv_off.numpy()))
+        for n in ("q", "k", "v", "dout", "bias"):
+            if d[n] is not None:
+                d[n].copy_(getattr(fresh, n).to(cuda_device))
+        graph.replay()
+        torch.cuda.synchronize()
+        jfa.jfa_check_error(ws_f)
+        jfa.jfa_check_error(ws_b)
+        e_out, e_lse = jfa.attention_forward(prob, d["q"], d["k"], d["v"], d["q_off"], d["kv_off"],
+                                             d["bias"], act, p.causal)
+        e_dq, e_dk, e_dv = jfa.attention_backward(prob, d["q"], d["k"], d["v"], e_out, e_lse,
+                                                  d["dout"], d["q_off"], d["kv_off"], d["bias"],
+                                                  act, p.causal)
+        torch.cuda.synchronize()
+        assert torch.equal(out, e_out) and torch.equal(dk, e_dk) and torch.equal(dv, e_dv)
+        if act == "softmax":
+            assert torch.equal(lse, e_lse)
+        ro, rl, (rdq, rdk, rdv) = run_oracle(fresh, act)
+        compare("O", out, ro, slice(None), BF16_MAX, BF16_MEAN)
+        compare("dQ", dq, rdq, slice(None), BF16_MAX, BF16_MEAN)
+        compare("dK", dk, rdk, slice(None), BF16_MAX, BF16_MEAN)
+        compare("dV", dv, rdv, slice(None), BF16_MAX, BF16_MEAN)
+    del graph
+
+
 # ---------------------------------------------------------------------------
 # the general backward's query tiles start at the first query that sees a key
 # tile: on 128-row block boundaries for self-attention and for n_kv - n_q a
