@@ -1,0 +1,75 @@
+"""Randomised batches on the GPU against the oracle.
+
+Each seed draws a workload (causal self-attention, short queries over long
+keys, GDPA), an activation, the causal rule, a bias kind, a head count, a
+sliding window or none, and sequence lengths mixed from tile edges (0, 1,
+63..65, 127..129, 255..257) and uniform draws, so that the tile schedules,
+the persistent backward's work queue, the forward's slot alternation and the
+short-query kernels meet shapes no hand-picked case lists.  Tolerances are
+those of the parity tests; GDPA sequences keep at least 8 keys (a single
+key leaves nothing to divide the score gradient, which the edge tests cover
+with their own bound).
+
+Pages: "Meta GEM Training Efficiency: Why LLM-Scale Recommenders Need a
+Different Stack", "Bottleneck move 1: dense-sequence kernels to jagged
+execution" (jagged tiles of uneven length, custom biases, GDPA).
+"""
+import numpy as np
+import pytest
+
+from jagged_attention_recommender_jfa_b200.inputs import make_problem
+from test_gpu_window import check_window
+
+pytestmark = pytest.mark.gpu
+
+EDGES = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257]
+
+
+def draw_case(seed):
+    rng = np.random.default_rng(1000 + seed)
+    workload = ["self_bf16", "cross_bf16", "gdpa_bf16"][rng.integers(0, 3)]
+    if workload == "gdpa_bf16":
+        act = ["silu", "gelu_tanh"][rng.integers(0, 2)]
+    else:
+        act = ["softmax", "softmax", "silu", "gelu_tanh"][rng.integers(0, 4)]
+    causal = bool(rng.integers(0, 2))
+    bias = ["none", "relpos", "dense"][rng.integers(0, 3)]
+    H = int(rng.integers(1, 4))
+    B = int(rng.integers(1, 7))
+
+    def lengths(hi):
+        return [int(EDGES[rng.integers(0, len(EDGES))]) if rng.random() < 0.5
+                else int(rng.integers(1, hi)) for _ in range(B)]
+
+    if workload == "self_bf16":
+        q_lens = lengths(700)
+        kv_lens = list(q_lens)
+    else:
+        short = rng.random() < 0.5
+        q_lens = [min(x, 64) for x in lengths(65)] if short else lengths(400)
+        kv_lens = lengths(900)
+    if act != "softmax":
+        kv_lens = [max(x, 8) for x in kv_lens]
+    if sum(q_lens) == 0:
+        q_lens[0] = 5
+    if sum(kv_lens) == 0:
+        kv_lens[0] = 9
+    window = int([0, 0, 1, 17, 128, 300][rng.integers(0, 6)])
+    return dict(workload=workload, act=act, causal=causal, bias=bias, H=H, q_lens=q_lens,
+                kv_lens=kv_lens, window=window)
+
+
+def test_draws_cover_the_kinds():
+    cases = [draw_case(s) for s in range(16)]
+    assert {c["workload"] for c in cases} == {"self_bf16", "cross_bf16", "gdpa_bf16"}
+    assert {c["bias"] for c in cases} == {"none", "relpos", "dense"}
+    assert any(c["window"] > 0 for c in cases) and any(c["window"] == 0 for c in cases)
+    assert any(max(c["q_lens"]) <= 64 for c in cases) and any(max(c["q_lens"]) > 128 for c in cases)
+
+
+@pytest.mark.parametrize("seed", range(64))
+def test_random_batch(cuda_device, seed):
+    c = draw_case(seed)
+    p = make_problem(c["workload"], seed, q_lens=c["q_lens"], kv_lens=c["kv_lens"], act=c["act"],
+                     causal=c["causal"], bias=c["bias"], H=c["H"])
+    check_window(p, cuda_device, c["window"], act=c["act"])
