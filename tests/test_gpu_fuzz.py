@@ -5,7 +5,10 @@ keys, GDPA), an activation, the causal rule, a bias kind, a head count, a
 sliding window or none, and sequence lengths mixed from tile edges (0, 1,
 63..65, 127..129, 255..257) and uniform draws, so that the tile schedules,
 the persistent backward's work queue, the forward's slot alternation and the
-short-query kernels meet shapes no hand-picked case lists.  Tolerances are
+short-query kernels meet shapes no hand-picked case lists.  Two more draws
+take the CUDA-core path (fp32 or bf16 storage, head_dim 32 / 64 / 128) and
+the MXFP8 path (softmax, its own 6e-2 bound on the oracle's dequantised
+operands).  Tolerances are
 those of the parity tests; GDPA sequences keep at least 8 keys (a single
 key leaves nothing to divide the score gradient, which the edge tests cover
 with their own bound).
@@ -18,6 +21,7 @@ import numpy as np
 import pytest
 
 from jagged_attention_recommender_jfa_b200.inputs import make_problem
+from test_gpu_parity import mx_dequantised_inputs
 from test_gpu_window import check_window
 
 pytestmark = pytest.mark.gpu
@@ -73,3 +77,23 @@ def test_random_batch(cuda_device, seed):
     p = make_problem(c["workload"], seed, q_lens=c["q_lens"], kv_lens=c["kv_lens"], act=c["act"],
                      causal=c["causal"], bias=c["bias"], H=c["H"])
     check_window(p, cuda_device, c["window"], act=c["act"])
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_batch_cuda_core(cuda_device, seed):
+    c = draw_case(seed)
+    rng = np.random.default_rng(2000 + seed)
+    d = int([32, 64, 128][rng.integers(0, 3)])
+    dtype = "f32" if (d == 128 or rng.random() < 0.5) else "bf16"
+    p = make_problem(c["workload"], seed, q_lens=c["q_lens"], kv_lens=c["kv_lens"], act=c["act"],
+                     causal=c["causal"], bias=c["bias"], H=c["H"], d=d, dtype=dtype)
+    check_window(p, cuda_device, c["window"], act=c["act"], strict_f32=(dtype == "f32"))
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_batch_mxfp8(cuda_device, seed):
+    c = draw_case(seed)
+    p = make_problem("self_mxfp8", seed, q_lens=c["q_lens"], kv_lens=c["kv_lens"], act="softmax",
+                     causal=c["causal"], bias=c["bias"], H=c["H"])
+    check_window(p, cuda_device, c["window"], inputs=mx_dequantised_inputs(p), quant_p=True,
+                 mx=True)
