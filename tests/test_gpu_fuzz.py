@@ -8,7 +8,9 @@ the persistent backward's work queue, the forward's slot alternation and the
 short-query kernels meet shapes no hand-picked case lists.  Two more draws
 take the CUDA-core path (fp32 or bf16 storage, head_dim 32 / 64 / 128) and
 the MXFP8 path (softmax, its own 6e-2 bound on the oracle's dequantised
-operands).  Tolerances are
+operands), and one more the bias gradient (relative-position table or dense
+jagged bias, against the oracle's, as the bias-gradient parity tests check
+it).  Tolerances are
 those of the parity tests; GDPA sequences keep at least 8 keys (a single
 key leaves nothing to divide the score gradient, which the edge tests cover
 with their own bound).
@@ -97,3 +99,19 @@ def test_random_batch_mxfp8(cuda_device, seed):
                      causal=c["causal"], bias=c["bias"], H=c["H"])
     check_window(p, cuda_device, c["window"], inputs=mx_dequantised_inputs(p), quant_p=True,
                  mx=True)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_batch_bias_gradient(cuda_device, seed):
+    from test_gpu_dbias import (BF16_MAX, BF16_MEAN, check_dense, check_relpos, dense_mask,
+                                oracle_dbias, pairs_per_entry, run_gpu)
+    c = draw_case(seed)
+    bias = c["bias"] if c["bias"] != "none" else ["relpos", "dense"][seed % 2]
+    p = make_problem(c["workload"], seed, q_lens=c["q_lens"], kv_lens=c["kv_lens"], act=c["act"],
+                     causal=c["causal"], bias=bias, H=c["H"])
+    db = run_gpu(p, cuda_device, c["act"])
+    ref = oracle_dbias(p, c["act"])
+    if bias == "relpos":
+        check_relpos("dtable", db, ref, pairs_per_entry(p), BF16_MAX, BF16_MEAN)
+    else:
+        check_dense("dbias", db, ref, BF16_MAX, BF16_MEAN, valid=dense_mask(p))
