@@ -10,7 +10,7 @@ take the CUDA-core path (fp32 or bf16 storage, head_dim 32 / 64 / 128) and
 the MXFP8 path (softmax, its own 6e-2 bound on the oracle's dequantised
 operands), and one more the bias gradient (relative-position table or dense
 jagged bias, against the oracle's, as the bias-gradient parity tests check
-it).  Tolerances are
+it); eight draws take a few sequences of 1,000 to 3,000 tokens.  Tolerances are
 those of the parity tests; GDPA sequences keep at least 8 keys (a single
 key leaves nothing to divide the score gradient, which the edge tests cover
 with their own bound).
@@ -115,3 +115,19 @@ def test_random_batch_bias_gradient(cuda_device, seed):
         check_relpos("dtable", db, ref, pairs_per_entry(p), BF16_MAX, BF16_MEAN)
     else:
         check_dense("dbias", db, ref, BF16_MAX, BF16_MEAN, valid=dense_mask(p))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_long_sequences(cuda_device, seed):
+    # a few sequences of 1,000 to 3,000 tokens: 8 to 24 key tiles per query
+    # row, the lazy rescale firing again and again, long persistent items
+    rng = np.random.default_rng(3000 + seed)
+    B = int(rng.integers(1, 4))
+    lens = [int(x) for x in rng.integers(1000, 3001, size=B)]
+    causal = bool(rng.integers(0, 2))
+    bias = ["none", "relpos"][rng.integers(0, 2)]
+    window = int([0, 0, 700][rng.integers(0, 3)])
+    act = ["softmax", "softmax", "silu"][rng.integers(0, 3)]
+    p = make_problem("self_bf16", seed, q_lens=lens, kv_lens=lens, act=act, causal=causal,
+                     bias=bias, H=2)
+    check_window(p, cuda_device, window, act=act)
