@@ -66,7 +66,7 @@ constexpr int kTestWaitLimitUs = 5000;  // the injected failure's wait limit
 
 const char* const kKernelNames[K_COUNT] = {
     "sched_prepare", "sched_rank", "simt_fwd", "simt_bwd_pre", "simt_bwd_dq", "simt_bwd_dkdv",
-    "quant_along_d", "quant_along_rows", "tc_fwd", "tc_bwd_pre", "tc_bwd", "tc_dq_finalize",
+    "mx_along_d", "mx_along_rows", "tc_fwd", "tc_bwd_pre", "tc_bwd", "tc_dq_finalize",
     "tc_fwd_mxfp8", "tc_bias_prep", "dbias_zero_masked", "norm_quantize_mxfp8", "tc_bwd_sq", "tc_fwd_sq"};
 
 }  // namespace
